@@ -1,0 +1,397 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 selective scan (S6) forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one forward scan (softplus, discretisation, recurrence, C
+contraction, D skip, SiLU gate, last_state) over one batch of the workload,
+inputs resident in HBM.  The default workload is the Mamba-2.8B layer shape
+(batch 4, L 8192, d_inner 5120, d_state 16, bf16 io, fp32 state).  Multi-GPU
+runs (torchrun, one rank per GPU) process one independent replica per rank:
+the scan's (batch, channel) rows are independent, so there is no collective
+(weak scaling).  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores (bounded samples
+of the same workload), the only reference implementation there is.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "selective-scan fwd/bwd tokens·channels/s and % of HBM/SFU roofline, 1 B200"
+UNIT = "tokens·channels/s"
+MUFU_EX2_PER_CLK_PER_SM = 16  # special-function unit ex2 rate per SM and clock
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fwd_lookback_mamba-2.8b-layer.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "selective_state_space_54_b200", "csrc", f)
+                  for f in ("ssm_fwd.cu", "ssm_common.cuh")]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba-2.8b-layer", choices=list(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "sm_max_mhz": d.get("sm_max_mhz", 1965.0),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def alg_bytes(w: synth.Workload) -> int:
+    """Bytes every input and output must cross HBM once."""
+    es = 2 if w.dtype == synth.BF16 else 4
+    bld = w.bld
+    b = 4 * bld * es                                   # u, delta, z in; y out
+    b += 2 * w.batch * w.seqlen * w.dstate * es        # B, C
+    b += w.dim * w.dstate * 4 + 2 * w.dim * 4          # A, D, delta_bias
+    if w.last_state:
+        b += w.batch * w.dim * w.dstate * 4
+    return b
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    vals = {}
+    for line in open(PROFILE_TRAFFIC):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ssm_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                             "power": float(parts[3]) if parts[3] not in ("[N/A]", "") else None,
+                             "active": parts[4], "hw": parts[5], "hw_thermal": parts[6],
+                             "sw_thermal": parts[7], "sw_power": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] is None or r["power"] > 250] or rows
+        reasons = set()
+        for r in loaded:
+            for k, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                            ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows), "samples": len(loaded),
+                "reasons": sorted(reasons)}
+
+
+def init_dist(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def cpu_baseline(w: synth.Workload, case: dict, target_s: float = 12.0) -> dict:
+    """The fp64 oracle as it stands, timed on the host cores on a bounded sample."""
+    import oracle
+    threads = oracle.default_threads()
+    nch = w.batch * w.dim
+    k = min(nch, max(threads, 16))
+    t_first = None
+    while True:
+        chans = synth.sample_channels(w, k)
+        subs = synth.subset_case(case, chans)
+        t0 = time.perf_counter()
+        for _, _, sub in subs:
+            oracle.fwd(sub, nthreads=threads)
+        dt = time.perf_counter() - t0
+        t_first = t_first or dt
+        if dt >= target_s * 0.5 or k >= nch:
+            break
+        k = min(nch, int(k * max(2.0, target_s / max(dt, 1e-3))))
+    return {"value": k * w.seqlen / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{k} of {nch} (batch, channel) rows over the full L={w.seqlen}, "
+                      f"fp64, {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    case = synth.make_workload(w)
+    threads = oracle.default_threads()
+    nch = w.batch * w.dim
+    # size one step to about 3 s of host work
+    k = min(nch, max(threads, 8))
+    chans = synth.sample_channels(w, k)
+    subs = synth.subset_case(case, chans)
+    t0 = time.perf_counter()
+    for _, _, sub in subs:
+        oracle.fwd(sub, nthreads=threads)
+    dt = time.perf_counter() - t0
+    k = min(nch, max(1, int(k * 3.0 / max(dt, 1e-3))))
+    chans = synth.sample_channels(w, k)
+    subs = synth.subset_case(case, chans)
+    for _ in range(args.warmup):
+        for _, _, sub in subs:
+            oracle.fwd(sub, nthreads=threads)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        for _, _, sub in subs:
+            oracle.fwd(sub, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    value = k * w.seqlen / per_step
+    sample = f"{k} of {nch} (batch, channel) rows over the full L={w.seqlen} per step, fp64"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, "oracle"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def to_torch(x, device):
+    """numpy input (bf16 bits as uint16, or fp32) -> torch tensor on device."""
+    import torch
+    if x.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device)
+
+
+def config_of(w, path):
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
+            "d_state": w.dstate, "io_dtype": w.dtype, "state_dtype": "f32",
+            "delta_softplus": True, "z_gate": True, "last_state": w.last_state, "path": path,
+            "l2": "inputs larger than L2 (no flush)" if alg_bytes(w) > 126e6 else "L2 resident",
+            "seed": w.seed}
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import selective_state_space_54_b200 as ssm
+    from selective_state_space_54_b200 import _lib
+
+    world, rank, local = init_dist(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if w.backward:
+        raise SystemExit("forward workloads only in this benchmark")
+
+    case = synth.make_workload(w)
+    g = {k: to_torch(case[k], dev) for k in ("u", "delta", "z", "B", "C")}
+    for k in ("A", "D", "delta_bias"):
+        g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
+    y = torch.empty_like(g["u"])
+    ls = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+    shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
+                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32)
+    path = ssm.fwd_path(shape)
+    ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    launches_per_step = {"lookback": 1, "per_group": 1, "split_l": 3}[path]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                     y=y, last_state=ls, return_last_state=True, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    ssm.check(ws)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if world == 1 else local) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ssm.check(ws)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    clocks = clk.summary()
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        host = {k: g[k].cpu().pin_memory() for k in ("u", "delta", "z", "B", "C", "A", "D", "delta_bias")}
+        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        ls_host = torch.empty(ls.shape, dtype=ls.dtype).pin_memory()
+        dbuf = {k: torch.empty_like(g[k]) for k in host}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = y_host.numel() * y_host.element_size() + ls_host.numel() * ls_host.element_size()
+
+        def e2e_step():
+            for k in host:
+                dbuf[k].copy_(host[k], non_blocking=True)
+            ssm.scan_fwd(dbuf["u"], dbuf["delta"], dbuf["A"], dbuf["B"], dbuf["C"], dbuf["D"],
+                         dbuf["z"], dbuf["delta_bias"], y=y, last_state=ls,
+                         return_last_state=True, workspace=ws)
+            y_host.copy_(y, non_blocking=True)
+            ls_host.copy_(ls, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        k_e2e = max(3, min(10, args.steps))
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / k_e2e)
+        e2e = {"value": world * w.bld / (ms_e2e * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+        del host, dbuf
+
+    pk = peaks()
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    sec = ms * 1e-3
+    ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
+    achieved = w.bldn / sec
+    roofline = {"bound": "alu", "achieved": achieved / 1e12, "peak": ex2_peak / 1e12,
+                "unit": "Tex2/s", "frac": achieved / ex2_peak,
+                "traffic": profiled_traffic(),
+                "kernel": "k_fwd_lookback" if path == "lookback" else f"k_fwd_segment ({path})",
+                "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
+                              f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})",
+                "algorithmic_bytes": alg_bytes(w),
+                "hbm_achieved_gbs": alg_bytes(w) / sec / 1e9, "hbm_peak_gbs": pk["hbm_gbs"],
+                "hbm_frac": alg_bytes(w) / sec / 1e9 / pk["hbm_gbs"]}
+    if clocks and clocks.get("sm_mhz"):
+        at_clock = sm_count * MUFU_EX2_PER_CLK_PER_SM * clocks["sm_mhz"] * 1e6
+        roofline["frac_at_measured_clock"] = achieved / at_clock
+
+    line = {"metric": METRIC, "value": world * w.bld / sec, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
+            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, case)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    _ = _lib
+
+
+if __name__ == "__main__":
+    main()

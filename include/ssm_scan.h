@@ -1,0 +1,164 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 selective-scan (S6) library, libssmscan.so.
+ *
+ * The operation (all entry points below compute parts of it):
+ *
+ *   Delta_t = softplus(delta_t + delta_bias)        (or delta_t + delta_bias)
+ *   Abar_t  = exp(Delta_t * A)                     diagonal A, per channel
+ *   h_t     = Abar_t (.) h_{t-1} + Delta_t * B_t * u_t
+ *   y_t     = (C_t . h_t + D * u_t) * SiLU(z_t)
+ *
+ * Sources: "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ * (xyznot.com reading guide), section "Metodo" (zero-order hold,
+ * Abar = exp(Delta A), recurrence h_t = Abar h_{t-1} + Bbar x_t) and section
+ * "O Mecanismo de Selecao (S6)" (B_t, C_t input dependent, Delta_t =
+ * softplus(Parameter + s_Delta(x_t))); "O que e um modelo Mamba?" (ibm.com),
+ * output equation y = C h + D x and the Mamba block walk-through (the SSM
+ * output is multiplied by the activated z branch); "Как работает Mamba
+ * (State Space Model)..." (aivaro.ru), section 3, the selective_scan(u,
+ * delta, A, B, C, D) example, whose Euler input term B_bar = delta * B this
+ * library uses.  The expanded (batch, seqlen, dim, dstate) state is never
+ * written to memory (reading guide, "Expansao de Estado Ciente de Hardware").
+ *
+ * Layouts (row-major, last index contiguous; "dim" is d_inner, "dstate" N):
+ *   u, delta, z, y, dout, du, ddelta, dz   [batch][dim][seqlen]   io dtype
+ *   B, C, dB, dC                           [batch][seqlen][dstate] io dtype
+ *   A, dA                                  [dim][dstate]          fp32
+ *   D, delta_bias, dD, ddelta_bias         [dim]                  fp32
+ *   initial_state, last_state, dinitial_state [batch][dim][dstate] fp32
+ * io dtype is fp32 or bf16 (ssm_shape.io_dtype).  State and all arithmetic
+ * are fp32.  bf16 results are rounded to nearest-even.
+ *
+ * Ownership and threading: the caller owns every buffer, device pointers
+ * throughout.  The library allocates no memory; scratch comes from the
+ * caller's workspace (sizes from the *_workspace_bytes queries).  Every call
+ * only enqueues work on `stream` and returns; nothing synchronises except
+ * ssm_scan_check().  Calls are thread-safe; two calls that share a workspace
+ * must be ordered on the GPU (same stream, or events).
+ *
+ * Errors: argument checks happen before any launch and return a status with
+ * nothing enqueued.  Launch failures return SSM_ERR_CUDA.  Kernels never trap:
+ * a bounded device-side wait that gives up records SSM_ERR_DEVICE_TIMEOUT in
+ * the workspace header, which ssm_scan_check() reports.
+ */
+#ifndef SSM_SCAN_H_
+#define SSM_SCAN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *ssm_stream_t;
+
+typedef enum {
+  SSM_OK = 0,
+  SSM_ERR_INVALID_ARG = -1,    /* null required pointer, bad size, misaligned */
+  SSM_ERR_UNSUPPORTED = -2,    /* dstate > 64, unknown dtype or path */
+  SSM_ERR_WORKSPACE = -3,      /* workspace missing or smaller than required */
+  SSM_ERR_CUDA = -4,           /* a CUDA runtime call or launch failed */
+  SSM_ERR_DEVICE_TIMEOUT = -5  /* a bounded device wait gave up */
+} ssm_status;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+/* Forward schedule.  AUTO picks from the shape and the device:
+ *  LOOKBACK  one persistent launch; every warp gets an equal share of
+ *            (8-channel group x 32-step chunk) items; a group split between
+ *            two warps passes its state through the workspace with a
+ *            bounded wait (taken only after the writer's first item);
+ *  SPLIT_L   two passes over time segments (segment end states from zero,
+ *            a sequential carry over segments, then the output pass);
+ *            for long sequences with few channels;
+ *  PER_GROUP one warp per 8-channel group over the whole sequence. */
+typedef enum {
+  SSM_PATH_AUTO = 0,
+  SSM_PATH_LOOKBACK = 1,
+  SSM_PATH_SPLIT_L = 2,
+  SSM_PATH_PER_GROUP = 3
+} ssm_path;
+
+typedef struct {
+  int64_t batch;    /* >= 0 */
+  int64_t dim;      /* d_inner, >= 0 */
+  int64_t seqlen;   /* L, >= 0; any value (ragged chunks are handled) */
+  int64_t dstate;   /* N, 1..64 */
+  int32_t io_dtype; /* ssm_dtype */
+  int32_t path;     /* ssm_path (forward only; ignored by the backward) */
+} ssm_shape;
+
+/* Bytes of workspace ssm_scan_fwd needs for `shape` on the current device
+ * (at least 256: the header holding the device error word).  Returns 0 for
+ * an invalid shape. */
+size_t ssm_scan_fwd_workspace_bytes(const ssm_shape *shape);
+
+/* Bytes of workspace ssm_scan_bwd needs (state checkpoints of the forward
+ * recomputation, fp32 dB/dC accumulators, header).  0 for an invalid shape. */
+size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape);
+
+/* Forward selective scan (the operation above).
+ *  u, delta, B, C, A, y          required
+ *  D, z, delta_bias              nullable (term omitted / no gate / no bias)
+ *  initial_state                 nullable: h_{-1} = 0 (aivaro.ru example)
+ *  last_state                    nullable: h_{L-1} is written when given
+ *  delta_softplus                nonzero: Delta = softplus(delta + bias)
+ *  workspace/ws_bytes            device scratch, >= ssm_scan_fwd_workspace_bytes
+ * Pointers must be aligned to their element size; 16-byte aligned rows take
+ * the vector path.  y may not alias an input. */
+ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta,
+                        const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *initial_state,
+                        void *y, float *last_state,
+                        void *workspace, size_t ws_bytes, ssm_stream_t stream);
+
+/* Backward of ssm_scan_fwd by recomputation: the states are recomputed from
+ * the inputs (never read from the forward), reading guide, "Expansao de
+ * Estado Ciente de Hardware".  Gradients of sum(dout * y):
+ *  du, ddelta, dz          [batch][dim][seqlen] io dtype (ddelta is with
+ *                          respect to the raw delta argument)
+ *  dB, dC                  [batch][seqlen][dstate] io dtype, summed over dim
+ *  dA                      [dim][dstate] fp32, summed over batch and seqlen
+ *  dD, ddelta_bias         [dim] fp32, summed over batch and seqlen
+ *  dinitial_state          [batch][dim][dstate] fp32 (nullable)
+ * dz must be given exactly when z is, dD exactly when D is, ddelta_bias when
+ * delta_bias is (else NULL).  Outputs are overwritten, not accumulated. */
+ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta,
+                        const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const float *initial_state,
+                        const void *dout,
+                        void *du, void *ddelta, float *dA, void *dB, void *dC,
+                        float *dD, void *dz, float *ddelta_bias,
+                        float *dinitial_state,
+                        void *workspace, size_t ws_bytes, ssm_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the device error word of
+ * `workspace`.  SSM_OK, SSM_ERR_DEVICE_TIMEOUT or SSM_ERR_CUDA. */
+ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream);
+
+/* Runs only the bounded inter-warp wait used by SSM_PATH_LOOKBACK on a flag
+ * that nothing sets, with a limit of `timeout_us` microseconds (1..10^6), so
+ * that the give-up path can be tested without faulting or hanging the GPU.
+ * Afterwards ssm_scan_check(workspace) must report SSM_ERR_DEVICE_TIMEOUT.
+ * workspace: >= 256 bytes. */
+ssm_status ssm_scan_test_wait_timeout(void *workspace, size_t ws_bytes,
+                                      int64_t timeout_us, ssm_stream_t stream);
+
+/* Path AUTO would choose for `shape` on the current device (for tests and
+ * the benchmark); SSM_PATH_AUTO itself for an invalid shape. */
+int32_t ssm_scan_fwd_path(const ssm_shape *shape);
+
+const char *ssm_status_string(ssm_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t ssm_scan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H_ */

@@ -1,0 +1,177 @@
+"""B200 selective scan (S6): Python binding of libssmscan.so.
+
+Argument marshalling only: torch tensors supply device pointers and the
+current CUDA stream; every step of the scan runs in the library's CUDA
+kernels (include/ssm_scan.h).  There is no CPU path.
+
+    y, last_state = scan_fwd(u, delta, A, B, C, D, z, delta_bias,
+                             delta_softplus=True, return_last_state=True)
+    grads = scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout)
+
+Layouts: u, delta, z, y, dout (batch, dim, seqlen); B, C (batch, seqlen,
+dstate); A (dim, dstate) fp32; D, delta_bias (dim,) fp32; states (batch, dim,
+dstate) fp32.  io tensors are all bf16 or all fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_PATH_AUTO, SSM_PATH_LOOKBACK,  # noqa: F401
+                   SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L, ssm_shape)
+
+__all__ = ["scan_fwd", "scan_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes",
+           "fwd_path", "check", "ScanError", "make_shape"]
+
+
+class ScanError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {_lib.status_string(code)} ({code})")
+        self.code = code
+
+
+def _io_dtype(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    if t.dtype == torch.float32:
+        return SSM_F32
+    raise TypeError(f"io tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+def make_shape(batch: int, dim: int, seqlen: int, dstate: int, io_dtype: int,
+               path: int = SSM_PATH_AUTO) -> ssm_shape:
+    return ssm_shape(batch, dim, seqlen, dstate, io_dtype, path)
+
+
+def fwd_workspace_bytes(shape: ssm_shape) -> int:
+    return int(_lib.load().ssm_scan_fwd_workspace_bytes(ctypes.byref(shape)))
+
+
+def bwd_workspace_bytes(shape: ssm_shape) -> int:
+    return int(_lib.load().ssm_scan_bwd_workspace_bytes(ctypes.byref(shape)))
+
+
+def fwd_path(shape: ssm_shape) -> str:
+    return PATH_NAMES[int(_lib.load().ssm_scan_fwd_path(ctypes.byref(shape)))]
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_io(name, t, shape, dtype, device):
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(nbytes, device, workspace):
+    import torch
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace holds {workspace.nbytes} bytes, needs {nbytes}")
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softplus=True,
+             initial_state=None, y=None, last_state=None, return_last_state=False,
+             workspace=None, path: int = SSM_PATH_AUTO, stream=None):
+    """Forward selective scan; returns y, or (y, last_state)."""
+    import torch
+    batch, dim, seqlen = u.shape
+    dstate = B.shape[-1]
+    dt = u.dtype
+    dev = u.device
+    f32 = torch.float32
+    _check_io("u", u, (batch, dim, seqlen), dt, dev)
+    _check_io("delta", delta, (batch, dim, seqlen), dt, dev)
+    _check_io("z", z, (batch, dim, seqlen), dt, dev)
+    _check_io("B", B, (batch, seqlen, dstate), dt, dev)
+    _check_io("C", C, (batch, seqlen, dstate), dt, dev)
+    _check_io("A", A, (dim, dstate), f32, dev)
+    _check_io("D", D, (dim,), f32, dev)
+    _check_io("delta_bias", delta_bias, (dim,), f32, dev)
+    _check_io("initial_state", initial_state, (batch, dim, dstate), f32, dev)
+    if y is None:
+        y = torch.empty_like(u)
+    _check_io("y", y, (batch, dim, seqlen), dt, dev)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, dim, dstate), dtype=f32, device=dev)
+    _check_io("last_state", last_state, (batch, dim, dstate), f32, dev)
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path)
+    nbytes = fwd_workspace_bytes(shape)
+    if nbytes == 0 and batch * dim * seqlen > 0:
+        raise ScanError(_lib.SSM_ERR_UNSUPPORTED, "ssm_scan_fwd_workspace_bytes")
+    ws = _workspace(nbytes, dev, workspace)
+    rc = _lib.load().ssm_scan_fwd(
+        ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(initial_state), _ptr(y),
+        _ptr(last_state), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
+    if rc != 0:
+        raise ScanError(rc, "ssm_scan_fwd")
+    if return_last_state:
+        return y, last_state
+    return y
+
+
+def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,
+             initial_state=None, want_dinitial_state=False, out=None, workspace=None,
+             stream=None):
+    """Backward of scan_fwd by recomputation; returns a dict of gradients."""
+    import torch
+    batch, dim, seqlen = u.shape
+    dstate = B.shape[-1]
+    dt, dev, f32 = u.dtype, u.device, torch.float32
+    for name, t, shp, ty in (("u", u, (batch, dim, seqlen), dt), ("delta", delta, (batch, dim, seqlen), dt),
+                             ("z", z, (batch, dim, seqlen), dt), ("B", B, (batch, seqlen, dstate), dt),
+                             ("C", C, (batch, seqlen, dstate), dt), ("A", A, (dim, dstate), f32),
+                             ("D", D, (dim,), f32), ("delta_bias", delta_bias, (dim,), f32),
+                             ("dout", dout, (batch, dim, seqlen), dt),
+                             ("initial_state", initial_state, (batch, dim, dstate), f32)):
+        _check_io(name, t, shp, ty, dev)
+    g = dict(out or {})
+    g.setdefault("du", torch.empty_like(u))
+    g.setdefault("ddelta", torch.empty_like(u))
+    g.setdefault("dA", torch.empty((dim, dstate), dtype=f32, device=dev))
+    g.setdefault("dB", torch.empty_like(B))
+    g.setdefault("dC", torch.empty_like(C))
+    g.setdefault("dD", torch.empty((dim,), dtype=f32, device=dev) if D is not None else None)
+    g.setdefault("dz", torch.empty_like(u) if z is not None else None)
+    g.setdefault("ddelta_bias",
+                 torch.empty((dim,), dtype=f32, device=dev) if delta_bias is not None else None)
+    g.setdefault("dinitial_state",
+                 torch.empty((batch, dim, dstate), dtype=f32, device=dev) if want_dinitial_state else None)
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u))
+    nbytes = bwd_workspace_bytes(shape)
+    ws = _workspace(nbytes, dev, workspace)
+    rc = _lib.load().ssm_scan_bwd(
+        ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(initial_state), _ptr(dout),
+        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+        _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]), _ptr(g["dinitial_state"]),
+        _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
+    if rc != 0:
+        raise ScanError(rc, "ssm_scan_bwd")
+    return g
+
+
+def check(workspace, stream=None) -> None:
+    """Synchronise and raise ScanError if a device-side wait gave up."""
+    rc = _lib.load().ssm_scan_check(_ptr(workspace), _stream(stream))
+    if rc != 0:
+        raise ScanError(rc, "ssm_scan_check")

@@ -1,0 +1,260 @@
+// C ABI of libssmscan.so: argument checks, schedule planning, workspace
+// layout and launches.  The public contract is include/ssm_scan.h.
+#include <stdio.h>
+#include <string.h>
+
+#include "ssm_common.cuh"
+#include "ssm_scan.h"
+
+using namespace ssm;
+
+namespace {
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool aligned(const void *p, size_t a) { return p == nullptr || ((uintptr_t)p % a) == 0; }
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+ssm_status check_shape(const ssm_shape *s) {
+  if (!s) return SSM_ERR_INVALID_ARG;
+  if (s->batch < 0 || s->dim < 0 || s->seqlen < 0 || s->dstate < 1) return SSM_ERR_INVALID_ARG;
+  if (s->dstate > 64) return SSM_ERR_UNSUPPORTED;
+  if (s->io_dtype != SSM_F32 && s->io_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_PER_GROUP) return SSM_ERR_UNSUPPORTED;
+  // index arithmetic is int64; keep every flat index well inside it
+  const double elems = (double)s->batch * (double)s->dim * (double)s->seqlen;
+  if (elems > 4.0e15 || (double)s->batch * s->seqlen * s->dstate > 4.0e15) return SSM_ERR_UNSUPPORTED;
+  return SSM_OK;
+}
+
+struct FwdPlan {
+  int path = SSM_PATH_AUTO;
+  int NP = 4;
+  int64_t gpb = 0, n_groups = 0, K = 0;
+  int64_t P = 0;                     // look-back warps
+  int64_t n_segs = 1, seg_chunks = 0;
+  size_t off_flags = 0, off_carry = 0, off_seg_h = 0, off_seg_dsum = 0, off_seg_carry = 0;
+  size_t total = kHeaderBytes;
+};
+
+ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
+  ssm_status st = check_shape(s);
+  if (st != SSM_OK) return st;
+  FwdPlan p;
+  p.NP = fwd_np_for(s->dstate);
+  p.gpb = (s->dim + kCPW - 1) / kCPW;
+  p.n_groups = s->batch * p.gpb;
+  p.K = (s->seqlen + kT - 1) / kT;
+  if (p.n_groups == 0 || p.K == 0) {
+    p.path = s->path == SSM_PATH_AUTO ? SSM_PATH_PER_GROUP : s->path;
+    *pl = p;
+    return SSM_OK;
+  }
+  const int sms = device_sms();
+  int occ = 0;
+  if (sms <= 0 || fwd_occupancy(s->io_dtype, p.NP, &occ) != cudaSuccess || occ <= 0) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  const int64_t unit = (int64_t)sms * kWarps;   // one warp per SM sub-partition
+  const int64_t slots = unit * occ;             // resident warps
+  int path = s->path;
+  if (path == SSM_PATH_AUTO) {
+    if (p.n_groups >= unit) path = SSM_PATH_LOOKBACK;
+    else if (p.K >= 64) path = SSM_PATH_SPLIT_L;
+    else path = SSM_PATH_PER_GROUP;
+  }
+  p.path = path;
+  if (path == SSM_PATH_LOOKBACK) {
+    // P <= groups keeps every warp's range at least one group long;
+    // a multiple of `unit` gives every sub-partition the same work.
+    int64_t r = p.n_groups / unit;
+    if (r > occ) r = occ;
+    p.P = r >= 1 ? r * unit : p.n_groups;
+    if (p.P > slots) p.P = slots;  // all warps co-resident
+    p.off_flags = kHeaderBytes;
+    p.off_carry = round_up(p.off_flags + sizeof(unsigned) * (size_t)p.P, 256);
+    p.total = round_up(p.off_carry + sizeof(float) * (size_t)p.P * kCPW * p.NP, 256);
+  } else if (path == SSM_PATH_SPLIT_L) {
+    // about two waves of resident warps; segments of at least 4 chunks
+    int64_t target = 2 * slots;
+    int64_t segs = (target + p.n_groups - 1) / p.n_groups;
+    int64_t max_segs = p.K / 4 > 1 ? p.K / 4 : 1;
+    if (segs > max_segs) segs = max_segs;
+    if (segs < 2 && p.K >= 2) segs = 2;
+    if (segs < 1) segs = 1;
+    p.seg_chunks = (p.K + segs - 1) / segs;
+    p.n_segs = (p.K + p.seg_chunks - 1) / p.seg_chunks;
+    const size_t items = (size_t)p.n_groups * (size_t)p.n_segs;
+    p.off_seg_h = kHeaderBytes;
+    p.off_seg_dsum = round_up(p.off_seg_h + sizeof(float) * items * kCPW * p.NP, 256);
+    p.off_seg_carry = round_up(p.off_seg_dsum + sizeof(float) * items * kCPW, 256);
+    p.total = round_up(p.off_seg_carry + sizeof(float) * items * kCPW * p.NP, 256);
+  } else {
+    p.n_segs = 1;
+    p.seg_chunks = p.K;
+  }
+  *pl = p;
+  return SSM_OK;
+}
+
+ssm_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SSM_OK;
+  fprintf(stderr, "ssm_scan: CUDA error %s\n", cudaGetErrorString(e));
+  return SSM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ssm_status_string(ssm_status s) {
+  switch (s) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_INVALID_ARG: return "invalid argument";
+    case SSM_ERR_UNSUPPORTED: return "unsupported shape, dtype or path";
+    case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+    case SSM_ERR_CUDA: return "CUDA error";
+    case SSM_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t ssm_scan_version(void) { return kVersion; }
+
+size_t ssm_scan_fwd_workspace_bytes(const ssm_shape *shape) {
+  FwdPlan p;
+  if (make_fwd_plan(shape, &p) != SSM_OK) return 0;
+  return p.total;
+}
+
+int32_t ssm_scan_fwd_path(const ssm_shape *shape) {
+  FwdPlan p;
+  if (make_fwd_plan(shape, &p) != SSM_OK) return SSM_PATH_AUTO;
+  return p.path;
+}
+
+ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta,
+                        const float *A, const void *B, const void *C, const float *D,
+                        const void *z, const float *delta_bias, int delta_softplus,
+                        const float *initial_state, void *y, float *last_state,
+                        void *workspace, size_t ws_bytes, ssm_stream_t stream) {
+  ssm_status st = check_shape(shape);
+  if (st != SSM_OK) return st;
+  const int64_t nch = shape->batch * shape->dim;
+  if (nch == 0) return SSM_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = shape->io_dtype == SSM_BF16 ? 2 : 4;
+  if (shape->seqlen == 0) {  // nothing to scan: last_state = initial state
+    if (!last_state) return SSM_OK;
+    if (!aligned(last_state, 4) || !aligned(initial_state, 4)) return SSM_ERR_INVALID_ARG;
+    const size_t bytes = sizeof(float) * (size_t)nch * (size_t)shape->dstate;
+    return cuda_status(initial_state
+                           ? cudaMemcpyAsync(last_state, initial_state, bytes, cudaMemcpyDeviceToDevice, s)
+                           : cudaMemsetAsync(last_state, 0, bytes, s));
+  }
+  if (!u || !delta || !A || !B || !C || !y) return SSM_ERR_INVALID_ARG;
+  if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) ||
+      !aligned(z, es) || !aligned(y, es) || !aligned(A, 4) || !aligned(D, 4) ||
+      !aligned(delta_bias, 4) || !aligned(initial_state, 4) || !aligned(last_state, 4))
+    return SSM_ERR_INVALID_ARG;
+  FwdPlan pl;
+  st = make_fwd_plan(shape, &pl);
+  if (st != SSM_OK) return st;
+  if (!workspace || ws_bytes < pl.total || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
+
+  FwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias; p.h0 = initial_state;
+  p.y = y; p.last_state = last_state;
+  p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = (int)shape->dstate;
+  p.softplus = delta_softplus ? 1 : 0;
+  p.io_vec = ((shape->seqlen * es) % 16 == 0) && aligned(u, 16) && aligned(delta, 16) &&
+             aligned(z, 16) && aligned(y, 16);
+  p.bc_vec = (shape->dstate == pl.NP) && ((shape->dstate * es) % 16 == 0) && aligned(B, 16) &&
+             aligned(C, 16);
+  p.gpb = pl.gpb; p.n_groups = pl.n_groups; p.n_chunks = pl.K;
+  p.n_workers = pl.P;
+  char *ws = static_cast<char *>(workspace);
+  p.err = reinterpret_cast<unsigned *>(ws);
+  p.wait_limit_ns = kWaitLimitNs;
+  p.n_segs = pl.n_segs; p.seg_chunks = pl.seg_chunks;
+
+  cudaError_t e;
+  if (pl.path == SSM_PATH_LOOKBACK) {
+    p.flags = reinterpret_cast<unsigned *>(ws + pl.off_flags);
+    p.carry = reinterpret_cast<float *>(ws + pl.off_carry);
+    e = cudaMemsetAsync(ws, 0, pl.off_carry, s);  // error word and flags
+    if (e != cudaSuccess) return cuda_status(e);
+    e = launch_fwd_lookback(shape->io_dtype, pl.NP, p, s);
+  } else {
+    if (pl.n_segs > 1) {
+      p.seg_h = reinterpret_cast<float *>(ws + pl.off_seg_h);
+      p.seg_dsum = reinterpret_cast<float *>(ws + pl.off_seg_dsum);
+      p.seg_carry = reinterpret_cast<float *>(ws + pl.off_seg_carry);
+    }
+    e = launch_fwd_splitl(shape->io_dtype, pl.NP, p, s);
+  }
+  return cuda_status(e);
+}
+
+size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
+  if (check_shape(shape) != SSM_OK) return 0;
+  return kHeaderBytes;
+}
+
+ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta,
+                        const float *A, const void *B, const void *C, const float *D,
+                        const void *z, const float *delta_bias, int delta_softplus,
+                        const float *initial_state, const void *dout, void *du, void *ddelta,
+                        float *dA, void *dB, void *dC, float *dD, void *dz,
+                        float *ddelta_bias, float *dinitial_state, void *workspace,
+                        size_t ws_bytes, ssm_stream_t stream) {
+  (void)u; (void)delta; (void)A; (void)B; (void)C; (void)D; (void)z; (void)delta_bias;
+  (void)delta_softplus; (void)initial_state; (void)dout; (void)du; (void)ddelta; (void)dA;
+  (void)dB; (void)dC; (void)dD; (void)dz; (void)ddelta_bias; (void)dinitial_state;
+  (void)workspace; (void)ws_bytes; (void)stream;
+  ssm_status st = check_shape(shape);
+  if (st != SSM_OK) return st;
+  return SSM_ERR_UNSUPPORTED;
+}
+
+ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream) {
+  if (!workspace) return SSM_ERR_WORKSPACE;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  unsigned word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (word == 0) return SSM_OK;
+  e = cudaMemset(workspace, 0, sizeof(word));
+  if (e != cudaSuccess) return cuda_status(e);
+  return SSM_ERR_DEVICE_TIMEOUT;
+}
+
+ssm_status ssm_scan_test_wait_timeout(void *workspace, size_t ws_bytes, int64_t timeout_us,
+                                      ssm_stream_t stream) {
+  if (!workspace || ws_bytes < kHeaderBytes || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
+  if (timeout_us < 1 || timeout_us > 1000000) return SSM_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  // the flag at byte 64 of the zeroed header is never set
+  e = launch_wait_timeout_probe(reinterpret_cast<unsigned *>(ws + 64),
+                                reinterpret_cast<unsigned *>(ws),
+                                (unsigned long long)timeout_us * 1000ull, s);
+  return cuda_status(e);
+}
+
+}  // extern "C"

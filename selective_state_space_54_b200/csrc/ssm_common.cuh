@@ -1,0 +1,199 @@
+// Internal definitions shared by the forward and backward kernels and the
+// C-ABI layer of libssmscan.so.  Not part of the public interface.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// ---- work decomposition ----------------------------------------------------
+// A warp owns an 8-channel group of one batch element.  Lane l handles
+// channel c = l / 4 and, of that channel's dstate states, the slice
+// n in [j*S, j*S + S) with j = l % 4 and S = NP / 4 (NP = dstate padded up to
+// a power of two >= 4).  Time is processed in chunks of kT steps; within a
+// chunk each lane walks the recurrence sequentially, so every (t, n) element
+// costs one exp2 and four fp32 ops and nothing of size (L, N) is stored.
+constexpr int kT = 32;           // time steps per chunk
+constexpr int kCPW = 8;          // channels per warp
+constexpr int kLPC = 4;          // lanes per channel
+constexpr int kWarps = 4;        // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kRowPad = 4;       // smem row padding (floats) against bank conflicts
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Workspace header: byte 0 holds the device error word.
+constexpr size_t kHeaderBytes = 256;
+constexpr unsigned kErrWaitTimeout = 1u;
+
+// Upper bound of one inter-warp wait in the look-back schedule, in ns of the
+// GPU global timer.  The wait is only ever reached after the producer warp's
+// first item, so in practice it never spins.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct FwdParams {
+  const void *u, *delta, *z, *B, *C;
+  const float *A, *D, *bias, *h0;
+  void *y;
+  float *last_state;
+  int64_t batch, dim, L;
+  int N;
+  int softplus;
+  int io_vec;   // u/delta/z/y rows 16-byte aligned: vector loads
+  int bc_vec;   // B/C chunk blocks 16-byte aligned and N == NP
+  int64_t gpb;        // 8-channel groups per batch element
+  int64_t n_groups;   // batch * gpb
+  int64_t n_chunks;   // ceil(L / kT)
+  // look-back schedule
+  int64_t n_workers;  // warps
+  float *carry;       // [n_workers][kCPW][NP]
+  unsigned *flags;    // [n_workers]
+  unsigned *err;      // workspace header
+  unsigned long long wait_limit_ns;
+  // split-L schedule
+  int64_t n_segs, seg_chunks;
+  float *seg_h;       // [n_groups * n_segs][kCPW][NP] segment end state from zero
+  float *seg_dsum;    // [n_groups * n_segs][kCPW]      sum of Delta over the segment
+  float *seg_carry;   // [n_groups * n_segs][kCPW][NP] state entering the segment
+};
+
+// ---- io helpers ---------------------------------------------------------------
+// bf16 values travel as raw 16-bit patterns; widening is a shift.
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+__device__ __forceinline__ float bf16_to_f(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&p);
+}
+
+template <typename T> struct IO;
+
+template <> struct IO<uint16_t> {
+  static constexpr int kBytes = 2;
+  __device__ __forceinline__ static float get(const uint16_t *p, int64_t i) { return bf16_to_f(p[i]); }
+  // 8 consecutive values row[t..t+8), zeros beyond L.
+  __device__ __forceinline__ static void load8(const uint16_t *row, int64_t t, int64_t L,
+                                               bool vec, float (&o)[8]) {
+    if (vec && t + 8 <= L) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(row + t));
+      o[0] = bf16_lo(v.x); o[1] = bf16_hi(v.x); o[2] = bf16_lo(v.y); o[3] = bf16_hi(v.y);
+      o[4] = bf16_lo(v.z); o[5] = bf16_hi(v.z); o[6] = bf16_lo(v.w); o[7] = bf16_hi(v.w);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = (t + i < L) ? bf16_to_f(row[t + i]) : 0.f;
+    }
+  }
+  __device__ __forceinline__ static void store8(uint16_t *row, int64_t t, int64_t L, bool vec,
+                                                const float (&v)[8]) {
+    if (vec && t + 8 <= L) {
+      uint4 o;
+      o.x = pack_bf16x2(v[0], v[1]); o.y = pack_bf16x2(v[2], v[3]);
+      o.z = pack_bf16x2(v[4], v[5]); o.w = pack_bf16x2(v[6], v[7]);
+      *reinterpret_cast<uint4 *>(row + t) = o;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (t + i < L) {
+          __nv_bfloat16 b = __float2bfloat16_rn(v[i]);
+          row[t + i] = *reinterpret_cast<uint16_t *>(&b);
+        }
+    }
+  }
+  __device__ __forceinline__ static void store1(uint16_t *p, int64_t i, float v) {
+    __nv_bfloat16 b = __float2bfloat16_rn(v);
+    p[i] = *reinterpret_cast<uint16_t *>(&b);
+  }
+};
+
+template <> struct IO<float> {
+  static constexpr int kBytes = 4;
+  __device__ __forceinline__ static float get(const float *p, int64_t i) { return p[i]; }
+  __device__ __forceinline__ static void load8(const float *row, int64_t t, int64_t L, bool vec,
+                                               float (&o)[8]) {
+    if (vec && t + 8 <= L) {
+      const float4 a = __ldg(reinterpret_cast<const float4 *>(row + t));
+      const float4 b = __ldg(reinterpret_cast<const float4 *>(row + t + 4));
+      o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = (t + i < L) ? row[t + i] : 0.f;
+    }
+  }
+  __device__ __forceinline__ static void store8(float *row, int64_t t, int64_t L, bool vec,
+                                                const float (&v)[8]) {
+    if (vec && t + 8 <= L) {
+      *reinterpret_cast<float4 *>(row + t) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4 *>(row + t + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (t + i < L) row[t + i] = v[i];
+    }
+  }
+  __device__ __forceinline__ static void store1(float *p, int64_t i, float v) { p[i] = v; }
+};
+
+// ---- math helpers -------------------------------------------------------------
+// 2^x on the special-function unit (flush-to-zero; 2^-big == 0 exactly).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// softplus(s) = log(1 + e^s); s itself above 20 (the difference is < 2e-9 relative).
+__device__ __forceinline__ float softplus_f(float s) { return s > 20.f ? s : log1pf(__expf(s)); }
+
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+
+// SiLU(z) = z * sigmoid(z)
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Lane 0 waits until *flag != 0 or limit_ns passed; the result is broadcast.
+// On give-up the error word gets kErrWaitTimeout.  Never traps, never spins
+// without bound.
+__device__ __forceinline__ bool warp_wait_flag(const unsigned *flag, unsigned *err,
+                                               unsigned long long limit_ns) {
+  unsigned ok = 0;
+  if ((threadIdx.x & 31) == 0) {
+    const unsigned long long t0 = global_ns();
+    while (true) {
+      if (ld_acquire(flag) != 0u) { ok = 1; break; }
+      if (global_ns() - t0 > limit_ns) break;
+      __nanosleep(256);
+    }
+    if (!ok) atomicOr(err, kErrWaitTimeout);
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __threadfence();
+  return ok != 0;
+}
+
+// ---- launchers (defined in ssm_fwd.cu / ssm_bwd.cu) ----------------------------
+int fwd_np_for(int64_t N);
+cudaError_t fwd_occupancy(int io_dtype, int NP, int *ctas_per_sm);
+cudaError_t launch_fwd_lookback(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
+cudaError_t launch_fwd_splitl(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
+cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,
+                                      cudaStream_t s);
+
+}  // namespace ssm

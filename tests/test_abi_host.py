@@ -1,0 +1,112 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and rejects bad arguments with the documented status before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_54_b200 import _lib
+from selective_state_space_54_b200.build import INCLUDE, LIB, build
+
+HEADER = os.path.join(INCLUDE, "ssm_scan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssm_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert sorted(_lib.EXPORTS) == declared_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert lib.ssm_status_string(0) == b"ok"
+    assert b"timed out" in lib.ssm_status_string(_lib.SSM_ERR_DEVICE_TIMEOUT)
+    assert lib.ssm_scan_version() >= 100
+
+
+def _shape(**kw):
+    d = dict(batch=2, dim=16, seqlen=64, dstate=16, io_dtype=_lib.SSM_BF16, path=0)
+    d.update(kw)
+    return _lib.ssm_shape(**d)
+
+
+BAD_SHAPES = [
+    (dict(batch=-1), _lib.SSM_ERR_INVALID_ARG),
+    (dict(dim=-3), _lib.SSM_ERR_INVALID_ARG),
+    (dict(seqlen=-1), _lib.SSM_ERR_INVALID_ARG),
+    (dict(dstate=0), _lib.SSM_ERR_INVALID_ARG),
+    (dict(dstate=65), _lib.SSM_ERR_UNSUPPORTED),
+    (dict(io_dtype=7), _lib.SSM_ERR_UNSUPPORTED),
+    (dict(path=9), _lib.SSM_ERR_UNSUPPORTED),
+]
+
+
+def _fwd(lib, shape, ptrs=None, ws=None, ws_bytes=0):
+    p = dict(u=8, delta=8, A=16, B=8, C=8, D=None, z=None, bias=None, h0=None, y=8, ls=None)
+    p.update(ptrs or {})
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ssm_scan_fwd(ctypes.byref(shape) if shape is not None else None, v(p["u"]),
+                            v(p["delta"]), v(p["A"]), v(p["B"]), v(p["C"]), v(p["D"]), v(p["z"]),
+                            v(p["bias"]), 1, v(p["h0"]), v(p["y"]), v(p["ls"]), v(ws), ws_bytes, None)
+
+
+def test_null_shape_rejected(lib):
+    assert _fwd(lib, None) == _lib.SSM_ERR_INVALID_ARG
+    assert lib.ssm_scan_fwd_workspace_bytes(None) == 0
+
+
+@pytest.mark.parametrize("kw,code", BAD_SHAPES)
+def test_bad_shapes_rejected(lib, kw, code):
+    assert _fwd(lib, _shape(**kw)) == code
+    assert lib.ssm_scan_fwd_workspace_bytes(ctypes.byref(_shape(**kw))) == 0
+    assert lib.ssm_scan_bwd_workspace_bytes(ctypes.byref(_shape(**kw))) == 0
+
+
+@pytest.mark.parametrize("missing", ["u", "delta", "A", "B", "C", "y"])
+def test_null_required_pointer_rejected(lib, missing):
+    assert _fwd(lib, _shape(), {missing: None}) == _lib.SSM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which,addr", [("u", 9), ("B", 3), ("A", 18), ("y", 1), ("z", 5),
+                                         ("D", 2), ("ls", 6)])
+def test_misaligned_pointer_rejected(lib, which, addr):
+    assert _fwd(lib, _shape(), {which: addr}) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_empty_problem_is_a_noop(lib):
+    # batch*dim == 0: nothing to do, nothing touched, even with null pointers
+    assert _fwd(lib, _shape(batch=0), {k: None for k in ("u", "delta", "A", "B", "C", "y")}) == 0
+    assert _fwd(lib, _shape(dim=0), {k: None for k in ("u", "delta", "A", "B", "C", "y")}) == 0
+
+
+def test_bwd_rejects_bad_shapes(lib):
+    # shape, 8 input pointers, delta_softplus, initial_state, dout, 9 outputs, ws, bytes, stream
+    for kw, code in BAD_SHAPES:
+        sh = _shape(**kw)
+        assert lib.ssm_scan_bwd(ctypes.byref(sh), *[None] * 8, 1, *[None] * 11, None, 0, None) == code
+
+
+def test_product_has_no_oracle_or_cpu_path():
+    # the package never imports the oracle and carries no CPU implementation
+    pkg = os.path.dirname(LIB)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith(".py") or f.endswith(".cu") or f.endswith(".cuh"):
+                text = open(os.path.join(root, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "ssm_oracle" not in text, f

@@ -1,0 +1,211 @@
+"""Forward parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small cases span several 32-step chunks, ragged chunk tails, ragged 8-channel
+groups and every dstate padding; the named workloads run at their full sizes
+in the launch configuration the benchmark uses and are checked on seeded
+channels the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import assert_close, to_f64, upload
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3}
+
+
+def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    g = upload(case, device)
+    h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
+    y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                         g["delta_bias"], delta_softplus=softplus, initial_state=h0_t,
+                         return_last_state=True, path=PATHS[path], y=y_out)
+    torch.cuda.synchronize()
+    return to_f64(y), to_f64(ls)
+
+
+def _check(case, device, path="auto", softplus=True, h0=None):
+    ref = oracle.fwd(case, delta_softplus=softplus, h0=h0)
+    y, ls = _run(case, device, path, softplus, h0)
+    st = assert_close(y, ref["y"], case["dtype"], f"y[{path}]")
+    # the state is fp32 on both io dtypes
+    assert_close(ls, ref["last_state"], synth.F32 if case["dtype"] == synth.F32 else synth.BF16,
+                 f"last_state[{path}]")
+    return st
+
+
+@pytest.mark.parametrize("path", ["auto", "lookback", "split_l", "per_group"])
+def test_tiny_fp32_workload(cuda_device, path):
+    case = synth.make_workload("tiny-fp32")
+    _check(case, cuda_device, path)
+
+
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("N", [1, 3, 4, 8, 12, 16, 32, 64])
+def test_dstate_sizes(cuda_device, dtype, N):
+    case = synth.make_case(2, 20, 200, N, dtype, seed=100 + N)
+    _check(case, cuda_device, "per_group")
+
+
+@pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
+@pytest.mark.parametrize("L", [1, 7, 31, 32, 33, 257, 1000, 1003])
+def test_ragged_lengths_and_groups(cuda_device, path, L):
+    # dim 44: five full 8-channel groups and a ragged one; L odd -> scalar loads
+    case = synth.make_case(3, 44, L, 16, synth.BF16, seed=L)
+    _check(case, cuda_device, path)
+
+
+@pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
+def test_fp32_several_chunks(cuda_device, path):
+    case = synth.make_case(2, 24, 777, 16, synth.F32, seed=7)
+    _check(case, cuda_device, path)
+
+
+@pytest.mark.parametrize("opt", ["no_z", "no_D", "no_bias", "no_softplus", "bare"])
+def test_optional_terms(cuda_device, opt):
+    kw = dict(with_z=opt not in ("no_z", "bare"), with_D=opt not in ("no_D", "bare"),
+              with_bias=opt not in ("no_bias", "bare"))
+    case = synth.make_case(2, 16, 300, 16, synth.F32, seed=3, **kw)
+    softplus = opt != "no_softplus"
+    if not softplus:
+        # raw delta must stay positive without softplus (|Abar| <= 1)
+        case["delta"] = np.abs(case["delta"]) * 0.05 + 1e-3
+        case["delta_bias"] = None
+    _check(case, cuda_device, "auto", softplus=softplus)
+
+
+@pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
+def test_initial_state(cuda_device, path):
+    case = synth.make_case(2, 16, 500, 16, synth.F32, seed=9)
+    h0 = np.random.default_rng(1).standard_normal((2, 16, 16)).astype(np.float32)
+    _check(case, cuda_device, path, h0=h0)
+
+
+def test_continuation_matches_one_scan(cuda_device):
+    # scan(L1) -> last_state -> scan(L2 from it) == scan(L1 + L2), on the GPU
+    import torch
+    import selective_state_space_54_b200 as ssm
+    case = synth.make_case(2, 16, 640, 16, synth.F32, seed=21)
+    g = upload(case, cuda_device)
+    y_full, ls_full = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                                   g["delta_bias"], return_last_state=True)
+    cut = 320
+    part = lambda t, lo, hi: t[..., lo:hi].contiguous()
+    y1, ls1 = ssm.scan_fwd(part(g["u"], 0, cut), part(g["delta"], 0, cut), g["A"],
+                           g["B"][:, :cut].contiguous(), g["C"][:, :cut].contiguous(), g["D"],
+                           part(g["z"], 0, cut), g["delta_bias"], return_last_state=True)
+    y2, ls2 = ssm.scan_fwd(part(g["u"], cut, 640), part(g["delta"], cut, 640), g["A"],
+                           g["B"][:, cut:].contiguous(), g["C"][:, cut:].contiguous(), g["D"],
+                           part(g["z"], cut, 640), g["delta_bias"], initial_state=ls1,
+                           return_last_state=True)
+    torch.cuda.synchronize()
+    got = torch.cat([y1, y2], dim=-1)
+    assert torch.allclose(got, y_full, rtol=1e-5, atol=1e-5)
+    assert torch.allclose(ls2, ls_full, rtol=1e-5, atol=1e-5)
+
+
+def test_large_delta_reset_bitwise(cuda_device):
+    # Reading guide, "Perguntas": a large Delta resets the state.  exp2 of a
+    # huge negative argument is exactly 0 in fp32 too, so outputs from t0 on
+    # must not depend on anything before t0, bit for bit.
+    case = synth.make_case(1, 16, 200, 16, synth.F32, seed=5, with_bias=False)
+    t0 = 97
+    case["delta"] = np.abs(case["delta"]) * 0.1 + 1e-3
+    case["delta"][:, :, t0] = 1e4
+    y0, ls0 = _run(case, cuda_device, "per_group", softplus=False)
+    c2 = dict(case)
+    rng = np.random.default_rng(3)
+    c2["u"] = case["u"].copy()
+    c2["u"][:, :, :t0] += rng.standard_normal((1, 16, t0)).astype(np.float32)
+    c2["B"] = case["B"].copy()
+    c2["B"][:, :t0] *= 3.0
+    y1, ls1 = _run(c2, cuda_device, "per_group", softplus=False)
+    assert np.array_equal(y0[..., t0:], y1[..., t0:])
+    assert np.array_equal(ls0, ls1)
+
+
+def test_paths_agree(cuda_device):
+    case = synth.make_case(4, 64, 2048, 16, synth.BF16, seed=31)
+    outs = {p: _run(case, cuda_device, p)[0] for p in ("lookback", "split_l", "per_group")}
+    for p in ("split_l", "per_group"):
+        d = np.max(np.abs(outs[p] - outs["lookback"]))
+        assert d <= 2e-2 * np.max(np.abs(outs["lookback"])), (p, d)
+
+
+def test_deterministic(cuda_device):
+    case = synth.make_case(2, 64, 1024, 16, synth.BF16, seed=41)
+    a = _run(case, cuda_device, "lookback")
+    b = _run(case, cuda_device, "lookback")
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_guard_bands_untouched(cuda_device):
+    # y is written into the middle of a larger buffer whose margins hold a
+    # NaN pattern; the kernel must not touch them (bounds check without a sanitizer)
+    import torch
+    case = synth.make_case(2, 20, 333, 16, synth.BF16, seed=51)
+    n = 2 * 20 * 333
+    pad = 4096
+    buf = torch.full((n + 2 * pad,), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    y_view = buf[pad:pad + n].view(2, 20, 333)
+    ref = oracle.fwd(case)
+    y, _ = _run(case, cuda_device, "auto", y_out=y_view)
+    assert_close(y, ref["y"], case["dtype"], "y")
+    assert torch.isnan(buf[:pad].float()).all() and torch.isnan(buf[pad + n:].float()).all()
+
+
+def test_wait_timeout_reports_status(cuda_device):
+    # the bounded inter-warp wait gives up, records the error and the context stays usable
+    import ctypes
+    import torch
+    import selective_state_space_54_b200 as ssm
+    from selective_state_space_54_b200 import _lib
+    lib = _lib.load()
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda_device)
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.ssm_scan_test_wait_timeout(ctypes.c_void_p(ws.data_ptr()), 256, 20000, s) == 0
+    assert lib.ssm_scan_check(ctypes.c_void_p(ws.data_ptr()), s) == _lib.SSM_ERR_DEVICE_TIMEOUT
+    assert lib.ssm_scan_check(ctypes.c_void_p(ws.data_ptr()), s) == 0  # cleared
+    _check(synth.make_workload("tiny-fp32"), cuda_device)  # still works
+    del ssm
+
+
+# ---- the named workloads at full size, checked on seeded channels ----------
+def _full_size(name, device, sample=None):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    w = synth.WORKLOADS[name]
+    case = synth.make_workload(w)
+    g = upload(case, device)
+    y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                         g["delta_bias"], return_last_state=True)
+    torch.cuda.synchronize()
+    chans = synth.sample_channels(w, sample)
+    for b, dims, sub in synth.subset_case(case, chans):
+        ref = oracle.fwd(sub)
+        yg = to_f64(y[b, dims])[None]
+        lg = to_f64(ls[b, dims])[None]
+        assert_close(yg, ref["y"], case["dtype"], f"{name} y b={b}")
+        assert_close(lg, ref["last_state"], synth.BF16, f"{name} last_state b={b}")
+    return y
+
+
+def test_full_mamba_130m_layer(cuda_device):
+    _full_size("mamba-130m-layer", cuda_device, sample=96)
+
+
+def test_full_mamba_2p8b_layer(cuda_device):
+    _full_size("mamba-2.8b-layer", cuda_device, sample=64)
+
+
+def test_full_million_length(cuda_device):
+    _full_size("million-length", cuda_device)
+
+
+def test_full_mamba_1p4b_layer_forward(cuda_device):
+    _full_size("mamba-1.4b-layer-train", cuda_device, sample=64)
