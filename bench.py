@@ -50,6 +50,11 @@ def parse():
     ap.add_argument("--workload", default="mamba-2.8b-layer", choices=list(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--lanes", type=int, default=0, choices=[0, 2, 4],
+                    help="lanes per channel (0: the library's choice)")
+    ap.add_argument("--path", default="auto", choices=["auto", "lookback", "split_l", "per_group"])
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling only)")
     return ap.parse_args()
 
 
@@ -261,6 +266,9 @@ def config_of(w, path):
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.batch, name=f"{w.name}[batch={args.batch}]")
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -280,8 +288,10 @@ def main():
         g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
     y = torch.empty_like(g["u"])
     ls = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+    path_id = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3}[args.path]
     shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
-                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32)
+                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32,
+                           path_id, args.lanes)
     path = ssm.fwd_path(shape)
     ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
     launches_per_step = {"lookback": 1, "per_group": 1, "split_l": 3}[path]
@@ -289,7 +299,8 @@ def main():
 
     def step():
         ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                     y=y, last_state=ls, return_last_state=True, workspace=ws)
+                     y=y, last_state=ls, return_last_state=True, workspace=ws, path=path_id,
+                     lanes=args.lanes)
 
     def barrier():
         if world > 1:
@@ -338,7 +349,7 @@ def main():
                 dbuf[k].copy_(host[k], non_blocking=True)
             ssm.scan_fwd(dbuf["u"], dbuf["delta"], dbuf["A"], dbuf["B"], dbuf["C"], dbuf["D"],
                          dbuf["z"], dbuf["delta_bias"], y=y, last_state=ls,
-                         return_last_state=True, workspace=ws)
+                         return_last_state=True, workspace=ws, path=path_id, lanes=args.lanes)
             y_host.copy_(y, non_blocking=True)
             ls_host.copy_(ls, non_blocking=True)
 

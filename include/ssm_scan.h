@@ -65,15 +65,16 @@ typedef enum {
 
 typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
 
-/* Forward schedule.  AUTO picks from the shape and the device:
+/* Forward schedule.  A warp holds 32/lanes channels, each walked by `lanes`
+ * lanes over dstate/lanes states.  AUTO picks from the shape and the device:
  *  LOOKBACK  one persistent launch; every warp gets an equal share of
- *            (8-channel group x 32-step chunk) items; a group split between
+ *            (channel group x 32-step chunk) items; a group split between
  *            two warps passes its state through the workspace with a
  *            bounded wait (taken only after the writer's first item);
  *  SPLIT_L   two passes over time segments (segment end states from zero,
  *            a sequential carry over segments, then the output pass);
  *            for long sequences with few channels;
- *  PER_GROUP one warp per 8-channel group over the whole sequence. */
+ *  PER_GROUP one warp per channel group over the whole sequence. */
 typedef enum {
   SSM_PATH_AUTO = 0,
   SSM_PATH_LOOKBACK = 1,
@@ -88,6 +89,8 @@ typedef struct {
   int64_t dstate;   /* N, 1..64 */
   int32_t io_dtype; /* ssm_dtype */
   int32_t path;     /* ssm_path (forward only; ignored by the backward) */
+  int32_t lanes;    /* lanes per channel in the forward: 0 = auto, 2 or 4 */
+  int32_t reserved; /* must be 0 */
 } ssm_shape;
 
 /* Bytes of workspace ssm_scan_fwd needs for `shape` on the current device

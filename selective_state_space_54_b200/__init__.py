@@ -40,8 +40,8 @@ def _io_dtype(t) -> int:
 
 
 def make_shape(batch: int, dim: int, seqlen: int, dstate: int, io_dtype: int,
-               path: int = SSM_PATH_AUTO) -> ssm_shape:
-    return ssm_shape(batch, dim, seqlen, dstate, io_dtype, path)
+               path: int = SSM_PATH_AUTO, lanes: int = 0) -> ssm_shape:
+    return ssm_shape(batch, dim, seqlen, dstate, io_dtype, path, lanes, 0)
 
 
 def fwd_workspace_bytes(shape: ssm_shape) -> int:
@@ -90,7 +90,7 @@ def _workspace(nbytes, device, workspace):
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softplus=True,
              initial_state=None, y=None, last_state=None, return_last_state=False,
-             workspace=None, path: int = SSM_PATH_AUTO, stream=None):
+             workspace=None, path: int = SSM_PATH_AUTO, lanes: int = 0, stream=None):
     """Forward selective scan; returns y, or (y, last_state)."""
     import torch
     batch, dim, seqlen = u.shape
@@ -113,7 +113,7 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, dstate), dtype=f32, device=dev)
     _check_io("last_state", last_state, (batch, dim, dstate), f32, dev)
-    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path)
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path, lanes)
     nbytes = fwd_workspace_bytes(shape)
     if nbytes == 0 and batch * dim * seqlen > 0:
         raise ScanError(_lib.SSM_ERR_UNSUPPORTED, "ssm_scan_fwd_workspace_bytes")

@@ -39,7 +39,8 @@ EXPORTS = (
 class ssm_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64),
                 ("seqlen", ctypes.c_int64), ("dstate", ctypes.c_int64),
-                ("io_dtype", ctypes.c_int32), ("path", ctypes.c_int32)]
+                ("io_dtype", ctypes.c_int32), ("path", ctypes.c_int32),
+                ("lanes", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _lib = None

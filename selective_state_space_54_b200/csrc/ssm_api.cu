@@ -29,6 +29,8 @@ ssm_status check_shape(const ssm_shape *s) {
   if (s->dstate > 64) return SSM_ERR_UNSUPPORTED;
   if (s->io_dtype != SSM_F32 && s->io_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_PER_GROUP) return SSM_ERR_UNSUPPORTED;
+  if (s->lanes != 0 && s->lanes != 2 && s->lanes != 4) return SSM_ERR_UNSUPPORTED;
+  if (s->reserved != 0) return SSM_ERR_INVALID_ARG;
   // index arithmetic is int64; keep every flat index well inside it
   const double elems = (double)s->batch * (double)s->dim * (double)s->seqlen;
   if (elems > 4.0e15 || (double)s->batch * s->seqlen * s->dstate > 4.0e15) return SSM_ERR_UNSUPPORTED;
@@ -38,6 +40,7 @@ ssm_status check_shape(const ssm_shape *s) {
 struct FwdPlan {
   int path = SSM_PATH_AUTO;
   int NP = 4;
+  int LPC = 4;                       // lanes per channel
   int64_t gpb = 0, n_groups = 0, K = 0;
   int64_t P = 0;                     // look-back warps
   int64_t n_segs = 1, seg_chunks = 0;
@@ -45,59 +48,82 @@ struct FwdPlan {
   size_t total = kHeaderBytes;
 };
 
+int64_t groups_for(const ssm_shape *s, int lpc) {
+  const int64_t cpw = 32 / lpc;
+  return s->batch * ((s->dim + cpw - 1) / cpw);
+}
+
+// Schedule choice.  The look-back schedule needs at least one channel group
+// per warp slot it uses (P <= groups) and balances work exactly, so it is
+// preferred whenever the problem has enough channel groups; two lanes per
+// channel (fewer instructions per element) when that still leaves two warps
+// per SM sub-partition, else four.  Long sequences with few channels take the
+// two-pass split-L schedule; tiny problems one warp per group.
 ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   ssm_status st = check_shape(s);
   if (st != SSM_OK) return st;
   FwdPlan p;
   p.NP = fwd_np_for(s->dstate);
-  p.gpb = (s->dim + kCPW - 1) / kCPW;
-  p.n_groups = s->batch * p.gpb;
   p.K = (s->seqlen + kT - 1) / kT;
-  if (p.n_groups == 0 || p.K == 0) {
+  if (s->batch * s->dim == 0 || p.K == 0) {
     p.path = s->path == SSM_PATH_AUTO ? SSM_PATH_PER_GROUP : s->path;
     *pl = p;
     return SSM_OK;
   }
   const int sms = device_sms();
-  int occ = 0;
-  if (sms <= 0 || fwd_occupancy(s->io_dtype, p.NP, &occ) != cudaSuccess || occ <= 0) {
-    cudaGetLastError();
-    return SSM_ERR_CUDA;
-  }
+  if (sms <= 0) return SSM_ERR_CUDA;
   const int64_t unit = (int64_t)sms * kWarps;   // one warp per SM sub-partition
-  const int64_t slots = unit * occ;             // resident warps
-  int path = s->path;
+  const int64_t g2 = groups_for(s, 2), g4 = groups_for(s, 4);
+  int path = s->path, lpc = s->lanes;
+  if (lpc == 0) {
+    if (path == SSM_PATH_SPLIT_L) lpc = 2;
+    else if (path == SSM_PATH_PER_GROUP) lpc = 4;
+    else if (g2 >= 2 * unit) lpc = 2;
+    else if (g4 >= unit || path == SSM_PATH_LOOKBACK) lpc = 4;
+    else lpc = p.K >= 64 ? 2 : 4;
+  }
+  const int64_t G = lpc == 2 ? g2 : g4;
   if (path == SSM_PATH_AUTO) {
-    if (p.n_groups >= unit) path = SSM_PATH_LOOKBACK;
+    if (G >= unit) path = SSM_PATH_LOOKBACK;
     else if (p.K >= 64) path = SSM_PATH_SPLIT_L;
     else path = SSM_PATH_PER_GROUP;
   }
+  int occ = 0;
+  if (fwd_occupancy(s->io_dtype, p.NP, lpc, &occ) != cudaSuccess || occ <= 0) {
+    cudaGetLastError();
+    return SSM_ERR_CUDA;
+  }
+  const int64_t slots = unit * occ;             // resident warps
+  const int cpw = 32 / lpc;
   p.path = path;
+  p.LPC = lpc;
+  p.gpb = (s->dim + cpw - 1) / cpw;
+  p.n_groups = G;
   if (path == SSM_PATH_LOOKBACK) {
     // P <= groups keeps every warp's range at least one group long;
     // a multiple of `unit` gives every sub-partition the same work.
-    int64_t r = p.n_groups / unit;
+    int64_t r = G / unit;
     if (r > occ) r = occ;
-    p.P = r >= 1 ? r * unit : p.n_groups;
+    p.P = r >= 1 ? r * unit : G;
     if (p.P > slots) p.P = slots;  // all warps co-resident
     p.off_flags = kHeaderBytes;
     p.off_carry = round_up(p.off_flags + sizeof(unsigned) * (size_t)p.P, 256);
-    p.total = round_up(p.off_carry + sizeof(float) * (size_t)p.P * kCPW * p.NP, 256);
+    p.total = round_up(p.off_carry + sizeof(float) * (size_t)p.P * cpw * p.NP, 256);
   } else if (path == SSM_PATH_SPLIT_L) {
     // about two waves of resident warps; segments of at least 4 chunks
     int64_t target = 2 * slots;
-    int64_t segs = (target + p.n_groups - 1) / p.n_groups;
+    int64_t segs = (target + G - 1) / G;
     int64_t max_segs = p.K / 4 > 1 ? p.K / 4 : 1;
     if (segs > max_segs) segs = max_segs;
     if (segs < 2 && p.K >= 2) segs = 2;
     if (segs < 1) segs = 1;
     p.seg_chunks = (p.K + segs - 1) / segs;
     p.n_segs = (p.K + p.seg_chunks - 1) / p.seg_chunks;
-    const size_t items = (size_t)p.n_groups * (size_t)p.n_segs;
+    const size_t items = (size_t)G * (size_t)p.n_segs;
     p.off_seg_h = kHeaderBytes;
-    p.off_seg_dsum = round_up(p.off_seg_h + sizeof(float) * items * kCPW * p.NP, 256);
-    p.off_seg_carry = round_up(p.off_seg_dsum + sizeof(float) * items * kCPW, 256);
-    p.total = round_up(p.off_seg_carry + sizeof(float) * items * kCPW * p.NP, 256);
+    p.off_seg_dsum = round_up(p.off_seg_h + sizeof(float) * items * cpw * p.NP, 256);
+    p.off_seg_carry = round_up(p.off_seg_dsum + sizeof(float) * items * cpw, 256);
+    p.total = round_up(p.off_seg_carry + sizeof(float) * items * cpw * p.NP, 256);
   } else {
     p.n_segs = 1;
     p.seg_chunks = p.K;
@@ -195,14 +221,14 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
     p.carry = reinterpret_cast<float *>(ws + pl.off_carry);
     e = cudaMemsetAsync(ws, 0, pl.off_carry, s);  // error word and flags
     if (e != cudaSuccess) return cuda_status(e);
-    e = launch_fwd_lookback(shape->io_dtype, pl.NP, p, s);
+    e = launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
   } else {
     if (pl.n_segs > 1) {
       p.seg_h = reinterpret_cast<float *>(ws + pl.off_seg_h);
       p.seg_dsum = reinterpret_cast<float *>(ws + pl.off_seg_dsum);
       p.seg_carry = reinterpret_cast<float *>(ws + pl.off_seg_carry);
     }
-    e = launch_fwd_splitl(shape->io_dtype, pl.NP, p, s);
+    e = launch_fwd_splitl(shape->io_dtype, pl.NP, pl.LPC, p, s);
   }
   return cuda_status(e);
 }

@@ -9,15 +9,14 @@
 namespace ssm {
 
 // ---- work decomposition ----------------------------------------------------
-// A warp owns an 8-channel group of one batch element.  Lane l handles
-// channel c = l / 4 and, of that channel's dstate states, the slice
-// n in [j*S, j*S + S) with j = l % 4 and S = NP / 4 (NP = dstate padded up to
-// a power of two >= 4).  Time is processed in chunks of kT steps; within a
-// chunk each lane walks the recurrence sequentially, so every (t, n) element
-// costs one exp2 and four fp32 ops and nothing of size (L, N) is stored.
+// A warp owns a group of 32/LPC channels of one batch element (LPC = lanes
+// per channel, 2 or 4).  Lane l handles channel c = l / LPC and, of that
+// channel's dstate states, the slice n in [j*S, j*S + S) with j = l % LPC and
+// S = NP / LPC (NP = dstate padded up to a power of two >= 4).  Time is
+// processed in chunks of kT steps; within a chunk each lane walks the
+// recurrence sequentially, so every (t, n) element costs one exp2 and four
+// fp32 ops and nothing of size (L, N) is stored.
 constexpr int kT = 32;           // time steps per chunk
-constexpr int kCPW = 8;          // channels per warp
-constexpr int kLPC = 4;          // lanes per channel
 constexpr int kWarps = 4;        // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowPad = 4;       // smem row padding (floats) against bank conflicts
@@ -42,20 +41,20 @@ struct FwdParams {
   int softplus;
   int io_vec;   // u/delta/z/y rows 16-byte aligned: vector loads
   int bc_vec;   // B/C chunk blocks 16-byte aligned and N == NP
-  int64_t gpb;        // 8-channel groups per batch element
+  int64_t gpb;        // channel groups per batch element
   int64_t n_groups;   // batch * gpb
   int64_t n_chunks;   // ceil(L / kT)
   // look-back schedule
   int64_t n_workers;  // warps
-  float *carry;       // [n_workers][kCPW][NP]
+  float *carry;       // [n_workers][32/LPC][NP]
   unsigned *flags;    // [n_workers]
   unsigned *err;      // workspace header
   unsigned long long wait_limit_ns;
   // split-L schedule
   int64_t n_segs, seg_chunks;
-  float *seg_h;       // [n_groups * n_segs][kCPW][NP] segment end state from zero
-  float *seg_dsum;    // [n_groups * n_segs][kCPW]      sum of Delta over the segment
-  float *seg_carry;   // [n_groups * n_segs][kCPW][NP] state entering the segment
+  float *seg_h;       // [n_groups * n_segs][32/LPC][NP] segment end state from zero
+  float *seg_dsum;    // [n_groups * n_segs][32/LPC]     sum of Delta over the segment
+  float *seg_carry;   // [n_groups * n_segs][32/LPC][NP] state entering the segment
 };
 
 // ---- io helpers ---------------------------------------------------------------
@@ -190,9 +189,9 @@ __device__ __forceinline__ bool warp_wait_flag(const unsigned *flag, unsigned *e
 
 // ---- launchers (defined in ssm_fwd.cu / ssm_bwd.cu) ----------------------------
 int fwd_np_for(int64_t N);
-cudaError_t fwd_occupancy(int io_dtype, int NP, int *ctas_per_sm);
-cudaError_t launch_fwd_lookback(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
-cudaError_t launch_fwd_splitl(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
+cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm);
+cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
+cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,
                                       cudaStream_t s);
 

@@ -12,49 +12,238 @@
 //             Mamba?" (ibm.com), output equation and block walk-through
 //
 // Design (B200): the path is bound by the special-function unit (one exp2 per
-// (t, n) element) and issue slots, not by HBM.  So each lane walks the
-// recurrence sequentially in time over a few states of one channel: per
-// element one MUFU ex2 and four fp32 ops (Delta*A, Delta*u*B, the state FMA,
-// the C contraction FMA), which is the minimum.  The reading guide's "parallel
-// associative scan" is used where time has to be split across warps: the
-// split-L schedule combines segment end states with the operator
-// (a, b) o (a', b') = (a a', a' b + b'), and the look-back schedule hands a
-// state across two warps.  Quantities computed once per (channel, step)
-// (softplus, Delta*u, the gate) are staged through shared memory so that the
-// four lanes of a channel share them; B and C chunks are widened to fp32 in
-// shared memory once per warp and read back as broadcasts.  Nothing of size
-// (L, N) is ever written to global memory.
+// (t, n) element) and by instruction issue, not by HBM.  So each lane walks
+// the recurrence sequentially in time over S states of one channel: per
+// element one MUFU ex2 plus four fp32 operations (Delta*A, Delta*u*B, the
+// state FMA, the C contraction FMA), issued as two-wide packed fp32 (f32x2)
+// instructions.  LPC lanes share a channel (LPC = 2 or 4; S = NP / LPC), so a
+// warp holds 32/LPC channels.
+//
+// The reading guide's "parallel associative scan" is used where time has to
+// be split across warps: the split-L schedule combines segment end states with
+// the operator (a, b) o (a', b') = (a a', a' b + b'), and the look-back
+// schedule hands a state across two warps.  Quantities computed once per
+// (channel, step) (softplus, Delta*u, the gate) are staged through shared
+// memory so that the LPC lanes of a channel share them; B and C chunks are
+// widened to fp32 in shared memory once per warp and read back as broadcasts.
+// The next chunk's inputs are loaded into registers before the current chunk's
+// recurrence runs.  Nothing of size (L, N) is ever written to global memory.
 #include "ssm_common.cuh"
 
 namespace ssm {
 
-template <int NP>
-struct __align__(16) FwdSmem {
-  float dl[kCPW][kT + kRowPad];   // Delta
-  float dlu[kCPW][kT + kRowPad];  // Delta * u
-  float ys[kCPW][kT + kRowPad];   // sum_n C h (reduced over the channel's lanes)
-  float Bs[kT][NP];               // B chunk, fp32, zero padded
-  float Cs[kT][NP];               // C chunk
+// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) -----------------------------
+typedef unsigned long long f2;
+
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ---- softplus without a second special-function op --------------------------
+// softplus(s) = max(s, 0) + log1p(x),  x = exp(-|s|) in (0, 1].
+// log1p(x) = x * p(x), p a degree-8 polynomial interpolating log1p(x)/x at the
+// Chebyshev nodes of [0, 1] (max relative error 2.3e-7 in fp32 evaluation,
+// fitted for this library).
+__device__ __forceinline__ float softplus_fast(float s) {
+  const float x = ex2(-fabsf(s) * kLog2e);
+  float p = 5.126102362e-03f;
+  p = fmaf(p, x, -2.907406539e-02f);
+  p = fmaf(p, x, 7.751608640e-02f);
+  p = fmaf(p, x, -1.360224783e-01f);
+  p = fmaf(p, x, 1.907688081e-01f);
+  p = fmaf(p, x, -2.483539879e-01f);
+  p = fmaf(p, x, 3.331812024e-01f);
+  p = fmaf(p, x, -4.999944568e-01f);
+  p = fmaf(p, x, 9.999999404e-01f);
+  return fmaf(x, p, fmaxf(s, 0.f));
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// SiLU(z) = z / (1 + e^-z)
+__device__ __forceinline__ float silu_fast(float z) {
+  return z * rcp_approx(1.f + ex2(-z * kLog2e));
+}
+
+// ---- raw io vectors of 8 values ------------------------------------------------
+template <typename T> struct Vec8;
+template <> struct Vec8<uint16_t> {
+  uint4 v;
+  __device__ __forceinline__ void load(const uint16_t *row, int64_t t, int64_t L, bool vec) {
+    if (vec && t + 8 <= L) {
+      v = __ldg(reinterpret_cast<const uint4 *>(row + t));
+    } else {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (t + 2 * i < L) ? row[t + 2 * i] : 0u;
+        const uint32_t hi = (t + 2 * i + 1 < L) ? row[t + 2 * i + 1] : 0u;
+        w[i] = lo | (hi << 16);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void unpack(float (&o)[8]) const {
+    o[0] = bf16_lo(v.x); o[1] = bf16_hi(v.x); o[2] = bf16_lo(v.y); o[3] = bf16_hi(v.y);
+    o[4] = bf16_lo(v.z); o[5] = bf16_hi(v.z); o[6] = bf16_lo(v.w); o[7] = bf16_hi(v.w);
+  }
+};
+template <> struct Vec8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *row, int64_t t, int64_t L, bool vec) {
+    if (vec && t + 8 <= L) {
+      a = __ldg(reinterpret_cast<const float4 *>(row + t));
+      b = __ldg(reinterpret_cast<const float4 *>(row + t + 4));
+    } else {
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = (t + i < L) ? row[t + i] : 0.f;
+      a = make_float4(o[0], o[1], o[2], o[3]);
+      b = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void unpack(float (&o)[8]) const {
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
 };
 
-template <int S>
-__device__ __forceinline__ void lds_vec(const float *p, float (&v)[S]) {
-  if constexpr (S % 4 == 0) {
+// ---- geometry ---------------------------------------------------------------------
+template <int NP, int LPC>
+struct Geo {
+  static constexpr int CPW = 32 / LPC;      // channels per warp
+  static constexpr int S = NP / LPC;        // states per lane
+  static constexpr int STEPS = kT / LPC;    // steps per lane in the per-step phases
+  static constexpr int VEC = STEPS / 8;     // 8-value vectors per lane and tensor
+};
+
+template <int NP, int LPC>
+struct __align__(16) FwdSmem {
+  float dl[32 / LPC][kT + kRowPad];   // Delta
+  float dlu[32 / LPC][kT + kRowPad];  // Delta * u
+  float ys[32 / LPC][kT + kRowPad];   // sum_n C h, reduced over the channel's lanes
+  float Bs[kT][NP];                   // B chunk, fp32, zero padded
+  float Cs[kT][NP];                   // C chunk
+};
+
+// B/C chunk in flight: raw 16-byte vectors of one chunk (vector path).
+template <typename T, int NP>
+struct BCChunk {
+  static constexpr int EPV = 16 / (int)sizeof(T);
+  static constexpr bool kVecOK = (NP % EPV) == 0;
+  static constexpr int NV = kVecOK ? kT * NP / EPV : 0;    // vectors per chunk and tensor
+  static constexpr int PER_LANE = (NV + 31) / 32;
+  static constexpr bool kPrefetch = kVecOK && PER_LANE <= 4;
+  uint4 b[kPrefetch ? PER_LANE : 1], c[kPrefetch ? PER_LANE : 1];
+};
+
+// Issue the global loads of one B/C chunk (vector path).
+template <typename T, int NP, bool EMIT>
+__device__ __forceinline__ void bc_load(BCChunk<T, NP> &r, const T *Bb, const T *Cb, int64_t t0,
+                                        int64_t L, int lane) {
+  using BC = BCChunk<T, NP>;
+  if constexpr (BC::kPrefetch) {
 #pragma unroll
-    for (int i = 0; i < S; i += 4) {
-      const float4 x = *reinterpret_cast<const float4 *>(p + i);
-      v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+    for (int i = 0; i < BC::PER_LANE; ++i) {
+      const int v = lane + 32 * i;
+      const int e = v * BC::EPV, t = e / NP;
+      if (v < BC::NV && t0 + t < L) {
+        r.b[i] = __ldg(reinterpret_cast<const uint4 *>(Bb + (t0 + t) * NP + (e - t * NP)));
+        if (EMIT) r.c[i] = __ldg(reinterpret_cast<const uint4 *>(Cb + (t0 + t) * NP + (e - t * NP)));
+      } else {
+        r.b[i] = make_uint4(0, 0, 0, 0);
+        r.c[i] = make_uint4(0, 0, 0, 0);
+      }
     }
-  } else if constexpr (S == 2) {
-    const float2 x = *reinterpret_cast<const float2 *>(p);
-    v[0] = x.x; v[1] = x.y;
-  } else {
-    v[0] = p[0];
   }
 }
 
-// The 4 lanes j = 0..3 of a channel each hold partial sums y0..y3 for 4
-// consecutive steps; lane j returns the full sum for step j (2 shuffle rounds).
+template <typename T, int NP>
+__device__ __forceinline__ void bc_store_vec(float (*dst)[NP], const uint4 &x, int v) {
+  using BC = BCChunk<T, NP>;
+  const int e = v * BC::EPV, t = e / NP, n = e - t * NP;
+  if constexpr (sizeof(T) == 2) {
+    *reinterpret_cast<float4 *>(&dst[t][n]) =
+        make_float4(bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y));
+    *reinterpret_cast<float4 *>(&dst[t][n + 4]) =
+        make_float4(bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w));
+  } else {
+    *reinterpret_cast<float4 *>(&dst[t][n]) =
+        make_float4(__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z), __uint_as_float(x.w));
+  }
+}
+
+// Stage one B/C chunk into smem: from the prefetched registers, or loading
+// it here (vector path without prefetch, or the scalar path when N != NP or
+// the rows are not 16-byte aligned).
+template <typename T, int NP, bool EMIT>
+__device__ __forceinline__ void bc_stage(float (*Bs)[NP], float (*Cs)[NP], const BCChunk<T, NP> &r,
+                                         const T *Bb, const T *Cb, int64_t t0, int64_t L, int N,
+                                         bool vec, int lane) {
+  using BC = BCChunk<T, NP>;
+  if constexpr (BC::kVecOK) {
+    if (vec) {
+      if constexpr (BC::kPrefetch) {
+#pragma unroll
+        for (int i = 0; i < BC::PER_LANE; ++i) {
+          const int v = lane + 32 * i;
+          if (v < BC::NV) {
+            bc_store_vec<T, NP>(Bs, r.b[i], v);
+            if (EMIT) bc_store_vec<T, NP>(Cs, r.c[i], v);
+          }
+        }
+      } else {
+        for (int v = lane; v < BC::NV; v += 32) {
+          const int e = v * BC::EPV, t = e / NP;
+          uint4 xb = make_uint4(0, 0, 0, 0), xc = make_uint4(0, 0, 0, 0);
+          if (t0 + t < L) {
+            xb = __ldg(reinterpret_cast<const uint4 *>(Bb + (t0 + t) * NP + (e - t * NP)));
+            if (EMIT) xc = __ldg(reinterpret_cast<const uint4 *>(Cb + (t0 + t) * NP + (e - t * NP)));
+          }
+          bc_store_vec<T, NP>(Bs, xb, v);
+          if (EMIT) bc_store_vec<T, NP>(Cs, xc, v);
+        }
+      }
+      return;
+    }
+  }
+  for (int e = lane; e < kT * NP; e += 32) {
+    const int t = e / NP, n = e - t * NP;
+    const bool in = n < N && t0 + t < L;
+    Bs[t][n] = in ? IO<T>::get(Bb, (t0 + t) * N + n) : 0.f;
+    if (EMIT) Cs[t][n] = in ? IO<T>::get(Cb, (t0 + t) * N + n) : 0.f;
+  }
+}
+
+// ---- reductions across the LPC lanes of a channel ------------------------------
+// LPC = 2: lanes j = 0, 1 hold partials y0, y1 for steps t, t+1; lane j returns step t+j.
+__device__ __forceinline__ float reduce2_transpose(float y0, float y1, int j) {
+  float keep = j ? y1 : y0;
+  const float send = j ? y0 : y1;
+  keep += __shfl_xor_sync(0xffffffffu, send, 1);
+  return keep;
+}
+// LPC = 4: lanes j = 0..3 hold partials for 4 steps; lane j returns step t+j.
 __device__ __forceinline__ float reduce4_transpose(float y0, float y1, float y2, float y3, int j) {
   const bool hi2 = (j & 2) != 0;
   float ka = hi2 ? y2 : y0, kb = hi2 ? y3 : y1;
@@ -68,67 +257,28 @@ __device__ __forceinline__ float reduce4_transpose(float y0, float y1, float y2,
   return k;
 }
 
-// B or C chunk [t0, t0 + kT) of one batch element into smem as fp32 [t][n],
-// zero for n >= N or t >= L.
-template <typename T, int NP>
-__device__ __forceinline__ void stage_bc(float (*dst)[NP], const T *src, int64_t t0, int64_t L,
-                                         int N, bool vec, int lane) {
-  constexpr int EPV = 16 / (int)sizeof(T);
-  if constexpr (NP % EPV == 0) {
-    if (vec) {  // N == NP and every 16-byte vector lies inside one row
-      constexpr int NV = kT * NP / EPV;
-#pragma unroll
-      for (int v = lane; v < NV; v += 32) {
-        const int e = v * EPV, t = e / NP, n = e - t * NP;
-        float o[EPV];
-        if (t0 + t < L) {
-          const T *ps = src + (t0 + t) * NP + n;
-          if constexpr (sizeof(T) == 2) {
-            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(ps));
-            o[0] = bf16_lo(x.x); o[1] = bf16_hi(x.x); o[2] = bf16_lo(x.y); o[3] = bf16_hi(x.y);
-            o[4] = bf16_lo(x.z); o[5] = bf16_hi(x.z); o[6] = bf16_lo(x.w); o[7] = bf16_hi(x.w);
-          } else {
-            const float4 x = __ldg(reinterpret_cast<const float4 *>(ps));
-            o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < EPV; ++i) o[i] = 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < EPV; i += 4)
-          *reinterpret_cast<float4 *>(&dst[t][n + i]) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-      }
-      return;
-    }
-  }
-  for (int e = lane; e < kT * NP; e += 32) {
-    const int t = e / NP, n = e - t * NP;
-    dst[t][n] = (n < N && t0 + t < L) ? IO<T>::get(src, (t0 + t) * N + n) : 0.f;
-  }
-}
-
-// Per-lane view of an 8-channel group.
+// ---- per-lane view of a channel group -----------------------------------------
 struct Lane {
   int lane, c, j;
   int64_t b, d;
   bool valid;
 };
 
+template <int LPC>
 __device__ __forceinline__ Lane lane_of(const FwdParams &p, int64_t g) {
   Lane r;
   r.lane = threadIdx.x & 31;
-  r.c = r.lane >> 2;
-  r.j = r.lane & 3;
+  r.c = r.lane / LPC;
+  r.j = r.lane % LPC;
   r.b = g / p.gpb;
-  r.d = (g - r.b * p.gpb) * kCPW + r.c;
+  r.d = (g - r.b * p.gpb) * (32 / LPC) + r.c;
   r.valid = r.d < p.dim;
   return r;
 }
 
-template <int NP>
-__device__ __forceinline__ void init_state(const FwdParams &p, const Lane &ln, float (&h)[NP / 4]) {
-  constexpr int S = NP / 4;
+template <int NP, int LPC>
+__device__ __forceinline__ void init_state(const FwdParams &p, const Lane &ln, float (&h)[NP / LPC]) {
+  constexpr int S = NP / LPC;
 #pragma unroll
   for (int s = 0; s < S; ++s) {
     const int n = ln.j * S + s;
@@ -136,10 +286,10 @@ __device__ __forceinline__ void init_state(const FwdParams &p, const Lane &ln, f
   }
 }
 
-template <int NP>
+template <int NP, int LPC>
 __device__ __forceinline__ void write_last_state(const FwdParams &p, const Lane &ln,
-                                                 const float (&h)[NP / 4]) {
-  constexpr int S = NP / 4;
+                                                 const float (&h)[NP / LPC]) {
+  constexpr int S = NP / LPC;
   if (!p.last_state || !ln.valid) return;
 #pragma unroll
   for (int s = 0; s < S; ++s) {
@@ -148,13 +298,16 @@ __device__ __forceinline__ void write_last_state(const FwdParams &p, const Lane 
   }
 }
 
-// Walk chunks [k0, k1) of group g from state h.  EMIT: write y (output pass);
-// otherwise only advance h and sum Delta (split-L pass 1).
-template <typename T, int NP, bool EMIT>
-__device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP> &sm, const Lane &ln,
-                                           int64_t k0, int64_t k1, float (&h)[NP / 4], float &dsum) {
-  constexpr int S = NP / 4;
-  const int c = ln.c, j = ln.j, q = ln.j;  // q: this lane's 8-step quarter of a chunk
+// ---- the chunk loop ------------------------------------------------------------------
+// Walk chunks [k0, k1) of the lane's channel group from state h.
+// EMIT: write y (output pass); otherwise advance h and sum Delta (split-L pass 1).
+template <typename T, int NP, int LPC, bool EMIT>
+__device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP, LPC> &sm, const Lane &ln,
+                                           int64_t k0, int64_t k1, float (&h)[NP / LPC],
+                                           float &dsum) {
+  using G = Geo<NP, LPC>;
+  constexpr int S = G::S, VEC = G::VEC, STEPS = G::STEPS;
+  const int c = ln.c, j = ln.j;
   const int64_t L = p.L;
   const int64_t row = (ln.b * p.dim + (ln.valid ? ln.d : 0)) * L;
   const T *u_row = static_cast<const T *>(p.u) + row;
@@ -166,6 +319,7 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP> &sm, 
   const float bias = (p.bias && ln.valid) ? p.bias[ln.d] : 0.f;
   const float Dd = (p.D && ln.valid) ? p.D[ln.d] : 0.f;
   const bool io_vec = p.io_vec != 0, bc_vec = p.bc_vec != 0;
+  const bool has_z = EMIT && z_row != nullptr;
   float A2[S];
 #pragma unroll
   for (int s = 0; s < S; ++s) {
@@ -173,37 +327,59 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP> &sm, 
     A2[s] = (ln.valid && n < p.N) ? p.A[ln.d * p.N + n] * kLog2e : 0.f;
   }
 
+  // registers of the chunk in flight
+  Vec8<T> ru[VEC], rd[VEC], rz[VEC];
+  BCChunk<T, NP> rbc;
+  auto issue_loads = [&](int64_t k) {
+    const int64_t ts = k * kT + j * STEPS;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      if (ln.valid) {
+        ru[v].load(u_row, ts + 8 * v, L, io_vec);
+        rd[v].load(dr_row, ts + 8 * v, L, io_vec);
+        if (has_z) rz[v].load(z_row, ts + 8 * v, L, io_vec);
+        else rz[v].zero();
+      } else {
+        ru[v].zero(); rd[v].zero(); rz[v].zero();
+      }
+    }
+    if (bc_vec) bc_load<T, NP, EMIT>(rbc, Bb, Cb, k * kT, L, ln.lane);
+  };
+  if (k0 < k1) issue_loads(k0);
+
   for (int64_t k = k0; k < k1; ++k) {
     const int64_t t0 = k * kT;
-    const int64_t tq = t0 + 8 * q;
-    // ---- per (channel, step) quantities of this lane's 8 steps ----
-    float uu[8], dr[8], zz[8];
-    if (ln.valid) {
-      IO<T>::load8(u_row, tq, L, io_vec, uu);
-      IO<T>::load8(dr_row, tq, L, io_vec, dr);
-      if (EMIT && z_row) IO<T>::load8(z_row, tq, L, io_vec, zz);
-    } else {
+    const int64_t ts = t0 + j * STEPS;
+    // ---- per (channel, step): Delta and Delta*u of this lane's STEPS steps ----
+    float uu[STEPS], zz[STEPS];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { uu[i] = 0.f; dr[i] = 0.f; zz[i] = 0.f; }
-    }
-    float dlv[8], dluv[8];
+    for (int v = 0; v < VEC; ++v) {
+      float u8[8], d8[8], z8[8];
+      ru[v].unpack(u8);
+      rd[v].unpack(d8);
+      rz[v].unpack(z8);
+      float dl8[8], du8[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float dl = 0.f;
-      if (ln.valid && tq + i < L) {
-        const float s = dr[i] + bias;
-        dl = p.softplus ? softplus_f(s) : s;
+      for (int i = 0; i < 8; ++i) {
+        float dl = d8[i] + bias;
+        dl = p.softplus ? softplus_fast(dl) : dl;
+        dl = (ln.valid && ts + 8 * v + i < L) ? dl : 0.f;  // padded steps: identity
+        dl8[i] = dl;
+        du8[i] = dl * u8[i];
+        uu[8 * v + i] = u8[i];
+        zz[8 * v + i] = z8[i];
       }
-      dlv[i] = dl;
-      dluv[i] = dl * uu[i];
+      float *pd = &sm.dl[c][j * STEPS + 8 * v];
+      float *pu = &sm.dlu[c][j * STEPS + 8 * v];
+      *reinterpret_cast<float4 *>(pd) = make_float4(dl8[0], dl8[1], dl8[2], dl8[3]);
+      *reinterpret_cast<float4 *>(pd + 4) = make_float4(dl8[4], dl8[5], dl8[6], dl8[7]);
+      *reinterpret_cast<float4 *>(pu) = make_float4(du8[0], du8[1], du8[2], du8[3]);
+      *reinterpret_cast<float4 *>(pu + 4) = make_float4(du8[4], du8[5], du8[6], du8[7]);
     }
-    *reinterpret_cast<float4 *>(&sm.dl[c][8 * q]) = make_float4(dlv[0], dlv[1], dlv[2], dlv[3]);
-    *reinterpret_cast<float4 *>(&sm.dl[c][8 * q + 4]) = make_float4(dlv[4], dlv[5], dlv[6], dlv[7]);
-    *reinterpret_cast<float4 *>(&sm.dlu[c][8 * q]) = make_float4(dluv[0], dluv[1], dluv[2], dluv[3]);
-    *reinterpret_cast<float4 *>(&sm.dlu[c][8 * q + 4]) = make_float4(dluv[4], dluv[5], dluv[6], dluv[7]);
-    stage_bc<T, NP>(sm.Bs, Bb, t0, L, p.N, bc_vec, ln.lane);
-    if (EMIT) stage_bc<T, NP>(sm.Cs, Cb, t0, L, p.N, bc_vec, ln.lane);
+    bc_stage<T, NP, EMIT>(sm.Bs, sm.Cs, rbc, Bb, Cb, t0, L, p.N, bc_vec, ln.lane);
     __syncwarp();
+    // the next chunk's loads fly while this chunk's recurrence runs
+    if (k + 1 < k1) issue_loads(k + 1);
 
     // ---- the recurrence: kT steps, S states per lane ----
 #pragma unroll 2
@@ -215,37 +391,65 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP> &sm, 
       float yp[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float Bv[S], Cv[S];
-        lds_vec<S>(&sm.Bs[tt + i][j * S], Bv);
-        if (EMIT) lds_vec<S>(&sm.Cs[tt + i][j * S], Cv);
-        float acc = 0.f;
+        const float *Brow = &sm.Bs[tt + i][j * S];
+        const float *Crow = &sm.Cs[tt + i][j * S];
+        if constexpr (S % 2 == 0) {
+          const f2 dl2 = pack2(dls[i], dls[i]), du2 = pack2(dus[i], dus[i]);
+          f2 acc = pack2(0.f, 0.f);
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-          const float a = ex2(dls[i] * A2[s]);
-          h[s] = fmaf(a, h[s], dus[i] * Bv[s]);
-          if (EMIT) acc = fmaf(Cv[s], h[s], acc);
+          for (int s = 0; s < S; s += 2) {
+            const f2 bv = *reinterpret_cast<const f2 *>(Brow + s);
+            float x0, x1;
+            unpack2(mul2(dl2, pack2(A2[s], A2[s + 1])), x0, x1);
+            const f2 a = pack2(ex2(x0), ex2(x1));
+            const f2 hh = fma2(a, pack2(h[s], h[s + 1]), mul2(du2, bv));
+            unpack2(hh, h[s], h[s + 1]);
+            if (EMIT) acc = fma2(*reinterpret_cast<const f2 *>(Crow + s), hh, acc);
+          }
+          float a0, a1;
+          unpack2(acc, a0, a1);
+          yp[i] = a0 + a1;
+        } else {
+          float acc = 0.f;
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            const float a = ex2(dls[i] * A2[s]);
+            h[s] = fmaf(a, h[s], dus[i] * Brow[s]);
+            if (EMIT) acc = fmaf(Crow[s], h[s], acc);
+          }
+          yp[i] = acc;
         }
-        yp[i] = acc;
         if (!EMIT) dsum += dls[i];
       }
-      if (EMIT) sm.ys[c][tt + j] = reduce4_transpose(yp[0], yp[1], yp[2], yp[3], j);
+      if (EMIT) {
+        if constexpr (LPC == 4) {
+          sm.ys[c][tt + j] = reduce4_transpose(yp[0], yp[1], yp[2], yp[3], j);
+        } else {
+          sm.ys[c][tt + j] = reduce2_transpose(yp[0], yp[1], j);
+          sm.ys[c][tt + 2 + j] = reduce2_transpose(yp[2], yp[3], j);
+        }
+      }
     }
 
-    // ---- epilogue: D skip, gate, store ----
+    // ---- epilogue: D skip, gate, store this lane's STEPS steps ----
     if (EMIT) {
       __syncwarp();
       if (ln.valid) {
-        const float4 a = *reinterpret_cast<const float4 *>(&sm.ys[c][8 * q]);
-        const float4 b4 = *reinterpret_cast<const float4 *>(&sm.ys[c][8 * q + 4]);
-        const float ys[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
-        float o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float v = fmaf(Dd, uu[i], ys[i]);
-          if (z_row) v *= silu_f(zz[i]);
-          o[i] = v;
+        for (int v = 0; v < VEC; ++v) {
+          const float *py = &sm.ys[c][j * STEPS + 8 * v];
+          const float4 a = *reinterpret_cast<const float4 *>(py);
+          const float4 b4 = *reinterpret_cast<const float4 *>(py + 4);
+          const float ys[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float val = fmaf(Dd, uu[8 * v + i], ys[i]);
+            if (has_z) val *= silu_fast(zz[8 * v + i]);
+            o[i] = val;
+          }
+          IO<T>::store8(y_row, ts + 8 * v, L, io_vec, o);
         }
-        IO<T>::store8(y_row, tq, L, io_vec, o);
       }
     }
     __syncwarp();
@@ -256,17 +460,17 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP> &sm, 
 // Warp w owns items [w*W/P, (w+1)*W/P) of the W = groups*chunks items in
 // (group, chunk) order.  Its range holds at most a tail of one group, whole
 // groups, and a head of another (the host keeps P <= groups, so a range is
-// never inside one group).  The head is done first, from the initial state,
-// and its end state published; the tail, which needs the state the previous
-// warp published from ITS head, is done last.  The bounded wait therefore
-// only spins if the previous warp has not finished its first item by the
-// time this warp has finished everything else.
-template <typename T, int NP>
+// never strictly inside one group).  The head is done first, from the initial
+// state, and its end state published; the tail, which needs the state the
+// previous warp published from ITS head, is done last.  The bounded wait
+// therefore only spins if the previous warp has not finished its first item
+// by the time this warp has finished everything else.
+template <typename T, int NP, int LPC>
 __global__ void __launch_bounds__(kThreads) k_fwd_lookback(FwdParams p) {
-  constexpr int S = NP / 4;
+  constexpr int S = NP / LPC, CPW = 32 / LPC;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
-  FwdSmem<NP> &sm = reinterpret_cast<FwdSmem<NP> *>(smem_raw)[warp];
+  FwdSmem<NP, LPC> &sm = reinterpret_cast<FwdSmem<NP, LPC> *>(smem_raw)[warp];
   const int64_t w = (int64_t)blockIdx.x * kWarps + warp;
   const int64_t P = p.n_workers;
   if (w >= P) return;
@@ -292,24 +496,24 @@ __global__ void __launch_bounds__(kThreads) k_fwd_lookback(FwdParams p) {
     else if (r < n_head) { g = g_last; k0 = 0; k1 = k_end; }
     else if (r < n_head + n_full) { g = g_lo + (r - n_head); k0 = 0; k1 = K; }
     else { g = g_first; k0 = k_first; k1 = K; }
-    const Lane ln = lane_of(p, g);
+    const Lane ln = lane_of<LPC>(p, g);
     if (k0 > 0) {  // continue the previous warp's head of this group
       warp_wait_flag(&p.flags[w - 1], p.err, p.wait_limit_ns);
 #pragma unroll
       for (int s = 0; s < S; ++s)
-        h[s] = __ldcg(&p.carry[((w - 1) * kCPW + ln.c) * NP + ln.j * S + s]);
+        h[s] = __ldcg(&p.carry[((w - 1) * CPW + ln.c) * NP + ln.j * S + s]);
     } else {
-      init_state<NP>(p, ln, h);
+      init_state<NP, LPC>(p, ln, h);
     }
-    run_chunks<T, NP, true>(p, sm, ln, k0, k1, h, dsum);
+    run_chunks<T, NP, LPC, true>(p, sm, ln, k0, k1, h, dsum);
     if (k1 < K) {  // publish the head's end state for warp w + 1
 #pragma unroll
-      for (int s = 0; s < S; ++s) p.carry[(w * kCPW + ln.c) * NP + ln.j * S + s] = h[s];
+      for (int s = 0; s < S; ++s) p.carry[(w * CPW + ln.c) * NP + ln.j * S + s] = h[s];
       __threadfence();
       __syncwarp();
       if (ln.lane == 0) st_release(&p.flags[w], 1u);
     } else {
-      write_last_state<NP>(p, ln, h);
+      write_last_state<NP, LPC>(p, ln, h);
     }
   }
 }
@@ -320,19 +524,19 @@ __global__ void __launch_bounds__(kThreads) k_fwd_lookback(FwdParams p) {
 // the segment's sum of Delta); EMIT=true is the output pass, entering each
 // segment with the state the carry kernel computed (or the initial state
 // when there is one segment).
-template <typename T, int NP, bool EMIT>
+template <typename T, int NP, int LPC, bool EMIT>
 __global__ void __launch_bounds__(kThreads) k_fwd_segment(FwdParams p) {
-  constexpr int S = NP / 4;
+  constexpr int S = NP / LPC, CPW = 32 / LPC;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
-  FwdSmem<NP> &sm = reinterpret_cast<FwdSmem<NP> *>(smem_raw)[warp];
+  FwdSmem<NP, LPC> &sm = reinterpret_cast<FwdSmem<NP, LPC> *>(smem_raw)[warp];
   const int64_t w = (int64_t)blockIdx.x * kWarps + warp;
   if (w >= p.n_groups * p.n_segs) return;
   const int64_t seg = w / p.n_groups, g = w - seg * p.n_groups;
   const int64_t k0 = seg * p.seg_chunks;
   const int64_t k1 = k0 + p.seg_chunks < p.n_chunks ? k0 + p.seg_chunks : p.n_chunks;
   const int64_t item = g * p.n_segs + seg;
-  const Lane ln = lane_of(p, g);
+  const Lane ln = lane_of<LPC>(p, g);
   float h[S];
   float dsum = 0.f;
   if (!EMIT) {
@@ -340,37 +544,38 @@ __global__ void __launch_bounds__(kThreads) k_fwd_segment(FwdParams p) {
     for (int s = 0; s < S; ++s) h[s] = 0.f;
   } else if (p.n_segs > 1) {
 #pragma unroll
-    for (int s = 0; s < S; ++s) h[s] = p.seg_carry[(item * kCPW + ln.c) * NP + ln.j * S + s];
+    for (int s = 0; s < S; ++s) h[s] = p.seg_carry[(item * CPW + ln.c) * NP + ln.j * S + s];
   } else {
-    init_state<NP>(p, ln, h);
+    init_state<NP, LPC>(p, ln, h);
   }
-  if (k0 < k1) run_chunks<T, NP, EMIT>(p, sm, ln, k0, k1, h, dsum);
+  if (k0 < k1) run_chunks<T, NP, LPC, EMIT>(p, sm, ln, k0, k1, h, dsum);
   if (!EMIT) {
 #pragma unroll
-    for (int s = 0; s < S; ++s) p.seg_h[(item * kCPW + ln.c) * NP + ln.j * S + s] = h[s];
-    if (ln.j == 0) p.seg_dsum[item * kCPW + ln.c] = dsum;
+    for (int s = 0; s < S; ++s) p.seg_h[(item * CPW + ln.c) * NP + ln.j * S + s] = h[s];
+    if (ln.j == 0) p.seg_dsum[item * CPW + ln.c] = dsum;
   } else if (k1 == p.n_chunks) {
-    write_last_state<NP>(p, ln, h);
+    write_last_state<NP, LPC>(p, ln, h);
   }
 }
 
 // Carry over segments, one thread per (group, channel, state):
 //   carry_0 = h0,  carry_{s+1} = exp(A * sum_s Delta) * carry_s + h_end_s
 // -- the associative operator of the recurrence applied segment by segment.
-template <int NP>
+template <int NP, int LPC>
 __global__ void k_fwd_carry(FwdParams p) {
+  constexpr int CPW = 32 / LPC;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= p.n_groups * kCPW * NP) return;
-  const int64_t g = idx / (kCPW * NP);
-  const int c = (int)((idx / NP) % kCPW), n = (int)(idx % NP);
-  const int64_t b = g / p.gpb, d = (g - b * p.gpb) * kCPW + c;
+  if (idx >= p.n_groups * CPW * NP) return;
+  const int64_t g = idx / (CPW * NP);
+  const int c = (int)((idx / NP) % CPW), n = (int)(idx % NP);
+  const int64_t b = g / p.gpb, d = (g - b * p.gpb) * CPW + c;
   const bool valid = d < p.dim && n < p.N;
   const float A2 = valid ? p.A[d * p.N + n] * kLog2e : 0.f;
   float carry = (valid && p.h0) ? p.h0[(b * p.dim + d) * p.N + n] : 0.f;
   for (int64_t s = 0; s < p.n_segs; ++s) {
     const int64_t item = g * p.n_segs + s;
-    p.seg_carry[(item * kCPW + c) * NP + n] = carry;
-    carry = fmaf(ex2(A2 * p.seg_dsum[item * kCPW + c]), carry, p.seg_h[(item * kCPW + c) * NP + n]);
+    p.seg_carry[(item * CPW + c) * NP + n] = carry;
+    carry = fmaf(ex2(A2 * p.seg_dsum[item * CPW + c]), carry, p.seg_h[(item * CPW + c) * NP + n]);
   }
 }
 
@@ -383,14 +588,19 @@ template <class V> struct TypeTag { using type = V; };
 template <int V> struct IntTag { static constexpr int value = V; };
 
 template <class F>
-static cudaError_t dispatch(int io_dtype, int NP, F &&f) {
+static cudaError_t dispatch(int io_dtype, int NP, int LPC, F &&f) {
+  auto by_lpc = [&](auto tt, auto np) -> cudaError_t {
+    if (LPC == 2) return f(tt, np, IntTag<2>{});
+    if (LPC == 4) return f(tt, np, IntTag<4>{});
+    return cudaErrorInvalidValue;
+  };
   auto by_np = [&](auto tt) -> cudaError_t {
     switch (NP) {
-      case 4: return f(tt, IntTag<4>{});
-      case 8: return f(tt, IntTag<8>{});
-      case 16: return f(tt, IntTag<16>{});
-      case 32: return f(tt, IntTag<32>{});
-      case 64: return f(tt, IntTag<64>{});
+      case 4: return by_lpc(tt, IntTag<4>{});
+      case 8: return by_lpc(tt, IntTag<8>{});
+      case 16: return by_lpc(tt, IntTag<16>{});
+      case 32: return by_lpc(tt, IntTag<32>{});
+      case 64: return by_lpc(tt, IntTag<64>{});
       default: return cudaErrorInvalidValue;
     }
   };
@@ -401,8 +611,8 @@ static cudaError_t dispatch(int io_dtype, int NP, F &&f) {
 
 int fwd_np_for(int64_t N) { return N <= 4 ? 4 : N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : 64; }
 
-template <typename T, int NP>
-static size_t fwd_smem_bytes() { return kWarps * sizeof(FwdSmem<NP>); }
+template <int NP, int LPC>
+static size_t fwd_smem_bytes() { return kWarps * sizeof(FwdSmem<NP, LPC>); }
 
 template <class K>
 static cudaError_t allow_smem(K kernel, size_t bytes) {
@@ -410,48 +620,48 @@ static cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-cudaError_t fwd_occupancy(int io_dtype, int NP, int *ctas_per_sm) {
-  return dispatch(io_dtype, NP, [&](auto tt, auto np) -> cudaError_t {
+cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm) {
+  return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
-    constexpr int kNP = decltype(np)::value;
-    const size_t smem = fwd_smem_bytes<T, kNP>();
-    cudaError_t e = allow_smem(k_fwd_lookback<T, kNP>, smem);
+    constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
+    const size_t smem = fwd_smem_bytes<kNP, kLPC>();
+    cudaError_t e = allow_smem(k_fwd_lookback<T, kNP, kLPC>, smem);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_lookback<T, kNP>,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_lookback<T, kNP, kLPC>,
                                                          kThreads, smem);
   });
 }
 
-cudaError_t launch_fwd_lookback(int io_dtype, int NP, const FwdParams &p, cudaStream_t s) {
-  return dispatch(io_dtype, NP, [&](auto tt, auto np) -> cudaError_t {
+cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s) {
+  return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
-    constexpr int kNP = decltype(np)::value;
-    const size_t smem = fwd_smem_bytes<T, kNP>();
-    cudaError_t e = allow_smem(k_fwd_lookback<T, kNP>, smem);
+    constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
+    const size_t smem = fwd_smem_bytes<kNP, kLPC>();
+    cudaError_t e = allow_smem(k_fwd_lookback<T, kNP, kLPC>, smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.n_workers + kWarps - 1) / kWarps);
-    k_fwd_lookback<T, kNP><<<grid, kThreads, smem, s>>>(p);
+    k_fwd_lookback<T, kNP, kLPC><<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }
 
-cudaError_t launch_fwd_splitl(int io_dtype, int NP, const FwdParams &p, cudaStream_t s) {
-  return dispatch(io_dtype, NP, [&](auto tt, auto np) -> cudaError_t {
+cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s) {
+  return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
-    constexpr int kNP = decltype(np)::value;
-    const size_t smem = fwd_smem_bytes<T, kNP>();
+    constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
+    const size_t smem = fwd_smem_bytes<kNP, kLPC>();
     const unsigned grid = (unsigned)((p.n_groups * p.n_segs + kWarps - 1) / kWarps);
     cudaError_t e;
     if (p.n_segs > 1) {
-      e = allow_smem(k_fwd_segment<T, kNP, false>, smem);
+      e = allow_smem(k_fwd_segment<T, kNP, kLPC, false>, smem);
       if (e != cudaSuccess) return e;
-      k_fwd_segment<T, kNP, false><<<grid, kThreads, smem, s>>>(p);
-      const int64_t nthreads = p.n_groups * kCPW * kNP;
-      k_fwd_carry<kNP><<<(unsigned)((nthreads + 255) / 256), 256, 0, s>>>(p);
+      k_fwd_segment<T, kNP, kLPC, false><<<grid, kThreads, smem, s>>>(p);
+      const int64_t nthreads = p.n_groups * (32 / kLPC) * kNP;
+      k_fwd_carry<kNP, kLPC><<<(unsigned)((nthreads + 255) / 256), 256, 0, s>>>(p);
     }
-    e = allow_smem(k_fwd_segment<T, kNP, true>, smem);
+    e = allow_smem(k_fwd_segment<T, kNP, kLPC, true>, smem);
     if (e != cudaSuccess) return e;
-    k_fwd_segment<T, kNP, true><<<grid, kThreads, smem, s>>>(p);
+    k_fwd_segment<T, kNP, kLPC, true><<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }

@@ -17,21 +17,21 @@ pytestmark = pytest.mark.gpu
 PATHS = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3}
 
 
-def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None):
+def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None, lanes=0):
     import torch
     import selective_state_space_54_b200 as ssm
     g = upload(case, device)
     h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
     y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
                          g["delta_bias"], delta_softplus=softplus, initial_state=h0_t,
-                         return_last_state=True, path=PATHS[path], y=y_out)
+                         return_last_state=True, path=PATHS[path], y=y_out, lanes=lanes)
     torch.cuda.synchronize()
     return to_f64(y), to_f64(ls)
 
 
-def _check(case, device, path="auto", softplus=True, h0=None):
+def _check(case, device, path="auto", softplus=True, h0=None, lanes=0):
     ref = oracle.fwd(case, delta_softplus=softplus, h0=h0)
-    y, ls = _run(case, device, path, softplus, h0)
+    y, ls = _run(case, device, path, softplus, h0, lanes=lanes)
     st = assert_close(y, ref["y"], case["dtype"], f"y[{path}]")
     # the state is fp32 on both io dtypes
     assert_close(ls, ref["last_state"], synth.F32 if case["dtype"] == synth.F32 else synth.BF16,
@@ -45,25 +45,28 @@ def test_tiny_fp32_workload(cuda_device, path):
     _check(case, cuda_device, path)
 
 
+@pytest.mark.parametrize("lanes", [2, 4])
 @pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
 @pytest.mark.parametrize("N", [1, 3, 4, 8, 12, 16, 32, 64])
-def test_dstate_sizes(cuda_device, dtype, N):
+def test_dstate_sizes(cuda_device, dtype, N, lanes):
     case = synth.make_case(2, 20, 200, N, dtype, seed=100 + N)
-    _check(case, cuda_device, "per_group")
+    _check(case, cuda_device, "per_group", lanes=lanes)
 
 
+@pytest.mark.parametrize("lanes", [2, 4])
 @pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
 @pytest.mark.parametrize("L", [1, 7, 31, 32, 33, 257, 1000, 1003])
-def test_ragged_lengths_and_groups(cuda_device, path, L):
-    # dim 44: five full 8-channel groups and a ragged one; L odd -> scalar loads
+def test_ragged_lengths_and_groups(cuda_device, path, L, lanes):
+    # dim 44: ragged 16- and 8-channel groups; L odd -> scalar loads
     case = synth.make_case(3, 44, L, 16, synth.BF16, seed=L)
-    _check(case, cuda_device, path)
+    _check(case, cuda_device, path, lanes=lanes)
 
 
+@pytest.mark.parametrize("lanes", [2, 4])
 @pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
-def test_fp32_several_chunks(cuda_device, path):
+def test_fp32_several_chunks(cuda_device, path, lanes):
     case = synth.make_case(2, 24, 777, 16, synth.F32, seed=7)
-    _check(case, cuda_device, path)
+    _check(case, cuda_device, path, lanes=lanes)
 
 
 @pytest.mark.parametrize("opt", ["no_z", "no_D", "no_bias", "no_softplus", "bare"])
@@ -79,11 +82,12 @@ def test_optional_terms(cuda_device, opt):
     _check(case, cuda_device, "auto", softplus=softplus)
 
 
+@pytest.mark.parametrize("lanes", [2, 4])
 @pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
-def test_initial_state(cuda_device, path):
+def test_initial_state(cuda_device, path, lanes):
     case = synth.make_case(2, 16, 500, 16, synth.F32, seed=9)
     h0 = np.random.default_rng(1).standard_normal((2, 16, 16)).astype(np.float32)
-    _check(case, cuda_device, path, h0=h0)
+    _check(case, cuda_device, path, h0=h0, lanes=lanes)
 
 
 def test_continuation_matches_one_scan(cuda_device):
@@ -131,10 +135,35 @@ def test_large_delta_reset_bitwise(cuda_device):
 
 def test_paths_agree(cuda_device):
     case = synth.make_case(4, 64, 2048, 16, synth.BF16, seed=31)
-    outs = {p: _run(case, cuda_device, p)[0] for p in ("lookback", "split_l", "per_group")}
-    for p in ("split_l", "per_group"):
-        d = np.max(np.abs(outs[p] - outs["lookback"]))
-        assert d <= 2e-2 * np.max(np.abs(outs["lookback"])), (p, d)
+    ref = oracle.fwd(case)["y"]
+    outs = {(p, ln): _run(case, cuda_device, p, lanes=ln)[0]
+            for p in ("lookback", "split_l", "per_group") for ln in (2, 4)}
+    for k, y in outs.items():
+        assert_close(y, ref, case["dtype"], str(k))
+        d = np.max(np.abs(y - outs[("lookback", 2)]))
+        assert d <= 2e-2 * np.max(np.abs(ref)), (k, d)
+
+
+def test_softplus_accuracy_through_the_kernel(cuda_device):
+    # N=1, B=1, C=1, u=1, no D, no gate, and A so negative that Abar = 0 at
+    # every step: then h_t = Delta_t and y_t = Delta_t = softplus(s_t) exactly,
+    # so the device softplus is checked against the oracle's log1p(exp(s))
+    # over s in [-30, 30], element by element.
+    L = 4096
+    s = np.linspace(-30.0, 30.0, L).astype(np.float32)
+    case = {"batch": 1, "dim": 1, "seqlen": L, "dstate": 1, "dtype": synth.F32,
+            "u": np.ones((1, 1, L), np.float32), "delta": s.reshape(1, 1, L),
+            "A": np.full((1, 1), -1e30, np.float32), "B": np.ones((1, L, 1), np.float32),
+            "C": np.ones((1, L, 1), np.float32), "D": None, "z": None, "delta_bias": None}
+    ref = oracle.fwd(case)["y"][0, 0]
+    assert np.all(ref > 0)
+    for lanes in (2, 4):
+        y, _ = _run(case, cuda_device, "per_group", lanes=lanes)
+        rel = np.abs(y[0, 0] - ref) / ref
+        # exp(-|s|) is 2^(-|s| log2 e): the fp32 rounding of that argument
+        # alone allows |s| * 6e-8 * ln 2 relative error
+        bound = 1e-6 + 1e-7 * np.abs(s.astype(np.float64))
+        assert np.all(rel <= bound), (lanes, float(rel.max()), float(s[np.argmax(rel / bound)]))
 
 
 def test_deterministic(cuda_device):
