@@ -139,6 +139,27 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
                         float *dinitial_state,
                         void *workspace, size_t ws_bytes, ssm_stream_t stream);
 
+/* Forward scan for callers that cannot allocate device memory: inference
+ * engine or framework plugins whose host owns every allocation and forbids
+ * one on the execute path, or real-time loops that allocate nothing after
+ * start-up.  The pages have no counterpart of this: it is a deployment
+ * convenience.  Same arguments and results as ssm_scan_fwd, without the
+ * workspace: the scratch lives in one 4 MiB device array inside the library
+ * (held on every GPU that loads it until the process exits).  path AUTO
+ * means SSM_PATH_LOOKBACK here, whose scratch does not grow with the
+ * problem.  Shapes needing more scratch than the array return
+ * SSM_ERR_UNSUPPORTED before any launch.  All calls share the array: calls
+ * whose kernels overlap on the GPU race, so order them on one stream.  The
+ * first call on a device looks up the array's address with that device
+ * current; make it before any stream capture.  The device error word sits
+ * in the array too, so a bounded look-back wait that gives up is not
+ * reported to the caller of this entry point. */
+ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u, const void *delta,
+                                const float *A, const void *B, const void *C,
+                                const float *D, const void *z, const float *delta_bias,
+                                int delta_softplus, const float *initial_state,
+                                void *y, float *last_state, ssm_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word of
  * `workspace`.  SSM_OK, SSM_ERR_DEVICE_TIMEOUT or SSM_ERR_CUDA. */
 ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream);
