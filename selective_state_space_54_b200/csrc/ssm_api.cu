@@ -235,7 +235,13 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
 
 size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
   if (check_shape(shape) != SSM_OK) return 0;
-  return kHeaderBytes;
+  const int NP = fwd_np_for(shape->dstate);
+  const size_t acc = sizeof(float) * (size_t)shape->batch * (size_t)shape->seqlen * NP;
+  size_t total = kHeaderBytes;
+  total = round_up(total + sizeof(float) * bwd_ckpt_floats(shape->batch, shape->dim, shape->seqlen, NP), 256);
+  total = round_up(total + acc, 256);
+  total = round_up(total + acc, 256);
+  return total;
 }
 
 ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta,
@@ -245,13 +251,62 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
                         float *dA, void *dB, void *dC, float *dD, void *dz,
                         float *ddelta_bias, float *dinitial_state, void *workspace,
                         size_t ws_bytes, ssm_stream_t stream) {
-  (void)u; (void)delta; (void)A; (void)B; (void)C; (void)D; (void)z; (void)delta_bias;
-  (void)delta_softplus; (void)initial_state; (void)dout; (void)du; (void)ddelta; (void)dA;
-  (void)dB; (void)dC; (void)dD; (void)dz; (void)ddelta_bias; (void)dinitial_state;
-  (void)workspace; (void)ws_bytes; (void)stream;
   ssm_status st = check_shape(shape);
   if (st != SSM_OK) return st;
-  return SSM_ERR_UNSUPPORTED;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t batch = shape->batch, dim = shape->dim, L = shape->seqlen, N = shape->dstate;
+  const size_t es = shape->io_dtype == SSM_BF16 ? 2 : 4;
+  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr) ||
+      (delta_bias == nullptr) != (ddelta_bias == nullptr))
+    return SSM_ERR_INVALID_ARG;
+  if (batch * dim == 0 || L == 0) {  // no step to differentiate: parameter gradients are zero
+    if (dim > 0 && (!dA || !aligned(dA, 4))) return SSM_ERR_INVALID_ARG;
+    cudaError_t e = cudaSuccess;
+    if (dim > 0) e = cudaMemsetAsync(dA, 0, sizeof(float) * dim * N, s);
+    if (e == cudaSuccess && dim > 0 && dD) e = cudaMemsetAsync(dD, 0, sizeof(float) * dim, s);
+    if (e == cudaSuccess && dim > 0 && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * dim, s);
+    if (e == cudaSuccess && batch * dim > 0 && dinitial_state)
+      e = cudaMemsetAsync(dinitial_state, 0, sizeof(float) * batch * dim * N, s);
+    return cuda_status(e);
+  }
+  if (!u || !delta || !A || !B || !C || !dout || !du || !ddelta || !dA || !dB || !dC)
+    return SSM_ERR_INVALID_ARG;
+  if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) ||
+      !aligned(z, es) || !aligned(dout, es) || !aligned(du, es) || !aligned(ddelta, es) ||
+      !aligned(dB, es) || !aligned(dC, es) || !aligned(dz, es) || !aligned(A, 4) ||
+      !aligned(D, 4) || !aligned(delta_bias, 4) || !aligned(initial_state, 4) ||
+      !aligned(dA, 4) || !aligned(dD, 4) || !aligned(ddelta_bias, 4) || !aligned(dinitial_state, 4))
+    return SSM_ERR_INVALID_ARG;
+  const size_t need = ssm_scan_bwd_workspace_bytes(shape);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
+  const int NP = fwd_np_for(N);
+  char *ws = static_cast<char *>(workspace);
+  const size_t acc = sizeof(float) * (size_t)batch * (size_t)L * NP;
+  const size_t off_ckpt = kHeaderBytes;
+  const size_t off_dB = round_up(off_ckpt + sizeof(float) * bwd_ckpt_floats(batch, dim, L, NP), 256);
+  const size_t off_dC = round_up(off_dB + acc, 256);
+
+  BwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C; p.dout = dout;
+  p.A = A; p.D = D; p.bias = delta_bias; p.h0 = initial_state;
+  p.du = du; p.ddelta = ddelta; p.dz = dz;
+  p.dA = dA; p.dD = dD; p.dbias = ddelta_bias; p.dh0 = dinitial_state;
+  p.ckpt = reinterpret_cast<float *>(ws + off_ckpt);
+  p.dB_acc = reinterpret_cast<float *>(ws + off_dB);
+  p.dC_acc = reinterpret_cast<float *>(ws + off_dC);
+  p.dB = dB; p.dC = dC;
+  p.batch = batch; p.dim = dim; p.L = L; p.N = (int)N;
+  p.softplus = delta_softplus ? 1 : 0;
+  p.io_vec = ((L * (int64_t)es) % 16 == 0) && aligned(u, 16) && aligned(delta, 16) &&
+             aligned(z, 16) && aligned(dout, 16) && aligned(du, 16) && aligned(ddelta, 16) &&
+             aligned(dz, 16);
+  cudaError_t e = cudaMemsetAsync(dA, 0, sizeof(float) * dim * N, s);
+  if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, sizeof(float) * dim, s);
+  if (e == cudaSuccess && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * dim, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws + off_dB, 0, (off_dC - off_dB) + acc, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_bwd(shape->io_dtype, NP, p, s));
 }
 
 ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream) {

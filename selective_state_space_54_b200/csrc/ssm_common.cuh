@@ -57,6 +57,23 @@ struct FwdParams {
   float *seg_carry;   // [n_groups * n_segs][32/LPC][NP] state entering the segment
 };
 
+// Backward parameters (ssm_bwd.cu).
+struct BwdParams {
+  const void *u, *delta, *z, *B, *C, *dout;
+  const float *A, *D, *bias, *h0;
+  void *du, *ddelta, *dz;
+  float *dA, *dD, *dbias, *dh0;
+  float *dB_acc, *dC_acc;     // [batch][L][NP] fp32
+  float *ckpt;                // [cta][K][32][NP]
+  void *dB, *dC;              // [batch][L][N] io dtype (finalize)
+  int64_t batch, dim, L;
+  int N;
+  int softplus;
+  int io_vec;
+  int64_t cpb;                // CTAs per batch element
+  int64_t K;                  // backward chunks
+};
+
 // ---- io helpers ---------------------------------------------------------------
 // bf16 values travel as raw 16-bit patterns; widening is a shift.
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -192,6 +209,8 @@ int fwd_np_for(int64_t N);
 cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm);
 cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
+size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
+cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,
                                       cudaStream_t s);
 

@@ -34,8 +34,7 @@ def _check(case, device, path="auto", softplus=True, h0=None, lanes=0):
     y, ls = _run(case, device, path, softplus, h0, lanes=lanes)
     st = assert_close(y, ref["y"], case["dtype"], f"y[{path}]")
     # the state is fp32 on both io dtypes
-    assert_close(ls, ref["last_state"], synth.F32 if case["dtype"] == synth.F32 else synth.BF16,
-                 f"last_state[{path}]")
+    assert_close(ls, ref["last_state"], case["dtype"], f"last_state[{path}]", stored_bf16=False)
     return st
 
 
@@ -220,7 +219,8 @@ def _full_size(name, device, sample=None):
         yg = to_f64(y[b, dims])[None]
         lg = to_f64(ls[b, dims])[None]
         assert_close(yg, ref["y"], case["dtype"], f"{name} y b={b}")
-        assert_close(lg, ref["last_state"], synth.BF16, f"{name} last_state b={b}")
+        assert_close(lg, ref["last_state"], case["dtype"], f"{name} last_state b={b}",
+                     stored_bf16=False)
     return y
 
 

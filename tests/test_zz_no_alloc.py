@@ -48,8 +48,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_device, dtype, batch, dim, L
         assert _noalloc(lib, shape, g, y, ls, stream) == 0
         torch.cuda.synchronize()
         assert_close(to_f64(y), ref_y, dtype, f"y, call {call}")
-        assert_close(to_f64(ls), ref_ls, synth.BF16 if dtype == synth.BF16 else synth.F32,
-                     f"last_state, call {call}")
+        assert_close(to_f64(ls), ref_ls, dtype, f"last_state, call {call}", stored_bf16=False)
 
 
 def test_noalloc_rejects_shapes_beyond_the_static_scratch(cuda_device):
