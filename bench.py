@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--workload", default="mamba-2.8b-layer", choices=list(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true",
+                    help="skip the training-workload forward+backward measurement")
     ap.add_argument("--lanes", type=int, default=0, choices=[0, 2, 4],
                     help="lanes per channel (0: the library's choice)")
     ap.add_argument("--path", default="auto", choices=["auto", "lookback", "split_l", "per_group"])
@@ -167,6 +169,22 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def dist_max(x: float, world: int, device) -> float:
+    """Max of a per-rank time over all ranks (every rank calls it, same order)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world: int, units_per_rank: float, seconds_max: float) -> float:
+    """Whole-job throughput: every rank processes its own replica (weak scaling)."""
+    return world * units_per_rank / seconds_max
+
+
 def init_dist(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -263,6 +281,65 @@ def config_of(w, path):
             "seed": w.seed}
 
 
+def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None):
+    """Forward + recomputation backward on the Mamba-1.4B layer training shape."""
+    w = w or synth.WORKLOADS["mamba-1.4b-layer-train"]
+    case = synth.make_workload(w)
+    g = {k: to_torch(case[k], dev) for k in ("u", "delta", "z", "B", "C", "dy")}
+    for k in ("A", "D", "delta_bias"):
+        g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
+    del case
+    y = torch.empty_like(g["u"])
+    shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
+                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32)
+    ws_f = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(ssm.bwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    out = {"du": torch.empty_like(g["u"]), "ddelta": torch.empty_like(g["u"]),
+           "dz": torch.empty_like(g["u"]), "dB": torch.empty_like(g["B"]),
+           "dC": torch.empty_like(g["C"]),
+           "dA": torch.empty((w.dim, w.dstate), dtype=torch.float32, device=dev),
+           "dD": torch.empty((w.dim,), dtype=torch.float32, device=dev),
+           "ddelta_bias": torch.empty((w.dim,), dtype=torch.float32, device=dev)}
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                     y=y, workspace=ws_f)
+
+    def bwd():
+        ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                     g["dy"], out=out, workspace=ws_b)
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    steps = max(3, min(args.steps, 10))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_f = t_b = 0.0
+    for _ in range(steps):
+        evs[0].record(stream)
+        fwd()
+        evs[1].record(stream)
+        bwd()
+        evs[2].record(stream)
+        torch.cuda.synchronize(dev)
+        t_f += evs[0].elapsed_time(evs[1])
+        t_b += evs[1].elapsed_time(evs[2])
+    barrier()
+    ms_f = max_over_ranks(t_f / steps)
+    ms_b = max_over_ranks(t_b / steps)
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
+            "d_state": w.dstate, "io_dtype": w.dtype, "steps": steps,
+            "fwd_ms": ms_f, "bwd_ms": ms_b,
+            "value": aggregate_value(world, w.bld, (ms_f + ms_b) * 1e-3), "unit": UNIT + " (fwd+bwd)",
+            "bwd_value": aggregate_value(world, w.bld, ms_b * 1e-3),
+            "bwd_ex2_per_element": 3,
+            "bwd_kernels_per_step": 2}
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -280,7 +357,27 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     if w.backward:
-        raise SystemExit("forward workloads only in this benchmark")
+        # the training step itself: forward + recomputation backward
+        def barrier0():
+            if world > 1:
+                import torch.distributed as dist
+                dist.barrier()
+
+        def max0(x):
+            return dist_max(x, world, dev)
+        tr = measure_training(ssm, torch, dev, args, world, barrier0, max0, w)
+        line = {"metric": METRIC, "value": tr["value"], "unit": UNIT, "n_gpus": world,
+                "steps": tr["steps"], "warmup": max(3, args.warmup),
+                "ms_per_step": tr["fwd_ms"] + tr["bwd_ms"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": dict(config_of(w, "lookback"), step="fwd+bwd"), "bwd": tr,
+                "gpu_launches": 3 * tr["steps"]}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
 
     case = synth.make_workload(w)
     g = {k: to_torch(case[k], dev) for k in ("u", "delta", "z", "B", "C")}
@@ -308,12 +405,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(x, world, dev)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -366,9 +458,13 @@ def main():
         torch.cuda.synchronize(dev)
         barrier()
         ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / k_e2e)
-        e2e = {"value": world * w.bld / (ms_e2e * 1e-3), "unit": UNIT,
+        e2e = {"value": aggregate_value(world, w.bld, ms_e2e * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
         del host, dbuf
+
+    bwd = None
+    if not args.no_bwd and not args.batch:
+        bwd = measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks)
 
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -388,11 +484,12 @@ def main():
         at_clock = sm_count * MUFU_EX2_PER_CLK_PER_SM * clocks["sm_mhz"] * 1e6
         roofline["frac_at_measured_clock"] = achieved / at_clock
 
-    line = {"metric": METRIC, "value": world * w.bld / sec, "unit": UNIT, "n_gpus": world,
+    line = {"metric": METRIC, "value": aggregate_value(world, w.bld, sec), "unit": UNIT,
+            "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
-            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, case)

@@ -110,3 +110,43 @@ def test_product_has_no_oracle_or_cpu_path():
                 text = open(os.path.join(root, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "ssm_oracle" not in text, f
+
+
+def _bwd(lib, shape, **over):
+    # shape, u, delta, A, B, C, D, z, bias, softplus, h0, dout,
+    # du, ddelta, dA, dB, dC, dD, dz, dbias, dh0, ws, ws_bytes, stream
+    p = dict(u=16, delta=16, A=16, B=16, C=16, D=None, z=None, bias=None, h0=None, dout=16,
+             du=16, ddelta=16, dA=16, dB=16, dC=16, dD=None, dz=None, dbias=None, dh0=None)
+    p.update(over)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ssm_scan_bwd(ctypes.byref(shape), v(p["u"]), v(p["delta"]), v(p["A"]), v(p["B"]),
+                            v(p["C"]), v(p["D"]), v(p["z"]), v(p["bias"]), 1, v(p["h0"]),
+                            v(p["dout"]), v(p["du"]), v(p["ddelta"]), v(p["dA"]), v(p["dB"]),
+                            v(p["dC"]), v(p["dD"]), v(p["dz"]), v(p["dbias"]), v(p["dh0"]),
+                            None, 0, None)
+
+
+@pytest.mark.parametrize("over", [dict(z=16), dict(dz=16), dict(D=16), dict(dD=16),
+                                  dict(bias=16), dict(dbias=16)])
+def test_bwd_gradient_pairs_must_match(lib, over):
+    # dz exactly when z, dD exactly when D, ddelta_bias exactly when delta_bias
+    assert _bwd(lib, _shape(), **over) == _lib.SSM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("missing", ["u", "delta", "A", "B", "C", "dout", "du", "ddelta", "dA",
+                                     "dB", "dC"])
+def test_bwd_null_required_pointer_rejected(lib, missing):
+    assert _bwd(lib, _shape(), **{missing: None}) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_bwd_misaligned_rejected(lib):
+    assert _bwd(lib, _shape(), du=17) == _lib.SSM_ERR_INVALID_ARG  # bf16 needs 2-byte
+    assert _bwd(lib, _shape(), dA=6) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_bad_shapes_before_launch(lib):
+    for kw, code in BAD_SHAPES:
+        sh = _shape(**kw)
+        rc = lib.ssm_scan_fwd_noalloc(ctypes.byref(sh), *[ctypes.c_void_p(16)] * 5, None, None,
+                                      None, 1, None, ctypes.c_void_p(16), None, None)
+        assert rc == code
