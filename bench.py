@@ -54,7 +54,8 @@ def parse():
                     help="skip the training-workload forward+backward measurement")
     ap.add_argument("--lanes", type=int, default=0, choices=[0, 2, 4],
                     help="lanes per channel (0: the library's choice)")
-    ap.add_argument("--path", default="auto", choices=["auto", "lookback", "split_l", "per_group"])
+    ap.add_argument("--path", default="auto",
+                    choices=["auto", "lookback", "split_l", "per_group", "lookback_ws"])
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling only)")
     return ap.parse_args()
@@ -385,13 +386,13 @@ def main():
         g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
     y = torch.empty_like(g["u"])
     ls = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
-    path_id = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3}[args.path]
+    path_id = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3, "lookback_ws": 4}[args.path]
     shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
                            ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32,
                            path_id, args.lanes)
     path = ssm.fwd_path(shape)
     ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
-    launches_per_step = {"lookback": 1, "per_group": 1, "split_l": 3}[path]
+    launches_per_step = {"lookback": 1, "per_group": 1, "split_l": 3, "lookback_ws": 1}[path]
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -474,7 +475,8 @@ def main():
     roofline = {"bound": "alu", "achieved": achieved / 1e12, "peak": ex2_peak / 1e12,
                 "unit": "Tex2/s", "frac": achieved / ex2_peak,
                 "traffic": profiled_traffic(),
-                "kernel": "k_fwd_lookback" if path == "lookback" else f"k_fwd_segment ({path})",
+                "kernel": {"lookback": "k_fwd_lookback", "lookback_ws": "k_fwd_ws"}.get(
+                    path, f"k_fwd_segment ({path})"),
                 "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                               f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})",
                 "algorithmic_bytes": alg_bytes(w),

@@ -74,12 +74,18 @@ typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
  *  SPLIT_L   two passes over time segments (segment end states from zero,
  *            a sequential carry over segments, then the output pass);
  *            for long sequences with few channels;
- *  PER_GROUP one warp per channel group over the whole sequence. */
+ *  PER_GROUP one warp per channel group over the whole sequence;
+ *  LOOKBACK_WS  the look-back schedule with warp specialisation (2 lanes per
+ *            channel): producer warps load inputs and compute softplus, the
+ *            gate and the output epilogue on the FMA pipe, consumer warps run
+ *            only the recurrence; AUTO picks it when it picks LOOKBACK with
+ *            2 lanes per channel. */
 typedef enum {
   SSM_PATH_AUTO = 0,
   SSM_PATH_LOOKBACK = 1,
   SSM_PATH_SPLIT_L = 2,
-  SSM_PATH_PER_GROUP = 3
+  SSM_PATH_PER_GROUP = 3,
+  SSM_PATH_LOOKBACK_WS = 4
 } ssm_path;
 
 typedef struct {

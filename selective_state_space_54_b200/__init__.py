@@ -18,7 +18,7 @@ import ctypes
 
 from . import _lib
 from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_PATH_AUTO, SSM_PATH_LOOKBACK,  # noqa: F401
-                   SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L, ssm_shape)
+                   SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L, ssm_shape)
 
 __all__ = ["scan_fwd", "scan_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes",
            "fwd_path", "check", "ScanError", "make_shape"]

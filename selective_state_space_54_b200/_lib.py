@@ -24,9 +24,11 @@ SSM_PATH_AUTO = 0
 SSM_PATH_LOOKBACK = 1
 SSM_PATH_SPLIT_L = 2
 SSM_PATH_PER_GROUP = 3
+SSM_PATH_LOOKBACK_WS = 4
 
 PATH_NAMES = {SSM_PATH_AUTO: "auto", SSM_PATH_LOOKBACK: "lookback",
-              SSM_PATH_SPLIT_L: "split_l", SSM_PATH_PER_GROUP: "per_group"}
+              SSM_PATH_SPLIT_L: "split_l", SSM_PATH_PER_GROUP: "per_group",
+              SSM_PATH_LOOKBACK_WS: "lookback_ws"}
 
 # every symbol include/ssm_scan.h declares
 EXPORTS = (

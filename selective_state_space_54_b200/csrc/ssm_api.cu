@@ -28,7 +28,8 @@ ssm_status check_shape(const ssm_shape *s) {
   if (s->batch < 0 || s->dim < 0 || s->seqlen < 0 || s->dstate < 1) return SSM_ERR_INVALID_ARG;
   if (s->dstate > 64) return SSM_ERR_UNSUPPORTED;
   if (s->io_dtype != SSM_F32 && s->io_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
-  if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_PER_GROUP) return SSM_ERR_UNSUPPORTED;
+  if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_LOOKBACK_WS) return SSM_ERR_UNSUPPORTED;
+  if (s->path == SSM_PATH_LOOKBACK_WS && s->lanes == 4) return SSM_ERR_UNSUPPORTED;
   if (s->lanes != 0 && s->lanes != 2 && s->lanes != 4) return SSM_ERR_UNSUPPORTED;
   if (s->reserved != 0) return SSM_ERR_INVALID_ARG;
   // index arithmetic is int64; keep every flat index well inside it
@@ -76,7 +77,7 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   const int64_t g2 = groups_for(s, 2), g4 = groups_for(s, 4);
   int path = s->path, lpc = s->lanes;
   if (lpc == 0) {
-    if (path == SSM_PATH_SPLIT_L) lpc = 2;
+    if (path == SSM_PATH_SPLIT_L || path == SSM_PATH_LOOKBACK_WS) lpc = 2;
     else if (path == SSM_PATH_PER_GROUP) lpc = 4;
     else if (g2 >= 2 * unit) lpc = 2;
     else if (g4 >= unit || path == SSM_PATH_LOOKBACK) lpc = 4;
@@ -84,14 +85,22 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   }
   const int64_t G = lpc == 2 ? g2 : g4;
   if (path == SSM_PATH_AUTO) {
-    if (G >= unit) path = SSM_PATH_LOOKBACK;
+    if (G >= unit) path = lpc == 2 ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
     else if (p.K >= 64) path = SSM_PATH_SPLIT_L;
     else path = SSM_PATH_PER_GROUP;
   }
   int occ = 0;
-  if (fwd_occupancy(s->io_dtype, p.NP, lpc, &occ) != cudaSuccess || occ <= 0) {
+  cudaError_t oe = path == SSM_PATH_LOOKBACK_WS ? fwd_ws_occupancy(s->io_dtype, p.NP, &occ)
+                                                : fwd_occupancy(s->io_dtype, p.NP, lpc, &occ);
+  if (oe != cudaSuccess || occ <= 0) {
     cudaGetLastError();
     return SSM_ERR_CUDA;
+  }
+  if (path == SSM_PATH_LOOKBACK_WS) {
+    // a CTA holds fwd_ws_pairs() consumer warps (one per sub-partition); the
+    // look-back items are (group, fwd_ws_chunk()-step chunk)
+    occ = occ * fwd_ws_pairs() / kWarps;
+    p.K = (s->seqlen + fwd_ws_chunk() - 1) / fwd_ws_chunk();
   }
   const int64_t slots = unit * occ;             // resident warps
   const int cpw = 32 / lpc;
@@ -99,7 +108,7 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   p.LPC = lpc;
   p.gpb = (s->dim + cpw - 1) / cpw;
   p.n_groups = G;
-  if (path == SSM_PATH_LOOKBACK) {
+  if (path == SSM_PATH_LOOKBACK || path == SSM_PATH_LOOKBACK_WS) {
     // P <= groups keeps every warp's range at least one group long;
     // a multiple of `unit` gives every sub-partition the same work.
     int64_t r = G / unit;
@@ -216,12 +225,13 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
   p.n_segs = pl.n_segs; p.seg_chunks = pl.seg_chunks;
 
   cudaError_t e;
-  if (pl.path == SSM_PATH_LOOKBACK) {
+  if (pl.path == SSM_PATH_LOOKBACK || pl.path == SSM_PATH_LOOKBACK_WS) {
     p.flags = reinterpret_cast<unsigned *>(ws + pl.off_flags);
     p.carry = reinterpret_cast<float *>(ws + pl.off_carry);
     e = cudaMemsetAsync(ws, 0, pl.off_carry, s);  // error word and flags
     if (e != cudaSuccess) return cuda_status(e);
-    e = launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
+    e = pl.path == SSM_PATH_LOOKBACK_WS ? launch_fwd_ws(shape->io_dtype, pl.NP, p, s)
+                                        : launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
   } else {
     if (pl.n_segs > 1) {
       p.seg_h = reinterpret_cast<float *>(ws + pl.off_seg_h);

@@ -89,12 +89,10 @@ template <int NP>
 struct __align__(16) BwdWarpSmem {
   float dl[kBCPW][kTB + kBPad];    // Delta
   float dlu[kBCPW][kTB + kBPad];   // Delta * u
-  float sg[kBCPW][kTB + kBPad];    // sigmoid(s): d softplus / ds
   float dy[kBCPW][kTB + kBPad];    // dout * SiLU(z)
   float ys[kBCPW][kTB + kBPad];    // sum_n C h
-  float ddl[kBCPW][kTB + kBPad];   // sum_n g (A a h_prev)
-  float s1[kBCPW][kTB + kBPad];    // sum_n g B
-  float dBC[kTB][2][NP];           // this warp's dB, dC over its 8 channels
+  float2 pd[kBCPW][kTB][4];        // per lane j: (sum_n g A a h_prev, sum_n g B) partials
+  float part[kTB / 2][kBCPW][2][NP];  // dB, dC contributions of half a chunk, per channel
 };
 
 template <int NP>
@@ -116,29 +114,41 @@ __device__ __forceinline__ void bwd_stage_bc(BwdSmem<NP> &sm, const T *Bb, const
   }
 }
 
-// Sum V values over the 8 lanes that share lane%4 (lane bits 2..4): after the
-// call lane l holds V/8 sums (V >= 8) at original indices
-// i + c2*V/2 + c1*V/4 + c0*V/8, (c2 c1 c0) = lane bits 4, 3, 2.
-template <int V>
-__device__ __forceinline__ void halve3(float (&v)[V], int lane) {
-  static_assert(V >= 8 && V % 8 == 0, "halve3 needs a multiple of 8 values");
-#pragma unroll
-  for (int lev = 0; lev < 3; ++lev) {
-    const int m = 16 >> lev;           // lane mask: 16, 8, 4
-    const int half = V >> (lev + 1);   // values kept after this level
-    const bool hi = (lane & m) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float keep = hi ? v[i + half] : v[i];
-      const float send = hi ? v[i] : v[i + half];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-    }
-  }
+// packed fp32 pairs (sm_100a f32x2 arithmetic)
+typedef unsigned long long bf2;
+__device__ __forceinline__ bf2 bpack(float lo, float hi) {
+  bf2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void bunpack(bf2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ bf2 bfma(bf2 a, bf2 b, bf2 c) {
+  bf2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ bf2 bmul(bf2 a, bf2 b) {
+  bf2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ bf2 badd(bf2 a, bf2 b) {
+  bf2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ bf2 bex2(bf2 x) {
+  float x0, x1;
+  bunpack(x, x0, x1);
+  return bpack(ex2(x0), ex2(x1));
 }
 
 template <typename T, int NP>
 __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
-  constexpr int S = NP / 4;
+  constexpr int S = NP / 4;              // states per lane
+  constexpr int SP = S >= 2 ? S / 2 : 1; // state pairs per lane (S = 1 pads one)
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem<NP> &sm = *reinterpret_cast<BwdSmem<NP> *>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -163,15 +173,30 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
   const T *Cb = static_cast<const T *>(p.C) + b * L * N;
   const float bias = (p.bias && valid) ? p.bias[d] : 0.f;
   const float Dd = (p.D && valid) ? p.D[d] : 0.f;
-  float A2[S], An[S];
+  // this lane's states n = j*S + s, as pairs; S = 1 uses the low half only
+  bf2 A2[SP], An[SP];
 #pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int n = j * S + s;
-    An[s] = (valid && n < N) ? p.A[d * N + n] : 0.f;
-    A2[s] = An[s] * kLog2e;
+  for (int i = 0; i < SP; ++i) {
+    float a[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int s = 2 * i + h2, n = j * S + s;
+      a[h2] = (s < S && valid && n < N) ? p.A[d * N + n] : 0.f;
+    }
+    An[i] = bpack(a[0], a[1]);
+    A2[i] = bpack(a[0] * kLog2e, a[1] * kLog2e);
   }
   float *ck = p.ckpt + cta * K * (kBW * kBCPW) * NP;
   const int ch = warp * kBCPW + c;   // channel within the CTA
+  auto ck_at = [&](int64_t k, int i) -> float * { return &ck[(k * (kBW * kBCPW) + ch) * NP + j * S + 2 * i]; };
+  auto Bpair = [&](int t, int i) -> bf2 {
+    if constexpr (S >= 2) return *reinterpret_cast<const bf2 *>(&sm.Bs[t][j * S + 2 * i]);
+    else return bpack(sm.Bs[t][j], 0.f);
+  };
+  auto Cpair = [&](int t, int i) -> bf2 {
+    if constexpr (S >= 2) return *reinterpret_cast<const bf2 *>(&sm.Cs[t][j * S + 2 * i]);
+    else return bpack(sm.Cs[t][j], 0.f);
+  };
 
   // per (channel, step) quantities for this lane's 4 steps of chunk k
   auto prepass = [&](int64_t t0, float (&uu)[4], float (&sgs)[4]) {
@@ -185,6 +210,7 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     float dr[4];
     vu.unpack(uu);
     vd.unpack(dr);
+    float dl4[4], du4[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float s = dr[i] + bias;
@@ -195,41 +221,55 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
       }
       const bool in = valid && t0 + 4 * q + i < L;
       dl = in ? dl : 0.f;
-      ws.dl[c][4 * q + i] = dl;
-      ws.dlu[c][4 * q + i] = dl * uu[i];
+      dl4[i] = dl;
+      du4[i] = dl * uu[i];
       sgs[i] = sg;
     }
+    *reinterpret_cast<float4 *>(&ws.dl[c][4 * q]) = make_float4(dl4[0], dl4[1], dl4[2], dl4[3]);
+    *reinterpret_cast<float4 *>(&ws.dlu[c][4 * q]) = make_float4(du4[0], du4[1], du4[2], du4[3]);
   };
 
   // ---- phase A: states entering every chunk ----
-  float h[S];
+  bf2 h[SP];
 #pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int n = j * S + s;
-    h[s] = (p.h0 && valid && n < N) ? p.h0[(b * p.dim + d) * N + n] : 0.f;
+  for (int i = 0; i < SP; ++i) {
+    float v[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int s = 2 * i + h2, n = j * S + s;
+      v[h2] = (s < S && p.h0 && valid && n < N) ? p.h0[(b * p.dim + d) * N + n] : 0.f;
+    }
+    h[i] = bpack(v[0], v[1]);
   }
   for (int64_t k = 0; k < K; ++k) {
     const int64_t t0 = k * kTB;
 #pragma unroll
-    for (int s = 0; s < S; ++s) ck[(k * (kBW * kBCPW) + ch) * NP + j * S + s] = h[s];
+    for (int i = 0; i < SP; ++i) {
+      float lo, hi;
+      bunpack(h[i], lo, hi);
+      float *dst = ck_at(k, i);
+      dst[0] = lo;
+      if (S >= 2) dst[1] = hi;
+    }
     float uu[4], sgs[4];
     prepass(t0, uu, sgs);
     bwd_stage_bc<T, NP>(sm, Bb, Cb, t0, L, N, false);
     __syncthreads();
 #pragma unroll 4
     for (int t = 0; t < kTB; ++t) {
-      const float dl = ws.dl[c][t], du = ws.dlu[c][t];
+      const bf2 dl2 = bpack(ws.dl[c][t], ws.dl[c][t]), du2 = bpack(ws.dlu[c][t], ws.dlu[c][t]);
 #pragma unroll
-      for (int s = 0; s < S; ++s) h[s] = fmaf(ex2(dl * A2[s]), h[s], du * sm.Bs[t][j * S + s]);
+      for (int i = 0; i < SP; ++i) h[i] = bfma(bex2(bmul(dl2, A2[i])), h[i], bmul(du2, Bpair(t, i)));
     }
     __syncthreads();
   }
 
   // ---- phase B: reverse ----
-  float g[S], dA_acc[S];
+  bf2 g[SP], dA_acc[SP];
 #pragma unroll
-  for (int s = 0; s < S; ++s) { g[s] = 0.f; dA_acc[s] = 0.f; }
+  for (int i = 0; i < SP; ++i) { g[i] = bpack(0.f, 0.f); dA_acc[i] = g[i]; }
   float dD_acc = 0.f, dbias_acc = 0.f;
+  constexpr int kRedOutputs = (kTB / 2) * 2 * NP / 4;   // float4 outputs of a half chunk
   for (int64_t k = K - 1; k >= 0; --k) {
     const int64_t t0 = k * kTB;
     float uu[4], sgs[4];
@@ -243,23 +283,29 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     __syncthreads();
 
     // recompute the chunk's states from its checkpoint
-    float H[kTB][S], h0c[S];
+    bf2 H[kTB][SP], h0c[SP];
 #pragma unroll
-    for (int s = 0; s < S; ++s) h0c[s] = ck[(k * (kBW * kBCPW) + ch) * NP + j * S + s];
+    for (int i = 0; i < SP; ++i) {
+      const float *src = ck_at(k, i);
+      h0c[i] = bpack(src[0], S >= 2 ? src[1] : 0.f);
+    }
 #pragma unroll
     for (int t = 0; t < kTB; t += 4) {
       float yp[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float dl = ws.dl[c][t + i], du = ws.dlu[c][t + i];
-        float acc = 0.f;
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const int tt = t + i4;
+        const bf2 dl2 = bpack(ws.dl[c][tt], ws.dl[c][tt]), du2 = bpack(ws.dlu[c][tt], ws.dlu[c][tt]);
+        bf2 acc = bpack(0.f, 0.f);
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-          const float hp = (t + i == 0) ? h0c[s] : H[t + i - 1][s];
-          H[t + i][s] = fmaf(ex2(dl * A2[s]), hp, du * sm.Bs[t + i][j * S + s]);
-          acc = fmaf(sm.Cs[t + i][j * S + s], H[t + i][s], acc);
+        for (int i = 0; i < SP; ++i) {
+          const bf2 hp = tt == 0 ? h0c[i] : H[tt - 1][i];
+          H[tt][i] = bfma(bex2(bmul(dl2, A2[i])), hp, bmul(du2, Bpair(tt, i)));
+          acc = bfma(Cpair(tt, i), H[tt][i], acc);
         }
-        yp[i] = acc;
+        float a0, a1;
+        bunpack(acc, a0, a1);
+        yp[i4] = a0 + a1;
       }
       // sum over the channel's 4 lanes; lane j keeps step t + j
       const bool hi2 = (j & 2) != 0, hi1 = (j & 1) != 0;
@@ -274,7 +320,7 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
 
     // output-side gradients of this lane's 4 steps
     {
-      float zz[4] = {0.f, 0.f, 0.f, 0.f}, oo[4] = {0.f, 0.f, 0.f, 0.f}, dzv[4];
+      float zz[4] = {0.f, 0.f, 0.f, 0.f}, oo[4] = {0.f, 0.f, 0.f, 0.f}, dzv[4], dyv[4];
       if (valid) {
         vo.unpack(oo);
         if (z_row) vz.unpack(zz);
@@ -289,60 +335,82 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
           dy = oo[i] * zz[i] * sz;
         }
         dy = (valid && t0 + 4 * q + i < L) ? dy : 0.f;
-        ws.dy[c][4 * q + i] = dy;
+        dyv[i] = dy;
         dD_acc = fmaf(dy, uu[i], dD_acc);
       }
+      *reinterpret_cast<float4 *>(&ws.dy[c][4 * q]) = make_float4(dyv[0], dyv[1], dyv[2], dyv[3]);
       if (z_row && valid) Vec4<T>::store(dz_row, t0 + 4 * q, L, io_vec, dzv);
     }
     __syncwarp();
 
-    // reverse recurrence over the chunk
+    // reverse recurrence over the chunk, in two halves; after each half the
+    // CTA sums its 32 channels' dB/dC contributions and adds them to the
+    // fp32 accumulators
 #pragma unroll
-    for (int t = kTB - 1; t >= 0; --t) {
-      const float dy = ws.dy[c][t], dl = ws.dl[c][t], du = ws.dlu[c][t];
-      float ddl = 0.f, s1 = 0.f;
-      float v[2 * S];
+    for (int half = 1; half >= 0; --half) {
 #pragma unroll
-      for (int s = 0; s < S; ++s) {
-        const float Bv = sm.Bs[t][j * S + s], Cv = sm.Cs[t][j * S + s];
-        g[s] = fmaf(dy, Cv, g[s]);
-        const float a = ex2(dl * A2[s]);
-        const float hp = (t == 0) ? h0c[s] : H[t - 1][s];
-        const float qv = g[s] * a * hp;
-        dA_acc[s] = fmaf(dl, qv, dA_acc[s]);
-        ddl = fmaf(An[s], qv, ddl);
-        s1 = fmaf(g[s], Bv, s1);
-        v[s] = g[s] * du;            // dB contribution
-        v[S + s] = dy * H[t][s];     // dC contribution
-        g[s] *= a;
-      }
-      ddl += __shfl_xor_sync(0xffffffffu, ddl, 1);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-      ddl += __shfl_xor_sync(0xffffffffu, ddl, 2);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-      if (j == 0) { ws.ddl[c][t] = ddl; ws.s1[c][t] = s1; }
-      // sum the dB/dC contributions over the warp's 8 channels
-      if constexpr (2 * S >= 8) {
-        halve3<2 * S>(v, lane);
-        const int base = ((c >> 2) & 1) * S + ((c >> 1) & 1) * (S / 2) + (c & 1) * (S / 4);
+      for (int tl = kTB / 2 - 1; tl >= 0; --tl) {
+        const int t = half * (kTB / 2) + tl;
+        const float dyv = ws.dy[c][t], dlv = ws.dl[c][t], duv = ws.dlu[c][t];
+        const bf2 dy2 = bpack(dyv, dyv), dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
+        bf2 ddl2 = bpack(0.f, 0.f), s12 = ddl2;
+        float *pp = &ws.part[tl][c][0][j * S];
 #pragma unroll
-        for (int i = 0; i < 2 * S / 8; ++i) {
-          const int o = base + i;
-          const int which = o >= S ? 1 : 0;
-          ws.dBC[t][which][j * S + (o - which * S)] = v[i];
+        for (int i = 0; i < SP; ++i) {
+          g[i] = bfma(dy2, Cpair(t, i), g[i]);
+          const bf2 a = bex2(bmul(dl2, A2[i]));
+          const bf2 hp = t == 0 ? h0c[i] : H[t - 1][i];
+          const bf2 ga = bmul(g[i], a);
+          const bf2 qv = bmul(ga, hp);
+          dA_acc[i] = bfma(dl2, qv, dA_acc[i]);
+          ddl2 = bfma(An[i], qv, ddl2);
+          s12 = bfma(g[i], Bpair(t, i), s12);
+          const bf2 vB = bmul(g[i], du2), vC = bmul(dy2, H[t][i]);
+          g[i] = ga;
+          if constexpr (S >= 2) {
+            *reinterpret_cast<bf2 *>(pp + 2 * i) = vB;
+            *reinterpret_cast<bf2 *>(pp + NP + 2 * i) = vC;
+          } else {
+            float lo, hi;
+            bunpack(vB, lo, hi);
+            pp[0] = lo;
+            bunpack(vC, lo, hi);
+            pp[NP] = lo;
+          }
         }
-      } else {
+        float d0, d1, s0, s1v;
+        bunpack(ddl2, d0, d1);
+        bunpack(s12, s0, s1v);
+        ws.pd[c][t][j] = make_float2(d0 + d1, s0 + s1v);
+      }
+      __syncthreads();
+      // dB, dC of this half chunk: 4 consecutive (which, n) per output,
+      // summed over the 4 warps x 8 channels, one vector atomic each
+      for (int o = threadIdx.x; o < kRedOutputs; o += kBW * 32) {
+        const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
+        const int t = half * (kTB / 2) + tl;
+        if (t0 + t < L) {
+          bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
+#pragma unroll 8
+          for (int w = 0; w < kBW; ++w) {
 #pragma unroll
-        for (int i = 0; i < 2 * S; ++i) {
-          float x = v[i];
-          x += __shfl_xor_sync(0xffffffffu, x, 4);
-          x += __shfl_xor_sync(0xffffffffu, x, 8);
-          x += __shfl_xor_sync(0xffffffffu, x, 16);
-          if (c == 0) ws.dBC[t][i >= S ? 1 : 0][j * S + (i % S)] = x;
+            for (int cc = 0; cc < kBCPW; ++cc) {
+              const float *src = &sm.w[w].part[tl][cc][0][0] + r4;
+              const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(src);
+              acc0 = badd(acc0, x.x);
+              acc1 = badd(acc1, x.y);
+            }
+          }
+          float4 acc;
+          bunpack(acc0, acc.x, acc.y);
+          bunpack(acc1, acc.z, acc.w);
+          const int which = r4 / NP, n = r4 - which * NP;
+          float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
+          atomicAdd(reinterpret_cast<float4 *>(dst), acc);
         }
       }
+      __syncthreads();
     }
-    __syncthreads();
 
     // input-side gradients of this lane's 4 steps
     {
@@ -350,9 +418,13 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = 4 * q + i;
-        const float s1 = ws.s1[c][t], dl = ws.dl[c][t];
+        const float4 pa = *reinterpret_cast<const float4 *>(&ws.pd[c][t][0]);
+        const float4 pb = *reinterpret_cast<const float4 *>(&ws.pd[c][t][2]);
+        const float ddl = (pa.x + pa.z) + (pb.x + pb.z);
+        const float s1 = (pa.y + pa.w) + (pb.y + pb.w);
+        const float dl = ws.dl[c][t];
         duv[i] = fmaf(dl, s1, ws.dy[c][t] * Dd);
-        float dd = fmaf(uu[i], s1, ws.ddl[c][t]);
+        float dd = fmaf(uu[i], s1, ddl);
         if (p.softplus) dd *= sgs[i];
         dd = (valid && t0 + t < L) ? dd : 0.f;
         ddv[i] = dd;
@@ -363,30 +435,23 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
         Vec4<T>::store(dd_row, t0 + 4 * q, L, io_vec, ddv);
       }
     }
-    // dB, dC of the chunk: sum the 4 warps, add to the fp32 accumulators
-    for (int e = threadIdx.x * 4; e < kTB * 2 * NP; e += kBW * 32 * 4) {
-      const int t = e / (2 * NP), r = e - t * 2 * NP, which = r / NP, n = r - which * NP;
-      if (t0 + t >= L) continue;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < kBW; ++w) {
-        const float4 x = *reinterpret_cast<const float4 *>(&sm.w[w].dBC[t][which][n]);
-        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
-      }
-      float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
-      atomicAdd(reinterpret_cast<float4 *>(dst), acc);
-    }
     __syncthreads();
   }
 
   // ---- per-channel sums ----
   if (valid) {
 #pragma unroll
-    for (int s = 0; s < S; ++s) {
-      const int n = j * S + s;
-      if (n < N) {
-        atomicAdd(&p.dA[d * N + n], dA_acc[s]);
-        if (p.dh0) p.dh0[(b * p.dim + d) * N + n] = g[s];
+    for (int i = 0; i < SP; ++i) {
+      float lo[2], gg[2];
+      bunpack(dA_acc[i], lo[0], lo[1]);
+      bunpack(g[i], gg[0], gg[1]);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int s = 2 * i + h2, n = j * S + s;
+        if (s < S && n < N) {
+          atomicAdd(&p.dA[d * N + n], lo[h2]);
+          if (p.dh0) p.dh0[(b * p.dim + d) * N + n] = gg[h2];
+        }
       }
     }
   }

@@ -209,6 +209,10 @@ int fwd_np_for(int64_t N);
 cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm);
 cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
+int fwd_ws_chunk();
+int fwd_ws_pairs();
+cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm);
+cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,

@@ -103,6 +103,7 @@ template <> struct Vec8<uint16_t> {
     }
   }
   __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void load_shared(const uint16_t *p) { v = *reinterpret_cast<const uint4 *>(p); }
   __device__ __forceinline__ void unpack(float (&o)[8]) const {
     o[0] = bf16_lo(v.x); o[1] = bf16_hi(v.x); o[2] = bf16_lo(v.y); o[3] = bf16_hi(v.y);
     o[4] = bf16_lo(v.z); o[5] = bf16_hi(v.z); o[6] = bf16_lo(v.w); o[7] = bf16_hi(v.w);
@@ -123,6 +124,10 @@ template <> struct Vec8<float> {
     }
   }
   __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void load_shared(const float *p) {
+    a = *reinterpret_cast<const float4 *>(p);
+    b = *reinterpret_cast<const float4 *>(p + 4);
+  }
   __device__ __forceinline__ void unpack(float (&o)[8]) const {
     o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
   }
@@ -146,22 +151,22 @@ struct __align__(16) FwdSmem {
   float Cs[kT][NP];                   // C chunk
 };
 
-// B/C chunk in flight: raw 16-byte vectors of one chunk (vector path).
-template <typename T, int NP>
+// B/C chunk in flight: raw 16-byte vectors of one TCH-step chunk (vector path).
+template <typename T, int NP, int TCH = kT>
 struct BCChunk {
   static constexpr int EPV = 16 / (int)sizeof(T);
   static constexpr bool kVecOK = (NP % EPV) == 0;
-  static constexpr int NV = kVecOK ? kT * NP / EPV : 0;    // vectors per chunk and tensor
+  static constexpr int NV = kVecOK ? TCH * NP / EPV : 0;   // vectors per chunk and tensor
   static constexpr int PER_LANE = (NV + 31) / 32;
   static constexpr bool kPrefetch = kVecOK && PER_LANE <= 4;
   uint4 b[kPrefetch ? PER_LANE : 1], c[kPrefetch ? PER_LANE : 1];
 };
 
 // Issue the global loads of one B/C chunk (vector path).
-template <typename T, int NP, bool EMIT>
-__device__ __forceinline__ void bc_load(BCChunk<T, NP> &r, const T *Bb, const T *Cb, int64_t t0,
-                                        int64_t L, int lane) {
-  using BC = BCChunk<T, NP>;
+template <typename T, int NP, bool EMIT, int TCH = kT>
+__device__ __forceinline__ void bc_load(BCChunk<T, NP, TCH> &r, const T *Bb, const T *Cb,
+                                        int64_t t0, int64_t L, int lane) {
+  using BC = BCChunk<T, NP, TCH>;
   if constexpr (BC::kPrefetch) {
 #pragma unroll
     for (int i = 0; i < BC::PER_LANE; ++i) {
@@ -180,7 +185,7 @@ __device__ __forceinline__ void bc_load(BCChunk<T, NP> &r, const T *Bb, const T 
 
 template <typename T, int NP>
 __device__ __forceinline__ void bc_store_vec(float (*dst)[NP], const uint4 &x, int v) {
-  using BC = BCChunk<T, NP>;
+  using BC = BCChunk<T, NP, kT>;
   const int e = v * BC::EPV, t = e / NP, n = e - t * NP;
   if constexpr (sizeof(T) == 2) {
     *reinterpret_cast<float4 *>(&dst[t][n]) =
@@ -196,11 +201,11 @@ __device__ __forceinline__ void bc_store_vec(float (*dst)[NP], const uint4 &x, i
 // Stage one B/C chunk into smem: from the prefetched registers, or loading
 // it here (vector path without prefetch, or the scalar path when N != NP or
 // the rows are not 16-byte aligned).
-template <typename T, int NP, bool EMIT>
-__device__ __forceinline__ void bc_stage(float (*Bs)[NP], float (*Cs)[NP], const BCChunk<T, NP> &r,
-                                         const T *Bb, const T *Cb, int64_t t0, int64_t L, int N,
-                                         bool vec, int lane) {
-  using BC = BCChunk<T, NP>;
+template <typename T, int NP, bool EMIT, int TCH = kT>
+__device__ __forceinline__ void bc_stage(float (*Bs)[NP], float (*Cs)[NP],
+                                         const BCChunk<T, NP, TCH> &r, const T *Bb, const T *Cb,
+                                         int64_t t0, int64_t L, int N, bool vec, int lane) {
+  using BC = BCChunk<T, NP, TCH>;
   if constexpr (BC::kVecOK) {
     if (vec) {
       if constexpr (BC::kPrefetch) {
@@ -227,7 +232,7 @@ __device__ __forceinline__ void bc_stage(float (*Bs)[NP], float (*Cs)[NP], const
       return;
     }
   }
-  for (int e = lane; e < kT * NP; e += 32) {
+  for (int e = lane; e < TCH * NP; e += 32) {
     const int t = e / NP, n = e - t * NP;
     const bool in = n < N && t0 + t < L;
     Bs[t][n] = in ? IO<T>::get(Bb, (t0 + t) * N + n) : 0.f;
@@ -583,6 +588,430 @@ __global__ void k_wait_probe(unsigned *flag, unsigned *err, unsigned long long l
   warp_wait_flag(flag, err, limit_ns);
 }
 
+// ---- warp-specialised look-back forward (2 lanes per channel) -------------------
+// A CTA holds kPairs producer warps (0..kPairs-1) and kPairs consumer warps
+// (kPairs..2*kPairs-1).  Producer i and consumer i form a pair that walks one
+// look-back share (same items as k_fwd_lookback, 16-step chunks).  The
+// consumer runs only the recurrence: per element one MUFU ex2 and two packed
+// fp32 pair operations, so the special-function unit is kept busy.  The
+// producer does everything else for the same chunks: the input copies
+// (cp.async into a ring of raw chunks, three chunks ahead), softplus,
+// Delta*u, the B/C widening, the gate, and the output epilogue of the chunk
+// before.  Two shared-memory stages alternate; named barriers carry "stage
+// full" (producer -> consumer) and "sums ready" (consumer -> producer) per
+// pair and stage.
+constexpr int kTW = 16;
+constexpr int kPairs = 4;
+constexpr int kWSThreads = 2 * kPairs * 32;
+
+template <int NP>
+struct __align__(16) WSStage {
+  float dl[16][kTW + 4];
+  float dlu[16][kTW + 4];
+  float ys[16][kTW + 4];
+  float Bs[kTW][NP];
+  float Cs[kTW][NP];
+};
+constexpr int kSlots = 4;  // raw-input ring: chunks k+1..k+3 in flight while k is processed
+
+template <typename T, int NP>
+struct __align__(16) WSRaw {
+  T u[16][kTW], d[16][kTW], z[16][kTW];  // [channel][step], io dtype
+  T B[kTW][NP], C[kTW][NP];              // [step][state], io dtype
+};
+
+template <typename T, int NP>
+struct __align__(16) WSPair {
+  WSStage<NP> st[2];
+  WSRaw<T, NP> raw[kSlots];
+};
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bar_sync_n(unsigned id, unsigned n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void bar_arrive_n(unsigned id, unsigned n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// The look-back share of worker w, as a list of runs (group, chunk range).
+struct Share {
+  int64_t K, g_first, k_first, g_last, k_end, n_head, g_lo, n_full, n_runs;
+  bool one;
+  __device__ __forceinline__ Share(int64_t w, int64_t P, int64_t n_groups, int64_t K_) {
+    K = K_;
+    const int64_t W = n_groups * K;
+    const int64_t s0 = w * W / P, e0 = (w + 1) * W / P;
+    g_first = s0 / K; k_first = s0 - g_first * K;
+    g_last = e0 > s0 ? (e0 - 1) / K : g_first;
+    k_end = e0 > s0 ? e0 - g_last * K : k_first;
+    one = g_first == g_last;
+    n_head = (!one && k_end < K) ? 1 : 0;
+    g_lo = k_first > 0 ? g_first + 1 : g_first;
+    const int64_t g_hi = k_end < K ? g_last : g_last + 1;
+    n_full = one ? 0 : (g_hi > g_lo ? g_hi - g_lo : 0);
+    const int64_t n_tail = (!one && k_first > 0) ? 1 : 0;
+    n_runs = e0 > s0 ? (one ? 1 : n_head + n_full + n_tail) : 0;
+  }
+  __device__ __forceinline__ void get(int64_t r, int64_t &g, int64_t &k0, int64_t &k1) const {
+    if (one) { g = g_first; k0 = k_first; k1 = k_end; }
+    else if (r < n_head) { g = g_last; k0 = 0; k1 = k_end; }
+    else if (r < n_head + n_full) { g = g_lo + (r - n_head); k0 = 0; k1 = K; }
+    else { g = g_first; k0 = k_first; k1 = K; }
+  }
+};
+
+template <typename T, int NP>
+__device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &sm, int64_t w,
+                                            const Share &sh, unsigned bar_full, unsigned bar_ys) {
+  constexpr int S = NP / 2, CPW = 16;
+  int64_t it = 0;
+  for (int64_t r = 0; r < sh.n_runs; ++r) {
+    int64_t g, k0, k1;
+    sh.get(r, g, k0, k1);
+    const Lane ln = lane_of<2>(p, g);
+    const int c = ln.c, j = ln.j;
+    f2 A2p[S / 2];
+#pragma unroll
+    for (int s = 0; s < S; s += 2) {
+      const int n = j * S + s;
+      const float a0 = (ln.valid && n < p.N) ? p.A[ln.d * p.N + n] * kLog2e : 0.f;
+      const float a1 = (ln.valid && n + 1 < p.N) ? p.A[ln.d * p.N + n + 1] * kLog2e : 0.f;
+      A2p[s / 2] = pack2(a0, a1);
+    }
+    float h[S];
+    if (k0 > 0) {
+      warp_wait_flag(&p.flags[w - 1], p.err, p.wait_limit_ns);
+#pragma unroll
+      for (int s = 0; s < S; ++s) h[s] = __ldcg(&p.carry[((w - 1) * CPW + c) * NP + j * S + s]);
+    } else {
+      init_state<NP, 2>(p, ln, h);
+    }
+    f2 hp[S / 2];
+#pragma unroll
+    for (int s = 0; s < S; s += 2) hp[s / 2] = pack2(h[s], h[s + 1]);
+    for (int64_t k = k0; k < k1; ++k, ++it) {
+      const int stage = (int)(it & 1);
+      WSStage<NP> &st = sm.st[stage];
+      bar_sync_n(bar_full + stage, 64);
+#pragma unroll
+      for (int tt = 0; tt < kTW; tt += 4) {
+        const float4 d4 = *reinterpret_cast<const float4 *>(&st.dl[c][tt]);
+        const float4 u4 = *reinterpret_cast<const float4 *>(&st.dlu[c][tt]);
+        const float dls[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float dus[4] = {u4.x, u4.y, u4.z, u4.w};
+        float yp[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float *Brow = &st.Bs[tt + i][j * S];
+          const float *Crow = &st.Cs[tt + i][j * S];
+          const f2 dl2 = pack2(dls[i], dls[i]), du2 = pack2(dus[i], dus[i]);
+          f2 acc[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};  // two chains
+#pragma unroll
+          for (int s = 0; s < S; s += 2) {
+            f2 bv, cv;
+            if constexpr (S % 4 == 0) {  // two pairs per 16-byte shared load
+              const ulonglong2 b4 = *reinterpret_cast<const ulonglong2 *>(Brow + (s & ~3));
+              const ulonglong2 c4 = *reinterpret_cast<const ulonglong2 *>(Crow + (s & ~3));
+              bv = (s & 2) ? b4.y : b4.x;
+              cv = (s & 2) ? c4.y : c4.x;
+            } else {
+              bv = *reinterpret_cast<const f2 *>(Brow + s);
+              cv = *reinterpret_cast<const f2 *>(Crow + s);
+            }
+            float x0, x1;
+            unpack2(mul2(dl2, A2p[s / 2]), x0, x1);
+            const f2 a = pack2(ex2(x0), ex2(x1));
+            hp[s / 2] = fma2(a, hp[s / 2], mul2(du2, bv));
+            acc[(s / 2) & 1] = fma2(cv, hp[s / 2], acc[(s / 2) & 1]);
+          }
+          float a0, a1, a2, a3;
+          unpack2(acc[0], a0, a1);
+          unpack2(acc[1], a2, a3);
+          yp[i] = (a0 + a1) + (a2 + a3);
+        }
+        // lane j keeps steps tt+2j, tt+2j+1 summed over the channel's 2 lanes
+        const float k0 = j ? yp[2] : yp[0], k1 = j ? yp[3] : yp[1];
+        const float s0 = j ? yp[0] : yp[2], s1 = j ? yp[1] : yp[3];
+        const float r0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);
+        const float r1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
+        *reinterpret_cast<float2 *>(&st.ys[c][tt + 2 * j]) = make_float2(r0, r1);
+      }
+      bar_arrive_n(bar_ys + stage, 64);
+    }
+#pragma unroll
+    for (int s = 0; s < S; s += 2) unpack2(hp[s / 2], h[s], h[s + 1]);
+    if (k1 < sh.K) {  // publish the head's end state for worker w + 1
+#pragma unroll
+      for (int s = 0; s < S; ++s) p.carry[(w * CPW + c) * NP + j * S + s] = h[s];
+      __threadfence();
+      __syncwarp();
+      if (ln.lane == 0) st_release(&p.flags[w], 1u);
+    } else {
+      write_last_state<NP, 2>(p, ln, h);
+    }
+  }
+}
+
+// Row pointers and per-channel constants of one run, computed once per run.
+template <typename T>
+struct RunRows {
+  const T *u, *dr, *z, *Bb, *Cb;
+  T *y;
+  float bias, Dd;
+  bool valid;
+  int c, j;
+  // Producer lanes take channel c = lane % 16 and steps [8j, 8j+8) with
+  // j = lane / 16, so that a quarter warp's 16-byte row accesses fall in
+  // distinct shared-memory banks.
+  __device__ __forceinline__ void set(const FwdParams &p, int64_t g) {
+    Lane ln;
+    ln.lane = threadIdx.x & 31;
+    ln.c = ln.lane & 15;
+    ln.j = ln.lane >> 4;
+    ln.b = g / p.gpb;
+    ln.d = (g - ln.b * p.gpb) * 16 + ln.c;
+    ln.valid = ln.d < p.dim;
+    const int64_t row = (ln.b * p.dim + (ln.valid ? ln.d : 0)) * p.L;
+    u = static_cast<const T *>(p.u) + row;
+    dr = static_cast<const T *>(p.delta) + row;
+    z = p.z ? static_cast<const T *>(p.z) + row : nullptr;
+    y = static_cast<T *>(p.y) + row;
+    Bb = static_cast<const T *>(p.B) + ln.b * p.L * p.N;
+    Cb = static_cast<const T *>(p.C) + ln.b * p.L * p.N;
+    bias = (p.bias && ln.valid) ? p.bias[ln.d] : 0.f;
+    Dd = (p.D && ln.valid) ? p.D[ln.d] : 0.f;
+    valid = ln.valid;
+    c = ln.c;
+    j = ln.j;
+  }
+};
+
+// Copy this lane's pieces of chunk k of run `rr` into raw slot `slot`:
+// u/delta/z steps [8j, 8j+8) of channel c, and B/C 16-byte pieces lane,
+// lane+32, ...  Asynchronous (cp.async, zero-filled past L) on 16-byte
+// aligned rows; plain loads otherwise.  Every lane later reads only the
+// pieces it copied itself.
+template <typename T, int NP>
+__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, const RunRows<T> &rr,
+                                         int64_t k, int lane) {
+  constexpr int ES = (int)sizeof(T), EPP = 16 / ES;   // elements per 16-byte piece
+  const int64_t L = p.L, t0 = k * kTW;
+  const int64_t ts = t0 + rr.j * 8;
+  if (p.io_vec) {
+#pragma unroll
+    for (int q = 0; q < 8 / EPP; ++q) {
+      const int64_t t = ts + q * EPP;
+      const int64_t left = rr.valid ? L - t : 0;
+      const int bytes = left >= EPP ? 16 : (left > 0 ? (int)left * ES : 0);
+      const int64_t off = bytes > 0 ? t : 0;
+      cp_async16(&raw.u[rr.c][rr.j * 8 + q * EPP], rr.u + off, bytes);
+      cp_async16(&raw.d[rr.c][rr.j * 8 + q * EPP], rr.dr + off, bytes);
+      if (rr.z) cp_async16(&raw.z[rr.c][rr.j * 8 + q * EPP], rr.z + off, bytes);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool in = rr.valid && ts + i < L;
+      raw.u[rr.c][rr.j * 8 + i] = in ? rr.u[ts + i] : T(0);
+      raw.d[rr.c][rr.j * 8 + i] = in ? rr.dr[ts + i] : T(0);
+      if (rr.z) raw.z[rr.c][rr.j * 8 + i] = in ? rr.z[ts + i] : T(0);
+    }
+  }
+  if (p.bc_vec && NP % EPP == 0) {
+    constexpr int NV = kTW * NP / EPP;
+    for (int v = lane; v < NV; v += 32) {
+      const int e = v * EPP, t = e / NP, n = e - t * NP;
+      const bool in = t0 + t < L;
+      const int64_t off = in ? (t0 + t) * NP + n : 0;
+      cp_async16(&raw.B[t][n], rr.Bb + off, in ? 16 : 0);
+      cp_async16(&raw.C[t][n], rr.Cb + off, in ? 16 : 0);
+    }
+  } else {
+    for (int e = lane; e < kTW * NP; e += 32) {
+      const int t = e / NP, n = e - t * NP;
+      const bool in = n < p.N && t0 + t < L;
+      raw.B[t][n] = in ? rr.Bb[(t0 + t) * p.N + n] : T(0);
+      raw.C[t][n] = in ? rr.Cb[(t0 + t) * p.N + n] : T(0);
+    }
+  }
+}
+
+__device__ __forceinline__ float io_to_f(uint16_t v) { return bf16_to_f(v); }
+__device__ __forceinline__ float io_to_f(float v) { return v; }
+
+template <typename T, int NP>
+__device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &sm, const Share &sh,
+                                            unsigned bar_full, unsigned bar_ys) {
+  constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
+  const int64_t L = p.L;
+  const int lane = threadIdx.x & 31;
+  const bool io_vec = p.io_vec != 0;
+  // the chunk whose output epilogue is pending
+  bool pend = false;
+  int pstage = 0;
+  T *py_row = nullptr;
+  int64_t pts = 0;
+  bool pvalid = false;
+  float gate[8], dg[8];
+
+  auto epilogue = [&]() {
+    bar_sync_n(bar_ys + pstage, 64);
+    if (pvalid) {
+      const float *py = &sm.st[pstage].ys[lane & 15][(lane >> 4) * 8];
+      const float4 a = *reinterpret_cast<const float4 *>(py);
+      const float4 b4 = *reinterpret_cast<const float4 *>(py + 4);
+      const float ys[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = fmaf(ys[i], gate[i], dg[i]);
+      IO<T>::store8(py_row, pts, L, io_vec, o);
+    }
+  };
+
+  // prefetch cursor: the item kSlots-1 chunks ahead of the one processed
+  int64_t pr = 0, pk = 0, pk1 = 0, pg = 0;
+  RunRows<T> pf;
+  bool pf_live = sh.n_runs > 0;
+  if (pf_live) {
+    sh.get(0, pg, pk, pk1);
+    pf.set(p, pg);
+  }
+  auto advance = [&]() {
+    if (!pf_live) return;
+    if (++pk >= pk1) {
+      if (++pr < sh.n_runs) {
+        sh.get(pr, pg, pk, pk1);
+        pf.set(p, pg);
+      } else {
+        pf_live = false;
+      }
+    }
+  };
+  int64_t it_f = 0;  // chunks fetched
+  for (int i = 0; i < kSlots - 1; ++i) {
+    if (pf_live && pk < pk1) ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+    cp_async_commit();
+    ++it_f;
+    advance();
+  }
+
+  int64_t it = 0;
+  for (int64_t r = 0; r < sh.n_runs; ++r) {
+    int64_t g, k0, k1;
+    sh.get(r, g, k0, k1);
+    RunRows<T> cur;
+    cur.set(p, g);
+    for (int64_t k = k0; k < k1; ++k, ++it) {
+      const int stage = (int)(it & 1);
+      WSStage<NP> &st = sm.st[stage];
+      WSRaw<T, NP> &raw = sm.raw[it % kSlots];
+      const int64_t ts = k * kTW + cur.j * 8;
+      cp_async_wait<kSlots - 2>();  // this chunk's copies have landed
+      // ---- pre-pass of chunk k into stage ----
+      float u8[8], d8[8], z8[8];
+      {
+        Vec8<T> vu, vd, vz;
+        vu.load_shared(&raw.u[cur.c][cur.j * 8]);
+        vd.load_shared(&raw.d[cur.c][cur.j * 8]);
+        vu.unpack(u8);
+        vd.unpack(d8);
+        if (cur.z) {
+          vz.load_shared(&raw.z[cur.c][cur.j * 8]);
+          vz.unpack(z8);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) z8[i] = 0.f;
+        }
+      }
+      float dl8[8], du8[8], ng[8], ndg[8];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const float s0 = d8[i] + cur.bias, s1 = d8[i + 1] + cur.bias;
+        float dl0 = s0, dl1 = s1;
+        if (p.softplus) {
+          dl0 = softplus_fast(s0);
+          dl1 = softplus_fast(s1);
+        }
+        dl0 = (cur.valid && ts + i < L) ? dl0 : 0.f;
+        dl1 = (cur.valid && ts + i + 1 < L) ? dl1 : 0.f;
+        dl8[i] = dl0; dl8[i + 1] = dl1;
+        du8[i] = dl0 * u8[i]; du8[i + 1] = dl1 * u8[i + 1];
+        float g0 = 1.f, g1 = 1.f;
+        if (cur.z) {
+          g0 = silu_fast(z8[i]);
+          g1 = silu_fast(z8[i + 1]);
+        }
+        ng[i] = g0; ng[i + 1] = g1;
+        ndg[i] = cur.Dd * u8[i] * g0; ndg[i + 1] = cur.Dd * u8[i + 1] * g1;
+      }
+      float *pd = &st.dl[cur.c][cur.j * 8];
+      float *pu = &st.dlu[cur.c][cur.j * 8];
+      *reinterpret_cast<float4 *>(pd) = make_float4(dl8[0], dl8[1], dl8[2], dl8[3]);
+      *reinterpret_cast<float4 *>(pd + 4) = make_float4(dl8[4], dl8[5], dl8[6], dl8[7]);
+      *reinterpret_cast<float4 *>(pu) = make_float4(du8[0], du8[1], du8[2], du8[3]);
+      *reinterpret_cast<float4 *>(pu + 4) = make_float4(du8[4], du8[5], du8[6], du8[7]);
+      // widen this lane's B/C pieces (the ones it fetched) to fp32
+      if (p.bc_vec && NP % EPP == 0) {
+        constexpr int NV = kTW * NP / EPP;
+        for (int v = lane; v < NV; v += 32) {
+          const int e = v * EPP, t = e / NP, n = e - t * NP;
+          bc_store_vec<T, NP>(st.Bs, *reinterpret_cast<const uint4 *>(&raw.B[t][n]), v);
+          bc_store_vec<T, NP>(st.Cs, *reinterpret_cast<const uint4 *>(&raw.C[t][n]), v);
+        }
+      } else {
+        for (int e = lane; e < kTW * NP; e += 32) {
+          const int t = e / NP, n = e - t * NP;
+          st.Bs[t][n] = io_to_f(raw.B[t][n]);
+          st.Cs[t][n] = io_to_f(raw.C[t][n]);
+        }
+      }
+      bar_arrive_n(bar_full + stage, 64);
+      // ---- copies of the chunk kSlots-1 ahead, into the slot just freed ----
+      if (pf_live && pk < pk1) ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+      cp_async_commit();
+      ++it_f;
+      advance();
+      // ---- epilogue of the previous chunk ----
+      if (pend) epilogue();
+      pend = true;
+      pstage = stage;
+      py_row = cur.y;
+      pts = ts;
+      pvalid = cur.valid;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { gate[i] = ng[i]; dg[i] = ndg[i]; }
+    }
+  }
+  if (pend) epilogue();
+  cp_async_wait<0>();
+}
+
+template <typename T, int NP>
+__global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5;
+  const bool producer = warp < kPairs;
+  const int pair = producer ? warp : warp - kPairs;
+  WSPair<T, NP> &sm = reinterpret_cast<WSPair<T, NP> *>(smem_raw)[pair];
+  const int64_t w = (int64_t)blockIdx.x * kPairs + pair;
+  if (w >= p.n_workers) return;  // both warps of a pair leave together
+  const Share sh(w, p.n_workers, p.n_groups, p.n_chunks);
+  const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
+  if (producer) ws_producer<T, NP>(p, sm, sh, bar_full, bar_ys);
+  else ws_consumer<T, NP>(p, sm, w, sh, bar_full, bar_ys);
+}
+
 // ---- host side ------------------------------------------------------------------
 template <class V> struct TypeTag { using type = V; };
 template <int V> struct IntTag { static constexpr int value = V; };
@@ -662,6 +1091,34 @@ cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p,
     e = allow_smem(k_fwd_segment<T, kNP, kLPC, true>, smem);
     if (e != cudaSuccess) return e;
     k_fwd_segment<T, kNP, kLPC, true><<<grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+  });
+}
+
+int fwd_ws_chunk() { return kTW; }
+int fwd_ws_pairs() { return kPairs; }
+
+cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm) {
+  return dispatch(io_dtype, NP, 2, [&](auto tt, auto np, auto) -> cudaError_t {
+    using T = typename decltype(tt)::type;
+    constexpr int kNP = decltype(np)::value;
+    const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
+    cudaError_t e = allow_smem(k_fwd_ws<T, kNP>, smem);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP>, kWSThreads,
+                                                         smem);
+  });
+}
+
+cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s) {
+  return dispatch(io_dtype, NP, 2, [&](auto tt, auto np, auto) -> cudaError_t {
+    using T = typename decltype(tt)::type;
+    constexpr int kNP = decltype(np)::value;
+    const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
+    cudaError_t e = allow_smem(k_fwd_ws<T, kNP>, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((p.n_workers + kPairs - 1) / kPairs);
+    k_fwd_ws<T, kNP><<<grid, kWSThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }

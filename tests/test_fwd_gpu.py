@@ -14,7 +14,10 @@ from gpu_util import assert_close, to_f64, upload
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3}
+PATHS = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3, "lookback_ws": 4}
+# every schedule with every lane split it supports
+PATH_LANES = [("lookback", 2), ("lookback", 4), ("split_l", 2), ("split_l", 4),
+              ("per_group", 2), ("per_group", 4), ("lookback_ws", 2)]
 
 
 def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None, lanes=0):
@@ -38,7 +41,7 @@ def _check(case, device, path="auto", softplus=True, h0=None, lanes=0):
     return st
 
 
-@pytest.mark.parametrize("path", ["auto", "lookback", "split_l", "per_group"])
+@pytest.mark.parametrize("path", ["auto", "lookback", "split_l", "per_group", "lookback_ws"])
 def test_tiny_fp32_workload(cuda_device, path):
     case = synth.make_workload("tiny-fp32")
     _check(case, cuda_device, path)
@@ -52,24 +55,23 @@ def test_dstate_sizes(cuda_device, dtype, N, lanes):
     _check(case, cuda_device, "per_group", lanes=lanes)
 
 
-@pytest.mark.parametrize("lanes", [2, 4])
-@pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
-@pytest.mark.parametrize("L", [1, 7, 31, 32, 33, 257, 1000, 1003])
+@pytest.mark.parametrize("path,lanes", PATH_LANES)
+@pytest.mark.parametrize("L", [1, 7, 15, 16, 17, 31, 32, 33, 257, 1000, 1003])
 def test_ragged_lengths_and_groups(cuda_device, path, L, lanes):
     # dim 44: ragged 16- and 8-channel groups; L odd -> scalar loads
     case = synth.make_case(3, 44, L, 16, synth.BF16, seed=L)
     _check(case, cuda_device, path, lanes=lanes)
 
 
-@pytest.mark.parametrize("lanes", [2, 4])
-@pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
+@pytest.mark.parametrize("path,lanes", PATH_LANES)
 def test_fp32_several_chunks(cuda_device, path, lanes):
     case = synth.make_case(2, 24, 777, 16, synth.F32, seed=7)
     _check(case, cuda_device, path, lanes=lanes)
 
 
+@pytest.mark.parametrize("path", ["auto", "lookback_ws"])
 @pytest.mark.parametrize("opt", ["no_z", "no_D", "no_bias", "no_softplus", "bare"])
-def test_optional_terms(cuda_device, opt):
+def test_optional_terms(cuda_device, opt, path):
     kw = dict(with_z=opt not in ("no_z", "bare"), with_D=opt not in ("no_D", "bare"),
               with_bias=opt not in ("no_bias", "bare"))
     case = synth.make_case(2, 16, 300, 16, synth.F32, seed=3, **kw)
@@ -78,11 +80,10 @@ def test_optional_terms(cuda_device, opt):
         # raw delta must stay positive without softplus (|Abar| <= 1)
         case["delta"] = np.abs(case["delta"]) * 0.05 + 1e-3
         case["delta_bias"] = None
-    _check(case, cuda_device, "auto", softplus=softplus)
+    _check(case, cuda_device, path, softplus=softplus)
 
 
-@pytest.mark.parametrize("lanes", [2, 4])
-@pytest.mark.parametrize("path", ["lookback", "split_l", "per_group"])
+@pytest.mark.parametrize("path,lanes", PATH_LANES)
 def test_initial_state(cuda_device, path, lanes):
     case = synth.make_case(2, 16, 500, 16, synth.F32, seed=9)
     h0 = np.random.default_rng(1).standard_normal((2, 16, 16)).astype(np.float32)
@@ -135,8 +136,7 @@ def test_large_delta_reset_bitwise(cuda_device):
 def test_paths_agree(cuda_device):
     case = synth.make_case(4, 64, 2048, 16, synth.BF16, seed=31)
     ref = oracle.fwd(case)["y"]
-    outs = {(p, ln): _run(case, cuda_device, p, lanes=ln)[0]
-            for p in ("lookback", "split_l", "per_group") for ln in (2, 4)}
+    outs = {(p, ln): _run(case, cuda_device, p, lanes=ln)[0] for p, ln in PATH_LANES}
     for k, y in outs.items():
         assert_close(y, ref, case["dtype"], str(k))
         d = np.max(np.abs(y - outs[("lookback", 2)]))
@@ -165,11 +165,24 @@ def test_softplus_accuracy_through_the_kernel(cuda_device):
         assert np.all(rel <= bound), (lanes, float(rel.max()), float(s[np.argmax(rel / bound)]))
 
 
-def test_deterministic(cuda_device):
+@pytest.mark.parametrize("path", ["lookback", "lookback_ws"])
+def test_deterministic(cuda_device, path):
     case = synth.make_case(2, 64, 1024, 16, synth.BF16, seed=41)
-    a = _run(case, cuda_device, "lookback")
-    b = _run(case, cuda_device, "lookback")
+    a = _run(case, cuda_device, path)
+    b = _run(case, cuda_device, path)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_lookback_splits_groups_between_warps(cuda_device):
+    # enough channel groups for several warps per SM sub-partition, with a
+    # length whose chunk count does not divide evenly: warp shares start and
+    # end inside groups, so the carried states are exercised on both paths
+    case = synth.make_case(8, 1536, 1000, 16, synth.BF16, seed=61)
+    ref = oracle.fwd(case)
+    for path in ("lookback", "lookback_ws"):
+        y, ls = _run(case, cuda_device, path)
+        assert_close(y, ref["y"], case["dtype"], path)
+        assert_close(ls, ref["last_state"], case["dtype"], path, stored_bf16=False)
 
 
 def test_guard_bands_untouched(cuda_device):
