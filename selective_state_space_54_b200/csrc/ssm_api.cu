@@ -311,6 +311,7 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
   p.io_vec = ((L * (int64_t)es) % 16 == 0) && aligned(u, 16) && aligned(delta, 16) &&
              aligned(z, 16) && aligned(dout, 16) && aligned(du, 16) && aligned(ddelta, 16) &&
              aligned(dz, 16);
+  p.bc_vec = (N == NP) && ((N * (int64_t)es) % 16 == 0) && aligned(B, 16) && aligned(C, 16);
   cudaError_t e = cudaMemsetAsync(dA, 0, sizeof(float) * dim * N, s);
   if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, sizeof(float) * dim, s);
   if (e == cudaSuccess && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * dim, s);

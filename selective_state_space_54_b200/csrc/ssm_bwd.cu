@@ -92,7 +92,10 @@ struct __align__(16) BwdWarpSmem {
   float dy[kBCPW][kTB + kBPad];    // dout * SiLU(z)
   float ys[kBCPW][kTB + kBPad];    // sum_n C h
   float2 pd[kBCPW][kTB][4];        // per lane j: (sum_n g A a h_prev, sum_n g B) partials
-  float part[kTB / 2][kBCPW][2][NP];  // dB, dC contributions of half a chunk, per channel
+  // dB, dC contributions of half a chunk: [step][B|C][lane slice j][channel, state]
+  // with 8 floats of padding per row so that a quarter warp's stores hit
+  // distinct banks
+  float part[kTB / 2][2][4][kBCPW * (NP / 4) + 8];
 };
 
 template <int NP>
@@ -113,6 +116,46 @@ __device__ __forceinline__ void bwd_stage_bc(BwdSmem<NP> &sm, const T *Bb, const
     if (with_c) sm.Cs[t][n] = in ? IO<T>::get(Cb, (t0 + t) * N + n) : 0.f;
   }
 }
+
+// One chunk of B and C in flight as raw 16-byte pieces, spread over the CTA
+// (vector path: N == NP, 16-byte aligned rows).
+template <typename T, int NP>
+struct BwdBC {
+  static constexpr int EPP = 16 / (int)sizeof(T);
+  static constexpr bool kVec = (NP % EPP) == 0;
+  static constexpr int NV = kVec ? kTB * NP / EPP : 1;              // pieces per tensor
+  static constexpr int PER = (2 * NV + kBW * 32 - 1) / (kBW * 32);  // pieces per thread
+  uint4 r[PER];
+  __device__ __forceinline__ void load(const T *Bb, const T *Cb, int64_t t0, int64_t L, bool with_c) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int v = threadIdx.x + i * kBW * 32;
+      const int which = v / NV, vv = v - which * NV;
+      const int e = vv * EPP, t = e / NP, n = e - t * NP;
+      if (v < 2 * NV && t0 + t < L && (which == 0 || with_c))
+        r[i] = __ldg(reinterpret_cast<const uint4 *>((which ? Cb : Bb) + (t0 + t) * NP + n));
+      else
+        r[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  __device__ __forceinline__ void stage(float (*Bs)[NP], float (*Cs)[NP]) const {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int v = threadIdx.x + i * kBW * 32;
+      if (v >= 2 * NV) continue;
+      const int which = v / NV, vv = v - which * NV;
+      const int e = vv * EPP, t = e / NP, n = e - t * NP;
+      float *dst = which ? &Cs[t][n] : &Bs[t][n];
+      if constexpr (sizeof(T) == 2) {
+        *reinterpret_cast<float4 *>(dst) = make_float4(bf16_lo(r[i].x), bf16_hi(r[i].x), bf16_lo(r[i].y), bf16_hi(r[i].y));
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(bf16_lo(r[i].z), bf16_hi(r[i].z), bf16_lo(r[i].w), bf16_hi(r[i].w));
+      } else {
+        *reinterpret_cast<float4 *>(dst) = make_float4(__uint_as_float(r[i].x), __uint_as_float(r[i].y),
+                                                       __uint_as_float(r[i].z), __uint_as_float(r[i].w));
+      }
+    }
+  }
+};
 
 // packed fp32 pairs (sm_100a f32x2 arithmetic)
 typedef unsigned long long bf2;
@@ -199,14 +242,10 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
   };
 
   // per (channel, step) quantities for this lane's 4 steps of chunk k
-  auto prepass = [&](int64_t t0, float (&uu)[4], float (&sgs)[4]) {
-    Vec4<T> vu, vd;
-    if (valid) {
-      vu.load(u_row, t0 + 4 * q, L, io_vec);
-      vd.load(dr_row, t0 + 4 * q, L, io_vec);
-    } else {
-      vu.v = {}; vd.v = {};
-    }
+  // per (channel, step) quantities for this lane's 4 steps of a chunk, from
+  // the chunk's preloaded u and delta
+  auto prepass = [&](int64_t t0, const Vec4<T> &vu, const Vec4<T> &vd, float (&uu)[4],
+                     float (&sgs)[4]) {
     float dr[4];
     vu.unpack(uu);
     vd.unpack(dr);
@@ -229,6 +268,31 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     *reinterpret_cast<float4 *>(&ws.dlu[c][4 * q]) = make_float4(du4[0], du4[1], du4[2], du4[3]);
   };
 
+  // inputs of one chunk, loaded a chunk ahead of their use
+  struct ChunkIn {
+    Vec4<T> u, d, o, z;
+    BwdBC<T, NP> bc;
+  };
+  const bool bc_vec = p.bc_vec != 0 && BwdBC<T, NP>::kVec;
+  auto load_chunk = [&](int64_t k, bool full, ChunkIn &in) {
+    const int64_t t0 = k * kTB;
+    if (valid) {
+      in.u.load(u_row, t0 + 4 * q, L, io_vec);
+      in.d.load(dr_row, t0 + 4 * q, L, io_vec);
+      if (full) {
+        in.o.load(do_row, t0 + 4 * q, L, io_vec);
+        if (z_row) in.z.load(z_row, t0 + 4 * q, L, io_vec);
+      }
+    } else {
+      in.u.v = {}; in.d.v = {}; in.o.v = {}; in.z.v = {};
+    }
+    if (bc_vec) in.bc.load(Bb, Cb, t0, L, full);
+  };
+  auto stage_chunk = [&](int64_t t0, const ChunkIn &in, bool full) {
+    if (bc_vec) in.bc.stage(sm.Bs, sm.Cs);
+    else bwd_stage_bc<T, NP>(sm, Bb, Cb, t0, L, N, full);
+  };
+
   // ---- phase A: states entering every chunk ----
   bf2 h[SP];
 #pragma unroll
@@ -241,6 +305,8 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     }
     h[i] = bpack(v[0], v[1]);
   }
+  ChunkIn nxt;
+  if (K > 0) load_chunk(0, false, nxt);
   for (int64_t k = 0; k < K; ++k) {
     const int64_t t0 = k * kTB;
 #pragma unroll
@@ -251,9 +317,11 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
       dst[0] = lo;
       if (S >= 2) dst[1] = hi;
     }
+    const ChunkIn cur = nxt;
+    if (k + 1 < K) load_chunk(k + 1, false, nxt);
     float uu[4], sgs[4];
-    prepass(t0, uu, sgs);
-    bwd_stage_bc<T, NP>(sm, Bb, Cb, t0, L, N, false);
+    prepass(t0, cur.u, cur.d, uu, sgs);
+    stage_chunk(t0, cur, false);
     __syncthreads();
 #pragma unroll 4
     for (int t = 0; t < kTB; ++t) {
@@ -270,16 +338,14 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
   for (int i = 0; i < SP; ++i) { g[i] = bpack(0.f, 0.f); dA_acc[i] = g[i]; }
   float dD_acc = 0.f, dbias_acc = 0.f;
   constexpr int kRedOutputs = (kTB / 2) * 2 * NP / 4;   // float4 outputs of a half chunk
+  if (K > 0) load_chunk(K - 1, true, nxt);
   for (int64_t k = K - 1; k >= 0; --k) {
     const int64_t t0 = k * kTB;
+    const ChunkIn cur = nxt;
+    if (k > 0) load_chunk(k - 1, true, nxt);
     float uu[4], sgs[4];
-    prepass(t0, uu, sgs);
-    Vec4<T> vz, vo;
-    if (valid) {
-      vo.load(do_row, t0 + 4 * q, L, io_vec);
-      if (z_row) vz.load(z_row, t0 + 4 * q, L, io_vec);
-    }
-    bwd_stage_bc<T, NP>(sm, Bb, Cb, t0, L, N, true);
+    prepass(t0, cur.u, cur.d, uu, sgs);
+    stage_chunk(t0, cur, true);
     __syncthreads();
 
     // recompute the chunk's states from its checkpoint
@@ -322,8 +388,8 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     {
       float zz[4] = {0.f, 0.f, 0.f, 0.f}, oo[4] = {0.f, 0.f, 0.f, 0.f}, dzv[4], dyv[4];
       if (valid) {
-        vo.unpack(oo);
-        if (z_row) vz.unpack(zz);
+        cur.o.unpack(oo);
+        if (z_row) cur.z.unpack(zz);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -354,7 +420,8 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
         const float dyv = ws.dy[c][t], dlv = ws.dl[c][t], duv = ws.dlu[c][t];
         const bf2 dy2 = bpack(dyv, dyv), dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
         bf2 ddl2 = bpack(0.f, 0.f), s12 = ddl2;
-        float *pp = &ws.part[tl][c][0][j * S];
+        float *pB = &ws.part[tl][0][j][c * S];
+        float *pC = &ws.part[tl][1][j][c * S];
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
           g[i] = bfma(dy2, Cpair(t, i), g[i]);
@@ -368,14 +435,14 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
           const bf2 vB = bmul(g[i], du2), vC = bmul(dy2, H[t][i]);
           g[i] = ga;
           if constexpr (S >= 2) {
-            *reinterpret_cast<bf2 *>(pp + 2 * i) = vB;
-            *reinterpret_cast<bf2 *>(pp + NP + 2 * i) = vC;
+            *reinterpret_cast<bf2 *>(pB + 2 * i) = vB;
+            *reinterpret_cast<bf2 *>(pC + 2 * i) = vC;
           } else {
             float lo, hi;
             bunpack(vB, lo, hi);
-            pp[0] = lo;
+            pB[0] = lo;
             bunpack(vC, lo, hi);
-            pp[NP] = lo;
+            pC[0] = lo;
           }
         }
         float d0, d1, s0, s1v;
@@ -384,29 +451,47 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
         ws.pd[c][t][j] = make_float2(d0 + d1, s0 + s1v);
       }
       __syncthreads();
-      // dB, dC of this half chunk: 4 consecutive (which, n) per output,
-      // summed over the 4 warps x 8 channels, one vector atomic each
-      for (int o = threadIdx.x; o < kRedOutputs; o += kBW * 32) {
-        const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
-        const int t = half * (kTB / 2) + tl;
-        if (t0 + t < L) {
-          bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
-#pragma unroll 8
-          for (int w = 0; w < kBW; ++w) {
-#pragma unroll
-            for (int cc = 0; cc < kBCPW; ++cc) {
-              const float *src = &sm.w[w].part[tl][cc][0][0] + r4;
-              const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(src);
-              acc0 = badd(acc0, x.x);
-              acc1 = badd(acc1, x.y);
-            }
-          }
-          float4 acc;
-          bunpack(acc0, acc.x, acc.y);
-          bunpack(acc1, acc.z, acc.w);
+      // dB, dC of this half chunk: sums over the 4 warps x 8 channels, added
+      // to the fp32 accumulators (16-byte vector atomics when S >= 4)
+      if constexpr (S >= 4) {
+        for (int o = threadIdx.x; o < kRedOutputs; o += kBW * 32) {
+          const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
           const int which = r4 / NP, n = r4 - which * NP;
-          float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
-          atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+          const int jj = n / S, s0 = n - jj * S;
+          const int t = half * (kTB / 2) + tl;
+          if (t0 + t < L) {
+            bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int w = 0; w < kBW; ++w) {
+#pragma unroll
+              for (int cc = 0; cc < kBCPW; ++cc) {
+                const float *src = &sm.w[w].part[tl][which][jj][cc * S + s0];
+                const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(src);
+                acc0 = badd(acc0, x.x);
+                acc1 = badd(acc1, x.y);
+              }
+            }
+            float4 acc;
+            bunpack(acc0, acc.x, acc.y);
+            bunpack(acc1, acc.z, acc.w);
+            float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
+            atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+          }
+        }
+      } else {
+        for (int o = threadIdx.x; o < (kTB / 2) * 2 * NP; o += kBW * 32) {
+          const int tl = o / (2 * NP), r = o % (2 * NP);
+          const int which = r / NP, n = r - which * NP;
+          const int jj = n / S, s0 = n - jj * S;
+          const int t = half * (kTB / 2) + tl;
+          if (t0 + t < L) {
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < kBW; ++w)
+#pragma unroll
+              for (int cc = 0; cc < kBCPW; ++cc) acc += sm.w[w].part[tl][which][jj][cc * S + s0];
+            atomicAdd((which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n), acc);
+          }
         }
       }
       __syncthreads();

@@ -70,6 +70,7 @@ struct BwdParams {
   int N;
   int softplus;
   int io_vec;
+  int bc_vec;                 // B/C rows 16-byte aligned and N == NP
   int64_t cpb;                // CTAs per batch element
   int64_t K;                  // backward chunks
 };
