@@ -36,7 +36,11 @@ import synth  # noqa: E402
 METRIC = "selective-scan fwd/bwd tokens·channels/s and % of HBM/SFU roofline, 1 B200"
 UNIT = "tokens·channels/s"
 MUFU_EX2_PER_CLK_PER_SM = 16  # special-function unit ex2 rate per SM and clock
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fwd_lookback_mamba-2.8b-layer.md")
+# ncu summaries holding the DRAM traffic of the dominant kernel, per forward path
+PROFILE_TRAFFIC = {
+    "lookback": os.path.join(ROOT, "profiles", "fwd_lookback_mamba-2.8b-layer.md"),
+    "lookback_ws": os.path.join(ROOT, "profiles", "fwd_ws_mamba-2.8b-layer.md"),
+}
 KERNEL_SOURCES = [os.path.join(ROOT, "selective_state_space_54_b200", "csrc", f)
                   for f in ("ssm_fwd.cu", "ssm_common.cuh")]
 
@@ -91,12 +95,13 @@ def source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
+def profiled_traffic(path: str):
     """dram bytes per launch from the committed ncu summary, if the kernel is unchanged."""
-    if not os.path.exists(PROFILE_TRAFFIC):
+    f = PROFILE_TRAFFIC.get(path)
+    if not f or not os.path.exists(f):
         return None
     vals = {}
-    for line in open(PROFILE_TRAFFIC):
+    for line in open(f):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
@@ -334,7 +339,7 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     ms_b = max_over_ranks(t_b / steps)
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
             "d_state": w.dstate, "io_dtype": w.dtype, "steps": steps,
-            "fwd_ms": ms_f, "bwd_ms": ms_b,
+            "fwd_path": ssm.fwd_path(shape), "fwd_ms": ms_f, "bwd_ms": ms_b,
             "value": aggregate_value(world, w.bld, (ms_f + ms_b) * 1e-3), "unit": UNIT + " (fwd+bwd)",
             "bwd_value": aggregate_value(world, w.bld, ms_b * 1e-3),
             "bwd_ex2_per_element": 3,
@@ -371,7 +376,7 @@ def main():
                 "steps": tr["steps"], "warmup": max(3, args.warmup),
                 "ms_per_step": tr["fwd_ms"] + tr["bwd_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": dict(config_of(w, "lookback"), step="fwd+bwd"), "bwd": tr,
+                "config": dict(config_of(w, tr["fwd_path"]), step="fwd+bwd"), "bwd": tr,
                 "gpu_launches": 3 * tr["steps"]}
         if rank == 0:
             print(json.dumps(line), flush=True)
@@ -474,7 +479,7 @@ def main():
     achieved = w.bldn / sec
     roofline = {"bound": "alu", "achieved": achieved / 1e12, "peak": ex2_peak / 1e12,
                 "unit": "Tex2/s", "frac": achieved / ex2_peak,
-                "traffic": profiled_traffic(),
+                "traffic": profiled_traffic(path),
                 "kernel": {"lookback": "k_fwd_lookback", "lookback_ws": "k_fwd_ws"}.get(
                     path, f"k_fwd_segment ({path})"),
                 "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
