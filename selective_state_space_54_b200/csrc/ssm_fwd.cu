@@ -48,6 +48,11 @@ __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ f2 mul2(f2 a, f2 b) {
   f2 d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -82,6 +87,30 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // SiLU(z) = z / (1 + e^-z)
 __device__ __forceinline__ float silu_fast(float z) {
   return z * rcp_approx(1.f + ex2(-z * kLog2e));
+}
+
+// The same two functions on a pair of values, the polynomial and the
+// products in packed fp32 pairs.
+__device__ __forceinline__ f2 splat2(float v) { return pack2(v, v); }
+__device__ __forceinline__ f2 softplus2(f2 s) {
+  float s0, s1;
+  unpack2(s, s0, s1);
+  const f2 x = pack2(ex2(-fabsf(s0) * kLog2e), ex2(-fabsf(s1) * kLog2e));
+  f2 q = fma2(splat2(5.126102362e-03f), x, splat2(-2.907406539e-02f));
+  q = fma2(q, x, splat2(7.751608640e-02f));
+  q = fma2(q, x, splat2(-1.360224783e-01f));
+  q = fma2(q, x, splat2(1.907688081e-01f));
+  q = fma2(q, x, splat2(-2.483539879e-01f));
+  q = fma2(q, x, splat2(3.331812024e-01f));
+  q = fma2(q, x, splat2(-4.999944568e-01f));
+  q = fma2(q, x, splat2(9.999999404e-01f));
+  return fma2(x, q, pack2(fmaxf(s0, 0.f), fmaxf(s1, 0.f)));
+}
+__device__ __forceinline__ f2 silu2(f2 z) {
+  float e0, e1, d0, d1;
+  unpack2(mul2(z, splat2(-kLog2e)), e0, e1);
+  unpack2(add2(pack2(ex2(e0), ex2(e1)), splat2(1.f)), d0, d1);
+  return mul2(z, pack2(rcp_approx(d0), rcp_approx(d1)));
 }
 
 // ---- raw io vectors of 8 values ------------------------------------------------
@@ -608,7 +637,7 @@ template <int NP>
 struct __align__(16) WSStage {
   float dl[16][kTW + 4];
   float dlu[16][kTW + 4];
-  float ys[16][kTW + 4];
+  float ys[2][16][kTW + 4];  // C.h partial sums of a channel's two lanes
   float Bs[kTW][NP];
   float Cs[kTW][NP];
 };
@@ -735,17 +764,12 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
             hp[s / 2] = fma2(a, hp[s / 2], mul2(du2, bv));
             acc[(s / 2) & 1] = fma2(cv, hp[s / 2], acc[(s / 2) & 1]);
           }
-          float a0, a1, a2, a3;
-          unpack2(acc[0], a0, a1);
-          unpack2(acc[1], a2, a3);
-          yp[i] = (a0 + a1) + (a2 + a3);
+          float a0, a1;
+          unpack2(add2(acc[0], acc[1]), a0, a1);
+          yp[i] = a0 + a1;
         }
-        // lane j keeps steps tt+2j, tt+2j+1 summed over the channel's 2 lanes
-        const float k0 = j ? yp[2] : yp[0], k1 = j ? yp[3] : yp[1];
-        const float s0 = j ? yp[0] : yp[2], s1 = j ? yp[1] : yp[3];
-        const float r0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);
-        const float r1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
-        *reinterpret_cast<float2 *>(&st.ys[c][tt + 2 * j]) = make_float2(r0, r1);
+        // this lane's half of the channel's C.h; the producer adds the halves
+        *reinterpret_cast<float4 *>(&st.ys[j][c][tt]) = make_float4(yp[0], yp[1], yp[2], yp[3]);
       }
       bar_arrive_n(bar_ys + stage, 64);
     }
@@ -764,78 +788,89 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
 }
 
 // Row pointers and per-channel constants of one run, computed once per run.
-template <typename T>
+// Producer lanes take channel c = lane % 16 and steps [8j, 8j+8) of every
+// chunk with j = lane / 16, so that a quarter warp's 16-byte row accesses fall
+// in distinct shared-memory banks.  The u/delta/z/y pointers already point at
+// step 8j of the channel's row; B/C at this lane's first 16-byte piece.
+template <typename T, int NP>
 struct RunRows {
-  const T *u, *dr, *z, *Bb, *Cb;
+  static constexpr int EPP = 16 / (int)sizeof(T);  // elements per 16-byte piece
+  const T *u, *dr, *z, *Bb, *Cb, *Bl, *Cl;
   T *y;
   float bias, Dd;
   bool valid;
-  int c, j;
-  // Producer lanes take channel c = lane % 16 and steps [8j, 8j+8) with
-  // j = lane / 16, so that a quarter warp's 16-byte row accesses fall in
-  // distinct shared-memory banks.
-  __device__ __forceinline__ void set(const FwdParams &p, int64_t g) {
-    Lane ln;
-    ln.lane = threadIdx.x & 31;
-    ln.c = ln.lane & 15;
-    ln.j = ln.lane >> 4;
-    ln.b = g / p.gpb;
-    ln.d = (g - ln.b * p.gpb) * 16 + ln.c;
-    ln.valid = ln.d < p.dim;
-    const int64_t row = (ln.b * p.dim + (ln.valid ? ln.d : 0)) * p.L;
+  __device__ __forceinline__ void set(const FwdParams &p, int64_t g, int lane) {
+    const int c = lane & 15, j = lane >> 4;
+    const int64_t b = g / p.gpb;
+    const int64_t d = (g - b * p.gpb) * 16 + c;
+    valid = d < p.dim;
+    const int64_t row = (b * p.dim + (valid ? d : 0)) * p.L + j * 8;
     u = static_cast<const T *>(p.u) + row;
     dr = static_cast<const T *>(p.delta) + row;
     z = p.z ? static_cast<const T *>(p.z) + row : nullptr;
     y = static_cast<T *>(p.y) + row;
-    Bb = static_cast<const T *>(p.B) + ln.b * p.L * p.N;
-    Cb = static_cast<const T *>(p.C) + ln.b * p.L * p.N;
-    bias = (p.bias && ln.valid) ? p.bias[ln.d] : 0.f;
-    Dd = (p.D && ln.valid) ? p.D[ln.d] : 0.f;
-    valid = ln.valid;
-    c = ln.c;
-    j = ln.j;
+    Bb = static_cast<const T *>(p.B) + b * p.L * p.N;
+    Cb = static_cast<const T *>(p.C) + b * p.L * p.N;
+    Bl = Bb + lane * EPP;
+    Cl = Cb + lane * EPP;
+    bias = (p.bias && valid) ? p.bias[d] : 0.f;
+    Dd = (p.D && valid) ? p.D[d] : 0.f;
   }
 };
 
 // Copy this lane's pieces of chunk k of run `rr` into raw slot `slot`:
-// u/delta/z steps [8j, 8j+8) of channel c, and B/C 16-byte pieces lane,
-// lane+32, ...  Asynchronous (cp.async, zero-filled past L) on 16-byte
-// aligned rows; plain loads otherwise.  Every lane later reads only the
-// pieces it copied itself.
+// u/delta/z steps [8j, 8j+8) of channel c, and the B/C 16-byte pieces lane,
+// lane+32, ...  Whole chunks of valid channels with 16-byte aligned rows take
+// the short path; the last chunk of a ragged L, padded channels and
+// unaligned rows take the checked one (zero fill past L).  Every lane later
+// reads only the pieces it copied itself.
 template <typename T, int NP>
-__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, const RunRows<T> &rr,
+__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, const RunRows<T, NP> &rr,
                                          int64_t k, int lane) {
-  constexpr int ES = (int)sizeof(T), EPP = 16 / ES;   // elements per 16-byte piece
+  constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
+  constexpr int NV = kTW * NP / EPP;  // B/C pieces per chunk
+  const int c = lane & 15, j8 = (lane >> 4) * 8;
   const int64_t L = p.L, t0 = k * kTW;
-  const int64_t ts = t0 + rr.j * 8;
-  if (p.io_vec) {
+  const bool whole = t0 + kTW <= L;
+  if (whole && rr.valid && p.io_vec) {
 #pragma unroll
     for (int q = 0; q < 8 / EPP; ++q) {
-      const int64_t t = ts + q * EPP;
+      cp_async16(&raw.u[c][j8 + q * EPP], rr.u + t0 + q * EPP, 16);
+      cp_async16(&raw.d[c][j8 + q * EPP], rr.dr + t0 + q * EPP, 16);
+      if (rr.z) cp_async16(&raw.z[c][j8 + q * EPP], rr.z + t0 + q * EPP, 16);
+    }
+  } else if (p.io_vec) {
+#pragma unroll
+    for (int q = 0; q < 8 / EPP; ++q) {
+      const int64_t t = t0 + j8 + q * EPP;
       const int64_t left = rr.valid ? L - t : 0;
       const int bytes = left >= EPP ? 16 : (left > 0 ? (int)left * ES : 0);
-      const int64_t off = bytes > 0 ? t : 0;
-      cp_async16(&raw.u[rr.c][rr.j * 8 + q * EPP], rr.u + off, bytes);
-      cp_async16(&raw.d[rr.c][rr.j * 8 + q * EPP], rr.dr + off, bytes);
-      if (rr.z) cp_async16(&raw.z[rr.c][rr.j * 8 + q * EPP], rr.z + off, bytes);
+      const int64_t off = bytes > 0 ? t0 + q * EPP : -j8;  // row start when nothing is read
+      cp_async16(&raw.u[c][j8 + q * EPP], rr.u + off, bytes);
+      cp_async16(&raw.d[c][j8 + q * EPP], rr.dr + off, bytes);
+      if (rr.z) cp_async16(&raw.z[c][j8 + q * EPP], rr.z + off, bytes);
     }
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const bool in = rr.valid && ts + i < L;
-      raw.u[rr.c][rr.j * 8 + i] = in ? rr.u[ts + i] : T(0);
-      raw.d[rr.c][rr.j * 8 + i] = in ? rr.dr[ts + i] : T(0);
-      if (rr.z) raw.z[rr.c][rr.j * 8 + i] = in ? rr.z[ts + i] : T(0);
+      const bool in = rr.valid && t0 + j8 + i < L;
+      raw.u[c][j8 + i] = in ? rr.u[t0 + i] : T(0);
+      raw.d[c][j8 + i] = in ? rr.dr[t0 + i] : T(0);
+      if (rr.z) raw.z[c][j8 + i] = in ? rr.z[t0 + i] : T(0);
     }
   }
   if (p.bc_vec && NP % EPP == 0) {
-    constexpr int NV = kTW * NP / EPP;
-    for (int v = lane; v < NV; v += 32) {
-      const int e = v * EPP, t = e / NP, n = e - t * NP;
-      const bool in = t0 + t < L;
-      const int64_t off = in ? (t0 + t) * NP + n : 0;
-      cp_async16(&raw.B[t][n], rr.Bb + off, in ? 16 : 0);
-      cp_async16(&raw.C[t][n], rr.Cb + off, in ? 16 : 0);
+    T *rB = &raw.B[0][0], *rC = &raw.C[0][0];
+#pragma unroll
+    for (int q = 0; q < (NV + 31) / 32; ++q) {
+      const int v = lane + 32 * q;
+      if (NV % 32 == 0 || v < NV) {
+        const int e = v * EPP;
+        const bool in = whole || t0 + e / NP < L;
+        const int64_t off = in ? t0 * NP + q * 32 * EPP : -(int64_t)lane * EPP;
+        cp_async16(rB + e, rr.Bl + off, in ? 16 : 0);
+        cp_async16(rC + e, rr.Cl + off, in ? 16 : 0);
+      }
     }
   } else {
     for (int e = lane; e < kTW * NP; e += 32) {
@@ -854,120 +889,106 @@ template <typename T, int NP>
 __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &sm, const Share &sh,
                                             unsigned bar_full, unsigned bar_ys) {
   constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
+  constexpr int NV = kTW * NP / EPP;
   const int64_t L = p.L;
   const int lane = threadIdx.x & 31;
+  const int c = lane & 15, j8 = (lane >> 4) * 8;
   const bool io_vec = p.io_vec != 0;
-  // the chunk whose output epilogue is pending
-  bool pend = false;
+  const bool has_z = p.z != nullptr;
+  // the chunk whose output epilogue is pending: its stage, row, gate, D*u
+  bool pend = false, pvalid = false;
   int pstage = 0;
-  T *py_row = nullptr;
-  int64_t pts = 0;
-  bool pvalid = false;
-  float gate[8], dg[8];
-
-  auto epilogue = [&]() {
-    bar_sync_n(bar_ys + pstage, 64);
-    if (pvalid) {
-      const float *py = &sm.st[pstage].ys[lane & 15][(lane >> 4) * 8];
-      const float4 a = *reinterpret_cast<const float4 *>(py);
-      const float4 b4 = *reinterpret_cast<const float4 *>(py + 4);
-      const float ys[8] = {a.x, a.y, a.z, a.w, b4.x, b4.y, b4.z, b4.w};
-      float o[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = fmaf(ys[i], gate[i], dg[i]);
-      IO<T>::store8(py_row, pts, L, io_vec, o);
-    }
-  };
+  T *py = nullptr;
+  int64_t pt = 0;
+  f2 gate2[4], du2[4];
 
   // prefetch cursor: the item kSlots-1 chunks ahead of the one processed
   int64_t pr = 0, pk = 0, pk1 = 0, pg = 0;
-  RunRows<T> pf;
+  RunRows<T, NP> pf;
   bool pf_live = sh.n_runs > 0;
   if (pf_live) {
     sh.get(0, pg, pk, pk1);
-    pf.set(p, pg);
+    pf.set(p, pg, lane);
   }
   auto advance = [&]() {
-    if (!pf_live) return;
     if (++pk >= pk1) {
       if (++pr < sh.n_runs) {
         sh.get(pr, pg, pk, pk1);
-        pf.set(p, pg);
+        pf.set(p, pg, lane);
       } else {
         pf_live = false;
       }
     }
   };
-  int64_t it_f = 0;  // chunks fetched
+  int it_f = 0;  // chunks fetched (slot cursor)
   for (int i = 0; i < kSlots - 1; ++i) {
-    if (pf_live && pk < pk1) ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+    if (pf_live) {
+      ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+      advance();
+    }
     cp_async_commit();
     ++it_f;
-    advance();
   }
 
-  int64_t it = 0;
+  int it = 0;
   for (int64_t r = 0; r < sh.n_runs; ++r) {
     int64_t g, k0, k1;
     sh.get(r, g, k0, k1);
-    RunRows<T> cur;
-    cur.set(p, g);
+    RunRows<T, NP> cur;
+    cur.set(p, g, lane);
     for (int64_t k = k0; k < k1; ++k, ++it) {
-      const int stage = (int)(it & 1);
+      const int stage = it & 1;
       WSStage<NP> &st = sm.st[stage];
       WSRaw<T, NP> &raw = sm.raw[it % kSlots];
-      const int64_t ts = k * kTW + cur.j * 8;
+      const int64_t t0 = k * kTW;
+      const bool whole = cur.valid && t0 + kTW <= L;
       cp_async_wait<kSlots - 2>();  // this chunk's copies have landed
-      // ---- pre-pass of chunk k into stage ----
-      float u8[8], d8[8], z8[8];
+      // ---- pre-pass of chunk k into the stage: Delta, Delta*u, B/C in fp32 ----
+      float u8[8], s8[8];
       {
-        Vec8<T> vu, vd, vz;
-        vu.load_shared(&raw.u[cur.c][cur.j * 8]);
-        vd.load_shared(&raw.d[cur.c][cur.j * 8]);
+        Vec8<T> vu, vd;
+        vu.load_shared(&raw.u[c][j8]);
+        vd.load_shared(&raw.d[c][j8]);
         vu.unpack(u8);
-        vd.unpack(d8);
-        if (cur.z) {
-          vz.load_shared(&raw.z[cur.c][cur.j * 8]);
-          vz.unpack(z8);
-        } else {
+        vd.unpack(s8);
+      }
+      f2 dl2[4], dlu2[4];
+      const f2 bias2 = pack2(cur.bias, cur.bias);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) z8[i] = 0.f;
+      for (int i = 0; i < 4; ++i) {
+        const f2 s = add2(pack2(s8[2 * i], s8[2 * i + 1]), bias2);
+        dl2[i] = p.softplus ? softplus2(s) : s;
+      }
+      if (!whole) {  // zero Delta past L and on padded channels: the state holds
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float a, b;
+          unpack2(dl2[i], a, b);
+          a = (cur.valid && t0 + j8 + 2 * i < L) ? a : 0.f;
+          b = (cur.valid && t0 + j8 + 2 * i + 1 < L) ? b : 0.f;
+          dl2[i] = pack2(a, b);
         }
       }
-      float dl8[8], du8[8], ng[8], ndg[8];
 #pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        const float s0 = d8[i] + cur.bias, s1 = d8[i + 1] + cur.bias;
-        float dl0 = s0, dl1 = s1;
-        if (p.softplus) {
-          dl0 = softplus_fast(s0);
-          dl1 = softplus_fast(s1);
-        }
-        dl0 = (cur.valid && ts + i < L) ? dl0 : 0.f;
-        dl1 = (cur.valid && ts + i + 1 < L) ? dl1 : 0.f;
-        dl8[i] = dl0; dl8[i + 1] = dl1;
-        du8[i] = dl0 * u8[i]; du8[i + 1] = dl1 * u8[i + 1];
-        float g0 = 1.f, g1 = 1.f;
-        if (cur.z) {
-          g0 = silu_fast(z8[i]);
-          g1 = silu_fast(z8[i + 1]);
-        }
-        ng[i] = g0; ng[i + 1] = g1;
-        ndg[i] = cur.Dd * u8[i] * g0; ndg[i + 1] = cur.Dd * u8[i + 1] * g1;
+      for (int i = 0; i < 4; ++i) dlu2[i] = mul2(dl2[i], pack2(u8[2 * i], u8[2 * i + 1]));
+      {
+        float *pd = &st.dl[c][j8];
+        float *pu = &st.dlu[c][j8];
+        *reinterpret_cast<ulonglong2 *>(pd) = make_ulonglong2(dl2[0], dl2[1]);
+        *reinterpret_cast<ulonglong2 *>(pd + 4) = make_ulonglong2(dl2[2], dl2[3]);
+        *reinterpret_cast<ulonglong2 *>(pu) = make_ulonglong2(dlu2[0], dlu2[1]);
+        *reinterpret_cast<ulonglong2 *>(pu + 4) = make_ulonglong2(dlu2[2], dlu2[3]);
       }
-      float *pd = &st.dl[cur.c][cur.j * 8];
-      float *pu = &st.dlu[cur.c][cur.j * 8];
-      *reinterpret_cast<float4 *>(pd) = make_float4(dl8[0], dl8[1], dl8[2], dl8[3]);
-      *reinterpret_cast<float4 *>(pd + 4) = make_float4(dl8[4], dl8[5], dl8[6], dl8[7]);
-      *reinterpret_cast<float4 *>(pu) = make_float4(du8[0], du8[1], du8[2], du8[3]);
-      *reinterpret_cast<float4 *>(pu + 4) = make_float4(du8[4], du8[5], du8[6], du8[7]);
       // widen this lane's B/C pieces (the ones it fetched) to fp32
       if (p.bc_vec && NP % EPP == 0) {
-        constexpr int NV = kTW * NP / EPP;
-        for (int v = lane; v < NV; v += 32) {
-          const int e = v * EPP, t = e / NP, n = e - t * NP;
-          bc_store_vec<T, NP>(st.Bs, *reinterpret_cast<const uint4 *>(&raw.B[t][n]), v);
-          bc_store_vec<T, NP>(st.Cs, *reinterpret_cast<const uint4 *>(&raw.C[t][n]), v);
+#pragma unroll
+        for (int q = 0; q < (NV + 31) / 32; ++q) {
+          const int v = lane + 32 * q;
+          if (NV % 32 == 0 || v < NV) {
+            const int e = v * EPP;
+            bc_store_vec<T, NP>(st.Bs, *reinterpret_cast<const uint4 *>(&raw.B[0][0] + e), v);
+            bc_store_vec<T, NP>(st.Cs, *reinterpret_cast<const uint4 *>(&raw.C[0][0] + e), v);
+          }
         }
       } else {
         for (int e = lane; e < kTW * NP; e += 32) {
@@ -977,23 +998,72 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
         }
       }
       bar_arrive_n(bar_full + stage, 64);
-      // ---- copies of the chunk kSlots-1 ahead, into the slot just freed ----
-      if (pf_live && pk < pk1) ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+      // ---- copies of the chunk kSlots-1 ahead, into the slot of chunk k-1 ----
+      if (pf_live) {
+        ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+        advance();
+      }
       cp_async_commit();
       ++it_f;
-      advance();
-      // ---- epilogue of the previous chunk ----
-      if (pend) epilogue();
+      // ---- epilogue of chunk k-1: y = (C.h + D*u) * SiLU(z) ----
+      if (pend) {
+        bar_sync_n(bar_ys + pstage, 64);
+        if (pvalid) {
+          const WSStage<NP> &ps = sm.st[pstage];
+          const ulonglong2 a0 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[0][c][j8]);
+          const ulonglong2 a1 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[0][c][j8 + 4]);
+          const ulonglong2 b0 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[1][c][j8]);
+          const ulonglong2 b1 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[1][c][j8 + 4]);
+          const f2 ya[4] = {a0.x, a0.y, a1.x, a1.y}, yb[4] = {b0.x, b0.y, b1.x, b1.y};
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            unpack2(mul2(add2(add2(ya[i], yb[i]), du2[i]), gate2[i]), o[2 * i], o[2 * i + 1]);
+          IO<T>::store8(py, pt, L - j8, io_vec, o);
+        }
+      }
+      // ---- gate and D*u of chunk k, for its epilogue in the next iteration ----
+      {
+        const f2 D2 = pack2(cur.Dd, cur.Dd);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) du2[i] = mul2(D2, pack2(u8[2 * i], u8[2 * i + 1]));
+        if (has_z) {
+          float z8[8];
+          Vec8<T> vz;
+          vz.load_shared(&raw.z[c][j8]);
+          vz.unpack(z8);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) gate2[i] = silu2(pack2(z8[2 * i], z8[2 * i + 1]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) gate2[i] = pack2(1.f, 1.f);
+        }
+      }
       pend = true;
       pstage = stage;
-      py_row = cur.y;
-      pts = ts;
+      py = cur.y;
+      pt = t0;
       pvalid = cur.valid;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { gate[i] = ng[i]; dg[i] = ndg[i]; }
     }
   }
-  if (pend) epilogue();
+  if (pend) {
+    bar_sync_n(bar_ys + pstage, 64);
+    if (pvalid) {
+      const WSStage<NP> &ps = sm.st[pstage];
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = ps.ys[0][c][j8 + i] + ps.ys[1][c][j8 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float d0, d1, g0, g1;
+        unpack2(du2[i], d0, d1);
+        unpack2(gate2[i], g0, g1);
+        o[2 * i] = (o[2 * i] + d0) * g0;
+        o[2 * i + 1] = (o[2 * i + 1] + d1) * g1;
+      }
+      IO<T>::store8(py, pt, L - j8, io_vec, o);
+    }
+  }
   cp_async_wait<0>();
 }
 
