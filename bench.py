@@ -346,6 +346,97 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
             "bwd_kernels_per_step": 2}
 
 
+def decode_bytes(w: synth.Workload) -> int:
+    """Bytes one decode step must move: the fp32 state read and written, the
+    per-channel token inputs and output, B/C, and A/D/bias once."""
+    es = 2 if w.dtype == synth.BF16 else 4
+    bd = w.batch * w.dim
+    return (8 * bd * w.dstate + 4 * es * bd + 2 * es * w.batch * w.dstate
+            + 4 * w.dim * w.dstate + 8 * w.dim)
+
+
+def measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None):
+    """Single-token steps on the decode workload, replayed from a CUDA graph.
+
+    Four independent (state, token) slots are cycled so that every step reads
+    and writes a state that is not in L2 (4 states > 126 MB of L2)."""
+    w = w or synth.WORKLOADS["mamba-2.8b-decode"]
+    slots = 4
+    case = synth.make_workload(w)
+    A = torch.from_numpy(np.asarray(case["A"], np.float32)).to(dev)
+    D = torch.from_numpy(np.asarray(case["D"], np.float32)).to(dev)
+    bias = torch.from_numpy(np.asarray(case["delta_bias"], np.float32)).to(dev)
+    tok = {k: to_torch(case[k], dev) for k in ("u", "delta", "z", "B", "C")}
+    xs, states, ys = [], [], []
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    for i in range(slots):
+        x = {k: tok[k][:, :, 0].contiguous() for k in ("u", "delta", "z")}
+        x.update({k: tok[k][:, 0, :].contiguous() for k in ("B", "C")})
+        if i:  # other tokens: the same values rolled along the channels
+            x = {k: torch.roll(v, i, dims=-1).contiguous() for k, v in x.items()}
+        xs.append(x)
+        states.append(torch.randn((w.batch, w.dim, w.dstate), generator=gen, device=dev,
+                                  dtype=torch.float32))
+        ys.append(torch.empty_like(x["u"]))
+
+    def step(i):
+        x = xs[i % slots]
+        ssm.scan_step(x["u"], x["delta"], A, x["B"], x["C"], D, x["z"], bias,
+                      state=states[i % slots], y=ys[i % slots])
+
+    stream = torch.cuda.current_stream(dev)
+    k = max(args.steps, 8) // slots * slots
+    for i in range(max(3, args.warmup) * slots):
+        step(i)
+    torch.cuda.synchronize(dev)
+    # eager: one library call per step from Python
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for i in range(k):
+        step(i)
+    ev[1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms_eager = max_over_ranks(ev[0].elapsed_time(ev[1]) / k)
+    # the same k steps captured once in a CUDA graph and replayed
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        step(0)  # warm the capture stream
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(k):
+                step(i)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev[2].record(stream)
+    g.replay()
+    ev[3].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(ev[2].elapsed_time(ev[3]) / k)
+    del g
+    nbytes = decode_bytes(w)
+    pk = peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate,
+            "io_dtype": w.dtype, "state_dtype": "f32", "steps": k, "state_slots": slots,
+            "l2": f"{slots} state slots of {8 * w.batch * w.dim * w.dstate // 2 / 1e6:.0f} MB cycled",
+            "us_per_step": ms * 1e3, "us_per_step_eager": ms_eager * 1e3,
+            "value": aggregate_value(world, w.batch * w.dim, ms * 1e-3),
+            "unit": "tokens·channels/s (single-token steps, CUDA graph replay)",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "kernel": "k_step", "algorithmic_bytes": nbytes,
+                         "peak_basis": f"measured copy bandwidth ({pk['source']})"},
+            "gpu_launches": k}
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -362,13 +453,31 @@ def main():
     world, rank, local = init_dist(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+
+    def barrier0():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    if w.extra.get("decode"):
+        dec = measure_decode(ssm, torch, dev, args, world, barrier0,
+                             lambda x: dist_max(x, world, dev), w)
+        line = {"metric": METRIC, "value": dec["value"], "unit": UNIT, "n_gpus": world,
+                "steps": dec["steps"], "warmup": max(3, args.warmup),
+                "ms_per_step": dec["us_per_step"] * 1e-3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": w.name, "batch": w.batch, "d_inner": w.dim,
+                           "d_state": w.dstate, "io_dtype": w.dtype, "step": "decode",
+                           "l2": dec["l2"], "seed": w.seed},
+                "roofline": dec["roofline"], "decode": dec, "gpu_launches": dec["gpu_launches"]}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if w.backward:
         # the training step itself: forward + recomputation backward
-        def barrier0():
-            if world > 1:
-                import torch.distributed as dist
-                dist.barrier()
-
         def max0(x):
             return dist_max(x, world, dev)
         tr = measure_training(ssm, torch, dev, args, world, barrier0, max0, w)
@@ -468,9 +577,10 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
         del host, dbuf
 
-    bwd = None
+    bwd = dec = None
     if not args.no_bwd and not args.batch:
         bwd = measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks)
+        dec = measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks)
 
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -496,7 +606,7 @@ def main():
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
-            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd,
+            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, case)

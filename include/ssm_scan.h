@@ -166,6 +166,31 @@ ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u, const voi
                                 int delta_softplus, const float *initial_state,
                                 void *y, float *last_state, ssm_stream_t stream);
 
+/* Single-step (recurrent) update: one new token for every (batch, channel),
+ * the constant-time-per-token inference mode in which only the fixed-size
+ * state is kept between tokens ("Mamba: Linear-Time Sequence Modeling with
+ * Selective State Spaces", xyznot.com reading guide, the question on KV
+ * caches; "O que e um modelo Mamba?", ibm.com, constant inference memory;
+ * "Как работает Mamba", aivaro.ru, O(1) per step).  Computes, with the same
+ * arithmetic as one step of ssm_scan_fwd:
+ *   Delta = softplus(delta + delta_bias)   (or delta + delta_bias)
+ *   state <- exp(Delta * A) (.) state + Delta * B * u      (in place)
+ *   y      = (C . state + D * u) * SiLU(z)
+ * shape->seqlen must be 1 (SSM_ERR_INVALID_ARG otherwise); path and lanes
+ * are ignored.  Layouts: u, delta, z, y [batch][dim] io dtype; B, C
+ * [batch][dstate] io dtype; A [dim][dstate], D and delta_bias [dim] fp32;
+ * state [batch][dim][dstate] fp32, read and overwritten.  D, z and
+ * delta_bias are nullable.  No workspace; nothing is allocated.  y may not
+ * alias an input; state must not alias any other argument.  Calling it
+ * seqlen times, feeding each token, gives the same y and final state as
+ * ssm_scan_fwd over the seqlen tokens with initial_state = state (up to
+ * rounding).  dstate % 4 == 0 with 16-byte aligned state and A (and B/C
+ * rows aligned to 4 elements) takes 16-byte accesses. */
+ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delta,
+                         const float *A, const void *B, const void *C,
+                         const float *D, const void *z, const float *delta_bias,
+                         int delta_softplus, float *state, void *y, ssm_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word of
  * `workspace`.  SSM_OK, SSM_ERR_DEVICE_TIMEOUT or SSM_ERR_CUDA. */
 ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream);

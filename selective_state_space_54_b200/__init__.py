@@ -7,6 +7,7 @@ kernels (include/ssm_scan.h).  There is no CPU path.
     y, last_state = scan_fwd(u, delta, A, B, C, D, z, delta_bias,
                              delta_softplus=True, return_last_state=True)
     grads = scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout)
+    y_t = scan_step(u_t, delta_t, A, B_t, C_t, D, z_t, delta_bias, state=state)
 
 Layouts: u, delta, z, y, dout (batch, dim, seqlen); B, C (batch, seqlen,
 dstate); A (dim, dstate) fp32; D, delta_bias (dim,) fp32; states (batch, dim,
@@ -20,7 +21,7 @@ from . import _lib
 from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_PATH_AUTO, SSM_PATH_LOOKBACK,  # noqa: F401
                    SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L, ssm_shape)
 
-__all__ = ["scan_fwd", "scan_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes",
+__all__ = ["scan_fwd", "scan_bwd", "scan_step", "fwd_workspace_bytes", "bwd_workspace_bytes",
            "fwd_path", "check", "ScanError", "make_shape"]
 
 
@@ -126,6 +127,38 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
         raise ScanError(rc, "ssm_scan_fwd")
     if return_last_state:
         return y, last_state
+    return y
+
+
+def scan_step(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, state,
+              delta_softplus=True, y=None, stream=None):
+    """One recurrent step for every (batch, channel): updates `state` in place
+    and returns y.  u, delta, z, y (batch, dim); B, C (batch, dstate); state
+    (batch, dim, dstate) fp32."""
+    import torch
+    batch, dim = u.shape
+    dstate = B.shape[-1]
+    dt = u.dtype
+    dev = u.device
+    f32 = torch.float32
+    _check_io("u", u, (batch, dim), dt, dev)
+    _check_io("delta", delta, (batch, dim), dt, dev)
+    _check_io("z", z, (batch, dim), dt, dev)
+    _check_io("B", B, (batch, dstate), dt, dev)
+    _check_io("C", C, (batch, dstate), dt, dev)
+    _check_io("A", A, (dim, dstate), f32, dev)
+    _check_io("D", D, (dim,), f32, dev)
+    _check_io("delta_bias", delta_bias, (dim,), f32, dev)
+    _check_io("state", state, (batch, dim, dstate), f32, dev)
+    if y is None:
+        y = torch.empty_like(u)
+    _check_io("y", y, (batch, dim), dt, dev)
+    shape = make_shape(batch, dim, 1, dstate, _io_dtype(u))
+    rc = _lib.load().ssm_scan_step(
+        ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(state), _ptr(y), _stream(stream))
+    if rc != 0:
+        raise ScanError(rc, "ssm_scan_step")
     return y
 
 

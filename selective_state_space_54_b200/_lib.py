@@ -34,7 +34,7 @@ PATH_NAMES = {SSM_PATH_AUTO: "auto", SSM_PATH_LOOKBACK: "lookback",
 EXPORTS = (
     "ssm_scan_fwd_workspace_bytes", "ssm_scan_bwd_workspace_bytes", "ssm_scan_fwd",
     "ssm_scan_bwd", "ssm_scan_check", "ssm_scan_test_wait_timeout", "ssm_scan_fwd_path",
-    "ssm_status_string", "ssm_scan_version", "ssm_scan_fwd_noalloc",
+    "ssm_status_string", "ssm_scan_version", "ssm_scan_fwd_noalloc", "ssm_scan_step",
 )
 
 
@@ -72,6 +72,8 @@ def load(path: str | None = None):
     lib.ssm_scan_bwd.restype = ci
     lib.ssm_scan_fwd_noalloc.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp]
     lib.ssm_scan_fwd_noalloc.restype = ci
+    lib.ssm_scan_step.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp]
+    lib.ssm_scan_step.restype = ci
     lib.ssm_scan_check.argtypes = [vp, vp]
     lib.ssm_scan_check.restype = ci
     lib.ssm_scan_test_wait_timeout.argtypes = [vp, sz, i64, vp]

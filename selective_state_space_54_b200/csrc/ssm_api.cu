@@ -243,6 +243,32 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
   return cuda_status(e);
 }
 
+ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delta,
+                         const float *A, const void *B, const void *C, const float *D,
+                         const void *z, const float *delta_bias, int delta_softplus,
+                         float *state, void *y, ssm_stream_t stream) {
+  ssm_status st = check_shape(shape);
+  if (st != SSM_OK) return st;
+  if (shape->seqlen != 1) return SSM_ERR_INVALID_ARG;
+  const int64_t nch = shape->batch * shape->dim;
+  if (nch == 0) return SSM_OK;
+  if (!u || !delta || !A || !B || !C || !state || !y) return SSM_ERR_INVALID_ARG;
+  const size_t es = shape->io_dtype == SSM_BF16 ? 2 : 4;
+  if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) ||
+      !aligned(z, es) || !aligned(y, es) || !aligned(A, 4) || !aligned(D, 4) ||
+      !aligned(delta_bias, 4) || !aligned(state, 4))
+    return SSM_ERR_INVALID_ARG;
+  StepParams p;
+  memset(&p, 0, sizeof(p));
+  p.u = u; p.delta = delta; p.z = z; p.B = B; p.C = C;
+  p.A = A; p.D = D; p.bias = delta_bias; p.state = state; p.y = y;
+  p.batch = shape->batch; p.dim = shape->dim; p.N = (int)shape->dstate;
+  p.softplus = delta_softplus ? 1 : 0;
+  p.vec = shape->dstate % 4 == 0 && aligned(state, 16) && aligned(A, 16) &&
+          aligned(B, 4 * es) && aligned(C, 4 * es);
+  return cuda_status(launch_step(shape->io_dtype, p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
   if (check_shape(shape) != SSM_OK) return 0;
   const int NP = fwd_np_for(shape->dstate);

@@ -57,6 +57,18 @@ struct FwdParams {
   float *seg_carry;   // [n_groups * n_segs][32/LPC][NP] state entering the segment
 };
 
+// Single-step (decode) parameters (ssm_step.cu).
+struct StepParams {
+  const void *u, *delta, *z, *B, *C;   // u/delta/z [batch][dim], B/C [batch][N], io dtype
+  const float *A, *D, *bias;
+  float *state;                        // [batch][dim][N] fp32, read and written in place
+  void *y;                             // [batch][dim] io dtype
+  int64_t batch, dim;
+  int N;
+  int softplus;
+  int vec;                             // N % 4 == 0, state/A 16-byte and B/C 4-element aligned
+};
+
 // Backward parameters (ssm_bwd.cu).
 struct BwdParams {
   const void *u, *delta, *z, *B, *C, *dout;
@@ -175,6 +187,36 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
+// ---- softplus without a second special-function op --------------------------
+// softplus(s) = max(s, 0) + log1p(x),  x = exp(-|s|) in (0, 1].
+// log1p(x) = x * p(x), p a degree-8 polynomial interpolating log1p(x)/x at the
+// Chebyshev nodes of [0, 1] (max relative error 2.3e-7 in fp32 evaluation,
+// fitted for this library).
+__device__ __forceinline__ float softplus_fast(float s) {
+  const float x = ex2(-fabsf(s) * kLog2e);
+  float p = 5.126102362e-03f;
+  p = fmaf(p, x, -2.907406539e-02f);
+  p = fmaf(p, x, 7.751608640e-02f);
+  p = fmaf(p, x, -1.360224783e-01f);
+  p = fmaf(p, x, 1.907688081e-01f);
+  p = fmaf(p, x, -2.483539879e-01f);
+  p = fmaf(p, x, 3.331812024e-01f);
+  p = fmaf(p, x, -4.999944568e-01f);
+  p = fmaf(p, x, 9.999999404e-01f);
+  return fmaf(x, p, fmaxf(s, 0.f));
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// SiLU(z) = z / (1 + e^-z)
+__device__ __forceinline__ float silu_fast(float z) {
+  return z * rcp_approx(1.f + ex2(-z * kLog2e));
+}
+
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -216,6 +258,7 @@ cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm);
 cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);
+cudaError_t launch_step(int io_dtype, const StepParams &p, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,
                                       cudaStream_t s);
 

@@ -59,35 +59,6 @@ __device__ __forceinline__ f2 mul2(f2 a, f2 b) {
   return d;
 }
 
-// ---- softplus without a second special-function op --------------------------
-// softplus(s) = max(s, 0) + log1p(x),  x = exp(-|s|) in (0, 1].
-// log1p(x) = x * p(x), p a degree-8 polynomial interpolating log1p(x)/x at the
-// Chebyshev nodes of [0, 1] (max relative error 2.3e-7 in fp32 evaluation,
-// fitted for this library).
-__device__ __forceinline__ float softplus_fast(float s) {
-  const float x = ex2(-fabsf(s) * kLog2e);
-  float p = 5.126102362e-03f;
-  p = fmaf(p, x, -2.907406539e-02f);
-  p = fmaf(p, x, 7.751608640e-02f);
-  p = fmaf(p, x, -1.360224783e-01f);
-  p = fmaf(p, x, 1.907688081e-01f);
-  p = fmaf(p, x, -2.483539879e-01f);
-  p = fmaf(p, x, 3.331812024e-01f);
-  p = fmaf(p, x, -4.999944568e-01f);
-  p = fmaf(p, x, 9.999999404e-01f);
-  return fmaf(x, p, fmaxf(s, 0.f));
-}
-
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// SiLU(z) = z / (1 + e^-z)
-__device__ __forceinline__ float silu_fast(float z) {
-  return z * rcp_approx(1.f + ex2(-z * kLog2e));
-}
 
 // The same two functions on a pair of values, the polynomial and the
 // products in packed fp32 pairs.

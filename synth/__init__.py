@@ -85,6 +85,10 @@ WORKLOADS = {
     "mamba-1.4b-layer-train": Workload("mamba-1.4b-layer-train", 8, 2048, 4096, 16,
                                        BF16, 4, backward=True,
                                        notes="Mamba-1.4B layer forward+backward"),
+    "mamba-2.8b-decode": Workload("mamba-2.8b-decode", 128, 1, 5120, 16, BF16, 5,
+                                  last_state=True, extra={"decode": True},
+                                  notes="Mamba-2.8B layer single-token step, fp32 state "
+                                        "(batch, d_inner, d_state) updated in place"),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 

@@ -150,3 +150,42 @@ def test_noalloc_rejects_bad_shapes_before_launch(lib):
         rc = lib.ssm_scan_fwd_noalloc(ctypes.byref(sh), *[ctypes.c_void_p(16)] * 5, None, None,
                                       None, 1, None, ctypes.c_void_p(16), None, None)
         assert rc == code
+
+
+def _step(lib, shape, ptrs=None):
+    p = dict(u=8, delta=8, A=16, B=8, C=8, D=None, z=None, bias=None, state=16, y=8)
+    p.update(ptrs or {})
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ssm_scan_step(ctypes.byref(shape) if shape is not None else None, v(p["u"]),
+                             v(p["delta"]), v(p["A"]), v(p["B"]), v(p["C"]), v(p["D"]), v(p["z"]),
+                             v(p["bias"]), 1, v(p["state"]), v(p["y"]), None)
+
+
+def test_step_rejects_bad_shapes_before_launch(lib):
+    assert _step(lib, None) == _lib.SSM_ERR_INVALID_ARG
+    for kw, code in BAD_SHAPES:
+        kw = dict(kw)
+        kw.setdefault("seqlen", 1)
+        if kw["seqlen"] == -1:
+            continue
+        assert _step(lib, _shape(**kw)) == code, kw
+    # a step is one token: any other seqlen is an error
+    for L in (0, 2, 64):
+        assert _step(lib, _shape(seqlen=L)) == _lib.SSM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("missing", ["u", "delta", "A", "B", "C", "state", "y"])
+def test_step_null_required_pointer_rejected(lib, missing):
+    assert _step(lib, _shape(seqlen=1), {missing: None}) == _lib.SSM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which,addr", [("u", 9), ("B", 3), ("A", 18), ("y", 1), ("z", 5),
+                                         ("D", 2), ("state", 6)])
+def test_step_misaligned_pointer_rejected(lib, which, addr):
+    assert _step(lib, _shape(seqlen=1), {which: addr}) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_step_empty_problem_is_a_noop(lib):
+    nulls = {k: None for k in ("u", "delta", "A", "B", "C", "state", "y")}
+    assert _step(lib, _shape(seqlen=1, batch=0), nulls) == 0
+    assert _step(lib, _shape(seqlen=1, dim=0), nulls) == 0
