@@ -437,6 +437,47 @@ def measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None
             "gpu_launches": k}
 
 
+def measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None, width=4):
+    """Causal depthwise conv1d + SiLU over the layer's x_proj shape (batch, d_inner, L)."""
+    w = w or synth.WORKLOADS["mamba-2.8b-layer"]
+    x = to_torch(synth.normal((w.batch, w.dim, w.seqlen), w.seed, "u", w.dtype), dev)
+    g = np.random.default_rng(w.seed)
+    wt = torch.from_numpy((g.standard_normal((w.dim, width)) / 2).astype(np.float32)).to(dev)
+    bt = torch.from_numpy(g.standard_normal(w.dim).astype(np.float32)).to(dev)
+    out = torch.empty_like(x)
+    fs = torch.empty((w.batch, w.dim, width - 1), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssm.causal_conv1d(x, wt, bt, out=out, final_state=fs)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    k = max(3, min(args.steps, 20))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(k):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / k)
+    es = x.element_size()
+    nbytes = 2 * es * w.bld + 4 * w.batch * w.dim * (width - 1) + 4 * w.dim * (width + 1)
+    pk = peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
+            "width": width, "io_dtype": w.dtype, "silu": True, "steps": k,
+            "l2": "inputs larger than L2 (no flush)", "ms_per_step": ms,
+            "value": aggregate_value(world, w.bld, ms * 1e-3), "unit": UNIT,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": "k_conv",
+                         "algorithmic_bytes": nbytes,
+                         "peak_basis": f"measured copy bandwidth ({pk['source']})"},
+            "gpu_launches": k}
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -577,10 +618,11 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
         del host, dbuf
 
-    bwd = dec = None
+    bwd = dec = conv = None
     if not args.no_bwd and not args.batch:
         bwd = measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks)
         dec = measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks)
+        conv = measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks)
 
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -606,7 +648,7 @@ def main():
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
-            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec,
+            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec, "conv1d": conv,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, case)

@@ -191,6 +191,27 @@ ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delt
                          const float *D, const void *z, const float *delta_bias,
                          int delta_softplus, float *state, void *y, ssm_stream_t stream);
 
+/* Causal depthwise 1-D convolution along seqlen, then SiLU if `silu`: the
+ * convolution layer the Mamba block applies to x_proj before the SSM, whose
+ * output goes through SiLU to become the SSM input ("O que e um modelo
+ * Mamba?", ibm.com, the Mamba block walk-through).  Per channel d:
+ *   out_t = act(bias[d] + sum_{k < width} weight[d][k] * x_{t - width + 1 + k})
+ * so weight[d][width-1] multiplies the current token.  Inputs before t = 0
+ * come from initial_state (zeros when NULL); final_state receives the last
+ * width-1 inputs, so that a sequence can be convolved in pieces.
+ *  x, out                     [batch][dim][seqlen]  io dtype (io_dtype)
+ *  weight                     [dim][width] fp32, required
+ *  bias                       [dim] fp32, nullable
+ *  initial_state, final_state [batch][dim][width-1] fp32, nullable
+ *                             (oldest input first; unused when width == 1)
+ * width is 1..8 (SSM_ERR_UNSUPPORTED above).  out may not alias x.  Rows
+ * whose bytes are a multiple of 16 on 16-byte aligned buffers take vector
+ * loads and stores. */
+ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
+                             int32_t io_dtype, const void *x, const float *weight,
+                             const float *bias, const float *initial_state, int silu,
+                             void *out, float *final_state, ssm_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word of
  * `workspace`.  SSM_OK, SSM_ERR_DEVICE_TIMEOUT or SSM_ERR_CUDA. */
 ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream);

@@ -5,11 +5,12 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
 package.  The product path (``selective_state_space_54_b200``) never does:
 it has no CPU fallback.
 
-The arithmetic lives in ``ssm_oracle.c`` (a plain per-channel loop, fp64,
-libm ``exp``/``log1p``/``expm1``); this module only widens the stored inputs
+The scan's arithmetic lives in ``ssm_oracle.c`` (a plain per-channel loop,
+fp64, libm ``exp``/``log1p``/``expm1``); this module widens the stored inputs
 to fp64 (exactly), calls it and returns numpy arrays.  See the header of
 ``ssm_oracle.c`` for the equations and the passages of the Mamba pages they
-follow.
+follow.  The causal convolution of the Mamba block (``conv1d``) is written
+here directly in numpy, fp64, as its definition: a sum of shifted inputs.
 """
 from __future__ import annotations
 
@@ -123,3 +124,31 @@ def bwd(case: dict, dout, *, delta_softplus: bool = True, h0=None,
     if rc != 0:
         raise RuntimeError(f"oracle_bwd failed: {rc}")
     return g
+
+
+def conv1d(x, weight, bias=None, *, dtype=None, initial_state=None, silu: bool = True):
+    """Causal depthwise 1-D convolution along seqlen, then SiLU.
+
+    The convolution layer the Mamba block applies to x_proj before the SSM,
+    whose output passes through SiLU ("O que e um modelo Mamba?", ibm.com,
+    the Mamba block walk-through).  Per channel d, width K:
+        out_t = act(bias[d] + sum_k weight[d, k] * x_{t-K+1+k}),
+    x_t for t < 0 taken from ``initial_state`` (batch, dim, K-1), zeros if None.
+    Returns (out, final_state): out (batch, dim, L) fp64 and the last K-1
+    inputs (batch, dim, K-1) fp64, oldest first.
+    """
+    xs = _f64(x, dtype)
+    w = np.asarray(weight, np.float64)
+    bt, dm, L = xs.shape
+    K = w.shape[1]
+    prev = np.zeros((bt, dm, K - 1)) if initial_state is None else \
+        np.asarray(initial_state, np.float64).reshape(bt, dm, K - 1)
+    xp = np.concatenate([prev, xs], axis=-1)  # x_{-(K-1)} .. x_{L-1}
+    out = np.zeros((bt, dm, L))
+    for k in range(K):
+        out += w[None, :, k, None] * xp[:, :, k:k + L]
+    if bias is not None:
+        out += np.asarray(bias, np.float64)[None, :, None]
+    if silu:
+        out = out / (1.0 + np.exp(-out))
+    return out, xp[:, :, L:L + K - 1].copy()

@@ -21,7 +21,7 @@ from . import _lib
 from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_PATH_AUTO, SSM_PATH_LOOKBACK,  # noqa: F401
                    SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L, ssm_shape)
 
-__all__ = ["scan_fwd", "scan_bwd", "scan_step", "fwd_workspace_bytes", "bwd_workspace_bytes",
+__all__ = ["scan_fwd", "scan_bwd", "scan_step", "causal_conv1d", "fwd_workspace_bytes", "bwd_workspace_bytes",
            "fwd_path", "check", "ScanError", "make_shape"]
 
 
@@ -160,6 +160,35 @@ def scan_step(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, state,
     if rc != 0:
         raise ScanError(rc, "ssm_scan_step")
     return y
+
+
+def causal_conv1d(x, weight, bias=None, *, initial_state=None, silu=True, out=None,
+                  return_final_state=False, final_state=None, stream=None):
+    """Causal depthwise conv1d along seqlen (+ SiLU); x, out (batch, dim, seqlen),
+    weight (dim, width) fp32, states (batch, dim, width - 1) fp32."""
+    import torch
+    batch, dim, seqlen = x.shape
+    width = weight.shape[-1]
+    dev = x.device
+    f32 = torch.float32
+    _check_io("x", x, (batch, dim, seqlen), x.dtype, dev)
+    _check_io("weight", weight, (dim, width), f32, dev)
+    _check_io("bias", bias, (dim,), f32, dev)
+    _check_io("initial_state", initial_state, (batch, dim, width - 1), f32, dev)
+    if out is None:
+        out = torch.empty_like(x)
+    _check_io("out", out, (batch, dim, seqlen), x.dtype, dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((batch, dim, width - 1), dtype=f32, device=dev)
+    _check_io("final_state", final_state, (batch, dim, width - 1), f32, dev)
+    rc = _lib.load().ssm_causal_conv1d(
+        batch, dim, seqlen, width, _io_dtype(x), _ptr(x), _ptr(weight), _ptr(bias),
+        _ptr(initial_state), int(bool(silu)), _ptr(out), _ptr(final_state), _stream(stream))
+    if rc != 0:
+        raise ScanError(rc, "ssm_causal_conv1d")
+    if return_final_state:
+        return out, final_state
+    return out
 
 
 def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,

@@ -269,6 +269,37 @@ ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delt
   return cuda_status(launch_step(shape->io_dtype, p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
+                             int32_t io_dtype, const void *x, const float *weight,
+                             const float *bias, const float *initial_state, int silu, void *out,
+                             float *final_state, ssm_stream_t stream) {
+  if (batch < 0 || dim < 0 || seqlen < 0 || width < 1) return SSM_ERR_INVALID_ARG;
+  if (width > 8) return SSM_ERR_UNSUPPORTED;
+  if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if ((double)batch * (double)dim * (double)seqlen > 4.0e15) return SSM_ERR_UNSUPPORTED;
+  const int64_t rows = batch * dim;
+  if (rows == 0) return SSM_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = io_dtype == SSM_BF16 ? 2 : 4;
+  if (!weight || !aligned(weight, 4) || !aligned(bias, 4) || !aligned(initial_state, 4) ||
+      !aligned(final_state, 4))
+    return SSM_ERR_INVALID_ARG;
+  if (seqlen == 0) {  // nothing to convolve: the state passes through
+    if (!final_state || width == 1) return SSM_OK;
+    const size_t bytes = sizeof(float) * (size_t)rows * (size_t)(width - 1);
+    return cuda_status(initial_state
+                           ? cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, s)
+                           : cudaMemsetAsync(final_state, 0, bytes, s));
+  }
+  if (!x || !out || !aligned(x, es) || !aligned(out, es)) return SSM_ERR_INVALID_ARG;
+  ConvParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = x; p.w = weight; p.bias = bias; p.s0 = initial_state; p.out = out; p.s1 = final_state;
+  p.batch = batch; p.dim = dim; p.L = seqlen; p.K = width; p.silu = silu ? 1 : 0;
+  p.vec = ((seqlen * (int64_t)es) % 16 == 0) && aligned(x, 16) && aligned(out, 16);
+  return cuda_status(launch_conv(io_dtype, p, s));
+}
+
 size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
   if (check_shape(shape) != SSM_OK) return 0;
   const int NP = fwd_np_for(shape->dstate);

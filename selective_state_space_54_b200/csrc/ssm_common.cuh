@@ -69,6 +69,19 @@ struct StepParams {
   int vec;                             // N % 4 == 0, state/A 16-byte and B/C 4-element aligned
 };
 
+// Causal depthwise conv1d parameters (ssm_conv.cu).
+struct ConvParams {
+  const void *x;                       // [batch][dim][L] io dtype
+  const float *w, *bias;               // [dim][K], [dim]
+  const float *s0;                     // [batch][dim][K-1] inputs before t = 0, nullable
+  void *out;                           // [batch][dim][L] io dtype
+  float *s1;                           // [batch][dim][K-1] last K-1 inputs, nullable
+  int64_t batch, dim, L;
+  int K;
+  int silu;
+  int vec;                             // 16-byte aligned rows: vector loads and stores
+};
+
 // Backward parameters (ssm_bwd.cu).
 struct BwdParams {
   const void *u, *delta, *z, *B, *C, *dout;
@@ -259,6 +272,7 @@ cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);
 cudaError_t launch_step(int io_dtype, const StepParams &p, cudaStream_t s);
+cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,
                                       cudaStream_t s);
 

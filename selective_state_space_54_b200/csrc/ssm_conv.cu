@@ -1,0 +1,183 @@
+// Causal depthwise 1-D convolution along the sequence, with optional SiLU,
+// for sm_100a: the convolution layer the Mamba block applies to x_proj
+// before the SSM, followed by its SiLU activation ("O que e um modelo
+// Mamba?", ibm.com, the walk-through of the Mamba block: the convolution
+// extracts local patterns between neighbouring tokens, its output goes
+// through SiLU and becomes the SSM's input).  Per channel d, width K:
+//   out_t = act(bias[d] + sum_{k<K} w[d][k] * x_{t-K+1+k}),
+// with x_t for t < 0 taken from the caller's initial state (zeros if none).
+//
+// Design (B200): 2 bytes in and 2 out per (b, d, t) in bf16, a few FMAs:
+// bound by HBM.  A warp takes 1024 consecutive steps of one (b, d) row in 4
+// passes; a lane takes 8 steps per pass with one 16-byte load and store,
+// all 4 loads issued before the first pass computes.  The K-1 steps before a
+// lane's chunk come from neighbouring lanes by shuffles, so every input byte
+// is read once.  Input and output are streamed with evict-first hints.
+#include "ssm_common.cuh"
+
+namespace ssm {
+
+constexpr int kConvThreads = 256;
+constexpr int kConvW = 8;                  // steps per lane and pass
+constexpr int kConvR = 4;                  // passes per warp, all loads issued first
+constexpr int kConvSeg = 32 * kConvW * kConvR;  // steps per warp
+
+// raw io vector of 8 values, kept packed until used
+template <typename T> struct Raw8;
+template <> struct Raw8<uint16_t> {
+  uint4 v;
+  __device__ __forceinline__ void load(const uint16_t *row, int64_t t, int64_t L, bool vec) {
+    if (vec && t + 8 <= L) {
+      v = __ldcs(reinterpret_cast<const uint4 *>(row + t));
+    } else {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = (t + 2 * i < L) ? row[t + 2 * i] : 0u;
+        const uint32_t hi = (t + 2 * i + 1 < L) ? row[t + 2 * i + 1] : 0u;
+        w[i] = lo | (hi << 16);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  __device__ __forceinline__ void unpack(float (&o)[8]) const {
+    o[0] = bf16_lo(v.x); o[1] = bf16_hi(v.x); o[2] = bf16_lo(v.y); o[3] = bf16_hi(v.y);
+    o[4] = bf16_lo(v.z); o[5] = bf16_hi(v.z); o[6] = bf16_lo(v.w); o[7] = bf16_hi(v.w);
+  }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *row, int64_t t, int64_t L, bool vec) {
+    if (vec && t + 8 <= L) {
+      a = __ldcs(reinterpret_cast<const float4 *>(row + t));
+      b = __ldcs(reinterpret_cast<const float4 *>(row + t + 4));
+    } else {
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = (t + i < L) ? row[t + i] : 0.f;
+      a = make_float4(o[0], o[1], o[2], o[3]);
+      b = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+  __device__ __forceinline__ void unpack(float (&o)[8]) const {
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+};
+
+// A warp takes kConvSeg consecutive steps of one row in kConvR passes of 256;
+// all passes' loads are issued before the first is used, so each lane keeps
+// kConvR 16-byte loads in flight.  The K-1 steps before a lane's chunk come
+// from the previous lane (shuffle up), or for lane 0 from lane 31 of the
+// previous pass; only the warp's first pass reads them from memory.
+template <typename T, int K>
+__global__ void __launch_bounds__(kConvThreads) k_conv(ConvParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
+  const int64_t L = p.L;
+  const int64_t segs = (L + kConvSeg - 1) / kConvSeg;
+  const int64_t row = warp / segs;
+  if (row >= p.batch * p.dim) return;  // whole warps leave together
+  const int64_t seg = warp - row * segs;
+  const int64_t d = row % p.dim;
+  const T *xr = static_cast<const T *>(p.x) + row * L;
+  T *orow = static_cast<T *>(p.out) + row * L;
+  const bool vec = p.vec != 0;
+  Raw8<T> raw[kConvR];
+#pragma unroll
+  for (int r = 0; r < kConvR; ++r) raw[r].load(xr, seg * kConvSeg + r * 32 * kConvW + lane * kConvW, L, vec);
+  float w[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) w[k] = p.w[d * K + k];
+  const float bias = p.bias ? p.bias[d] : 0.f;
+  float carry[K > 1 ? K - 1 : 1];  // the K-1 inputs before the pass, as lane 31 of the last pass saw them
+#pragma unroll
+  for (int r = 0; r < kConvR; ++r) {
+    const int64_t t0 = seg * kConvSeg + r * 32 * kConvW + lane * kConvW;
+    if (seg * kConvSeg + r * 32 * kConvW >= L) break;  // warp-uniform
+    float v[kConvW];
+    raw[r].unpack(v);
+    float halo[K > 1 ? K - 1 : 1];
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) {
+      const float up = __shfl_up_sync(0xffffffffu, v[kConvW - (K - 1) + i], 1);
+      const float last = __shfl_sync(0xffffffffu, v[kConvW - (K - 1) + i], 31);
+      if (lane > 0) {
+        halo[i] = up;
+      } else if (r > 0) {
+        halo[i] = carry[i];
+      } else {
+        const int64_t t = t0 - (K - 1) + i;  // the warp's first pass: memory or the initial state
+        halo[i] = t >= 0 ? IO<T>::get(xr, t) : (p.s0 ? p.s0[row * (K - 1) + (K - 1) + t] : 0.f);
+      }
+      carry[i] = last;
+    }
+    float o[kConvW];
+#pragma unroll
+    for (int i = 0; i < kConvW; ++i) {
+      float acc = bias;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int idx = i - (K - 1) + k;  // position in [halo | v]
+        acc = fmaf(w[k], idx < 0 ? halo[idx + K - 1] : v[idx], acc);
+      }
+      o[i] = p.silu ? silu_fast(acc) : acc;
+    }
+    if (t0 < L) {
+      if (vec && t0 + kConvW <= L) {
+        if constexpr (sizeof(T) == 2) {
+          uint4 q;
+          q.x = pack_bf16x2(o[0], o[1]); q.y = pack_bf16x2(o[2], o[3]);
+          q.z = pack_bf16x2(o[4], o[5]); q.w = pack_bf16x2(o[6], o[7]);
+          __stcs(reinterpret_cast<uint4 *>(orow + t0), q);
+        } else {
+          __stcs(reinterpret_cast<float4 *>(orow + t0), make_float4(o[0], o[1], o[2], o[3]));
+          __stcs(reinterpret_cast<float4 *>(orow + t0 + 4), make_float4(o[4], o[5], o[6], o[7]));
+        }
+      } else {
+        IO<T>::store8(orow, t0, L, false, o);
+      }
+    }
+    // final state: the last K-1 inputs of the row, written by the lane holding step L-1
+    if (K > 1 && p.s1 && t0 <= L - 1 && L - 1 < t0 + kConvW) {
+#pragma unroll
+      for (int i = 0; i < K - 1; ++i) {
+        const int idx = (int)(L - (K - 1) + i - t0);  // position in v, or in halo when negative
+        float val = 0.f;                             // (idx >= -(K - 1) always holds here)
+#pragma unroll
+        for (int m = 0; m < kConvW; ++m)
+          if (m == idx) val = v[m];
+#pragma unroll
+        for (int m = 0; m < K - 1; ++m)
+          if (m - (K - 1) == idx) val = halo[m];
+        p.s1[row * (K - 1) + i] = val;
+      }
+    }
+  }
+}
+
+template <typename T>
+static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
+  const int64_t segs = (p.L + kConvSeg - 1) / kConvSeg;
+  const int64_t warps = p.batch * p.dim * segs;
+  const int64_t blocks = (warps * 32 + kConvThreads - 1) / kConvThreads;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  const unsigned g = (unsigned)blocks;
+  switch (p.K) {
+    case 1: k_conv<T, 1><<<g, kConvThreads, 0, s>>>(p); break;
+    case 2: k_conv<T, 2><<<g, kConvThreads, 0, s>>>(p); break;
+    case 3: k_conv<T, 3><<<g, kConvThreads, 0, s>>>(p); break;
+    case 4: k_conv<T, 4><<<g, kConvThreads, 0, s>>>(p); break;
+    case 5: k_conv<T, 5><<<g, kConvThreads, 0, s>>>(p); break;
+    case 6: k_conv<T, 6><<<g, kConvThreads, 0, s>>>(p); break;
+    case 7: k_conv<T, 7><<<g, kConvThreads, 0, s>>>(p); break;
+    case 8: k_conv<T, 8><<<g, kConvThreads, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s) {
+  return io_dtype == 1 ? launch_conv_t<uint16_t>(p, s) : launch_conv_t<float>(p, s);
+}
+
+}  // namespace ssm

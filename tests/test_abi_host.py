@@ -21,7 +21,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ssm_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ssm_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_and_binding_agree():
@@ -189,3 +189,29 @@ def test_step_empty_problem_is_a_noop(lib):
     nulls = {k: None for k in ("u", "delta", "A", "B", "C", "state", "y")}
     assert _step(lib, _shape(seqlen=1, batch=0), nulls) == 0
     assert _step(lib, _shape(seqlen=1, dim=0), nulls) == 0
+
+
+def _conv(lib, batch=2, dim=4, L=64, K=4, dtype=_lib.SSM_BF16, **ptrs):
+    p = dict(x=16, w=16, bias=None, s0=None, out=16, s1=None)
+    p.update(ptrs)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.ssm_causal_conv1d(batch, dim, L, K, dtype, v(p["x"]), v(p["w"]), v(p["bias"]),
+                                 v(p["s0"]), 1, v(p["out"]), v(p["s1"]), None)
+
+
+def test_conv_rejects_bad_arguments_before_launch(lib):
+    assert _conv(lib, batch=-1) == _lib.SSM_ERR_INVALID_ARG
+    assert _conv(lib, L=-1) == _lib.SSM_ERR_INVALID_ARG
+    assert _conv(lib, K=0) == _lib.SSM_ERR_INVALID_ARG
+    assert _conv(lib, K=9) == _lib.SSM_ERR_UNSUPPORTED
+    assert _conv(lib, dtype=5) == _lib.SSM_ERR_UNSUPPORTED
+    for k in ("x", "w", "out"):
+        assert _conv(lib, **{k: None}) == _lib.SSM_ERR_INVALID_ARG, k
+    assert _conv(lib, x=17) == _lib.SSM_ERR_INVALID_ARG
+    assert _conv(lib, w=6) == _lib.SSM_ERR_INVALID_ARG
+    assert _conv(lib, s1=2) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_conv_empty_problem_is_a_noop(lib):
+    assert _conv(lib, batch=0, x=None, w=None, out=None) == 0
+    assert _conv(lib, dim=0, x=None, w=None, out=None) == 0

@@ -1,0 +1,97 @@
+"""Causal depthwise conv1d (+ SiLU) parity: ssm_causal_conv1d through the C ABI
+against the fp64 oracle, on seeded inputs of the Mamba block's shapes."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import assert_close, to_f64, to_torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(batch, dim, L, K, dtype, seed):
+    x = synth.normal((batch, dim, L), seed, "u", dtype)
+    g = np.random.default_rng(seed)
+    w = (g.standard_normal((dim, K)) / np.sqrt(K)).astype(np.float32)
+    b = g.standard_normal(dim).astype(np.float32)
+    s0 = g.standard_normal((batch, dim, K - 1)).astype(np.float32)
+    return x, w, b, s0
+
+
+def _run(x, w, b, s0, dtype, device, silu=True):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    xt = to_torch(x, dtype, device)
+    f = lambda a: None if a is None else torch.from_numpy(a).to(device)
+    out, fs = ssm.causal_conv1d(xt, f(w), f(b), initial_state=f(s0), silu=silu,
+                                return_final_state=True)
+    torch.cuda.synchronize()
+    return to_f64(out), to_f64(fs)
+
+
+def _check(batch, dim, L, K, dtype, seed, device, with_bias=True, with_state=True, silu=True):
+    x, w, b, s0 = _inputs(batch, dim, L, K, dtype, seed)
+    b = b if with_bias else None
+    s0 = s0 if with_state else None
+    ref, ref_s = oracle.conv1d(x, w, b, dtype=dtype, initial_state=s0, silu=silu)
+    out, fs = _run(x, w, b, s0, dtype, device, silu)
+    assert_close(out, ref, dtype, "out")
+    if K > 1:
+        # the state is a copy of inputs: exact
+        assert np.array_equal(fs, ref_s)
+
+
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 5, 8])
+def test_conv_widths(cuda_device, dtype, K):
+    _check(2, 24, 700, K, dtype, 50 + K, cuda_device)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 7, 8, 9, 255, 256, 257, 1000])
+def test_conv_ragged_lengths(cuda_device, L):
+    _check(2, 5, L, 4, synth.BF16, L, cuda_device)
+
+
+@pytest.mark.parametrize("opt", ["no_bias", "no_state", "no_silu"])
+def test_conv_optional_terms(cuda_device, opt):
+    _check(1, 16, 300, 4, synth.F32, 7, cuda_device, with_bias=opt != "no_bias",
+           with_state=opt != "no_state", silu=opt != "no_silu")
+
+
+def test_conv_streaming_in_pieces(cuda_device):
+    # two calls chained through the state equal one call over the whole sequence
+    import torch
+    import selective_state_space_54_b200 as ssm
+    x, w, b, s0 = _inputs(2, 40, 1000, 4, synth.F32, 9)
+    dev = cuda_device
+    xt = torch.from_numpy(x).to(dev)
+    wt, bt, st = (torch.from_numpy(a).to(dev) for a in (w, b, s0))
+    full, fs = ssm.causal_conv1d(xt, wt, bt, initial_state=st, return_final_state=True)
+    a, sa = ssm.causal_conv1d(xt[:, :, :333].contiguous(), wt, bt, initial_state=st,
+                              return_final_state=True)
+    c, sc = ssm.causal_conv1d(xt[:, :, 333:].contiguous(), wt, bt, initial_state=sa,
+                              return_final_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([a, c], dim=-1), full)
+    assert torch.equal(sc, fs)
+
+
+def test_conv_unaligned_rows_take_the_scalar_path(cuda_device):
+    # L * 2 bytes not a multiple of 16: no vector access, same results
+    _check(3, 7, 77, 4, synth.BF16, 11, cuda_device)
+
+
+def test_conv_full_mamba_2p8b_layer(cuda_device):
+    # the Mamba-2.8B layer's x_proj shape (batch 4, d_inner 5120, L 8192), sampled rows
+    import torch
+    import selective_state_space_54_b200 as ssm
+    w_ = synth.WORKLOADS["mamba-2.8b-layer"]
+    x, w, b, _ = _inputs(w_.batch, w_.dim, w_.seqlen, 4, synth.BF16, 21)
+    out, fs = _run(x, w, b, None, synth.BF16, cuda_device)
+    rows = np.random.default_rng(3).choice(w_.batch * w_.dim, 64, replace=False)
+    for r in rows:
+        bi, d = divmod(int(r), w_.dim)
+        ref, ref_s = oracle.conv1d(x[bi:bi + 1, d:d + 1], w[d:d + 1], b[d:d + 1], dtype=synth.BF16)
+        assert_close(out[bi:bi + 1, d:d + 1], ref, synth.BF16, f"row {r}")
+        assert np.array_equal(fs[bi:bi + 1, d:d + 1], ref_s)

@@ -318,3 +318,51 @@ def test_synth_recipe():
     # RNE: 1+2^-8 is a tie between 1 and 1+2^-7 -> even (1.0)
     assert back[0] == 1.0 and back[1] == 1.0 and back[2] == np.float32(1.0078125)
     assert back[3] == -2.5
+
+
+# -- the causal convolution of the Mamba block (ibm.com walk-through) --------
+def _conv_inputs(seed, bt=2, dm=3, L=40, K=4):
+    g = np.random.default_rng(seed)
+    return (g.standard_normal((bt, dm, L)), g.standard_normal((dm, K)), g.standard_normal(dm),
+            g.standard_normal((bt, dm, K - 1)))
+
+
+def test_conv_matches_numpy_convolve():
+    # a library routine: np.convolve(x, w reversed)[:L] is the causal filter
+    x, w, b, _ = _conv_inputs(1)
+    out, _ = oracle.conv1d(x, w, b, silu=False)
+    for i in range(x.shape[0]):
+        for d in range(x.shape[1]):
+            ref = np.convolve(x[i, d], w[d][::-1])[:x.shape[2]] + b[d]
+            np.testing.assert_allclose(out[i, d], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_conv_identity_and_shift_kernels():
+    x, _, _, _ = _conv_inputs(2)
+    ident = np.zeros((3, 4)); ident[:, 3] = 1.0   # weight on the current token
+    out, st = oracle.conv1d(x, ident, silu=False)
+    assert np.array_equal(out, x)
+    assert np.array_equal(st, x[:, :, -3:])
+    shift = np.zeros((3, 4)); shift[:, 0] = 1.0   # weight on the token 3 steps back
+    out, _ = oracle.conv1d(x, shift, silu=False)
+    assert np.array_equal(out[:, :, 3:], x[:, :, :-3]) and not out[:, :, :3].any()
+
+
+def test_conv_silu_closed_form():
+    x, w, b, _ = _conv_inputs(3)
+    lin, _ = oracle.conv1d(x, w, b, silu=False)
+    act, _ = oracle.conv1d(x, w, b, silu=True)
+    np.testing.assert_allclose(act, lin * (1.0 / (1.0 + np.exp(-lin))), rtol=1e-15)
+
+
+def test_conv_streaming_in_pieces():
+    # convolving [x1 | x2] equals convolving x1, then x2 from x1's final state
+    x, w, b, s0 = _conv_inputs(4, L=50)
+    full, fs = oracle.conv1d(x, w, b, initial_state=s0)
+    a, sa = oracle.conv1d(x[:, :, :17], w, b, initial_state=s0)
+    c, sc = oracle.conv1d(x[:, :, 17:], w, b, initial_state=sa)
+    np.testing.assert_allclose(np.concatenate([a, c], axis=-1), full, rtol=1e-14, atol=1e-14)
+    assert np.array_equal(sc, fs)
+    # shorter than the window: the state shifts through
+    e, se = oracle.conv1d(x[:, :, :2], w, b, initial_state=s0)
+    assert np.array_equal(se, np.concatenate([s0[:, :, 2:], x[:, :, :2]], axis=-1))
