@@ -96,8 +96,21 @@ typedef struct {
   int32_t io_dtype; /* ssm_dtype */
   int32_t path;     /* ssm_path (forward only; ignored by the backward) */
   int32_t lanes;    /* lanes per channel in the forward: 0 = auto, 2 or 4 */
-  int32_t reserved; /* must be 0 */
+  int32_t flags;    /* ssm_flags bits; others must be 0 */
 } ssm_shape;
+
+/* Discretisation of the input term (ssm_shape.flags).
+ *  default             Euler: Bbar = Delta * B, as in the aivaro.ru
+ *                      selective_scan example (section 3).
+ *  SSM_FLAG_ZOH_EXACT  exact zero-order hold for diagonal A, the reading
+ *                      guide's "Metodo" formula Bbar = (Delta A)^-1
+ *                      (exp(Delta A) - I) Delta B, i.e. per state
+ *                      Bbar_n = (exp(Delta A_n) - 1) / A_n * B_n (Delta * B_n
+ *                      where A_n = 0).  Forward on path LOOKBACK (AUTO
+ *                      picks it; other explicit paths return
+ *                      SSM_ERR_UNSUPPORTED) and ssm_scan_step; ssm_scan_bwd
+ *                      returns SSM_ERR_UNSUPPORTED for it. */
+typedef enum { SSM_FLAG_ZOH_EXACT = 1 } ssm_flags;
 
 /* Bytes of workspace ssm_scan_fwd needs for `shape` on the current device
  * (at least 256: the header holding the device error word).  Returns 0 for

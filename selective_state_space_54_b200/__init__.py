@@ -18,8 +18,9 @@ from __future__ import annotations
 import ctypes
 
 from . import _lib
-from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_PATH_AUTO, SSM_PATH_LOOKBACK,  # noqa: F401
-                   SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L, ssm_shape)
+from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_FLAG_ZOH_EXACT, SSM_PATH_AUTO,  # noqa: F401
+                   SSM_PATH_LOOKBACK, SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L,
+                   ssm_shape)
 
 __all__ = ["scan_fwd", "scan_bwd", "scan_step", "causal_conv1d", "fwd_workspace_bytes", "bwd_workspace_bytes",
            "fwd_path", "check", "ScanError", "make_shape"]
@@ -41,8 +42,8 @@ def _io_dtype(t) -> int:
 
 
 def make_shape(batch: int, dim: int, seqlen: int, dstate: int, io_dtype: int,
-               path: int = SSM_PATH_AUTO, lanes: int = 0) -> ssm_shape:
-    return ssm_shape(batch, dim, seqlen, dstate, io_dtype, path, lanes, 0)
+               path: int = SSM_PATH_AUTO, lanes: int = 0, flags: int = 0) -> ssm_shape:
+    return ssm_shape(batch, dim, seqlen, dstate, io_dtype, path, lanes, flags)
 
 
 def fwd_workspace_bytes(shape: ssm_shape) -> int:
@@ -91,8 +92,10 @@ def _workspace(nbytes, device, workspace):
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softplus=True,
              initial_state=None, y=None, last_state=None, return_last_state=False,
-             workspace=None, path: int = SSM_PATH_AUTO, lanes: int = 0, stream=None):
-    """Forward selective scan; returns y, or (y, last_state)."""
+             workspace=None, path: int = SSM_PATH_AUTO, lanes: int = 0, zoh_exact=False,
+             stream=None):
+    """Forward selective scan; returns y, or (y, last_state).  zoh_exact selects the
+    exact zero-order-hold input term instead of the Euler one (Delta * B)."""
     import torch
     batch, dim, seqlen = u.shape
     dstate = B.shape[-1]
@@ -114,7 +117,8 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, dstate), dtype=f32, device=dev)
     _check_io("last_state", last_state, (batch, dim, dstate), f32, dev)
-    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path, lanes)
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path, lanes,
+                       SSM_FLAG_ZOH_EXACT if zoh_exact else 0)
     nbytes = fwd_workspace_bytes(shape)
     if nbytes == 0 and batch * dim * seqlen > 0:
         raise ScanError(_lib.SSM_ERR_UNSUPPORTED, "ssm_scan_fwd_workspace_bytes")
@@ -131,7 +135,7 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
 
 
 def scan_step(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, state,
-              delta_softplus=True, y=None, stream=None):
+              delta_softplus=True, zoh_exact=False, y=None, stream=None):
     """One recurrent step for every (batch, channel): updates `state` in place
     and returns y.  u, delta, z, y (batch, dim); B, C (batch, dstate); state
     (batch, dim, dstate) fp32."""
@@ -153,7 +157,8 @@ def scan_step(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, state,
     if y is None:
         y = torch.empty_like(u)
     _check_io("y", y, (batch, dim), dt, dev)
-    shape = make_shape(batch, dim, 1, dstate, _io_dtype(u))
+    shape = make_shape(batch, dim, 1, dstate, _io_dtype(u),
+                       flags=SSM_FLAG_ZOH_EXACT if zoh_exact else 0)
     rc = _lib.load().ssm_scan_step(
         ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(state), _ptr(y), _stream(stream))

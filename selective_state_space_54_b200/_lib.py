@@ -26,6 +26,8 @@ SSM_PATH_SPLIT_L = 2
 SSM_PATH_PER_GROUP = 3
 SSM_PATH_LOOKBACK_WS = 4
 
+SSM_FLAG_ZOH_EXACT = 1
+
 PATH_NAMES = {SSM_PATH_AUTO: "auto", SSM_PATH_LOOKBACK: "lookback",
               SSM_PATH_SPLIT_L: "split_l", SSM_PATH_PER_GROUP: "per_group",
               SSM_PATH_LOOKBACK_WS: "lookback_ws"}
@@ -43,7 +45,7 @@ class ssm_shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64),
                 ("seqlen", ctypes.c_int64), ("dstate", ctypes.c_int64),
                 ("io_dtype", ctypes.c_int32), ("path", ctypes.c_int32),
-                ("lanes", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("lanes", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 _lib = None

@@ -31,7 +31,9 @@ ssm_status check_shape(const ssm_shape *s) {
   if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_LOOKBACK_WS) return SSM_ERR_UNSUPPORTED;
   if (s->path == SSM_PATH_LOOKBACK_WS && s->lanes == 4) return SSM_ERR_UNSUPPORTED;
   if (s->lanes != 0 && s->lanes != 2 && s->lanes != 4) return SSM_ERR_UNSUPPORTED;
-  if (s->reserved != 0) return SSM_ERR_INVALID_ARG;
+  if (s->flags & ~SSM_FLAG_ZOH_EXACT) return SSM_ERR_INVALID_ARG;
+  if ((s->flags & SSM_FLAG_ZOH_EXACT) && s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK)
+    return SSM_ERR_UNSUPPORTED;
   // index arithmetic is int64; keep every flat index well inside it
   const double elems = (double)s->batch * (double)s->dim * (double)s->seqlen;
   if (elems > 4.0e15 || (double)s->batch * s->seqlen * s->dstate > 4.0e15) return SSM_ERR_UNSUPPORTED;
@@ -84,14 +86,17 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
     else lpc = p.K >= 64 ? 2 : 4;
   }
   const int64_t G = lpc == 2 ? g2 : g4;
+  // the exact-ZOH input term is built into the look-back kernel only
+  const bool zoh = (s->flags & SSM_FLAG_ZOH_EXACT) != 0;
   if (path == SSM_PATH_AUTO) {
-    if (G >= unit) path = lpc == 2 ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
+    if (zoh) path = SSM_PATH_LOOKBACK;
+    else if (G >= unit) path = lpc == 2 ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
     else if (p.K >= 64) path = SSM_PATH_SPLIT_L;
     else path = SSM_PATH_PER_GROUP;
   }
   int occ = 0;
   cudaError_t oe = path == SSM_PATH_LOOKBACK_WS ? fwd_ws_occupancy(s->io_dtype, p.NP, &occ)
-                                                : fwd_occupancy(s->io_dtype, p.NP, lpc, &occ);
+                                                : fwd_occupancy(s->io_dtype, p.NP, lpc, zoh, &occ);
   if (oe != cudaSuccess || occ <= 0) {
     cudaGetLastError();
     return SSM_ERR_CUDA;
@@ -213,6 +218,7 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
   p.y = y; p.last_state = last_state;
   p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = (int)shape->dstate;
   p.softplus = delta_softplus ? 1 : 0;
+  p.zoh = (shape->flags & SSM_FLAG_ZOH_EXACT) ? 1 : 0;
   p.io_vec = ((shape->seqlen * es) % 16 == 0) && aligned(u, 16) && aligned(delta, 16) &&
              aligned(z, 16) && aligned(y, 16);
   p.bc_vec = (shape->dstate == pl.NP) && ((shape->dstate * es) % 16 == 0) && aligned(B, 16) &&
@@ -264,6 +270,7 @@ ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delt
   p.A = A; p.D = D; p.bias = delta_bias; p.state = state; p.y = y;
   p.batch = shape->batch; p.dim = shape->dim; p.N = (int)shape->dstate;
   p.softplus = delta_softplus ? 1 : 0;
+  p.zoh = (shape->flags & SSM_FLAG_ZOH_EXACT) ? 1 : 0;
   p.vec = shape->dstate % 4 == 0 && aligned(state, 16) && aligned(A, 16) &&
           aligned(B, 4 * es) && aligned(C, 4 * es);
   return cuda_status(launch_step(shape->io_dtype, p, reinterpret_cast<cudaStream_t>(stream)));
@@ -320,6 +327,7 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
                         size_t ws_bytes, ssm_stream_t stream) {
   ssm_status st = check_shape(shape);
   if (st != SSM_OK) return st;
+  if (shape->flags & SSM_FLAG_ZOH_EXACT) return SSM_ERR_UNSUPPORTED;  // Euler backward only
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t batch = shape->batch, dim = shape->dim, L = shape->seqlen, N = shape->dstate;
   const size_t es = shape->io_dtype == SSM_BF16 ? 2 : 4;

@@ -39,6 +39,7 @@ struct FwdParams {
   int64_t batch, dim, L;
   int N;
   int softplus;
+  int zoh;      // exact zero-order-hold input term instead of Euler
   int io_vec;   // u/delta/z/y rows 16-byte aligned: vector loads
   int bc_vec;   // B/C chunk blocks 16-byte aligned and N == NP
   int64_t gpb;        // channel groups per batch element
@@ -66,6 +67,7 @@ struct StepParams {
   int64_t batch, dim;
   int N;
   int softplus;
+  int zoh;                             // exact zero-order-hold input term instead of Euler
   int vec;                             // N % 4 == 0, state/A 16-byte and B/C 4-element aligned
 };
 
@@ -230,6 +232,25 @@ __device__ __forceinline__ float silu_fast(float z) {
   return z * rcp_approx(1.f + ex2(-z * kLog2e));
 }
 
+// Exact zero-order hold for diagonal A: Bbar_n / (Delta B_n) = (e^x - 1) / x
+// with x = Delta A_n, given x2 = x / ln 2 (the ex2 argument) and a = 2^x2.
+// For |x| < 1/2 the Taylor series sum_k x^k / (k+1)!, k <= 7 (remainder below
+// 1.1e-8); otherwise (a - 1) / x, where a - 1 loses nothing (|a - 1| > 0.39).
+// x = 0 (A_n = 0 or Delta = 0) gives 1: the Euler term, the exact limit.
+constexpr float kLn2 = 0.6931471805599453f;
+__device__ __forceinline__ float expm1_over_x(float x2, float a) {
+  const float x = x2 * kLn2;
+  float q = 2.48015873015873e-05f;         // 1/8!
+  q = fmaf(q, x, 1.984126984126984e-04f);  // 1/7!
+  q = fmaf(q, x, 1.388888888888889e-03f);  // 1/6!
+  q = fmaf(q, x, 8.333333333333333e-03f);  // 1/5!
+  q = fmaf(q, x, 4.166666666666667e-02f);  // 1/4!
+  q = fmaf(q, x, 1.666666666666667e-01f);  // 1/3!
+  q = fmaf(q, x, 0.5f);                    // 1/2!
+  q = fmaf(q, x, 1.f);
+  return fabsf(x) < 0.5f ? q : (a - 1.f) * rcp_approx(x);
+}
+
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -262,7 +283,7 @@ __device__ __forceinline__ bool warp_wait_flag(const unsigned *flag, unsigned *e
 
 // ---- launchers (defined in ssm_fwd.cu / ssm_bwd.cu) ----------------------------
 int fwd_np_for(int64_t N);
-cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm);
+cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int zoh, int *ctas_per_sm);
 cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 int fwd_ws_chunk();

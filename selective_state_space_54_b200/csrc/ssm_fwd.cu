@@ -306,7 +306,7 @@ __device__ __forceinline__ void write_last_state(const FwdParams &p, const Lane 
 // ---- the chunk loop ------------------------------------------------------------------
 // Walk chunks [k0, k1) of the lane's channel group from state h.
 // EMIT: write y (output pass); otherwise advance h and sum Delta (split-L pass 1).
-template <typename T, int NP, int LPC, bool EMIT>
+template <typename T, int NP, int LPC, bool EMIT, bool ZOH = false>
 __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP, LPC> &sm, const Lane &ln,
                                            int64_t k0, int64_t k1, float (&h)[NP / LPC],
                                            float &dsum) {
@@ -387,6 +387,36 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP, LPC> 
     if (k + 1 < k1) issue_loads(k + 1);
 
     // ---- the recurrence: kT steps, S states per lane ----
+    if constexpr (ZOH) {  // exact zero-order hold: Bbar_n = Delta * (e^x - 1) / x * B_n, x = Delta A_n
+#pragma unroll 1
+      for (int tt = 0; tt < kT; tt += 4) {
+        float yp[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float dl = sm.dl[c][tt + i], du = sm.dlu[c][tt + i];
+          const float *Brow = &sm.Bs[tt + i][j * S];
+          const float *Crow = &sm.Cs[tt + i][j * S];
+          float acc = 0.f;
+#pragma unroll
+          for (int s = 0; s < S; ++s) {
+            const float x2 = dl * A2[s];
+            const float a = ex2(x2);
+            h[s] = fmaf(a, h[s], du * expm1_over_x(x2, a) * Brow[s]);
+            if (EMIT) acc = fmaf(Crow[s], h[s], acc);
+          }
+          yp[i] = acc;
+          if (!EMIT) dsum += dl;
+        }
+        if (EMIT) {
+          if constexpr (LPC == 4) {
+            sm.ys[c][tt + j] = reduce4_transpose(yp[0], yp[1], yp[2], yp[3], j);
+          } else {
+            sm.ys[c][tt + j] = reduce2_transpose(yp[0], yp[1], j);
+            sm.ys[c][tt + 2 + j] = reduce2_transpose(yp[2], yp[3], j);
+          }
+        }
+      }
+    } else {
 #pragma unroll 2
     for (int tt = 0; tt < kT; tt += 4) {
       const float4 d4 = *reinterpret_cast<const float4 *>(&sm.dl[c][tt]);
@@ -435,6 +465,7 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP, LPC> 
         }
       }
     }
+    }
 
     // ---- epilogue: D skip, gate, store this lane's STEPS steps ----
     if (EMIT) {
@@ -470,7 +501,7 @@ __device__ __forceinline__ void run_chunks(const FwdParams &p, FwdSmem<NP, LPC> 
 // previous warp published from ITS head, is done last.  The bounded wait
 // therefore only spins if the previous warp has not finished its first item
 // by the time this warp has finished everything else.
-template <typename T, int NP, int LPC>
+template <typename T, int NP, int LPC, bool ZOH>
 __global__ void __launch_bounds__(kThreads) k_fwd_lookback(FwdParams p) {
   constexpr int S = NP / LPC, CPW = 32 / LPC;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -510,7 +541,7 @@ __global__ void __launch_bounds__(kThreads) k_fwd_lookback(FwdParams p) {
     } else {
       init_state<NP, LPC>(p, ln, h);
     }
-    run_chunks<T, NP, LPC, true>(p, sm, ln, k0, k1, h, dsum);
+    run_chunks<T, NP, LPC, true, ZOH>(p, sm, ln, k0, k1, h, dsum);
     if (k1 < K) {  // publish the head's end state for warp w + 1
 #pragma unroll
       for (int s = 0; s < S; ++s) p.carry[(w * CPW + ln.c) * NP + ln.j * S + s] = h[s];
@@ -1090,15 +1121,15 @@ static cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm) {
+cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int zoh, int *ctas_per_sm) {
   return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
     const size_t smem = fwd_smem_bytes<kNP, kLPC>();
-    cudaError_t e = allow_smem(k_fwd_lookback<T, kNP, kLPC>, smem);
+    auto kern = zoh ? k_fwd_lookback<T, kNP, kLPC, true> : k_fwd_lookback<T, kNP, kLPC, false>;
+    cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_lookback<T, kNP, kLPC>,
-                                                         kThreads, smem);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, kern, kThreads, smem);
   });
 }
 
@@ -1107,10 +1138,11 @@ cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
     const size_t smem = fwd_smem_bytes<kNP, kLPC>();
-    cudaError_t e = allow_smem(k_fwd_lookback<T, kNP, kLPC>, smem);
+    auto kern = p.zoh ? k_fwd_lookback<T, kNP, kLPC, true> : k_fwd_lookback<T, kNP, kLPC, false>;
+    cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.n_workers + kWarps - 1) / kWarps);
-    k_fwd_lookback<T, kNP, kLPC><<<grid, kThreads, smem, s>>>(p);
+    kern<<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }

@@ -104,8 +104,12 @@ __global__ void __launch_bounds__(kStepThreads) k_step(StepParams p) {
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int i = 0; i < S; i += 2) {
-      h[i] = fmaf(ex2(dl * a[i] * kLog2e), h[i], du * Bv[i]);
-      h[i + 1] = fmaf(ex2(dl * a[i + 1] * kLog2e), h[i + 1], du * Bv[i + 1]);
+      const float x0 = dl * a[i] * kLog2e, x1 = dl * a[i + 1] * kLog2e;
+      const float e0 = ex2(x0), e1 = ex2(x1);
+      const float b0 = p.zoh ? du * expm1_over_x(x0, e0) : du;
+      const float b1 = p.zoh ? du * expm1_over_x(x1, e1) : du;
+      h[i] = fmaf(e0, h[i], b0 * Bv[i]);
+      h[i + 1] = fmaf(e1, h[i + 1], b1 * Bv[i + 1]);
       y0 = fmaf(Cv[i], h[i], y0);  // states past N have C = 0 and h = 0
       y1 = fmaf(Cv[i + 1], h[i + 1], y1);
     }
@@ -233,8 +237,12 @@ __global__ void __launch_bounds__(kStepThreads) k_step_rows(StepParams p) {
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int i = 0; i < S; i += 2) {
-      h[i] = fmaf(ex2(dl * a[i]), h[i], du * Bv[i]);
-      h[i + 1] = fmaf(ex2(dl * a[i + 1]), h[i + 1], du * Bv[i + 1]);
+      const float x0 = dl * a[i], x1 = dl * a[i + 1];  // a holds A * log2(e)
+      const float e0 = ex2(x0), e1 = ex2(x1);
+      const float b0 = p.zoh ? du * expm1_over_x(x0, e0) : du;
+      const float b1 = p.zoh ? du * expm1_over_x(x1, e1) : du;
+      h[i] = fmaf(e0, h[i], b0 * Bv[i]);
+      h[i + 1] = fmaf(e1, h[i + 1], b1 * Bv[i + 1]);
       y0 = fmaf(Cv[i], h[i], y0);
       y1 = fmaf(Cv[i + 1], h[i + 1], y1);
     }

@@ -215,3 +215,15 @@ def test_conv_rejects_bad_arguments_before_launch(lib):
 def test_conv_empty_problem_is_a_noop(lib):
     assert _conv(lib, batch=0, x=None, w=None, out=None) == 0
     assert _conv(lib, dim=0, x=None, w=None, out=None) == 0
+
+
+def test_flags_checked_before_launch(lib):
+    assert _fwd(lib, _shape(flags=2)) == _lib.SSM_ERR_INVALID_ARG
+    # exact ZOH runs on the look-back path only; other explicit paths are refused
+    for path in (_lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP, _lib.SSM_PATH_LOOKBACK_WS):
+        assert _fwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path)) == \
+            _lib.SSM_ERR_UNSUPPORTED
+        assert lib.ssm_scan_fwd_workspace_bytes(
+            ctypes.byref(_shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path))) == 0
+    # the backward is Euler only
+    assert _bwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED

@@ -251,3 +251,67 @@ def test_full_million_length(cuda_device):
 
 def test_full_mamba_1p4b_layer_forward(cuda_device):
     _full_size("mamba-1.4b-layer-train", cuda_device, sample=64)
+
+
+# ---- exact zero-order hold (the reading guide's "Metodo" discretisation) ----
+def _run_zoh(case, device, path="auto", lanes=0, h0=None):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    g = upload(case, device)
+    h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
+    y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                         g["delta_bias"], initial_state=h0_t, return_last_state=True,
+                         path=PATHS[path], lanes=lanes, zoh_exact=True)
+    torch.cuda.synchronize()
+    return to_f64(y), to_f64(ls)
+
+
+@pytest.mark.parametrize("lanes", [0, 2, 4])
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("N", [1, 4, 16, 64])
+def test_zoh_exact_matches_oracle(cuda_device, dtype, N, lanes):
+    case = synth.make_case(2, 40, 333, N, dtype, seed=400 + N)
+    ref = oracle.fwd(case, zoh_exact=True)
+    y, ls = _run_zoh(case, cuda_device, "lookback" if lanes else "auto", lanes)
+    assert_close(y, ref["y"], dtype, "y")
+    assert_close(ls, ref["last_state"], dtype, "last_state", stored_bf16=False)
+
+
+def test_zoh_exact_with_initial_state_and_large_steps(cuda_device):
+    # Delta A spans both branches of (e^x - 1) / x (|x| < 1/2 and beyond)
+    case = synth.make_case(1, 64, 200, 16, synth.F32, seed=410)
+    case["delta_bias"] = np.full(64, 1.5, np.float32)
+    h0 = np.random.default_rng(5).standard_normal((1, 64, 16)).astype(np.float32)
+    ref = oracle.fwd(case, zoh_exact=True, h0=h0)
+    y, ls = _run_zoh(case, cuda_device, h0=h0)
+    assert_close(y, ref["y"], synth.F32, "y")
+    assert_close(ls, ref["last_state"], synth.F32, "last_state")
+
+
+def test_zoh_exact_gate_reduction(cuda_device):
+    # N = 1, A = -1, B = 1, C = 1, no D, no z: exp(-softplus(s)) = sigmoid(-s), so
+    # h_t = (1 - sigmoid(s_t)) h_{t-1} + sigmoid(s_t) u_t exactly (reading guide,
+    # the question on Delta and recurrent gating)
+    L = 500
+    case = synth.make_case(1, 8, L, 1, synth.F32, seed=411, with_z=False, with_D=False)
+    case["A"] = -np.ones((8, 1), np.float32)
+    case["B"] = np.ones((1, L, 1), np.float32)
+    case["C"] = np.ones((1, L, 1), np.float32)
+    y, _ = _run_zoh(case, cuda_device)
+    s = case["delta"].astype(np.float64) + case["delta_bias"].astype(np.float64)[None, :, None]
+    sig = 1.0 / (1.0 + np.exp(-s))
+    u = case["u"].astype(np.float64)
+    h = np.zeros((1, 8))
+    ref = np.zeros_like(u)
+    for t in range(L):
+        h = (1 - sig[:, :, t]) * h + sig[:, :, t] * u[:, :, t]
+        ref[:, :, t] = h
+    assert_close(y, ref, synth.F32, "gate recurrence")
+
+
+def test_zoh_exact_is_not_euler(cuda_device):
+    case = synth.make_case(1, 32, 128, 16, synth.F32, seed=412)
+    case["delta_bias"] = np.full(32, 0.5, np.float32)
+    y_zoh, _ = _run_zoh(case, cuda_device)
+    y_eul, _ = _run(case, cuda_device)
+    assert np.linalg.norm(y_zoh - y_eul) > 1e-2 * np.linalg.norm(y_eul)

@@ -149,3 +149,21 @@ def test_step_full_decode_workload(cuda_device):
     h0 = _state(w.batch, w.dim, w.dstate, 7)
     _check(case, cuda_device, h0)
 
+
+
+@pytest.mark.parametrize("N", [4, 16, 12])
+def test_step_zoh_exact_matches_oracle(cuda_device, N):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    case = synth.make_case(3, 64, 1, N, synth.F32, seed=500 + N)
+    case["delta_bias"] = np.linspace(-4, 2, 64).astype(np.float32)  # both (e^x - 1)/x branches
+    h0 = _state(3, 64, N, 9)
+    ref = oracle.fwd(case, h0=h0, zoh_exact=True)
+    g = upload(case, cuda_device)
+    x = _step_inputs(g, 0)
+    st = torch.from_numpy(h0).to(cuda_device)
+    y = ssm.scan_step(x["u"], x["delta"], g["A"], x["B"], x["C"], g["D"], x["z"], g["delta_bias"],
+                      state=st, zoh_exact=True)
+    torch.cuda.synchronize()
+    assert_close(to_f64(y), ref["y"][:, :, 0], synth.F32, "y")
+    assert_close(to_f64(st), ref["last_state"], synth.F32, "state")
