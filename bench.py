@@ -337,9 +337,21 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     barrier()
     ms_f = max_over_ranks(t_f / steps)
     ms_b = max_over_ranks(t_b / steps)
+    # the backward's special-function work: ex2 of the checkpoint pass, the
+    # recomputation and the reverse pass, one each per (b, t, d, n) element
+    pk = peaks()
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
+    bwd_achieved = 3 * w.bldn / (ms_b * 1e-3)
+    bwd_roofline = {"bound": "alu", "achieved": bwd_achieved / 1e12, "peak": ex2_peak / 1e12,
+                    "unit": "Tex2/s", "frac": bwd_achieved / ex2_peak, "traffic": None,
+                    "kernel": "k_bwd", "ex2_per_element": 3,
+                    "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
+                                  f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
             "d_state": w.dstate, "io_dtype": w.dtype, "steps": steps,
             "fwd_path": ssm.fwd_path(shape), "fwd_ms": ms_f, "bwd_ms": ms_b,
+            "bwd_roofline": bwd_roofline,
             "value": aggregate_value(world, w.bld, (ms_f + ms_b) * 1e-3), "unit": UNIT + " (fwd+bwd)",
             "bwd_value": aggregate_value(world, w.bld, ms_b * 1e-3),
             "bwd_ex2_per_element": 3,
@@ -527,7 +539,7 @@ def main():
                 "ms_per_step": tr["fwd_ms"] + tr["bwd_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": dict(config_of(w, tr["fwd_path"]), step="fwd+bwd"), "bwd": tr,
-                "gpu_launches": 3 * tr["steps"]}
+                "roofline": tr["bwd_roofline"], "gpu_launches": 3 * tr["steps"]}
         if rank == 0:
             print(json.dumps(line), flush=True)
         if world > 1:
