@@ -96,3 +96,8 @@ def test_bwd_full_mamba_1p4b_layer(cuda_device):
     case = synth.make_workload(w)
     stats = _check(case, cuda_device)
     assert set(stats) >= {"du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias"}
+
+
+def test_bwd_single_step_and_single_channel(cuda_device):
+    _check(_case(1, 1, 1, 16, synth.F32, 78), cuda_device)
+    _check(_case(1, 3, 2, 4, synth.BF16, 79), cuda_device)

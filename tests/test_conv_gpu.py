@@ -95,3 +95,16 @@ def test_conv_full_mamba_2p8b_layer(cuda_device):
         ref, ref_s = oracle.conv1d(x[bi:bi + 1, d:d + 1], w[d:d + 1], b[d:d + 1], dtype=synth.BF16)
         assert_close(out[bi:bi + 1, d:d + 1], ref, synth.BF16, f"row {r}")
         assert np.array_equal(fs[bi:bi + 1, d:d + 1], ref_s)
+
+
+def test_conv_zero_length_passes_the_state_through(cuda_device):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    dev = cuda_device
+    x = torch.zeros((2, 6, 0), dtype=torch.bfloat16, device=dev)
+    w = torch.randn((6, 4), device=dev)
+    s0 = torch.randn((2, 6, 3), device=dev)
+    out, fs = ssm.causal_conv1d(x, w, initial_state=s0, return_final_state=True)
+    out2, fs2 = ssm.causal_conv1d(x, w, return_final_state=True)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and torch.equal(fs, s0) and not fs2.any()

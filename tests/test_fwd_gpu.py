@@ -315,3 +315,23 @@ def test_zoh_exact_is_not_euler(cuda_device):
     y_zoh, _ = _run_zoh(case, cuda_device)
     y_eul, _ = _run(case, cuda_device)
     assert np.linalg.norm(y_zoh - y_eul) > 1e-2 * np.linalg.norm(y_eul)
+
+
+# ---- degenerate sizes ----------------------------------------------------------
+def test_zero_length_passes_the_state_through(cuda_device):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    dev = cuda_device
+    u = torch.zeros((2, 8, 0), dtype=torch.bfloat16, device=dev)
+    Bm = torch.zeros((2, 0, 16), dtype=torch.bfloat16, device=dev)
+    A = torch.from_numpy(synth.s4d_real_A(8, 16)).to(dev)
+    h0 = torch.randn((2, 8, 16), device=dev)
+    y, ls = ssm.scan_fwd(u, u, A, Bm, Bm, initial_state=h0, return_last_state=True)
+    y2, ls2 = ssm.scan_fwd(u, u, A, Bm, Bm, return_last_state=True)
+    torch.cuda.synchronize()
+    assert y.numel() == 0 and torch.equal(ls, h0) and not ls2.any()
+
+
+def test_single_channel_single_step(cuda_device):
+    for dtype in (synth.F32, synth.BF16):
+        _check(synth.make_case(1, 1, 1, 16, dtype, seed=77), cuda_device)

@@ -167,3 +167,11 @@ def test_step_zoh_exact_matches_oracle(cuda_device, N):
     torch.cuda.synchronize()
     assert_close(to_f64(y), ref["y"][:, :, 0], synth.F32, "y")
     assert_close(to_f64(st), ref["last_state"], synth.F32, "state")
+
+
+def test_step_batch_beyond_the_grid_y_limit(cuda_device):
+    # more row groups than one grid dimension holds (4 * 65535 rows): the
+    # one-row-per-block kernel with its row loop takes over
+    batch, dim, N = 270000, 1, 16
+    case = synth.make_case(batch, dim, 1, N, synth.BF16, seed=16)
+    _check(case, cuda_device, _state(batch, dim, N, 10))
