@@ -92,10 +92,10 @@ struct __align__(16) BwdWarpSmem {
   float dy[kBCPW][kTB + kBPad];    // dout * SiLU(z)
   float ys[kBCPW][kTB + kBPad];    // sum_n C h
   float2 pd[kBCPW][kTB][4];        // per lane j: (sum_n g A a h_prev, sum_n g B) partials
-  // dB, dC contributions of half a chunk: [step][B|C][lane slice j][channel, state]
-  // with 8 floats of padding per row so that a quarter warp's stores hit
-  // distinct banks
-  float part[kTB / 2][2][4][kBCPW * (NP / 4) + 8];
+  // dB, dC contributions of a 4-step group: [step][B|C][lane slice j][channel,
+  // state] with 8 floats of padding per row so that a quarter warp's stores
+  // hit distinct banks
+  float part[4][2][4][kBCPW * (NP / 4) + 8];
 };
 
 template <int NP>
@@ -189,7 +189,7 @@ __device__ __forceinline__ bf2 bex2(bf2 x) {
 }
 
 template <typename T, int NP>
-__global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
+__global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4 ? 3 : 2)) k_bwd(BwdParams p) {
   constexpr int S = NP / 4;              // states per lane
   constexpr int SP = S >= 2 ? S / 2 : 1; // state pairs per lane (S = 1 pads one)
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
 #pragma unroll
   for (int i = 0; i < SP; ++i) { g[i] = bpack(0.f, 0.f); dA_acc[i] = g[i]; }
   float dD_acc = 0.f, dbias_acc = 0.f;
-  constexpr int kRedOutputs = (kTB / 2) * 2 * NP / 4;   // float4 outputs of a half chunk
+  constexpr int kRedOutputs = 4 * 2 * NP / 4;   // float4 outputs of a 4-step group
   if (K > 0) load_chunk(K - 1, true, nxt);
   for (int64_t k = K - 1; k >= 0; --k) {
     const int64_t t0 = k * kTB;
@@ -348,16 +348,22 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     stage_chunk(t0, cur, true);
     __syncthreads();
 
-    // recompute the chunk's states from its checkpoint
-    bf2 H[kTB][SP], h0c[SP];
+    // recompute the chunk's states from its checkpoint, keeping only the
+    // state entering each 4-step group (the reverse pass recomputes a group's
+    // states again right before it needs them)
+    bf2 H4[kTB / 4][SP];
+    {
+      bf2 hh[SP];
 #pragma unroll
-    for (int i = 0; i < SP; ++i) {
-      const float *src = ck_at(k, i);
-      h0c[i] = bpack(src[0], S >= 2 ? src[1] : 0.f);
-    }
+      for (int i = 0; i < SP; ++i) {
+        const float *src = ck_at(k, i);
+        hh[i] = bpack(src[0], S >= 2 ? src[1] : 0.f);
+      }
 #pragma unroll
     for (int t = 0; t < kTB; t += 4) {
       float yp[4];
+#pragma unroll
+      for (int i = 0; i < SP; ++i) H4[t / 4][i] = hh[i];
 #pragma unroll
       for (int i4 = 0; i4 < 4; ++i4) {
         const int tt = t + i4;
@@ -365,9 +371,8 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
         bf2 acc = bpack(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
-          const bf2 hp = tt == 0 ? h0c[i] : H[tt - 1][i];
-          H[tt][i] = bfma(bex2(bmul(dl2, A2[i])), hp, bmul(du2, Bpair(tt, i)));
-          acc = bfma(Cpair(tt, i), H[tt][i], acc);
+          hh[i] = bfma(bex2(bmul(dl2, A2[i])), hh[i], bmul(du2, Bpair(tt, i)));
+          acc = bfma(Cpair(tt, i), hh[i], acc);
         }
         float a0, a1;
         bunpack(acc, a0, a1);
@@ -381,6 +386,7 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
       float kk = hi1 ? kb : ka;
       kk += __shfl_xor_sync(0xffffffffu, hi1 ? ka : kb, 1);
       ws.ys[c][t + j] = kk;
+    }
     }
     __syncwarp();
 
@@ -409,30 +415,42 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
     }
     __syncwarp();
 
-    // reverse recurrence over the chunk, in two halves; after each half the
-    // CTA sums its 32 channels' dB/dC contributions and adds them to the
-    // fp32 accumulators
+    // reverse recurrence over the chunk, in 4-step groups: each group's states
+    // and decays are recomputed from the state entering it, then walked in
+    // reverse; after each group the CTA sums its 32 channels' dB/dC
+    // contributions and adds them to the fp32 accumulators
 #pragma unroll
-    for (int half = 1; half >= 0; --half) {
+    for (int grp = kTB / 4 - 1; grp >= 0; --grp) {
+      bf2 hg[4][SP], ag[4][SP];
 #pragma unroll
-      for (int tl = kTB / 2 - 1; tl >= 0; --tl) {
-        const int t = half * (kTB / 2) + tl;
+      for (int u = 0; u < 4; ++u) {
+        const int t = 4 * grp + u;
+        const float dlv = ws.dl[c][t], duv = ws.dlu[c][t];
+        const bf2 dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
+#pragma unroll
+        for (int i = 0; i < SP; ++i) {
+          ag[u][i] = bex2(bmul(dl2, A2[i]));
+          hg[u][i] = bfma(ag[u][i], u == 0 ? H4[grp][i] : hg[u - 1][i], bmul(du2, Bpair(t, i)));
+        }
+      }
+#pragma unroll
+      for (int u = 3; u >= 0; --u) {
+        const int t = 4 * grp + u;
         const float dyv = ws.dy[c][t], dlv = ws.dl[c][t], duv = ws.dlu[c][t];
         const bf2 dy2 = bpack(dyv, dyv), dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
         bf2 ddl2 = bpack(0.f, 0.f), s12 = ddl2;
-        float *pB = &ws.part[tl][0][j][c * S];
-        float *pC = &ws.part[tl][1][j][c * S];
+        float *pB = &ws.part[u][0][j][c * S];
+        float *pC = &ws.part[u][1][j][c * S];
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
           g[i] = bfma(dy2, Cpair(t, i), g[i]);
-          const bf2 a = bex2(bmul(dl2, A2[i]));
-          const bf2 hp = t == 0 ? h0c[i] : H[t - 1][i];
-          const bf2 ga = bmul(g[i], a);
+          const bf2 hp = u == 0 ? H4[grp][i] : hg[u - 1][i];
+          const bf2 ga = bmul(g[i], ag[u][i]);
           const bf2 qv = bmul(ga, hp);
           dA_acc[i] = bfma(dl2, qv, dA_acc[i]);
           ddl2 = bfma(An[i], qv, ddl2);
           s12 = bfma(g[i], Bpair(t, i), s12);
-          const bf2 vB = bmul(g[i], du2), vC = bmul(dy2, H[t][i]);
+          const bf2 vB = bmul(g[i], du2), vC = bmul(dy2, hg[u][i]);
           g[i] = ga;
           if constexpr (S >= 2) {
             *reinterpret_cast<bf2 *>(pB + 2 * i) = vB;
@@ -451,14 +469,14 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
         ws.pd[c][t][j] = make_float2(d0 + d1, s0 + s1v);
       }
       __syncthreads();
-      // dB, dC of this half chunk: sums over the 4 warps x 8 channels, added
-      // to the fp32 accumulators (16-byte vector atomics when S >= 4)
+      // dB, dC of this group: sums over the 4 warps x 8 channels, added to
+      // the fp32 accumulators (16-byte vector atomics when S >= 4)
       if constexpr (S >= 4) {
         for (int o = threadIdx.x; o < kRedOutputs; o += kBW * 32) {
           const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
           const int which = r4 / NP, n = r4 - which * NP;
           const int jj = n / S, s0 = n - jj * S;
-          const int t = half * (kTB / 2) + tl;
+          const int t = 4 * grp + tl;
           if (t0 + t < L) {
             bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
@@ -479,11 +497,11 @@ __global__ void __launch_bounds__(kBW * 32) k_bwd(BwdParams p) {
           }
         }
       } else {
-        for (int o = threadIdx.x; o < (kTB / 2) * 2 * NP; o += kBW * 32) {
+        for (int o = threadIdx.x; o < 4 * 2 * NP; o += kBW * 32) {
           const int tl = o / (2 * NP), r = o % (2 * NP);
           const int which = r / NP, n = r - which * NP;
           const int jj = n / S, s0 = n - jj * S;
-          const int t = half * (kTB / 2) + tl;
+          const int t = 4 * grp + tl;
           if (t0 + t < L) {
             float acc = 0.f;
 #pragma unroll
