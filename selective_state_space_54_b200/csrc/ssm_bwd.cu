@@ -91,7 +91,9 @@ struct __align__(16) BwdWarpSmem {
   float dlu[kBCPW][kTB + kBPad];   // Delta * u
   float dy[kBCPW][kTB + kBPad];    // dout * SiLU(z)
   float ys[kBCPW][kTB + kBPad];    // sum_n C h
-  float2 pd[kBCPW][kTB][4];        // per lane j: (sum_n g A a h_prev, sum_n g B) partials
+  // per step, channel and lane j: (sum_n g A a h_prev, sum_n g B) partials;
+  // step-major so that a warp's stores of one step are contiguous
+  float2 pd[kTB][kBCPW][4];
   // dB, dC contributions of a 4-step group: [step][B|C][lane slice j][channel,
   // state] with 8 floats of padding per row so that a quarter warp's stores
   // hit distinct banks
@@ -103,6 +105,8 @@ struct __align__(16) BwdSmem {
   float Bs[kTB][NP];
   float Cs[kTB][NP];
   BwdWarpSmem<NP> w[kBW];
+  // per-warp sums of one 4-step group's dB/dC outputs (16-byte vectors)
+  ulonglong2 red[kBW][NP / 4 >= 1 ? 4 * 2 * NP / 4 : 1];
 };
 
 // B and C chunk [t0, t0 + kTB) into smem (fp32, zero padded), by the whole CTA.
@@ -466,34 +470,48 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         float d0, d1, s0, s1v;
         bunpack(ddl2, d0, d1);
         bunpack(s12, s0, s1v);
-        ws.pd[c][t][j] = make_float2(d0 + d1, s0 + s1v);
+        ws.pd[t][c][j] = make_float2(d0 + d1, s0 + s1v);
       }
       __syncthreads();
       // dB, dC of this group: sums over the 4 warps x 8 channels, added to
       // the fp32 accumulators (16-byte vector atomics when S >= 4)
       if constexpr (S >= 4) {
-        for (int o = threadIdx.x; o < kRedOutputs; o += kBW * 32) {
+        // every warp sums its own 8 channels for each output; warp 0 then
+        // adds the 4 warps' sums and issues the atomics
+        for (int o = lane; o < kRedOutputs; o += 32) {
           const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
           const int which = r4 / NP, n = r4 - which * NP;
           const int jj = n / S, s0 = n - jj * S;
-          const int t = 4 * grp + tl;
-          if (t0 + t < L) {
+          bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+          for (int cc = 0; cc < kBCPW; ++cc) {
+            const float *src = &ws.part[tl][which][jj][cc * S + s0];
+            const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(src);
+            acc0 = badd(acc0, x.x);
+            acc1 = badd(acc1, x.y);
+          }
+          sm.red[warp][o] = make_ulonglong2(acc0, acc1);
+        }
+        __syncthreads();
+        if (warp == 0) {
+          for (int o = lane; o < kRedOutputs; o += 32) {
+            const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
+            const int which = r4 / NP, n = r4 - which * NP;
+            const int t = 4 * grp + tl;
             bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
             for (int w = 0; w < kBW; ++w) {
-#pragma unroll
-              for (int cc = 0; cc < kBCPW; ++cc) {
-                const float *src = &sm.w[w].part[tl][which][jj][cc * S + s0];
-                const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(src);
-                acc0 = badd(acc0, x.x);
-                acc1 = badd(acc1, x.y);
-              }
+              const ulonglong2 x = sm.red[w][o];
+              acc0 = badd(acc0, x.x);
+              acc1 = badd(acc1, x.y);
             }
-            float4 acc;
-            bunpack(acc0, acc.x, acc.y);
-            bunpack(acc1, acc.z, acc.w);
-            float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
-            atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+            if (t0 + t < L) {
+              float4 acc;
+              bunpack(acc0, acc.x, acc.y);
+              bunpack(acc1, acc.z, acc.w);
+              float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
+              atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+            }
           }
         }
       } else {
@@ -511,8 +529,11 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
             atomicAdd((which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n), acc);
           }
         }
+        __syncthreads();  // the next group rewrites part
       }
-      __syncthreads();
+      // (S >= 4: the barrier between the per-warp sums and warp 0's combine
+      // already orders this group's reads of part before the next group's
+      // writes, and warp 0's reads of red before the next group's barrier)
     }
 
     // input-side gradients of this lane's 4 steps
@@ -521,8 +542,8 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = 4 * q + i;
-        const float4 pa = *reinterpret_cast<const float4 *>(&ws.pd[c][t][0]);
-        const float4 pb = *reinterpret_cast<const float4 *>(&ws.pd[c][t][2]);
+        const float4 pa = *reinterpret_cast<const float4 *>(&ws.pd[t][c][0]);
+        const float4 pb = *reinterpret_cast<const float4 *>(&ws.pd[t][c][2]);
         const float ddl = (pa.x + pa.z) + (pb.x + pb.z);
         const float s1 = (pa.y + pa.w) + (pb.y + pb.w);
         const float dl = ws.dl[c][t];
