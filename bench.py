@@ -296,8 +296,11 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
         g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
     del case
     y = torch.empty_like(g["u"])
+    # the training step: the forward saves the state entering every 16-step
+    # chunk in its workspace, and the backward starts from those
     shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
-                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32)
+                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32,
+                           flags=ssm.SSM_FLAG_SAVE_STATES)
     ws_f = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(ssm.bwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
     out = {"du": torch.empty_like(g["u"]), "ddelta": torch.empty_like(g["u"]),
@@ -310,11 +313,11 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
 
     def fwd():
         ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                     y=y, workspace=ws_f)
+                     y=y, workspace=ws_f, save_states=True)
 
     def bwd():
         ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                     g["dy"], out=out, workspace=ws_b)
+                     g["dy"], out=out, workspace=ws_b, fwd_workspace=ws_f)
 
     for _ in range(max(3, args.warmup)):
         fwd()
@@ -337,24 +340,27 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     barrier()
     ms_f = max_over_ranks(t_f / steps)
     ms_b = max_over_ranks(t_b / steps)
-    # the backward's special-function work: ex2 of the checkpoint pass, the
-    # recomputation and the reverse pass, one each per (b, t, d, n) element
+    # the backward's special-function work per (b, t, d, n) element: one ex2
+    # for the chunk recomputation and one for the group recomputation whose
+    # decays the reverse pass reuses (the chunk-entry states come from the
+    # forward, so the backward's own checkpoint pass does not run)
+    ex2_per_element = 2
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
-    bwd_achieved = 3 * w.bldn / (ms_b * 1e-3)
+    bwd_achieved = ex2_per_element * w.bldn / (ms_b * 1e-3)
     bwd_roofline = {"bound": "alu", "achieved": bwd_achieved / 1e12, "peak": ex2_peak / 1e12,
                     "unit": "Tex2/s", "frac": bwd_achieved / ex2_peak, "traffic": None,
-                    "kernel": "k_bwd", "ex2_per_element": 3,
+                    "kernel": "k_bwd", "ex2_per_element": ex2_per_element,
                     "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                                   f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
             "d_state": w.dstate, "io_dtype": w.dtype, "steps": steps,
-            "fwd_path": ssm.fwd_path(shape), "fwd_ms": ms_f, "bwd_ms": ms_b,
+            "fwd_path": ssm.fwd_path(shape), "saved_states": True, "fwd_ms": ms_f, "bwd_ms": ms_b,
             "bwd_roofline": bwd_roofline,
             "value": aggregate_value(world, w.bld, (ms_f + ms_b) * 1e-3), "unit": UNIT + " (fwd+bwd)",
             "bwd_value": aggregate_value(world, w.bld, ms_b * 1e-3),
-            "bwd_ex2_per_element": 3,
+            "bwd_ex2_per_element": ex2_per_element,
             "bwd_kernels_per_step": 2}
 
 

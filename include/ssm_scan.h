@@ -110,7 +110,16 @@ typedef struct {
  *                      picks it; other explicit paths return
  *                      SSM_ERR_UNSUPPORTED) and ssm_scan_step; ssm_scan_bwd
  *                      returns SSM_ERR_UNSUPPORTED for it. */
-typedef enum { SSM_FLAG_ZOH_EXACT = 1 } ssm_flags;
+typedef enum { SSM_FLAG_ZOH_EXACT = 1, SSM_FLAG_SAVE_STATES = 2 } ssm_flags;
+
+/* SSM_FLAG_SAVE_STATES (forward, with the Euler term): besides y, the forward
+ * writes into its workspace the state entering every 16-step chunk of every
+ * channel (fp32, 4 * batch * ceil(dim/32) * 32 * ceil(seqlen/16) * NP bytes,
+ * NP = dstate rounded up to a power of two >= 4; ssm_scan_fwd_workspace_bytes
+ * counts them).  Passing that workspace as fwd_workspace to ssm_scan_bwd, with
+ * the same shape and flag, lets the backward skip its own forward pass over
+ * the chunks.  It runs on path LOOKBACK_WS (AUTO picks it; other explicit
+ * paths, lanes = 4 and SSM_FLAG_ZOH_EXACT return SSM_ERR_UNSUPPORTED). */
 
 /* Bytes of workspace ssm_scan_fwd needs for `shape` on the current device
  * (at least 256: the header holding the device error word).  Returns 0 for
@@ -137,9 +146,13 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
                         void *y, float *last_state,
                         void *workspace, size_t ws_bytes, ssm_stream_t stream);
 
-/* Backward of ssm_scan_fwd by recomputation: the states are recomputed from
- * the inputs (never read from the forward), reading guide, "Expansao de
- * Estado Ciente de Hardware".  Gradients of sum(dout * y):
+/* Backward of ssm_scan_fwd by recomputation: the states inside each 16-step
+ * chunk are recomputed from the inputs, reading guide, "Expansao de Estado
+ * Ciente de Hardware"; only the state entering each chunk may come from the
+ * forward (fwd_workspace, nullable: a workspace that ssm_scan_fwd filled with
+ * SSM_FLAG_SAVE_STATES for the same shape, inputs and initial state; the
+ * shape passed here must carry that flag too).  Without it the backward
+ * first recomputes those chunk states itself.  Gradients of sum(dout * y):
  *  du, ddelta, dz          [batch][dim][seqlen] io dtype (ddelta is with
  *                          respect to the raw delta argument)
  *  dB, dC                  [batch][seqlen][dstate] io dtype, summed over dim
@@ -152,7 +165,7 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
                         const float *A, const void *B, const void *C,
                         const float *D, const void *z, const float *delta_bias,
                         int delta_softplus, const float *initial_state,
-                        const void *dout,
+                        const void *dout, const void *fwd_workspace,
                         void *du, void *ddelta, float *dA, void *dB, void *dC,
                         float *dD, void *dz, float *ddelta_bias,
                         float *dinitial_state,

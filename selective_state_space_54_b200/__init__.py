@@ -18,7 +18,8 @@ from __future__ import annotations
 import ctypes
 
 from . import _lib
-from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_FLAG_ZOH_EXACT, SSM_PATH_AUTO,  # noqa: F401
+from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_FLAG_SAVE_STATES,  # noqa: F401
+                   SSM_FLAG_ZOH_EXACT, SSM_PATH_AUTO,
                    SSM_PATH_LOOKBACK, SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L,
                    ssm_shape)
 
@@ -93,9 +94,11 @@ def _workspace(nbytes, device, workspace):
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softplus=True,
              initial_state=None, y=None, last_state=None, return_last_state=False,
              workspace=None, path: int = SSM_PATH_AUTO, lanes: int = 0, zoh_exact=False,
-             stream=None):
+             save_states=False, stream=None):
     """Forward selective scan; returns y, or (y, last_state).  zoh_exact selects the
-    exact zero-order-hold input term instead of the Euler one (Delta * B)."""
+    exact zero-order-hold input term instead of the Euler one (Delta * B).
+    save_states also writes the state entering every 16-step chunk into
+    ``workspace`` (which must then be given), for scan_bwd(fwd_workspace=...)."""
     import torch
     batch, dim, seqlen = u.shape
     dstate = B.shape[-1]
@@ -117,8 +120,10 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, dstate), dtype=f32, device=dev)
     _check_io("last_state", last_state, (batch, dim, dstate), f32, dev)
-    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path, lanes,
-                       SSM_FLAG_ZOH_EXACT if zoh_exact else 0)
+    flags = (SSM_FLAG_ZOH_EXACT if zoh_exact else 0) | (SSM_FLAG_SAVE_STATES if save_states else 0)
+    if save_states and workspace is None:
+        raise ValueError("save_states writes into the workspace: pass workspace=")
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path, lanes, flags)
     nbytes = fwd_workspace_bytes(shape)
     if nbytes == 0 and batch * dim * seqlen > 0:
         raise ScanError(_lib.SSM_ERR_UNSUPPORTED, "ssm_scan_fwd_workspace_bytes")
@@ -198,8 +203,10 @@ def causal_conv1d(x, weight, bias=None, *, initial_state=None, silu=True, out=No
 
 def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,
              initial_state=None, want_dinitial_state=False, out=None, workspace=None,
-             stream=None):
-    """Backward of scan_fwd by recomputation; returns a dict of gradients."""
+             fwd_workspace=None, stream=None):
+    """Backward of scan_fwd by recomputation; returns a dict of gradients.
+    fwd_workspace: the workspace of a scan_fwd(save_states=True) call on the same
+    inputs, whose saved chunk states the backward then uses."""
     import torch
     batch, dim, seqlen = u.shape
     dstate = B.shape[-1]
@@ -223,13 +230,14 @@ def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,
                  torch.empty((dim,), dtype=f32, device=dev) if delta_bias is not None else None)
     g.setdefault("dinitial_state",
                  torch.empty((batch, dim, dstate), dtype=f32, device=dev) if want_dinitial_state else None)
-    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u))
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u),
+                       flags=SSM_FLAG_SAVE_STATES if fwd_workspace is not None else 0)
     nbytes = bwd_workspace_bytes(shape)
     ws = _workspace(nbytes, dev, workspace)
     rc = _lib.load().ssm_scan_bwd(
         ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(initial_state), _ptr(dout),
-        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+        _ptr(fwd_workspace), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
         _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]), _ptr(g["dinitial_state"]),
         _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
     if rc != 0:

@@ -27,6 +27,7 @@ SSM_PATH_PER_GROUP = 3
 SSM_PATH_LOOKBACK_WS = 4
 
 SSM_FLAG_ZOH_EXACT = 1
+SSM_FLAG_SAVE_STATES = 2
 
 PATH_NAMES = {SSM_PATH_AUTO: "auto", SSM_PATH_LOOKBACK: "lookback",
               SSM_PATH_SPLIT_L: "split_l", SSM_PATH_PER_GROUP: "per_group",
@@ -70,7 +71,7 @@ def load(path: str | None = None):
     lib.ssm_scan_bwd_workspace_bytes.restype = sz
     lib.ssm_scan_fwd.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, sz, vp]
     lib.ssm_scan_fwd.restype = ci
-    lib.ssm_scan_bwd.argtypes = ([shp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp]
+    lib.ssm_scan_bwd.argtypes = ([shp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp]
                                  + [vp] * 9 + [vp, sz, vp])
     lib.ssm_scan_bwd.restype = ci
     lib.ssm_scan_fwd_noalloc.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp]

@@ -31,8 +31,13 @@ ssm_status check_shape(const ssm_shape *s) {
   if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_LOOKBACK_WS) return SSM_ERR_UNSUPPORTED;
   if (s->path == SSM_PATH_LOOKBACK_WS && s->lanes == 4) return SSM_ERR_UNSUPPORTED;
   if (s->lanes != 0 && s->lanes != 2 && s->lanes != 4) return SSM_ERR_UNSUPPORTED;
-  if (s->flags & ~SSM_FLAG_ZOH_EXACT) return SSM_ERR_INVALID_ARG;
+  if (s->flags & ~(SSM_FLAG_ZOH_EXACT | SSM_FLAG_SAVE_STATES)) return SSM_ERR_INVALID_ARG;
   if ((s->flags & SSM_FLAG_ZOH_EXACT) && s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK)
+    return SSM_ERR_UNSUPPORTED;
+  // saved states are written by the warp-specialised kernel, which is Euler only
+  if ((s->flags & SSM_FLAG_SAVE_STATES) &&
+      ((s->flags & SSM_FLAG_ZOH_EXACT) || (s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK_WS) ||
+       s->lanes == 4))
     return SSM_ERR_UNSUPPORTED;
   // index arithmetic is int64; keep every flat index well inside it
   const double elems = (double)s->batch * (double)s->dim * (double)s->seqlen;
@@ -48,6 +53,7 @@ struct FwdPlan {
   int64_t P = 0;                     // look-back warps
   int64_t n_segs = 1, seg_chunks = 0;
   size_t off_flags = 0, off_carry = 0, off_seg_h = 0, off_seg_dsum = 0, off_seg_carry = 0;
+  size_t ckpt_bytes = 0;             // saved states, right after the header
   size_t total = kHeaderBytes;
 };
 
@@ -78,6 +84,12 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   const int64_t unit = (int64_t)sms * kWarps;   // one warp per SM sub-partition
   const int64_t g2 = groups_for(s, 2), g4 = groups_for(s, 4);
   int path = s->path, lpc = s->lanes;
+  const bool save = (s->flags & SSM_FLAG_SAVE_STATES) != 0;
+  if (save) {
+    path = SSM_PATH_LOOKBACK_WS;
+    lpc = 2;
+    p.ckpt_bytes = sizeof(float) * bwd_ckpt_floats(s->batch, s->dim, s->seqlen, p.NP);
+  }
   if (lpc == 0) {
     if (path == SSM_PATH_SPLIT_L || path == SSM_PATH_LOOKBACK_WS) lpc = 2;
     else if (path == SSM_PATH_PER_GROUP) lpc = 4;
@@ -120,7 +132,7 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
     if (r > occ) r = occ;
     p.P = r >= 1 ? r * unit : G;
     if (p.P > slots) p.P = slots;  // all warps co-resident
-    p.off_flags = kHeaderBytes;
+    p.off_flags = round_up(kHeaderBytes + p.ckpt_bytes, 256);
     p.off_carry = round_up(p.off_flags + sizeof(unsigned) * (size_t)p.P, 256);
     p.total = round_up(p.off_carry + sizeof(float) * (size_t)p.P * cpw * p.NP, 256);
   } else if (path == SSM_PATH_SPLIT_L) {
@@ -229,12 +241,18 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
   p.err = reinterpret_cast<unsigned *>(ws);
   p.wait_limit_ns = kWaitLimitNs;
   p.n_segs = pl.n_segs; p.seg_chunks = pl.seg_chunks;
+  if (pl.ckpt_bytes) {
+    p.ckpt_out = reinterpret_cast<float *>(ws + kHeaderBytes);
+    p.ck_cpb = (shape->dim + kCkptChannels - 1) / kCkptChannels;
+    p.ck_K = (shape->seqlen + kCkptSteps - 1) / kCkptSteps;
+  }
 
   cudaError_t e;
   if (pl.path == SSM_PATH_LOOKBACK || pl.path == SSM_PATH_LOOKBACK_WS) {
     p.flags = reinterpret_cast<unsigned *>(ws + pl.off_flags);
     p.carry = reinterpret_cast<float *>(ws + pl.off_carry);
-    e = cudaMemsetAsync(ws, 0, pl.off_carry, s);  // error word and flags
+    e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);  // error word
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + pl.off_flags, 0, pl.off_carry - pl.off_flags, s);  // flags
     if (e != cudaSuccess) return cuda_status(e);
     e = pl.path == SSM_PATH_LOOKBACK_WS ? launch_fwd_ws(shape->io_dtype, pl.NP, p, s)
                                         : launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
@@ -321,13 +339,17 @@ size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
 ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta,
                         const float *A, const void *B, const void *C, const float *D,
                         const void *z, const float *delta_bias, int delta_softplus,
-                        const float *initial_state, const void *dout, void *du, void *ddelta,
+                        const float *initial_state, const void *dout, const void *fwd_workspace,
+                        void *du, void *ddelta,
                         float *dA, void *dB, void *dC, float *dD, void *dz,
                         float *ddelta_bias, float *dinitial_state, void *workspace,
                         size_t ws_bytes, ssm_stream_t stream) {
   ssm_status st = check_shape(shape);
   if (st != SSM_OK) return st;
   if (shape->flags & SSM_FLAG_ZOH_EXACT) return SSM_ERR_UNSUPPORTED;  // Euler backward only
+  // saved states come from a forward run with the same shape and flag
+  if (fwd_workspace && (!(shape->flags & SSM_FLAG_SAVE_STATES) || !aligned(fwd_workspace, 256)))
+    return SSM_ERR_INVALID_ARG;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t batch = shape->batch, dim = shape->dim, L = shape->seqlen, N = shape->dstate;
   const size_t es = shape->io_dtype == SSM_BF16 ? 2 : 4;
@@ -367,7 +389,12 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
   p.A = A; p.D = D; p.bias = delta_bias; p.h0 = initial_state;
   p.du = du; p.ddelta = ddelta; p.dz = dz;
   p.dA = dA; p.dD = dD; p.dbias = ddelta_bias; p.dh0 = dinitial_state;
-  p.ckpt = reinterpret_cast<float *>(ws + off_ckpt);
+  if (fwd_workspace) {  // the forward's saved states, right after its header
+    p.ckpt = reinterpret_cast<float *>(const_cast<char *>(static_cast<const char *>(fwd_workspace)) + kHeaderBytes);
+    p.ckpt_given = 1;
+  } else {
+    p.ckpt = reinterpret_cast<float *>(ws + off_ckpt);
+  }
   p.dB_acc = reinterpret_cast<float *>(ws + off_dB);
   p.dC_acc = reinterpret_cast<float *>(ws + off_dC);
   p.dB = dB; p.dC = dC;

@@ -25,10 +25,11 @@
 
 namespace ssm {
 
-constexpr int kTB = 16;       // steps per backward chunk
+constexpr int kTB = kCkptSteps;  // steps per backward chunk (the saved-state chunk)
 constexpr int kBW = 4;        // warps per CTA
 constexpr int kBCPW = 8;      // channels per warp
 constexpr int kBPad = 4;
+static_assert(kBW * kBCPW == kCkptChannels, "a backward CTA covers one saved-state channel block");
 
 // 4 consecutive io values
 template <typename T> struct Vec4;
@@ -310,8 +311,8 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     h[i] = bpack(v[0], v[1]);
   }
   ChunkIn nxt;
-  if (K > 0) load_chunk(0, false, nxt);
-  for (int64_t k = 0; k < K; ++k) {
+  if (K > 0 && !p.ckpt_given) load_chunk(0, false, nxt);
+  for (int64_t k = 0; k < (p.ckpt_given ? 0 : K); ++k) {
     const int64_t t0 = k * kTB;
 #pragma unroll
     for (int i = 0; i < SP; ++i) {
@@ -360,8 +361,8 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
       bf2 hh[SP];
 #pragma unroll
       for (int i = 0; i < SP; ++i) {
-        const float *src = ck_at(k, i);
-        hh[i] = bpack(src[0], S >= 2 ? src[1] : 0.f);
+        const float *src = ck_at(k, i);  // padded channels: saved states may be unwritten
+        hh[i] = valid ? bpack(src[0], S >= 2 ? src[1] : 0.f) : bpack(0.f, 0.f);
       }
 #pragma unroll
     for (int t = 0; t < kTB; t += 4) {

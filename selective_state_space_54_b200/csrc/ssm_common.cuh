@@ -22,6 +22,12 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kRowPad = 4;       // smem row padding (floats) against bank conflicts
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Saved-state layout shared by the forward (writer) and the backward (reader):
+// the state entering every kCkptSteps-step chunk, per block of kCkptChannels
+// channels of one batch element.
+constexpr int kCkptSteps = 16;
+constexpr int kCkptChannels = 32;
+
 // Workspace header: byte 0 holds the device error word.
 constexpr size_t kHeaderBytes = 256;
 constexpr unsigned kErrWaitTimeout = 1u;
@@ -53,6 +59,11 @@ struct FwdParams {
   unsigned long long wait_limit_ns;
   // split-L schedule
   int64_t n_segs, seg_chunks;
+  // saved states for the backward (nullable): the state entering every
+  // kCkptSteps-step chunk, laid out [cta][chunk][kCkptChannels][NP] with
+  // cta = b * ck_cpb + d / kCkptChannels (the backward's own layout)
+  float *ckpt_out;
+  int64_t ck_cpb, ck_K;
   float *seg_h;       // [n_groups * n_segs][32/LPC][NP] segment end state from zero
   float *seg_dsum;    // [n_groups * n_segs][32/LPC]     sum of Delta over the segment
   float *seg_carry;   // [n_groups * n_segs][32/LPC][NP] state entering the segment
@@ -92,6 +103,7 @@ struct BwdParams {
   float *dA, *dD, *dbias, *dh0;
   float *dB_acc, *dC_acc;     // [batch][L][NP] fp32
   float *ckpt;                // [cta][K][32][NP]
+  int ckpt_given;             // ckpt holds states saved by the forward: skip the checkpoint pass
   void *dB, *dC;              // [batch][L][N] io dtype (finalize)
   int64_t batch, dim, L;
   int N;

@@ -632,6 +632,7 @@ __global__ void k_wait_probe(unsigned *flag, unsigned *err, unsigned long long l
 // full" (producer -> consumer) and "sums ready" (consumer -> producer) per
 // pair and stage.
 constexpr int kTW = 16;
+static_assert(kTW == kCkptSteps, "the saved states are written at warp-specialised chunk starts");
 constexpr int kPairs = 4;
 constexpr int kWSThreads = 2 * kPairs * 32;
 
@@ -731,9 +732,25 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
     f2 hp[S / 2];
 #pragma unroll
     for (int s = 0; s < S; s += 2) hp[s / 2] = pack2(h[s], h[s + 1]);
+    // saved states for the backward: this lane's S states of the channel
+    float *ck = nullptr;
+    if (p.ckpt_out && ln.valid)
+      ck = p.ckpt_out + ((ln.b * p.ck_cpb + ln.d / kCkptChannels) * p.ck_K * kCkptChannels +
+                         ln.d % kCkptChannels) * NP + j * S;
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = (int)(it & 1);
       WSStage<NP> &st = sm.st[stage];
+      if (ck) {  // the state entering chunk k
+        float *dst = ck + k * kCkptChannels * NP;
+        if constexpr (S % 4 == 0) {
+#pragma unroll
+          for (int s = 0; s < S; s += 4)
+            __stcg(reinterpret_cast<ulonglong2 *>(dst + s), make_ulonglong2(hp[s / 2], hp[s / 2 + 1]));
+        } else {
+#pragma unroll
+          for (int s = 0; s < S; s += 2) __stcg(reinterpret_cast<unsigned long long *>(dst + s), hp[s / 2]);
+        }
+      }
       bar_sync_n(bar_full + stage, 64);
 #pragma unroll
       for (int tt = 0; tt < kTW; tt += 4) {

@@ -95,10 +95,11 @@ def test_empty_problem_is_a_noop(lib):
 
 
 def test_bwd_rejects_bad_shapes(lib):
-    # shape, 8 input pointers, delta_softplus, initial_state, dout, 9 outputs, ws, bytes, stream
+    # shape, 8 input pointers, delta_softplus, initial_state, dout, fwd_workspace, 9 outputs,
+    # ws, bytes, stream
     for kw, code in BAD_SHAPES:
         sh = _shape(**kw)
-        assert lib.ssm_scan_bwd(ctypes.byref(sh), *[None] * 8, 1, *[None] * 11, None, 0, None) == code
+        assert lib.ssm_scan_bwd(ctypes.byref(sh), *[None] * 8, 1, *[None] * 12, None, 0, None) == code
 
 
 def test_product_has_no_oracle_or_cpu_path():
@@ -113,15 +114,15 @@ def test_product_has_no_oracle_or_cpu_path():
 
 
 def _bwd(lib, shape, **over):
-    # shape, u, delta, A, B, C, D, z, bias, softplus, h0, dout,
+    # shape, u, delta, A, B, C, D, z, bias, softplus, h0, dout, fwd_ws,
     # du, ddelta, dA, dB, dC, dD, dz, dbias, dh0, ws, ws_bytes, stream
-    p = dict(u=16, delta=16, A=16, B=16, C=16, D=None, z=None, bias=None, h0=None, dout=16,
+    p = dict(u=16, delta=16, A=16, B=16, C=16, D=None, z=None, bias=None, h0=None, dout=16, fws=None,
              du=16, ddelta=16, dA=16, dB=16, dC=16, dD=None, dz=None, dbias=None, dh0=None)
     p.update(over)
     v = lambda x: None if x is None else ctypes.c_void_p(x)
     return lib.ssm_scan_bwd(ctypes.byref(shape), v(p["u"]), v(p["delta"]), v(p["A"]), v(p["B"]),
                             v(p["C"]), v(p["D"]), v(p["z"]), v(p["bias"]), 1, v(p["h0"]),
-                            v(p["dout"]), v(p["du"]), v(p["ddelta"]), v(p["dA"]), v(p["dB"]),
+                            v(p["dout"]), v(p["fws"]), v(p["du"]), v(p["ddelta"]), v(p["dA"]), v(p["dB"]),
                             v(p["dC"]), v(p["dD"]), v(p["dz"]), v(p["dbias"]), v(p["dh0"]),
                             None, 0, None)
 
@@ -218,7 +219,7 @@ def test_conv_empty_problem_is_a_noop(lib):
 
 
 def test_flags_checked_before_launch(lib):
-    assert _fwd(lib, _shape(flags=2)) == _lib.SSM_ERR_INVALID_ARG
+    assert _fwd(lib, _shape(flags=4)) == _lib.SSM_ERR_INVALID_ARG  # an unknown bit
     # exact ZOH runs on the look-back path only; other explicit paths are refused
     for path in (_lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP, _lib.SSM_PATH_LOOKBACK_WS):
         assert _fwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path)) == \
@@ -227,3 +228,15 @@ def test_flags_checked_before_launch(lib):
             ctypes.byref(_shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path))) == 0
     # the backward is Euler only
     assert _bwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED
+
+
+def test_saved_states_flag_checked_before_launch(lib):
+    save, zoh = _lib.SSM_FLAG_SAVE_STATES, _lib.SSM_FLAG_ZOH_EXACT
+    # written by the warp-specialised kernel only: Euler, 2 lanes, AUTO or LOOKBACK_WS
+    assert _fwd(lib, _shape(flags=save | zoh)) == _lib.SSM_ERR_UNSUPPORTED
+    for path in (_lib.SSM_PATH_LOOKBACK, _lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP):
+        assert _fwd(lib, _shape(flags=save, path=path)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, _shape(flags=save, lanes=4)) == _lib.SSM_ERR_UNSUPPORTED
+    # a forward workspace for the backward needs the flag, and 256-byte alignment
+    assert _bwd(lib, _shape(), fws=256) == _lib.SSM_ERR_INVALID_ARG
+    assert _bwd(lib, _shape(flags=save), fws=272) == _lib.SSM_ERR_INVALID_ARG

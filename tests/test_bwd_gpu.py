@@ -101,3 +101,53 @@ def test_bwd_full_mamba_1p4b_layer(cuda_device):
 def test_bwd_single_step_and_single_channel(cuda_device):
     _check(_case(1, 1, 1, 16, synth.F32, 78), cuda_device)
     _check(_case(1, 3, 2, 4, synth.BF16, 79), cuda_device)
+
+
+# ---- states saved by the forward (the chunk checkpoints of the training step) ----
+def _bwd_saved(case, device, h0=None):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    g = upload(case, device)
+    h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
+    shape = ssm.make_shape(case["batch"], case["dim"], case["seqlen"], case["dstate"],
+                           ssm.SSM_BF16 if case["dtype"] == synth.BF16 else ssm.SSM_F32,
+                           flags=ssm.SSM_FLAG_SAVE_STATES)
+    ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=device)
+    y = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                     initial_state=h0_t, workspace=ws, save_states=True)
+    out = ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                       g["delta_bias"], g["dy"], initial_state=h0_t, fwd_workspace=ws,
+                       want_dinitial_state=h0 is not None)
+    torch.cuda.synchronize()
+    return to_f64(y), {k: (None if v is None else to_f64(v)) for k, v in out.items()}
+
+
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("N", [4, 16, 32])
+def test_bwd_with_saved_states(cuda_device, dtype, N):
+    # 40 channels: a partial 32-channel block; 333 steps: a partial 16-step chunk
+    case = _case(2, 40, 333, N, dtype, 600 + N)
+    h0 = np.random.default_rng(N).standard_normal((2, 40, N)).astype(np.float32)
+    ref = oracle.bwd(case, case["dy"], h0=h0, want_dh0=True)
+    y, got = _bwd_saved(case, cuda_device, h0)
+    assert_close(y, oracle.fwd(case, h0=h0)["y"], dtype, "y")
+    for k in GRADS:
+        assert_close(got[k], ref[k], dtype, k, stored_bf16=k in IO_GRADS)
+    assert_close(got["dinitial_state"], ref["dh0"], dtype, "dh0", stored_bf16=False)
+
+
+def test_bwd_saved_states_agree_with_recomputed(cuda_device):
+    case = _case(2, 64, 512, 16, synth.F32, 610)
+    _, saved = _bwd_saved(case, cuda_device)
+    recomputed = _bwd(case, cuda_device)
+    for k in GRADS:
+        assert_close(saved[k], recomputed[k], synth.F32, k)
+
+
+def test_bwd_full_mamba_1p4b_layer_with_saved_states(cuda_device):
+    w = synth.WORKLOADS["mamba-1.4b-layer-train"]
+    case = synth.make_workload(w)
+    ref = oracle.bwd(case, case["dy"])
+    _, got = _bwd_saved(case, cuda_device)
+    for k in GRADS:
+        assert_close(got[k], ref[k], case["dtype"], k, stored_bf16=k in IO_GRADS)
