@@ -600,6 +600,32 @@ def main():
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
     clocks = clk.summary()
 
+    # the same forward on token-major activations (batch, seqlen, d_inner)
+    tok = None
+    if not args.no_bwd and not args.batch and w.dtype == synth.BF16 and w.dim % 8 == 0:
+        tm = {k: g[k].transpose(1, 2).contiguous() for k in ("u", "delta", "z")}
+        y_tm = torch.empty_like(tm["u"])
+
+        def step_tm():
+            ssm.scan_fwd(tm["u"], tm["delta"], g["A"], g["B"], g["C"], g["D"], tm["z"],
+                         g["delta_bias"], y=y_tm, last_state=ls, return_last_state=True,
+                         workspace=ws, token_major=True)
+
+        for _ in range(max(3, args.warmup)):
+            step_tm()
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step_tm()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_tm = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+        tok = {"layout": "[batch][seqlen][d_inner] u, delta, z, y", "ms_per_step": ms_tm,
+               "value": aggregate_value(world, w.bld, ms_tm * 1e-3), "unit": UNIT}
+        del tm, y_tm
+
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
     if not args.no_e2e:
@@ -666,7 +692,7 @@ def main():
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
-            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec, "conv1d": conv,
+            "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec, "conv1d": conv, "token_major": tok,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, case)

@@ -110,7 +110,19 @@ typedef struct {
  *                      picks it; other explicit paths return
  *                      SSM_ERR_UNSUPPORTED) and ssm_scan_step; ssm_scan_bwd
  *                      returns SSM_ERR_UNSUPPORTED for it. */
-typedef enum { SSM_FLAG_ZOH_EXACT = 1, SSM_FLAG_SAVE_STATES = 2 } ssm_flags;
+typedef enum {
+  SSM_FLAG_ZOH_EXACT = 1,
+  SSM_FLAG_SAVE_STATES = 2,
+  SSM_FLAG_TOKEN_MAJOR = 4
+} ssm_flags;
+
+/* SSM_FLAG_TOKEN_MAJOR (forward): u, delta, z and y are laid out
+ * [batch][seqlen][dim] (dim contiguous), as a projection produces them, instead
+ * of [batch][dim][seqlen]; B and C keep their layout.  bf16 only, dim % 8 == 0,
+ * u/delta/z/y 16-byte aligned; path AUTO or LOOKBACK_WS with the Euler term
+ * (SSM_ERR_UNSUPPORTED otherwise, SSM_ERR_INVALID_ARG for misaligned
+ * pointers).  ssm_scan_bwd returns SSM_ERR_UNSUPPORTED for it; ssm_scan_step
+ * ignores it (one token has no time axis). */
 
 /* SSM_FLAG_SAVE_STATES (forward, with the Euler term): besides y, the forward
  * writes into its workspace the state entering every 16-step chunk of every

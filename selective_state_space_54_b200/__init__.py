@@ -19,7 +19,7 @@ import ctypes
 
 from . import _lib
 from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_FLAG_SAVE_STATES,  # noqa: F401
-                   SSM_FLAG_ZOH_EXACT, SSM_PATH_AUTO,
+                   SSM_FLAG_TOKEN_MAJOR, SSM_FLAG_ZOH_EXACT, SSM_PATH_AUTO,
                    SSM_PATH_LOOKBACK, SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L,
                    ssm_shape)
 
@@ -94,20 +94,25 @@ def _workspace(nbytes, device, workspace):
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softplus=True,
              initial_state=None, y=None, last_state=None, return_last_state=False,
              workspace=None, path: int = SSM_PATH_AUTO, lanes: int = 0, zoh_exact=False,
-             save_states=False, stream=None):
+             save_states=False, token_major=False, stream=None):
     """Forward selective scan; returns y, or (y, last_state).  zoh_exact selects the
     exact zero-order-hold input term instead of the Euler one (Delta * B).
     save_states also writes the state entering every 16-step chunk into
-    ``workspace`` (which must then be given), for scan_bwd(fwd_workspace=...)."""
+    ``workspace`` (which must then be given), for scan_bwd(fwd_workspace=...).
+    token_major: u, delta, z and y are (batch, seqlen, dim) instead."""
     import torch
-    batch, dim, seqlen = u.shape
+    if token_major:
+        batch, seqlen, dim = u.shape
+    else:
+        batch, dim, seqlen = u.shape
     dstate = B.shape[-1]
     dt = u.dtype
     dev = u.device
     f32 = torch.float32
-    _check_io("u", u, (batch, dim, seqlen), dt, dev)
-    _check_io("delta", delta, (batch, dim, seqlen), dt, dev)
-    _check_io("z", z, (batch, dim, seqlen), dt, dev)
+    act = (batch, seqlen, dim) if token_major else (batch, dim, seqlen)
+    _check_io("u", u, act, dt, dev)
+    _check_io("delta", delta, act, dt, dev)
+    _check_io("z", z, act, dt, dev)
     _check_io("B", B, (batch, seqlen, dstate), dt, dev)
     _check_io("C", C, (batch, seqlen, dstate), dt, dev)
     _check_io("A", A, (dim, dstate), f32, dev)
@@ -116,11 +121,12 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
     _check_io("initial_state", initial_state, (batch, dim, dstate), f32, dev)
     if y is None:
         y = torch.empty_like(u)
-    _check_io("y", y, (batch, dim, seqlen), dt, dev)
+    _check_io("y", y, act, dt, dev)
     if last_state is None and return_last_state:
         last_state = torch.empty((batch, dim, dstate), dtype=f32, device=dev)
     _check_io("last_state", last_state, (batch, dim, dstate), f32, dev)
-    flags = (SSM_FLAG_ZOH_EXACT if zoh_exact else 0) | (SSM_FLAG_SAVE_STATES if save_states else 0)
+    flags = ((SSM_FLAG_ZOH_EXACT if zoh_exact else 0) | (SSM_FLAG_SAVE_STATES if save_states else 0)
+             | (SSM_FLAG_TOKEN_MAJOR if token_major else 0))
     if save_states and workspace is None:
         raise ValueError("save_states writes into the workspace: pass workspace=")
     shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), path, lanes, flags)

@@ -28,6 +28,7 @@ SSM_PATH_LOOKBACK_WS = 4
 
 SSM_FLAG_ZOH_EXACT = 1
 SSM_FLAG_SAVE_STATES = 2
+SSM_FLAG_TOKEN_MAJOR = 4
 
 PATH_NAMES = {SSM_PATH_AUTO: "auto", SSM_PATH_LOOKBACK: "lookback",
               SSM_PATH_SPLIT_L: "split_l", SSM_PATH_PER_GROUP: "per_group",

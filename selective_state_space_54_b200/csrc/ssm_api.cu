@@ -31,7 +31,13 @@ ssm_status check_shape(const ssm_shape *s) {
   if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_LOOKBACK_WS) return SSM_ERR_UNSUPPORTED;
   if (s->path == SSM_PATH_LOOKBACK_WS && s->lanes == 4) return SSM_ERR_UNSUPPORTED;
   if (s->lanes != 0 && s->lanes != 2 && s->lanes != 4) return SSM_ERR_UNSUPPORTED;
-  if (s->flags & ~(SSM_FLAG_ZOH_EXACT | SSM_FLAG_SAVE_STATES)) return SSM_ERR_INVALID_ARG;
+  if (s->flags & ~(SSM_FLAG_ZOH_EXACT | SSM_FLAG_SAVE_STATES | SSM_FLAG_TOKEN_MAJOR))
+    return SSM_ERR_INVALID_ARG;
+  // token-major activations: bf16, 16-byte channel rows, warp-specialised Euler path
+  if ((s->flags & SSM_FLAG_TOKEN_MAJOR) &&
+      (s->io_dtype != SSM_BF16 || s->dim % 8 != 0 || (s->flags & SSM_FLAG_ZOH_EXACT) ||
+       (s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK_WS) || s->lanes == 4))
+    return SSM_ERR_UNSUPPORTED;
   if ((s->flags & SSM_FLAG_ZOH_EXACT) && s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK)
     return SSM_ERR_UNSUPPORTED;
   // saved states are written by the warp-specialised kernel, which is Euler only
@@ -85,11 +91,11 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   const int64_t g2 = groups_for(s, 2), g4 = groups_for(s, 4);
   int path = s->path, lpc = s->lanes;
   const bool save = (s->flags & SSM_FLAG_SAVE_STATES) != 0;
-  if (save) {
+  if (save || (s->flags & SSM_FLAG_TOKEN_MAJOR)) {  // both live in the warp-specialised kernel
     path = SSM_PATH_LOOKBACK_WS;
     lpc = 2;
-    p.ckpt_bytes = sizeof(float) * bwd_ckpt_floats(s->batch, s->dim, s->seqlen, p.NP);
   }
+  if (save) p.ckpt_bytes = sizeof(float) * bwd_ckpt_floats(s->batch, s->dim, s->seqlen, p.NP);
   if (lpc == 0) {
     if (path == SSM_PATH_SPLIT_L || path == SSM_PATH_LOOKBACK_WS) lpc = 2;
     else if (path == SSM_PATH_PER_GROUP) lpc = 4;
@@ -231,6 +237,9 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
   p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = (int)shape->dstate;
   p.softplus = delta_softplus ? 1 : 0;
   p.zoh = (shape->flags & SSM_FLAG_ZOH_EXACT) ? 1 : 0;
+  p.tok = (shape->flags & SSM_FLAG_TOKEN_MAJOR) ? 1 : 0;
+  if (p.tok && !(aligned(u, 16) && aligned(delta, 16) && aligned(z, 16) && aligned(y, 16)))
+    return SSM_ERR_INVALID_ARG;
   p.io_vec = ((shape->seqlen * es) % 16 == 0) && aligned(u, 16) && aligned(delta, 16) &&
              aligned(z, 16) && aligned(y, 16);
   p.bc_vec = (shape->dstate == pl.NP) && ((shape->dstate * es) % 16 == 0) && aligned(B, 16) &&
@@ -346,7 +355,8 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
                         size_t ws_bytes, ssm_stream_t stream) {
   ssm_status st = check_shape(shape);
   if (st != SSM_OK) return st;
-  if (shape->flags & SSM_FLAG_ZOH_EXACT) return SSM_ERR_UNSUPPORTED;  // Euler backward only
+  if (shape->flags & (SSM_FLAG_ZOH_EXACT | SSM_FLAG_TOKEN_MAJOR))  // Euler, channel-major only
+    return SSM_ERR_UNSUPPORTED;
   // saved states come from a forward run with the same shape and flag
   if (fwd_workspace && (!(shape->flags & SSM_FLAG_SAVE_STATES) || !aligned(fwd_workspace, 256)))
     return SSM_ERR_INVALID_ARG;

@@ -46,6 +46,7 @@ struct FwdParams {
   int N;
   int softplus;
   int zoh;      // exact zero-order-hold input term instead of Euler
+  int tok;      // u/delta/z/y laid out [batch][L][dim] (bf16, warp-specialised path)
   int io_vec;   // u/delta/z/y rows 16-byte aligned: vector loads
   int bc_vec;   // B/C chunk blocks 16-byte aligned and N == NP
   int64_t gpb;        // channel groups per batch element

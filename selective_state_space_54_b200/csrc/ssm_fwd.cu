@@ -818,12 +818,16 @@ struct RunRows {
   T *y;
   float bias, Dd;
   bool valid;
+  int64_t tok_c0;  // token-major: the group's first channel
   __device__ __forceinline__ void set(const FwdParams &p, int64_t g, int lane) {
     const int c = lane & 15, j = lane >> 4;
     const int64_t b = g / p.gpb;
     const int64_t d = (g - b * p.gpb) * 16 + c;
     valid = d < p.dim;
-    const int64_t row = (b * p.dim + (valid ? d : 0)) * p.L + j * 8;
+    // channel-major: this lane's row at step 8j; token-major: the group's
+    // first channel at step 0 (time stride dim)
+    const int64_t row = p.tok ? b * p.L * p.dim + (g - b * p.gpb) * 16
+                              : (b * p.dim + (valid ? d : 0)) * p.L + j * 8;
     u = static_cast<const T *>(p.u) + row;
     dr = static_cast<const T *>(p.delta) + row;
     z = p.z ? static_cast<const T *>(p.z) + row : nullptr;
@@ -834,6 +838,7 @@ struct RunRows {
     Cl = Cb + lane * EPP;
     bias = (p.bias && valid) ? p.bias[d] : 0.f;
     Dd = (p.D && valid) ? p.D[d] : 0.f;
+    tok_c0 = (g - b * p.gpb) * 16;
   }
 };
 
@@ -851,7 +856,26 @@ __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, 
   const int c = lane & 15, j8 = (lane >> 4) * 8;
   const int64_t L = p.L, t0 = k * kTW;
   const bool whole = t0 + kTW <= L;
-  if (whole && rr.valid && p.io_vec) {
+  bool tok_done = false;
+  if constexpr (sizeof(T) == 2) {
+   if (p.tok) {
+    // token-major: the tile is [step][16 channels]; lane l copies step l / 2,
+    // channels 8 (l % 2) .. +8 (16 bytes of bf16; dim % 8 == 0, 16-byte rows)
+    tok_done = true;
+    const int t = lane >> 1, half = lane & 1;
+    const int64_t g0 = rr.tok_c0;
+    const bool in = t0 + t < L && g0 + half * 8 < p.dim;
+    const int64_t off = in ? (t0 + t) * p.dim + half * 8 : 0;
+    T *du = &raw.u[0][0] + t * 16 + half * 8;
+    T *dd = &raw.d[0][0] + t * 16 + half * 8;
+    T *dz = &raw.z[0][0] + t * 16 + half * 8;
+    cp_async16(du, rr.u + off, in ? 16 : 0);
+    cp_async16(dd, rr.dr + off, in ? 16 : 0);
+    if (rr.z) cp_async16(dz, rr.z + off, in ? 16 : 0);
+   }
+  }
+  if (tok_done) {
+  } else if (whole && rr.valid && p.io_vec) {
 #pragma unroll
     for (int q = 0; q < 8 / EPP; ++q) {
       cp_async16(&raw.u[c][j8 + q * EPP], rr.u + t0 + q * EPP, 16);
@@ -914,6 +938,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   const int c = lane & 15, j8 = (lane >> 4) * 8;
   const bool io_vec = p.io_vec != 0;
   const bool has_z = p.z != nullptr;
+  const bool tok = p.tok != 0;  // u/delta/z/y laid out [batch][seqlen][dim]
   // the chunk whose output epilogue is pending: its stage, row, gate, D*u
   bool pend = false, pvalid = false;
   int pstage = 0;
@@ -962,9 +987,16 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
       const int64_t t0 = k * kTW;
       const bool whole = cur.valid && t0 + kTW <= L;
       cp_async_wait<kSlots - 2>();  // this chunk's copies have landed
+      if (tok) __syncwarp();  // token-major tiles hold other lanes' copies
       // ---- pre-pass of chunk k into the stage: Delta, Delta*u, B/C in fp32 ----
       float u8[8], s8[8];
-      {
+      if (tok) {  // [step][channel] tile: this lane's channel c at steps j8..j8+7
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          u8[i] = io_to_f((&raw.u[0][0])[(j8 + i) * 16 + c]);
+          s8[i] = io_to_f((&raw.d[0][0])[(j8 + i) * 16 + c]);
+        }
+      } else {
         Vec8<T> vu, vd;
         vu.load_shared(&raw.u[c][j8]);
         vd.load_shared(&raw.d[c][j8]);
@@ -1038,7 +1070,13 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             unpack2(mul2(add2(add2(ya[i], yb[i]), du2[i]), gate2[i]), o[2 * i], o[2 * i + 1]);
-          IO<T>::store8(py, pt, L - j8, io_vec, o);
+          if (tok) {  // time stride dim; a warp's 16 channels of a step are contiguous
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (pt + j8 + i < L) IO<T>::store1(py, (pt + j8 + i) * p.dim + c, o[i]);
+          } else {
+            IO<T>::store8(py, pt, L - j8, io_vec, o);
+          }
         }
       }
       // ---- gate and D*u of chunk k, for its epilogue in the next iteration ----
@@ -1048,9 +1086,14 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
         for (int i = 0; i < 4; ++i) du2[i] = mul2(D2, pack2(u8[2 * i], u8[2 * i + 1]));
         if (has_z) {
           float z8[8];
-          Vec8<T> vz;
-          vz.load_shared(&raw.z[c][j8]);
-          vz.unpack(z8);
+          if (tok) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) z8[i] = io_to_f((&raw.z[0][0])[(j8 + i) * 16 + c]);
+          } else {
+            Vec8<T> vz;
+            vz.load_shared(&raw.z[c][j8]);
+            vz.unpack(z8);
+          }
 #pragma unroll
           for (int i = 0; i < 4; ++i) gate2[i] = silu2(pack2(z8[2 * i], z8[2 * i + 1]));
         } else {
@@ -1080,7 +1123,13 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
         o[2 * i] = (o[2 * i] + d0) * g0;
         o[2 * i + 1] = (o[2 * i + 1] + d1) * g1;
       }
-      IO<T>::store8(py, pt, L - j8, io_vec, o);
+      if (tok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (pt + j8 + i < L) IO<T>::store1(py, (pt + j8 + i) * p.dim + c, o[i]);
+      } else {
+        IO<T>::store8(py, pt, L - j8, io_vec, o);
+      }
     }
   }
   cp_async_wait<0>();

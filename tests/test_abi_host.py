@@ -219,7 +219,7 @@ def test_conv_empty_problem_is_a_noop(lib):
 
 
 def test_flags_checked_before_launch(lib):
-    assert _fwd(lib, _shape(flags=4)) == _lib.SSM_ERR_INVALID_ARG  # an unknown bit
+    assert _fwd(lib, _shape(flags=8)) == _lib.SSM_ERR_INVALID_ARG  # an unknown bit
     # exact ZOH runs on the look-back path only; other explicit paths are refused
     for path in (_lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP, _lib.SSM_PATH_LOOKBACK_WS):
         assert _fwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path)) == \
@@ -240,3 +240,12 @@ def test_saved_states_flag_checked_before_launch(lib):
     # a forward workspace for the backward needs the flag, and 256-byte alignment
     assert _bwd(lib, _shape(), fws=256) == _lib.SSM_ERR_INVALID_ARG
     assert _bwd(lib, _shape(flags=save), fws=272) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_token_major_flag_checked_before_launch(lib):
+    tok = _lib.SSM_FLAG_TOKEN_MAJOR
+    assert _fwd(lib, _shape(flags=tok, io_dtype=_lib.SSM_F32)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, _shape(flags=tok, dim=20)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, _shape(flags=tok | _lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, _shape(flags=tok, path=_lib.SSM_PATH_LOOKBACK)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _bwd(lib, _shape(flags=tok)) == _lib.SSM_ERR_UNSUPPORTED

@@ -335,3 +335,23 @@ def test_zero_length_passes_the_state_through(cuda_device):
 def test_single_channel_single_step(cuda_device):
     for dtype in (synth.F32, synth.BF16):
         _check(synth.make_case(1, 1, 1, 16, dtype, seed=77), cuda_device)
+
+
+# ---- token-major activations (batch, seqlen, dim), as a projection writes them ----
+@pytest.mark.parametrize("batch,dim,L", [(2, 64, 256), (1, 40, 333), (3, 8, 17), (2, 1024, 1000)])
+def test_token_major_equals_channel_major(cuda_device, batch, dim, L):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    case = synth.make_case(batch, dim, L, 16, synth.BF16, seed=700 + dim)
+    g = upload(case, cuda_device)
+    y_cm, ls_cm = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                               g["delta_bias"], return_last_state=True, path=PATHS["lookback_ws"])
+    tm = {k: g[k].transpose(1, 2).contiguous() for k in ("u", "delta", "z")}
+    y_tm, ls_tm = ssm.scan_fwd(tm["u"], tm["delta"], g["A"], g["B"], g["C"], g["D"], tm["z"],
+                               g["delta_bias"], return_last_state=True, token_major=True)
+    torch.cuda.synchronize()
+    # the same arithmetic in the same order: only the loads and stores move
+    assert torch.equal(y_tm.transpose(1, 2), y_cm)
+    assert torch.equal(ls_tm, ls_cm)
+    ref = oracle.fwd(case)
+    assert_close(to_f64(y_tm.transpose(1, 2)), ref["y"], synth.BF16, "y")
