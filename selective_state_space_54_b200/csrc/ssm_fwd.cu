@@ -819,6 +819,7 @@ struct RunRows {
   float bias, Dd;
   bool valid;
   int64_t tok_c0;  // token-major: the group's first channel
+  template <bool TOK>
   __device__ __forceinline__ void set(const FwdParams &p, int64_t g, int lane) {
     const int c = lane & 15, j = lane >> 4;
     const int64_t b = g / p.gpb;
@@ -826,8 +827,8 @@ struct RunRows {
     valid = d < p.dim;
     // channel-major: this lane's row at step 8j; token-major: the group's
     // first channel at step 0 (time stride dim)
-    const int64_t row = p.tok ? b * p.L * p.dim + (g - b * p.gpb) * 16
-                              : (b * p.dim + (valid ? d : 0)) * p.L + j * 8;
+    const int64_t row = TOK ? b * p.L * p.dim + (g - b * p.gpb) * 16
+                            : (b * p.dim + (valid ? d : 0)) * p.L + j * 8;
     u = static_cast<const T *>(p.u) + row;
     dr = static_cast<const T *>(p.delta) + row;
     z = p.z ? static_cast<const T *>(p.z) + row : nullptr;
@@ -848,7 +849,7 @@ struct RunRows {
 // the short path; the last chunk of a ragged L, padded channels and
 // unaligned rows take the checked one (zero fill past L).  Every lane later
 // reads only the pieces it copied itself.
-template <typename T, int NP>
+template <typename T, int NP, bool TOK>
 __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, const RunRows<T, NP> &rr,
                                          int64_t k, int lane) {
   constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
@@ -857,8 +858,8 @@ __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, 
   const int64_t L = p.L, t0 = k * kTW;
   const bool whole = t0 + kTW <= L;
   bool tok_done = false;
-  if constexpr (sizeof(T) == 2) {
-   if (p.tok) {
+  if constexpr (TOK && sizeof(T) == 2) {
+   {
     // token-major: the tile is [step][16 channels]; lane l copies step l / 2,
     // channels 8 (l % 2) .. +8 (16 bytes of bf16; dim % 8 == 0, 16-byte rows)
     tok_done = true;
@@ -928,7 +929,7 @@ __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, 
 __device__ __forceinline__ float io_to_f(uint16_t v) { return bf16_to_f(v); }
 __device__ __forceinline__ float io_to_f(float v) { return v; }
 
-template <typename T, int NP>
+template <typename T, int NP, bool TOK>
 __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &sm, const Share &sh,
                                             unsigned bar_full, unsigned bar_ys) {
   constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
@@ -938,7 +939,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   const int c = lane & 15, j8 = (lane >> 4) * 8;
   const bool io_vec = p.io_vec != 0;
   const bool has_z = p.z != nullptr;
-  const bool tok = p.tok != 0;  // u/delta/z/y laid out [batch][seqlen][dim]
+  constexpr bool tok = TOK;  // u/delta/z/y laid out [batch][seqlen][dim]
   // the chunk whose output epilogue is pending: its stage, row, gate, D*u
   bool pend = false, pvalid = false;
   int pstage = 0;
@@ -952,13 +953,13 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   bool pf_live = sh.n_runs > 0;
   if (pf_live) {
     sh.get(0, pg, pk, pk1);
-    pf.set(p, pg, lane);
+    pf.template set<TOK>(p, pg, lane);
   }
   auto advance = [&]() {
     if (++pk >= pk1) {
       if (++pr < sh.n_runs) {
         sh.get(pr, pg, pk, pk1);
-        pf.set(p, pg, lane);
+        pf.template set<TOK>(p, pg, lane);
       } else {
         pf_live = false;
       }
@@ -967,7 +968,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   int it_f = 0;  // chunks fetched (slot cursor)
   for (int i = 0; i < kSlots - 1; ++i) {
     if (pf_live) {
-      ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+      ws_fetch<T, NP, TOK>(p, sm.raw[it_f % kSlots], pf, pk, lane);
       advance();
     }
     cp_async_commit();
@@ -979,7 +980,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
     int64_t g, k0, k1;
     sh.get(r, g, k0, k1);
     RunRows<T, NP> cur;
-    cur.set(p, g, lane);
+    cur.template set<TOK>(p, g, lane);
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = it & 1;
       WSStage<NP> &st = sm.st[stage];
@@ -987,10 +988,10 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
       const int64_t t0 = k * kTW;
       const bool whole = cur.valid && t0 + kTW <= L;
       cp_async_wait<kSlots - 2>();  // this chunk's copies have landed
-      if (tok) __syncwarp();  // token-major tiles hold other lanes' copies
+      if constexpr (tok) __syncwarp();  // token-major tiles hold other lanes' copies
       // ---- pre-pass of chunk k into the stage: Delta, Delta*u, B/C in fp32 ----
       float u8[8], s8[8];
-      if (tok) {  // [step][channel] tile: this lane's channel c at steps j8..j8+7
+      if constexpr (tok) {  // [step][channel] tile: this lane's channel c at steps j8..j8+7
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           u8[i] = io_to_f((&raw.u[0][0])[(j8 + i) * 16 + c]);
@@ -1051,7 +1052,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
       bar_arrive_n(bar_full + stage, 64);
       // ---- copies of the chunk kSlots-1 ahead, into the slot of chunk k-1 ----
       if (pf_live) {
-        ws_fetch<T, NP>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+        ws_fetch<T, NP, TOK>(p, sm.raw[it_f % kSlots], pf, pk, lane);
         advance();
       }
       cp_async_commit();
@@ -1070,7 +1071,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             unpack2(mul2(add2(add2(ya[i], yb[i]), du2[i]), gate2[i]), o[2 * i], o[2 * i + 1]);
-          if (tok) {  // time stride dim; a warp's 16 channels of a step are contiguous
+          if constexpr (tok) {  // time stride dim; a warp's 16 channels of a step are contiguous
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               if (pt + j8 + i < L) IO<T>::store1(py, (pt + j8 + i) * p.dim + c, o[i]);
@@ -1086,7 +1087,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
         for (int i = 0; i < 4; ++i) du2[i] = mul2(D2, pack2(u8[2 * i], u8[2 * i + 1]));
         if (has_z) {
           float z8[8];
-          if (tok) {
+          if constexpr (tok) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) z8[i] = io_to_f((&raw.z[0][0])[(j8 + i) * 16 + c]);
           } else {
@@ -1123,7 +1124,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
         o[2 * i] = (o[2 * i] + d0) * g0;
         o[2 * i + 1] = (o[2 * i + 1] + d1) * g1;
       }
-      if (tok) {
+      if constexpr (tok) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           if (pt + j8 + i < L) IO<T>::store1(py, (pt + j8 + i) * p.dim + c, o[i]);
@@ -1135,7 +1136,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   cp_async_wait<0>();
 }
 
-template <typename T, int NP>
+template <typename T, int NP, bool TOK>
 __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
@@ -1146,7 +1147,7 @@ __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   if (w >= p.n_workers) return;  // both warps of a pair leave together
   const Share sh(w, p.n_workers, p.n_groups, p.n_chunks);
   const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
-  if (producer) ws_producer<T, NP>(p, sm, sh, bar_full, bar_ys);
+  if (producer) ws_producer<T, NP, TOK>(p, sm, sh, bar_full, bar_ys);
   else ws_consumer<T, NP>(p, sm, w, sh, bar_full, bar_ys);
 }
 
@@ -1242,9 +1243,9 @@ cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm) {
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value;
     const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
-    cudaError_t e = allow_smem(k_fwd_ws<T, kNP>, smem);
+    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false>, smem);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP>, kWSThreads,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP, false>, kWSThreads,
                                                          smem);
   });
 }
@@ -1254,10 +1255,20 @@ cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value;
     const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
-    cudaError_t e = allow_smem(k_fwd_ws<T, kNP>, smem);
-    if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((p.n_workers + kPairs - 1) / kPairs);
-    k_fwd_ws<T, kNP><<<grid, kWSThreads, smem, s>>>(p);
+    if (p.tok) {  // token-major tiles: bf16 only (the API checks)
+      if constexpr (sizeof(T) == 2) {
+        cudaError_t e = allow_smem(k_fwd_ws<T, kNP, true>, smem);
+        if (e != cudaSuccess) return e;
+        k_fwd_ws<T, kNP, true><<<grid, kWSThreads, smem, s>>>(p);
+        return cudaGetLastError();
+      } else {
+        return cudaErrorInvalidValue;
+      }
+    }
+    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false>, smem);
+    if (e != cudaSuccess) return e;
+    k_fwd_ws<T, kNP, false><<<grid, kWSThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }
