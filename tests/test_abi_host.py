@@ -249,3 +249,19 @@ def test_token_major_flag_checked_before_launch(lib):
     assert _fwd(lib, _shape(flags=tok | _lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED
     assert _fwd(lib, _shape(flags=tok, path=_lib.SSM_PATH_LOOKBACK)) == _lib.SSM_ERR_UNSUPPORTED
     assert _bwd(lib, _shape(flags=tok)) == _lib.SSM_ERR_UNSUPPORTED
+
+
+def test_c_program_against_the_header(lib, tmp_path):
+    # the ABI from C: compile a small C caller against include/ssm_scan.h and link it
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(os.path.dirname(__file__), "c_abi", "abi_check.c")
+    exe = str(tmp_path / "abi_check")
+    libdir = os.path.dirname(LIB)
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-I", INCLUDE, src, "-o", exe,
+                           "-L", libdir, "-lssmscan", "-Wl,-rpath," + libdir])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
