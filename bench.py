@@ -481,8 +481,25 @@ def measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None, 
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(ev0.elapsed_time(ev1) / k)
+    # the backward on the same shape: x and dout read, dx written
+    dout = torch.empty_like(x).normal_()
+
+    def step_bwd():
+        ssm.causal_conv1d_bwd(x, wt, bt, dout)
+
+    for _ in range(max(3, args.warmup)):
+        step_bwd()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(k):
+        step_bwd()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_b = max_over_ranks(ev0.elapsed_time(ev1) / k)
     es = x.element_size()
     nbytes = 2 * es * w.bld + 4 * w.batch * w.dim * (width - 1) + 4 * w.dim * (width + 1)
+    nbytes_b = 3 * es * w.bld + 4 * w.dim * (2 * width + 2)
     pk = peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
@@ -493,6 +510,9 @@ def measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None, 
                          "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": "k_conv",
                          "algorithmic_bytes": nbytes,
                          "peak_basis": f"measured copy bandwidth ({pk['source']})"},
+            "bwd": {"ms_per_step": ms_b, "algorithmic_bytes": nbytes_b,
+                    "achieved_gbs": nbytes_b / (ms_b * 1e-3) / 1e9,
+                    "frac": nbytes_b / (ms_b * 1e-3) / 1e9 / pk["hbm_gbs"], "kernel": "k_conv_bwd"},
             "gpu_launches": k}
 
 

@@ -250,6 +250,23 @@ ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t
                              const float *bias, const float *initial_state, int silu,
                              void *out, float *final_state, ssm_stream_t stream);
 
+/* Backward of ssm_causal_conv1d: gradients of sum(dout * out) with respect
+ * to x, weight, bias and the initial state, for the same arguments as the
+ * forward call.  With a_t = bias + sum_k weight_k x_{t-width+1+k} and
+ * out_t = act(a_t): da_t = dout_t act'(a_t); dx_s = sum_k weight_k
+ * da_{s+width-1-k}; dweight_k = sum over batch and t of da_t x_{t-width+1+k};
+ * dbias = sum of da_t.  The activations are recomputed, never stored.
+ *  dout, dx                  [batch][dim][seqlen] io dtype (dx overwritten)
+ *  dweight                   [dim][width] fp32, overwritten (required)
+ *  dbias                     [dim] fp32, exactly when bias is given
+ *  dinitial_state            [batch][dim][width-1] fp32, nullable
+ * Argument checks as in the forward.  dx may not alias x or dout. */
+ssm_status ssm_causal_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
+                                 int32_t io_dtype, const void *x, const float *weight,
+                                 const float *bias, const float *initial_state, int silu,
+                                 const void *dout, void *dx, float *dweight, float *dbias,
+                                 float *dinitial_state, ssm_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the device error word of
  * `workspace`.  SSM_OK, SSM_ERR_DEVICE_TIMEOUT or SSM_ERR_CUDA. */
 ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream);

@@ -152,3 +152,41 @@ def conv1d(x, weight, bias=None, *, dtype=None, initial_state=None, silu: bool =
     if silu:
         out = out / (1.0 + np.exp(-out))
     return out, xp[:, :, L:L + K - 1].copy()
+
+
+def conv1d_bwd(x, weight, bias, dout, *, dtype=None, initial_state=None, silu: bool = True):
+    """Gradients of sum(dout * conv1d(x, weight, bias, initial_state, silu)).
+
+    Written from the forward's definition (``conv1d`` above): with
+    a_t = bias + sum_k w_k x_{t-K+1+k} and out_t = act(a_t),
+        da_t    = dout_t * act'(a_t)           (SiLU'(a) = s (1 + a (1 - s)), s = sigmoid(a))
+        dx_s    = sum_k w_k da_{s+K-1-k}       (terms with s+K-1-k < L)
+        dw_k    = sum_{b,t} da_t x_{t-K+1+k}   (x_{<0} from the initial state)
+        dbias   = sum_{b,t} da_t
+    and the initial state's gradient is dx for the K-1 inputs before t = 0.
+    Returns a dict of fp64 arrays: dx, dweight, dbias, dinitial_state.
+    """
+    xs = _f64(x, dtype)
+    g = _f64(dout, dtype)
+    w = np.asarray(weight, np.float64)
+    bt, dm, L = xs.shape
+    K = w.shape[1]
+    prev = np.zeros((bt, dm, K - 1)) if initial_state is None else \
+        np.asarray(initial_state, np.float64).reshape(bt, dm, K - 1)
+    xp = np.concatenate([prev, xs], axis=-1)          # x_{-(K-1)} .. x_{L-1}
+    a = np.zeros((bt, dm, L))
+    for k in range(K):
+        a += w[None, :, k, None] * xp[:, :, k:k + L]
+    if bias is not None:
+        a += np.asarray(bias, np.float64)[None, :, None]
+    if silu:
+        sg = 1.0 / (1.0 + np.exp(-a))
+        da = g * sg * (1.0 + a * (1.0 - sg))
+    else:
+        da = g
+    dxp = np.zeros((bt, dm, L + K - 1))              # gradient of every entry of xp
+    for k in range(K):
+        dxp[:, :, k:k + L] += w[None, :, k, None] * da
+    dw = np.stack([(da * xp[:, :, k:k + L]).sum(axis=(0, 2)) for k in range(K)], axis=1)
+    return {"dx": dxp[:, :, K - 1:], "dweight": dw, "dbias": da.sum(axis=(0, 2)),
+            "dinitial_state": dxp[:, :, :K - 1].copy()}

@@ -23,7 +23,7 @@ from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_FLAG_SAVE_STATES,  # noqa:
                    SSM_PATH_LOOKBACK, SSM_PATH_LOOKBACK_WS, SSM_PATH_PER_GROUP, SSM_PATH_SPLIT_L,
                    ssm_shape)
 
-__all__ = ["scan_fwd", "scan_bwd", "scan_step", "causal_conv1d", "fwd_workspace_bytes", "bwd_workspace_bytes",
+__all__ = ["scan_fwd", "scan_bwd", "scan_step", "causal_conv1d", "causal_conv1d_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes",
            "fwd_path", "check", "ScanError", "make_shape"]
 
 
@@ -205,6 +205,31 @@ def causal_conv1d(x, weight, bias=None, *, initial_state=None, silu=True, out=No
     if return_final_state:
         return out, final_state
     return out
+
+
+def causal_conv1d_bwd(x, weight, bias, dout, *, initial_state=None, silu=True,
+                      want_dinitial_state=False, stream=None):
+    """Backward of causal_conv1d: returns dict(dx, dweight, dbias, dinitial_state)."""
+    import torch
+    batch, dim, seqlen = x.shape
+    width = weight.shape[-1]
+    dev, f32 = x.device, torch.float32
+    _check_io("x", x, (batch, dim, seqlen), x.dtype, dev)
+    _check_io("dout", dout, (batch, dim, seqlen), x.dtype, dev)
+    _check_io("weight", weight, (dim, width), f32, dev)
+    _check_io("bias", bias, (dim,), f32, dev)
+    _check_io("initial_state", initial_state, (batch, dim, width - 1), f32, dev)
+    g = {"dx": torch.empty_like(x), "dweight": torch.empty((dim, width), dtype=f32, device=dev),
+         "dbias": torch.empty((dim,), dtype=f32, device=dev) if bias is not None else None,
+         "dinitial_state": (torch.empty((batch, dim, width - 1), dtype=f32, device=dev)
+                            if want_dinitial_state else None)}
+    rc = _lib.load().ssm_causal_conv1d_bwd(
+        batch, dim, seqlen, width, _io_dtype(x), _ptr(x), _ptr(weight), _ptr(bias),
+        _ptr(initial_state), int(bool(silu)), _ptr(dout), _ptr(g["dx"]), _ptr(g["dweight"]),
+        _ptr(g["dbias"]), _ptr(g["dinitial_state"]), _stream(stream))
+    if rc != 0:
+        raise ScanError(rc, "ssm_causal_conv1d_bwd")
+    return g
 
 
 def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,

@@ -39,7 +39,7 @@ EXPORTS = (
     "ssm_scan_fwd_workspace_bytes", "ssm_scan_bwd_workspace_bytes", "ssm_scan_fwd",
     "ssm_scan_bwd", "ssm_scan_check", "ssm_scan_test_wait_timeout", "ssm_scan_fwd_path",
     "ssm_status_string", "ssm_scan_version", "ssm_scan_fwd_noalloc", "ssm_scan_step",
-    "ssm_causal_conv1d",
+    "ssm_causal_conv1d", "ssm_causal_conv1d_bwd",
 )
 
 
@@ -81,6 +81,9 @@ def load(path: str | None = None):
     lib.ssm_scan_step.restype = ci
     lib.ssm_causal_conv1d.argtypes = [i64, i64, i64, i32, i32, vp, vp, vp, vp, ci, vp, vp, vp]
     lib.ssm_causal_conv1d.restype = ci
+    lib.ssm_causal_conv1d_bwd.argtypes = [i64, i64, i64, i32, i32, vp, vp, vp, vp, ci, vp, vp, vp, vp,
+                                          vp, vp]
+    lib.ssm_causal_conv1d_bwd.restype = ci
     lib.ssm_scan_check.argtypes = [vp, vp]
     lib.ssm_scan_check.restype = ci
     lib.ssm_scan_test_wait_timeout.argtypes = [vp, sz, i64, vp]

@@ -334,6 +334,41 @@ ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t
   return cuda_status(launch_conv(io_dtype, p, s));
 }
 
+ssm_status ssm_causal_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
+                                 int32_t io_dtype, const void *x, const float *weight,
+                                 const float *bias, const float *initial_state, int silu,
+                                 const void *dout, void *dx, float *dweight, float *dbias,
+                                 float *dinitial_state, ssm_stream_t stream) {
+  if (batch < 0 || dim < 0 || seqlen < 0 || width < 1) return SSM_ERR_INVALID_ARG;
+  if (width > 8) return SSM_ERR_UNSUPPORTED;
+  if (io_dtype != SSM_F32 && io_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if ((double)batch * (double)dim * (double)seqlen > 4.0e15) return SSM_ERR_UNSUPPORTED;
+  if ((bias == nullptr) != (dbias == nullptr)) return SSM_ERR_INVALID_ARG;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = io_dtype == SSM_BF16 ? 2 : 4;
+  if (dim > 0 && (!weight || !dweight)) return SSM_ERR_INVALID_ARG;
+  if (!aligned(weight, 4) || !aligned(bias, 4) || !aligned(initial_state, 4) || !aligned(dweight, 4) ||
+      !aligned(dbias, 4) || !aligned(dinitial_state, 4))
+    return SSM_ERR_INVALID_ARG;
+  const int64_t rows = batch * dim;
+  // parameter gradients are sums: start from zero (also when there is no step)
+  cudaError_t e = cudaSuccess;
+  if (dim > 0) e = cudaMemsetAsync(dweight, 0, sizeof(float) * dim * width, s);
+  if (e == cudaSuccess && dim > 0 && dbias) e = cudaMemsetAsync(dbias, 0, sizeof(float) * dim, s);
+  if (e == cudaSuccess && rows > 0 && dinitial_state && width > 1)
+    e = cudaMemsetAsync(dinitial_state, 0, sizeof(float) * rows * (width - 1), s);
+  if (e != cudaSuccess || rows == 0 || seqlen == 0) return cuda_status(e);
+  if (!x || !dout || !dx || !aligned(x, es) || !aligned(dout, es) || !aligned(dx, es))
+    return SSM_ERR_INVALID_ARG;
+  ConvBwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.x = x; p.dout = dout; p.w = weight; p.bias = bias; p.s0 = initial_state;
+  p.dx = dx; p.dw = dweight; p.dbias = dbias; p.ds0 = dinitial_state;
+  p.batch = batch; p.dim = dim; p.L = seqlen; p.K = width; p.silu = silu ? 1 : 0;
+  p.vec = ((seqlen * (int64_t)es) % 16 == 0) && aligned(x, 16) && aligned(dout, 16) && aligned(dx, 16);
+  return cuda_status(launch_conv_bwd(io_dtype, p, s));
+}
+
 size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
   if (check_shape(shape) != SSM_OK) return 0;
   const int NP = fwd_np_for(shape->dstate);

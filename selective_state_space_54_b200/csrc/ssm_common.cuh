@@ -96,6 +96,18 @@ struct ConvParams {
   int vec;                             // 16-byte aligned rows: vector loads and stores
 };
 
+// Causal depthwise conv1d backward parameters (ssm_conv.cu).
+struct ConvBwdParams {
+  const void *x, *dout;                // [batch][dim][L] io dtype
+  const float *w, *bias, *s0;          // [dim][K], [dim] nullable, [batch][dim][K-1] nullable
+  void *dx;                            // [batch][dim][L] io dtype
+  float *dw, *dbias, *ds0;             // [dim][K] (zeroed), [dim] (zeroed) nullable, [batch][dim][K-1] nullable
+  int64_t batch, dim, L;
+  int K;
+  int silu;
+  int vec;                             // 16-byte aligned rows
+};
+
 // Backward parameters (ssm_bwd.cu).
 struct BwdParams {
   const void *u, *delta, *z, *B, *C, *dout;
@@ -307,6 +319,7 @@ size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);
 cudaError_t launch_step(int io_dtype, const StepParams &p, cudaStream_t s);
 cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s);
+cudaError_t launch_conv_bwd(int io_dtype, const ConvBwdParams &p, cudaStream_t s);
 cudaError_t launch_wait_timeout_probe(unsigned *flag, unsigned *err, unsigned long long limit_ns,
                                       cudaStream_t s);
 

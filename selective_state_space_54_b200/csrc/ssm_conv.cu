@@ -155,6 +155,178 @@ __global__ void __launch_bounds__(kConvThreads) k_conv(ConvParams p) {
   }
 }
 
+// ---- backward -------------------------------------------------------------
+// Gradients of sum(dout * out): with a_t = bias + sum_k w_k x_{t-K+1+k} and
+// out_t = act(a_t), da_t = dout_t act'(a_t); dx_s = sum_k w_k da_{s+K-1-k};
+// dw_k = sum_{b,t} da_t x_{t-K+1+k}; dbias = sum_{b,t} da_t; the initial
+// state's gradient is dx of the K-1 inputs before t = 0.  Same warp layout as
+// the forward: a warp recomputes a and da pass by pass, accumulates its dw and
+// dbias partials, and writes dx of the pass before once it has the next pass's
+// first K-1 values of da (a shuffle from lane 0).  The warp's last pass takes
+// them from the next segment, recomputed by lane 31 from memory.
+template <typename T, int K>
+__device__ __forceinline__ float conv_act_grad(float a, float g, bool silu) {
+  if (!silu) return g;
+  const float sg = rcp_approx(1.f + ex2(-a * kLog2e));
+  return g * sg * fmaf(a, 1.f - sg, 1.f);
+}
+
+template <typename T, int K>
+__global__ void __launch_bounds__(kConvThreads) k_conv_bwd(ConvBwdParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
+  const int64_t L = p.L;
+  const int64_t segs = (L + kConvSeg - 1) / kConvSeg;
+  const int64_t row = warp / segs;
+  if (row >= p.batch * p.dim) return;  // whole warps leave together
+  const int64_t seg = warp - row * segs;
+  const int64_t d = row % p.dim;
+  const T *xr = static_cast<const T *>(p.x) + row * L;
+  const T *gr = static_cast<const T *>(p.dout) + row * L;
+  T *dxr = static_cast<T *>(p.dx) + row * L;
+  const bool vec = p.vec != 0;
+  const bool silu = p.silu != 0;
+  Raw8<T> rx[kConvR], rg[kConvR];
+#pragma unroll
+  for (int r = 0; r < kConvR; ++r) {
+    const int64_t t0 = seg * kConvSeg + r * 32 * kConvW + lane * kConvW;
+    rx[r].load(xr, t0, L, vec);
+    rg[r].load(gr, t0, L, vec);
+  }
+  float w[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) w[k] = p.w[d * K + k];
+  const float bias = p.bias ? p.bias[d] : 0.f;
+  // x_t for t < 0: the initial state, else zero
+  auto x_before = [&](int64_t t) -> float {
+    return p.s0 ? p.s0[row * (K - 1) + (K - 1) + t] : 0.f;
+  };
+  float dwp[K], dbp = 0.f;
+#pragma unroll
+  for (int k = 0; k < K; ++k) dwp[k] = 0.f;
+  float carry[K > 1 ? K - 1 : 1];  // x before the pass, as lane 31 of the last pass saw it
+  float da_prev[kConvW];           // da of the pass before, waiting for its dx
+  int64_t t0_prev = 0;
+  bool have_prev = false;
+  // dx of one pass from its da and the next K-1 values of da after the lane's chunk
+  auto emit_dx = [&](const float (&da)[kConvW], const float (&nxt)[K > 1 ? K - 1 : 1], int64_t t0) {
+    float o[kConvW];
+#pragma unroll
+    for (int i = 0; i < kConvW; ++i) {
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int idx = i + (K - 1) - k;  // position of da_{s+K-1-k} in [da | nxt]
+        acc = fmaf(w[k], idx < kConvW ? da[idx] : nxt[idx - kConvW], acc);
+      }
+      o[i] = acc;
+    }
+    if (t0 < L) IO<T>::store8(dxr, t0, L, vec, o);
+  };
+#pragma unroll
+  for (int r = 0; r < kConvR; ++r) {
+    const int64_t t0 = seg * kConvSeg + r * 32 * kConvW + lane * kConvW;
+    const bool live = seg * kConvSeg + r * 32 * kConvW < L;  // warp-uniform
+    float v[kConvW], gv[kConvW];
+    rx[r].unpack(v);
+    rg[r].unpack(gv);
+    float halo[K > 1 ? K - 1 : 1];
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) {
+      const float up = __shfl_up_sync(0xffffffffu, v[kConvW - (K - 1) + i], 1);
+      const float last = __shfl_sync(0xffffffffu, v[kConvW - (K - 1) + i], 31);
+      if (lane > 0) {
+        halo[i] = up;
+      } else if (r > 0) {
+        halo[i] = carry[i];
+      } else {
+        const int64_t t = t0 - (K - 1) + i;
+        halo[i] = t >= 0 ? IO<T>::get(xr, t) : x_before(t);
+      }
+      carry[i] = last;
+    }
+    float da[kConvW];
+#pragma unroll
+    for (int i = 0; i < kConvW; ++i) {
+      float acc = bias;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int idx = i - (K - 1) + k;
+        acc = fmaf(w[k], idx < 0 ? halo[idx + K - 1] : v[idx], acc);
+      }
+      da[i] = (t0 + i < L) ? conv_act_grad<T, K>(acc, gv[i], silu) : 0.f;
+      dbp += da[i];
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int idx = i - (K - 1) + k;
+        dwp[k] = fmaf(da[i], idx < 0 ? halo[idx + K - 1] : v[idx], dwp[k]);
+      }
+    }
+    // the next K-1 values of da after each lane's chunk of the pass before: the
+    // next lane's first values, or for lane 31 this pass's lane 0
+    if (have_prev) {
+      float nxt[K > 1 ? K - 1 : 1];
+#pragma unroll
+      for (int m = 0; m < K - 1; ++m) {
+        const float down = __shfl_down_sync(0xffffffffu, da_prev[m], 1);
+        const float first = __shfl_sync(0xffffffffu, da[m], 0);
+        nxt[m] = lane < 31 ? down : (live ? first : 0.f);
+      }
+      emit_dx(da_prev, nxt, t0_prev);
+    }
+    if (!live) { have_prev = false; break; }
+#pragma unroll
+    for (int i = 0; i < kConvW; ++i) da_prev[i] = da[i];
+    t0_prev = t0;
+    have_prev = true;
+    // initial-state gradient: dx of x_{-(K-1)+j} = sum_k w_k da_{j-k}, j - k >= 0
+    if (K > 1 && p.ds0 && seg == 0 && r == 0 && lane == 0) {
+#pragma unroll
+      for (int j = 0; j < K - 1; ++j) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+          if (j - k >= 0) acc = fmaf(w[k], da[j - k], acc);
+        p.ds0[row * (K - 1) + j] = acc;
+      }
+    }
+  }
+  if (have_prev) {  // the last pass: its next values come from the next segment
+    float nxt[K > 1 ? K - 1 : 1];
+#pragma unroll
+    for (int m = 0; m < K - 1; ++m) {
+      const float down = __shfl_down_sync(0xffffffffu, da_prev[m], 1);
+      nxt[m] = down;
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int m = 0; m < K - 1; ++m) {
+        const int64_t t = t0_prev + kConvW + m;  // a step of the next segment
+        float acc = bias;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const int64_t tx = t - (K - 1) + k;
+          acc = fmaf(w[k], tx < L ? IO<T>::get(xr, tx) : 0.f, acc);
+        }
+        nxt[m] = t < L ? conv_act_grad<T, K>(acc, IO<T>::get(gr, t), silu) : 0.f;
+      }
+    }
+    emit_dx(da_prev, nxt, t0_prev);
+  }
+  // dw and dbias: warp sums, one atomic per warp
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) dwp[k] += __shfl_xor_sync(0xffffffffu, dwp[k], o);
+    dbp += __shfl_xor_sync(0xffffffffu, dbp, o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) atomicAdd(&p.dw[d * K + k], dwp[k]);
+    if (p.dbias) atomicAdd(&p.dbias[d], dbp);
+  }
+}
+
 template <typename T>
 static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
   const int64_t segs = (p.L + kConvSeg - 1) / kConvSeg;
@@ -178,6 +350,31 @@ static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
 
 cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s) {
   return io_dtype == 1 ? launch_conv_t<uint16_t>(p, s) : launch_conv_t<float>(p, s);
+}
+
+template <typename T>
+static cudaError_t launch_conv_bwd_t(const ConvBwdParams &p, cudaStream_t s) {
+  const int64_t segs = (p.L + kConvSeg - 1) / kConvSeg;
+  const int64_t warps = p.batch * p.dim * segs;
+  const int64_t blocks = (warps * 32 + kConvThreads - 1) / kConvThreads;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  const unsigned g = (unsigned)blocks;
+  switch (p.K) {
+    case 1: k_conv_bwd<T, 1><<<g, kConvThreads, 0, s>>>(p); break;
+    case 2: k_conv_bwd<T, 2><<<g, kConvThreads, 0, s>>>(p); break;
+    case 3: k_conv_bwd<T, 3><<<g, kConvThreads, 0, s>>>(p); break;
+    case 4: k_conv_bwd<T, 4><<<g, kConvThreads, 0, s>>>(p); break;
+    case 5: k_conv_bwd<T, 5><<<g, kConvThreads, 0, s>>>(p); break;
+    case 6: k_conv_bwd<T, 6><<<g, kConvThreads, 0, s>>>(p); break;
+    case 7: k_conv_bwd<T, 7><<<g, kConvThreads, 0, s>>>(p); break;
+    case 8: k_conv_bwd<T, 8><<<g, kConvThreads, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv_bwd(int io_dtype, const ConvBwdParams &p, cudaStream_t s) {
+  return io_dtype == 1 ? launch_conv_bwd_t<uint16_t>(p, s) : launch_conv_bwd_t<float>(p, s);
 }
 
 }  // namespace ssm

@@ -265,3 +265,17 @@ def test_c_program_against_the_header(lib, tmp_path):
                            "-L", libdir, "-lssmscan", "-Wl,-rpath," + libdir])
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
+
+
+def test_conv_bwd_rejects_bad_arguments_before_launch(lib):
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(batch=2, dim=4, L=64, K=4, dtype=_lib.SSM_BF16, x=16, w=16, bias=None, dout=16, dx=16,
+             dw=16, db=None):
+        return lib.ssm_causal_conv1d_bwd(batch, dim, L, K, dtype, v(x), v(w), v(bias), None, 1,
+                                         v(dout), v(dx), v(dw), v(db), None, None)
+    assert call(batch=-1) == _lib.SSM_ERR_INVALID_ARG
+    assert call(K=9) == _lib.SSM_ERR_UNSUPPORTED
+    assert call(bias=16) == _lib.SSM_ERR_INVALID_ARG          # dbias missing
+    assert call(dw=None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(w=6) == _lib.SSM_ERR_INVALID_ARG

@@ -108,3 +108,60 @@ def test_conv_zero_length_passes_the_state_through(cuda_device):
     out2, fs2 = ssm.causal_conv1d(x, w, return_final_state=True)
     torch.cuda.synchronize()
     assert out.numel() == 0 and torch.equal(fs, s0) and not fs2.any()
+
+
+# ---- backward --------------------------------------------------------------------
+def _run_bwd(x, w, b, s0, dout, dtype, device, silu=True):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    f = lambda a: None if a is None else torch.from_numpy(a).to(device)
+    g = ssm.causal_conv1d_bwd(to_torch(x, dtype, device), f(w), f(b), to_torch(dout, dtype, device),
+                              initial_state=f(s0), silu=silu, want_dinitial_state=True)
+    torch.cuda.synchronize()
+    return {k: (None if v is None else to_f64(v)) for k, v in g.items()}
+
+
+def _check_bwd(batch, dim, L, K, dtype, seed, device, with_bias=True, with_state=True, silu=True):
+    x, w, b, s0 = _inputs(batch, dim, L, K, dtype, seed)
+    dout = synth.normal((batch, dim, L), seed, "dy", dtype)
+    b = b if with_bias else None
+    s0 = s0 if with_state else None
+    ref = oracle.conv1d_bwd(x, w, b, dout, dtype=dtype, initial_state=s0, silu=silu)
+    got = _run_bwd(x, w, b, s0, dout, dtype, device, silu)
+    assert_close(got["dx"], ref["dx"], dtype, "dx")
+    # parameter sums are fp32 sums of bf16-input terms: the bf16 path's tolerance
+    assert_close(got["dweight"], ref["dweight"], dtype, "dweight", stored_bf16=False)
+    if with_bias:
+        assert_close(got["dbias"], ref["dbias"], dtype, "dbias", stored_bf16=False)
+    if K > 1:
+        assert_close(got["dinitial_state"], ref["dinitial_state"], dtype, "dinitial_state",
+                     stored_bf16=False)
+
+
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("K", [1, 2, 4, 8])
+def test_conv_bwd_widths(cuda_device, dtype, K):
+    _check_bwd(2, 24, 1500, K, dtype, 80 + K, cuda_device)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 7, 8, 9, 255, 256, 257, 1023, 1024, 1025, 3000])
+def test_conv_bwd_ragged_lengths(cuda_device, L):
+    _check_bwd(2, 5, L, 4, synth.F32, 90 + L, cuda_device)
+
+
+@pytest.mark.parametrize("opt", ["no_bias", "no_state", "no_silu"])
+def test_conv_bwd_optional_terms(cuda_device, opt):
+    _check_bwd(1, 16, 700, 4, synth.F32, 13, cuda_device, with_bias=opt != "no_bias",
+               with_state=opt != "no_state", silu=opt != "no_silu")
+
+
+def test_conv_bwd_full_mamba_2p8b_layer(cuda_device):
+    # the x_proj shape at full size; dx on sampled rows, parameter sums in full
+    w_ = synth.WORKLOADS["mamba-2.8b-layer"]
+    x, w, b, _ = _inputs(w_.batch, w_.dim, w_.seqlen, 4, synth.BF16, 22)
+    dout = synth.normal((w_.batch, w_.dim, w_.seqlen), 22, "dy", synth.BF16)
+    got = _run_bwd(x, w, b, None, dout, synth.BF16, cuda_device)
+    ref = oracle.conv1d_bwd(x, w, b, dout, dtype=synth.BF16)
+    assert_close(got["dx"], ref["dx"], synth.BF16, "dx")
+    assert_close(got["dweight"], ref["dweight"], synth.BF16, "dweight", stored_bf16=False)
+    assert_close(got["dbias"], ref["dbias"], synth.BF16, "dbias", stored_bf16=False)

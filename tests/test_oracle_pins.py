@@ -366,3 +366,35 @@ def test_conv_streaming_in_pieces():
     # shorter than the window: the state shifts through
     e, se = oracle.conv1d(x[:, :, :2], w, b, initial_state=s0)
     assert np.array_equal(se, np.concatenate([s0[:, :, 2:], x[:, :, :2]], axis=-1))
+
+
+def test_conv_backward_matches_finite_differences():
+    # central differences of L = sum(dout * conv1d(...)) in fp64, every input
+    x, w, b, s0 = _conv_inputs(5, bt=1, dm=2, L=12, K=4)
+    dout = np.random.default_rng(6).standard_normal(x.shape)
+    g = oracle.conv1d_bwd(x, w, b, dout, initial_state=s0)
+    loss = lambda xx, ww, bb, ss: float((dout * oracle.conv1d(xx, ww, bb, initial_state=ss)[0]).sum())
+    eps = 1e-6
+    for name, arr, key in (("x", x, "dx"), ("w", w, "dweight"), ("b", b, "dbias"),
+                           ("s0", s0, "dinitial_state")):
+        num = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            args = {"x": x.copy(), "w": w.copy(), "b": b.copy(), "s0": s0.copy()}
+            args[name][i] += eps
+            hi = loss(args["x"], args["w"], args["b"], args["s0"])
+            args[name][i] -= 2 * eps
+            lo = loss(args["x"], args["w"], args["b"], args["s0"])
+            num[i] = (hi - lo) / (2 * eps)
+        np.testing.assert_allclose(g[key], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_conv_backward_without_activation_is_the_adjoint():
+    # linear case: <dout, conv(x)> = <conv^T(dout), x> for the x part (bias and state zero)
+    x, w, _, _ = _conv_inputs(7, bt=2, dm=3, L=30, K=3)
+    dout = np.random.default_rng(8).standard_normal(x.shape)
+    out, _ = oracle.conv1d(x, w, silu=False)
+    g = oracle.conv1d_bwd(x, w, None, dout, silu=False)
+    np.testing.assert_allclose((dout * out).sum(), (g["dx"] * x).sum(), rtol=1e-12)
+    np.testing.assert_allclose(g["dbias"], dout.sum(axis=(0, 2)), rtol=1e-12)
