@@ -172,7 +172,7 @@ __device__ __forceinline__ float conv_act_grad(float a, float g, bool silu) {
 }
 
 template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads) k_conv_bwd(ConvBwdParams p) {
+__global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 : 1) k_conv_bwd(ConvBwdParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
   const int64_t L = p.L;
