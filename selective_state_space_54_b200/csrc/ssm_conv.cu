@@ -18,6 +18,32 @@
 namespace ssm {
 
 constexpr int kConvThreads = 256;
+
+// packed fp32 pairs (sm_100a f32x2 arithmetic)
+typedef unsigned long long f2;
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 constexpr int kConvW = 8;                  // steps per lane and pass
 constexpr int kConvR = 4;                  // passes per warp, all loads issued first
 constexpr int kConvSeg = 32 * kConvW * kConvR;  // steps per warp
@@ -245,7 +271,7 @@ __global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 :
       }
       carry[i] = last;
     }
-    float da[kConvW];
+    float da[kConvW], pre[kConvW];
 #pragma unroll
     for (int i = 0; i < kConvW; ++i) {
       float acc = bias;
@@ -254,7 +280,31 @@ __global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 :
         const int idx = i - (K - 1) + k;
         acc = fmaf(w[k], idx < 0 ? halo[idx + K - 1] : v[idx], acc);
       }
-      da[i] = (t0 + i < L) ? conv_act_grad<T, K>(acc, gv[i], silu) : 0.f;
+      pre[i] = acc;
+    }
+    // da = dout * SiLU'(a) = g s (1 + a (1 - s)), s = 1 / (1 + e^-a), on pairs
+#pragma unroll
+    for (int i = 0; i < kConvW; i += 2) {
+      if (silu) {
+        float e0, e1, s0, s1;
+        unpack2(mul2(pack2(pre[i], pre[i + 1]), pack2(-kLog2e, -kLog2e)), e0, e1);
+        unpack2(add2(pack2(ex2(e0), ex2(e1)), pack2(1.f, 1.f)), s0, s1);
+        const f2 sg = pack2(rcp_approx(s0), rcp_approx(s1));
+        const f2 a2 = pack2(pre[i], pre[i + 1]);
+        const f2 one_m = fma2(sg, pack2(-1.f, -1.f), pack2(1.f, 1.f));
+        const f2 fac = fma2(a2, one_m, pack2(1.f, 1.f));
+        unpack2(mul2(mul2(pack2(gv[i], gv[i + 1]), sg), fac), da[i], da[i + 1]);
+      } else {
+        da[i] = gv[i];
+        da[i + 1] = gv[i + 1];
+      }
+    }
+    if (!(t0 + kConvW <= L)) {  // the chunk holding step L-1: no gradient past L
+#pragma unroll
+      for (int i = 0; i < kConvW; ++i) da[i] = t0 + i < L ? da[i] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kConvW; ++i) {
       dbp += da[i];
 #pragma unroll
       for (int k = 0; k < K; ++k) {
