@@ -146,7 +146,17 @@ __global__ void __launch_bounds__(kConvThreads) k_conv(ConvParams p) {
         const int idx = i - (K - 1) + k;  // position in [halo | v]
         acc = fmaf(w[k], idx < 0 ? halo[idx + K - 1] : v[idx], acc);
       }
-      o[i] = p.silu ? silu_fast(acc) : acc;
+      o[i] = acc;
+    }
+    if (p.silu) {  // SiLU(a) = a / (1 + e^-a), on pairs
+#pragma unroll
+      for (int i = 0; i < kConvW; i += 2) {
+        const f2 a2 = pack2(o[i], o[i + 1]);
+        float e0, e1, d0, d1;
+        unpack2(mul2(a2, pack2(-kLog2e, -kLog2e)), e0, e1);
+        unpack2(add2(pack2(ex2(e0), ex2(e1)), pack2(1.f, 1.f)), d0, d1);
+        unpack2(mul2(a2, pack2(rcp_approx(d0), rcp_approx(d1))), o[i], o[i + 1]);
+      }
     }
     if (t0 < L) {
       if (vec && t0 + kConvW <= L) {
