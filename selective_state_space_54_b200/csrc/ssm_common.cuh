@@ -218,8 +218,6 @@ __device__ __forceinline__ float softplus_f(float s) { return s > 20.f ? s : log
 
 __device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
-// SiLU(z) = z * sigmoid(z)
-__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.f + __expf(-z)); }
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
