@@ -340,11 +340,13 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     barrier()
     ms_f = max_over_ranks(t_f / steps)
     ms_b = max_over_ranks(t_b / steps)
-    # the backward's special-function work per (b, t, d, n) element: one ex2
-    # for the chunk recomputation and one for the group recomputation whose
-    # decays the reverse pass reuses (the chunk-entry states come from the
-    # forward, so the backward's own checkpoint pass does not run)
-    ex2_per_element = 2
+    # The roofline counts the method's own special-function work: one exp2
+    # per (b, t, d, n) element (the decay exp(Delta A) the backward must
+    # recompute).  The kernel's own count is reported beside it: it
+    # exponentiates each element twice (once to recompute the 16-step chunk's
+    # sums, once for the 4-step group whose decays the reverse pass reuses).
+    ex2_per_element = 1
+    kernel_ex2 = 2
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
@@ -352,6 +354,8 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     bwd_roofline = {"bound": "alu", "achieved": bwd_achieved / 1e12, "peak": ex2_peak / 1e12,
                     "unit": "Tex2/s", "frac": bwd_achieved / ex2_peak, "traffic": None,
                     "kernel": "k_bwd", "ex2_per_element": ex2_per_element,
+                    "kernel_ex2_per_element": kernel_ex2,
+                    "kernel_mufu_frac": kernel_ex2 * w.bldn / (ms_b * 1e-3) / ex2_peak,
                     "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                                   f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
@@ -360,8 +364,69 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
             "bwd_roofline": bwd_roofline,
             "value": aggregate_value(world, w.bld, (ms_f + ms_b) * 1e-3), "unit": UNIT + " (fwd+bwd)",
             "bwd_value": aggregate_value(world, w.bld, ms_b * 1e-3),
-            "bwd_ex2_per_element": ex2_per_element,
+            "bwd_ex2_per_element": ex2_per_element, "bwd_kernel_ex2_per_element": kernel_ex2,
             "bwd_kernels_per_step": 2}
+
+
+def measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks, name):
+    """The forward alone on another workload (path AUTO, inputs resident in
+    HBM), with its special-function roofline.  The roofline counts the
+    method's one exp2 per (b, t, d, n) element; the split-L schedule's own
+    count (each element exponentiated in both passes) is reported beside it."""
+    w = synth.WORKLOADS[name]
+    case = synth.make_workload(w)
+    g = {k: to_torch(case[k], dev) for k in ("u", "delta", "z", "B", "C")}
+    for k in ("A", "D", "delta_bias"):
+        g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
+    del case
+    y = torch.empty_like(g["u"])
+    ls = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+    shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
+                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32)
+    path = ssm.fwd_path(shape)
+    ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                     y=y, last_state=ls, return_last_state=True, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    ssm.check(ws)
+    k = max(3, min(args.steps, 10 if w.bld > 5e8 else 20))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(k):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ssm.check(ws)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / k)
+    pk = peaks()
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
+    kernel_ex2 = 2 if path == "split_l" else 1
+    achieved = w.bldn / (ms * 1e-3)
+    nbytes = alg_bytes(w)
+    del g, y, ls, ws
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
+            "d_state": w.dstate, "io_dtype": w.dtype, "path": path, "steps": k,
+            "l2": "inputs larger than L2 (no flush)" if nbytes > 126e6 else "L2 resident",
+            "ms_per_step": ms, "value": aggregate_value(world, w.bld, ms * 1e-3), "unit": UNIT,
+            "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": ex2_peak / 1e12,
+                         "unit": "Tex2/s", "frac": achieved / ex2_peak, "traffic": None,
+                         "ex2_per_element": 1, "kernel_ex2_per_element": kernel_ex2,
+                         "kernel_mufu_frac": kernel_ex2 * achieved / ex2_peak,
+                         "algorithmic_bytes": nbytes,
+                         "hbm_achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                         "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
+                                       f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"},
+            "gpu_launches": k * (3 if path == "split_l" else 1)}
 
 
 def decode_bytes(w: synth.Workload) -> int:
@@ -682,8 +747,12 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
         del host, dbuf
 
-    bwd = dec = conv = None
+    bwd = dec = conv = m130 = mlen = None
     if not args.no_bwd and not args.batch:
+        m130 = measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks,
+                               "mamba-130m-layer")
+        mlen = measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks,
+                               "million-length")
         bwd = measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks)
         dec = measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks)
         conv = measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks)
@@ -713,6 +782,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
             "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec, "conv1d": conv, "token_major": tok,
+            "mamba_130m_layer": m130, "million_length": mlen,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, case)

@@ -189,15 +189,25 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
  * start-up.  The pages have no counterpart of this: it is a deployment
  * convenience.  Same arguments and results as ssm_scan_fwd, without the
  * workspace: the scratch lives in one 4 MiB device array inside the library
- * (held on every GPU that loads it until the process exits).  path AUTO
- * means SSM_PATH_LOOKBACK here, whose scratch does not grow with the
- * problem.  Shapes needing more scratch than the array return
- * SSM_ERR_UNSUPPORTED before any launch.  All calls share the array: calls
- * whose kernels overlap on the GPU race, so order them on one stream.  The
- * first call on a device looks up the array's address with that device
- * current; make it before any stream capture.  The device error word sits
- * in the array too, so a bounded look-back wait that gives up is not
- * reported to the caller of this entry point. */
+ * (held on every GPU that loads it until the process exits).
+ *  - path AUTO keeps ssm_scan_fwd's own choice when that is LOOKBACK,
+ *    LOOKBACK_WS (the default for Mamba layer shapes, token-major included)
+ *    or PER_GROUP, whose scratch is bounded by the resident warps or is
+ *    just the error word; where AUTO would pick SPLIT_L, whose scratch grows
+ *    with the problem, it takes LOOKBACK instead.
+ *  - SSM_FLAG_SAVE_STATES returns SSM_ERR_UNSUPPORTED: the saved states
+ *    would sit in the shared array, out of the backward's reach.  The other
+ *    flags behave as in ssm_scan_fwd.
+ *  - Shapes needing more scratch than the array return SSM_ERR_UNSUPPORTED
+ *    before any launch.
+ *  - All calls share the array: calls whose kernels overlap on the GPU
+ *    race, so order them on one stream.
+ *  - Every call looks up the array's address for the current device and
+ *    context (a host-side query; nothing is allocated or cached), so a
+ *    device reset between calls is harmless and a failed lookup fails only
+ *    that call (SSM_ERR_CUDA).
+ *  - The device error word sits in the array too, so a bounded look-back
+ *    wait that gives up is not reported to the caller of this entry point. */
 ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u, const void *delta,
                                 const float *A, const void *B, const void *C,
                                 const float *D, const void *z, const float *delta_bias,

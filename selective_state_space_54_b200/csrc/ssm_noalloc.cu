@@ -16,10 +16,12 @@
 //  - every call shares the one array, so two calls whose kernels overlap on
 //    the GPU (different streams without ordering, or several host threads)
 //    race on it; order them on one stream;
-//  - the first call on a device looks up the array's device address for
-//    that device (cudaGetSymbolAddress, with that device current); make that
-//    first call before any stream capture.
-#include <mutex>
+//  - every call looks up the array's device address for the current device
+//    and context (cudaGetSymbolAddress, a host-side query that allocates
+//    nothing); nothing is cached, so a device reset or a new context between
+//    calls is harmless, and a lookup that fails (for example because the
+//    module cannot be loaded while a stream is being captured) fails only
+//    that call.
 #include <stdio.h>
 #include <string.h>
 
@@ -29,18 +31,10 @@
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;
-constexpr int kMaxDevices = 64;
 
 // The scratch itself.  Host code may not use the symbol as an address: it is
-// a host-side stand-in, so the device address is looked up per device below.
+// a host-side stand-in, so the device address is looked up on every call.
 __device__ __align__(256) unsigned char g_scan_scratch[kStaticScratchBytes];
-
-struct DeviceScratch {
-  std::once_flag once;
-  void *ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-DeviceScratch g_scratch[kMaxDevices];
 
 }  // namespace
 
@@ -51,12 +45,24 @@ extern "C" ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u
                                            float *last_state, ssm_stream_t stream) {
   if (!shape) return SSM_ERR_INVALID_ARG;
   ssm_shape s = *shape;
-  // AUTO takes the look-back schedule here: its scratch is bounded by the
-  // resident warps, not by the problem size.
-  if (s.path == SSM_PATH_AUTO) s.path = SSM_PATH_LOOKBACK;
+  // Saved chunk states would sit in the shared array, where no backward call
+  // can reach them and the next call overwrites them.
+  if (s.flags & SSM_FLAG_SAVE_STATES) {
+    fprintf(stderr, "ssm_scan_fwd_noalloc: SSM_FLAG_SAVE_STATES needs a caller-owned workspace; "
+                    "use ssm_scan_fwd\n");
+    return SSM_ERR_UNSUPPORTED;
+  }
   if (s.batch * s.dim * s.seqlen == 0)  // nothing that needs scratch
     return ssm_scan_fwd(&s, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, y,
                         last_state, nullptr, 0, stream);
+  // AUTO keeps the regular choice when its scratch is bounded by the resident
+  // warps (the look-back schedules, warp-specialised or not) or needs none
+  // (one warp per group); the split-L schedule, whose scratch grows with the
+  // problem, is replaced by the look-back one.
+  if (s.path == SSM_PATH_AUTO) {
+    const int32_t p = ssm_scan_fwd_path(&s);
+    if (p == SSM_PATH_SPLIT_L) s.path = SSM_PATH_LOOKBACK;
+  }
   const size_t need = ssm_scan_fwd_workspace_bytes(&s);
   if (need == 0) {
     // invalid shape, or no device: let the regular checks give the status
@@ -70,21 +76,15 @@ extern "C" ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u
             need, kStaticScratchBytes);
     return SSM_ERR_UNSUPPORTED;
   }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSM_ERR_CUDA;
-  DeviceScratch &ds = g_scratch[dev];
-  std::call_once(ds.once, [&ds]() {
-    void *p = nullptr;
-    ds.err = cudaGetSymbolAddress(&p, g_scan_scratch);
-    ds.ptr = ds.err == cudaSuccess ? p : nullptr;
-  });
-  if (ds.err != cudaSuccess || !ds.ptr) {
-    fprintf(stderr, "ssm_scan_fwd_noalloc: cudaGetSymbolAddress failed: %s\n",
-            cudaGetErrorString(ds.err));
+  void *ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_scan_scratch);
+  if (e != cudaSuccess || !ptr) {
+    fprintf(stderr, "ssm_scan_fwd_noalloc: cudaGetSymbolAddress failed: %s\n", cudaGetErrorString(e));
+    cudaGetLastError();  // the failure belongs to this call only
     return SSM_ERR_CUDA;
   }
   // ssm_scan_fwd clears the error word and the flags on `stream` first, so
   // nothing left in the array by an earlier call is read.
   return ssm_scan_fwd(&s, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, y,
-                      last_state, ds.ptr, kStaticScratchBytes, stream);
+                      last_state, ptr, kStaticScratchBytes, stream);
 }

@@ -153,6 +153,22 @@ def test_noalloc_rejects_bad_shapes_before_launch(lib):
         assert rc == code
 
 
+def test_noalloc_flags_checked_before_launch(lib):
+    # each flag on the allocation-free entry point, without a GPU: saved states
+    # are refused (they would sit in the shared array, out of the backward's
+    # reach); the other flags get ssm_scan_fwd's own checks
+    def call(**kw):
+        sh = _shape(**kw)
+        return lib.ssm_scan_fwd_noalloc(ctypes.byref(sh), *[ctypes.c_void_p(16)] * 5, None, None,
+                                        None, 1, None, ctypes.c_void_p(16), None, None)
+    assert call(flags=_lib.SSM_FLAG_SAVE_STATES) == _lib.SSM_ERR_UNSUPPORTED
+    assert call(flags=8) == _lib.SSM_ERR_INVALID_ARG
+    assert call(flags=_lib.SSM_FLAG_ZOH_EXACT, path=_lib.SSM_PATH_SPLIT_L) == _lib.SSM_ERR_UNSUPPORTED
+    assert call(flags=_lib.SSM_FLAG_TOKEN_MAJOR, io_dtype=_lib.SSM_F32) == _lib.SSM_ERR_UNSUPPORTED
+    assert call(flags=_lib.SSM_FLAG_TOKEN_MAJOR, path=_lib.SSM_PATH_LOOKBACK) == \
+        _lib.SSM_ERR_UNSUPPORTED
+
+
 def _step(lib, shape, ptrs=None):
     p = dict(u=8, delta=8, A=16, B=8, C=8, D=None, z=None, bias=None, state=16, y=8)
     p.update(ptrs or {})

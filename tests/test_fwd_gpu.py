@@ -2,8 +2,9 @@
 
 Small cases span several 32-step chunks, ragged chunk tails, ragged 8-channel
 groups and every dstate padding; the named workloads run at their full sizes
-in the launch configuration the benchmark uses and are checked on seeded
-channels the oracle computes one by one.
+in the launch configuration the benchmark uses and are checked on every
+output element (the million-length workload on its 64 seeded channels over
+the full length).  Every forward reads the workspace's device error word.
 """
 import numpy as np
 import pytest
@@ -20,15 +21,24 @@ PATH_LANES = [("lookback", 2), ("lookback", 4), ("split_l", 2), ("split_l", 4),
               ("per_group", 2), ("per_group", 4), ("lookback_ws", 2)]
 
 
-def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None, lanes=0):
+def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None, lanes=0,
+         zoh=False):
+    """One forward through the C ABI with an explicit workspace, whose device
+    error word is read afterwards: a bounded look-back wait that gave up
+    fails the test instead of passing silently."""
     import torch
     import selective_state_space_54_b200 as ssm
     g = upload(case, device)
     h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
+    shape = ssm.make_shape(case["batch"], case["dim"], case["seqlen"], case["dstate"],
+                           ssm.SSM_BF16 if case["dtype"] == synth.BF16 else ssm.SSM_F32,
+                           PATHS[path], lanes, ssm.SSM_FLAG_ZOH_EXACT if zoh else 0)
+    ws = torch.empty(max(256, ssm.fwd_workspace_bytes(shape)), dtype=torch.uint8, device=device)
     y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
                          g["delta_bias"], delta_softplus=softplus, initial_state=h0_t,
-                         return_last_state=True, path=PATHS[path], y=y_out, lanes=lanes)
-    torch.cuda.synchronize()
+                         return_last_state=True, path=PATHS[path], y=y_out, lanes=lanes,
+                         zoh_exact=zoh, workspace=ws)
+    ssm.check(ws)  # synchronises; raises on a device-side wait that gave up
     return to_f64(y), to_f64(ls)
 
 
@@ -216,54 +226,83 @@ def test_wait_timeout_reports_status(cuda_device):
     del ssm
 
 
-# ---- the named workloads at full size, checked on seeded channels ----------
-def _full_size(name, device, sample=None):
+# ---- the named workloads at full size ---------------------------------------
+def _forward_full_size(name, device):
+    """Run the workload at full size in the benchmark's launch configuration
+    (path AUTO, inputs resident on the device) and return the case and the
+    device outputs as fp64 host arrays, after reading the error word."""
     import torch
     import selective_state_space_54_b200 as ssm
     w = synth.WORKLOADS[name]
     case = synth.make_workload(w)
     g = upload(case, device)
+    shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
+                           ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32)
+    ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=device)
     y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
-                         g["delta_bias"], return_last_state=True)
-    torch.cuda.synchronize()
-    chans = synth.sample_channels(w, sample)
-    for b, dims, sub in synth.subset_case(case, chans):
+                         g["delta_bias"], return_last_state=True, workspace=ws)
+    ssm.check(ws)
+    del g
+    return w, case, to_f64(y), to_f64(ls)
+
+
+def _every_element(name, device):
+    """The whole y and last_state against the fp64 oracle, one batch element
+    at a time (bounded host memory), with the contract's tolerances applied
+    to the totals: rel-L2 <= 2e-3 and max-abs <= 1e-2 max|ref| on y (bf16),
+    rel-L2 <= 2e-3 on the fp32 state."""
+    w, case, y, ls = _forward_full_size(name, device)
+    acc = {"y": [0.0, 0.0, 0.0, 0.0], "last_state": [0.0, 0.0, 0.0, 0.0]}  # err2, ref2, maxerr, maxref
+    for b in range(w.batch):
+        _, dims, sub = synth.subset_case(case, np.arange(b * w.dim, (b + 1) * w.dim))[0]
         ref = oracle.fwd(sub)
-        yg = to_f64(y[b, dims])[None]
-        lg = to_f64(ls[b, dims])[None]
-        assert_close(yg, ref["y"], case["dtype"], f"{name} y b={b}")
-        assert_close(lg, ref["last_state"], case["dtype"], f"{name} last_state b={b}",
-                     stored_bf16=False)
-    return y
+        for k, got in (("y", y[b:b + 1]), ("last_state", ls[b:b + 1])):
+            r = ref[k]
+            assert np.all(np.isfinite(got)), f"{name} {k} b={b}: non-finite"
+            a = acc[k]
+            a[0] += float(np.sum((got - r) ** 2))
+            a[1] += float(np.sum(r ** 2))
+            a[2] = max(a[2], float(np.max(np.abs(got - r))))
+            a[3] = max(a[3], float(np.max(np.abs(r))))
+        del ref, sub
+    out = {}
+    for k, (e2, r2, me, mr) in acc.items():
+        rel = (e2 / r2) ** 0.5
+        out[k] = rel
+        print(f"{name} {k}: rel-L2 {rel:.3e} over every element, max-abs {me:.3e} (max|ref| {mr:.3e})")
+        assert rel <= 2e-3, f"{name} {k}: rel-L2 {rel:.3e} > 2e-3"
+        if k == "y":
+            assert me <= 1e-2 * mr, f"{name} y: max-abs {me:.3e} > 1e-2 * {mr:.3e}"
+    return out
 
 
 def test_full_mamba_130m_layer(cuda_device):
-    _full_size("mamba-130m-layer", cuda_device, sample=96)
+    _every_element("mamba-130m-layer", cuda_device)
 
 
 def test_full_mamba_2p8b_layer(cuda_device):
-    _full_size("mamba-2.8b-layer", cuda_device, sample=64)
-
-
-def test_full_million_length(cuda_device):
-    _full_size("million-length", cuda_device)
+    _every_element("mamba-2.8b-layer", cuda_device)
 
 
 def test_full_mamba_1p4b_layer_forward(cuda_device):
-    _full_size("mamba-1.4b-layer-train", cuda_device, sample=64)
+    _every_element("mamba-1.4b-layer-train", cuda_device)
+
+
+def test_full_million_length(cuda_device):
+    # the seeded 64 channels over the full 2^20 steps (the oracle is serial in t)
+    w, case, y, ls = _forward_full_size("million-length", cuda_device)
+    chans = synth.sample_channels(w)
+    for b, dims, sub in synth.subset_case(case, chans):
+        ref = oracle.fwd(sub)
+        st = assert_close(y[b, dims][None], ref["y"], case["dtype"], f"million-length y b={b}")
+        assert_close(ls[b, dims][None], ref["last_state"], case["dtype"],
+                     f"million-length last_state b={b}", stored_bf16=False)
+        print(f"million-length y: rel-L2 {st['rel_l2']:.3e} on {len(dims)} channels")
 
 
 # ---- exact zero-order hold (the reading guide's "Metodo" discretisation) ----
 def _run_zoh(case, device, path="auto", lanes=0, h0=None):
-    import torch
-    import selective_state_space_54_b200 as ssm
-    g = upload(case, device)
-    h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
-    y, ls = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
-                         g["delta_bias"], initial_state=h0_t, return_last_state=True,
-                         path=PATHS[path], lanes=lanes, zoh_exact=True)
-    torch.cuda.synchronize()
-    return to_f64(y), to_f64(ls)
+    return _run(case, device, path, lanes=lanes, h0=h0, zoh=True)
 
 
 @pytest.mark.parametrize("lanes", [0, 2, 4])

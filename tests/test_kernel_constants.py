@@ -1,0 +1,65 @@
+"""CPU pins of the constants the kernels carry.
+
+The forward's softplus evaluates log1p(x) for x = exp(-|s|) in (0, 1] as
+x * p(x), with p the degree-8 polynomial that interpolates log1p(x)/x at the
+9 Chebyshev nodes of [0, 1].  This test re-derives p by that method (numpy
+polynomial interpolation at the nodes), checks that every coefficient in the
+source is the fp32 rounding of the derived one, and that the fp32 Horner
+evaluation stays within the stated 2.3e-7 relative error of log1p on (0, 1].
+"""
+import os
+import re
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "selective_state_space_54_b200", "csrc")
+FLOAT = r"(-?\d\.\d+e[-+]\d+)f"
+
+
+def _chebyshev_interpolant():
+    k = np.arange(9)
+    x = 0.5 + 0.5 * np.cos((2 * k + 1) * np.pi / 18)  # Chebyshev nodes of [0, 1]
+    return np.polyfit(x, np.log1p(x) / x, 8)          # highest degree first
+
+
+def _source_coefficients(path, func):
+    src = open(path).read()
+    body = src[src.index(func):]
+    body = body[:body.index("\n}\n")]
+    return [float(v) for v in re.findall(FLOAT, body)]
+
+
+def test_softplus_polynomial_is_the_chebyshev_interpolant():
+    ref = _chebyshev_interpolant()
+    ref32 = ref.astype(np.float32)
+    for path, func in ((os.path.join(CSRC, "ssm_common.cuh"), "float softplus_fast("),
+                       (os.path.join(CSRC, "ssm_fwd.cu"), "f2 softplus2(")):
+        got = _source_coefficients(path, func)
+        # the log2(e) factor of the exp argument comes first in softplus_fast
+        got = [g for g in got if abs(g - 1.4426950408889634) > 1e-6]
+        assert len(got) == 9, (path, got)
+        got = np.array(got)
+        # each printed coefficient is the derived one to fp32 precision
+        assert np.all(np.abs(got - ref) <= 2 ** -23 * np.abs(ref) + 1e-12), (path, got - ref)
+        assert np.array_equal(got.astype(np.float32), ref32) or \
+            np.max(np.abs(got.astype(np.float32) - ref32) / np.abs(ref32)) <= 2 ** -23
+
+
+def test_softplus_polynomial_error_bound():
+    coef = np.array(_source_coefficients(os.path.join(CSRC, "ssm_common.cuh"),
+                                         "float softplus_fast("))
+    coef = coef[np.abs(coef - 1.4426950408889634) > 1e-6].astype(np.float32)
+    x = np.concatenate([np.geomspace(1e-30, 1e-3, 2000), np.linspace(1e-3, 1.0, 400001)])
+    x = x.astype(np.float32)
+    # Horner with fused multiply-adds, as the kernel evaluates it (fmaf): the
+    # product of two fp32 values is exact in fp64, so one rounding to fp32
+    # after the fp64 sum stands for the FMA's single rounding
+    x64 = x.astype(np.float64)
+    p = np.full_like(x64, coef[0])
+    for c in coef[1:]:
+        p = (p * x64 + np.float64(c)).astype(np.float32).astype(np.float64)
+    got = (x64 * p).astype(np.float32).astype(np.float64)
+    ref = np.log1p(x.astype(np.float64))
+    rel = np.abs(got - ref) / ref
+    assert rel.max() <= 2.3e-7, rel.max()

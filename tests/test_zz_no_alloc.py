@@ -12,6 +12,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 import synth
 from gpu_util import assert_close, to_f64, upload
 
@@ -19,6 +20,8 @@ pytestmark = pytest.mark.gpu
 
 
 def _noalloc(lib, shape, g, y, ls, stream):
+    """The entry point itself, through ctypes: the caller passes inputs and
+    outputs only, no workspace."""
     p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
     return lib.ssm_scan_fwd_noalloc(ctypes.byref(shape), p(g["u"]), p(g["delta"]), p(g["A"]),
                                     p(g["B"]), p(g["C"]), p(g["D"]), p(g["z"]),
@@ -49,6 +52,52 @@ def test_noalloc_matches_workspace_entry_point(cuda_device, dtype, batch, dim, L
         torch.cuda.synchronize()
         assert_close(to_f64(y), ref_y, dtype, f"y, call {call}")
         assert_close(to_f64(ls), ref_ls, dtype, f"last_state, call {call}", stored_bf16=False)
+
+
+def test_noalloc_against_the_oracle(cuda_device):
+    # directly against the fp64 oracle, on a shape where AUTO keeps the
+    # warp-specialised look-back schedule
+    import torch
+    import selective_state_space_54_b200 as ssm
+    from selective_state_space_54_b200 import _lib
+    lib = _lib.load()
+    batch, dim, L = 4, 5120, 512
+    case = synth.make_case(batch, dim, L, 16, synth.BF16, seed=78)
+    g = upload(case, cuda_device)
+    shape = ssm.make_shape(batch, dim, L, 16, ssm.SSM_BF16)
+    assert ssm.fwd_path(shape) == "lookback_ws"
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    y = torch.full_like(g["u"], float("nan"))
+    ls = torch.full((batch, dim, 16), float("nan"), dtype=torch.float32, device=cuda_device)
+    assert _noalloc(lib, shape, g, y, ls, stream) == 0
+    torch.cuda.synchronize()
+    ref = oracle.fwd(case)
+    assert_close(to_f64(y), ref["y"], synth.BF16, "y")
+    assert_close(to_f64(ls), ref["last_state"], synth.BF16, "last_state", stored_bf16=False)
+
+
+def test_noalloc_token_major(cuda_device):
+    # token-major activations through the entry point equal ssm_scan_fwd's, bit for bit
+    import torch
+    import selective_state_space_54_b200 as ssm
+    from selective_state_space_54_b200 import _lib
+    lib = _lib.load()
+    batch, dim, L = 2, 1024, 1000
+    case = synth.make_case(batch, dim, L, 16, synth.BF16, seed=79)
+    g = upload(case, cuda_device)
+    tm = dict(g)
+    for k in ("u", "delta", "z"):
+        tm[k] = g[k].transpose(1, 2).contiguous()
+    y_ref, ls_ref = ssm.scan_fwd(tm["u"], tm["delta"], g["A"], g["B"], g["C"], g["D"], tm["z"],
+                                 g["delta_bias"], return_last_state=True, token_major=True)
+    shape = ssm.make_shape(batch, dim, L, 16, ssm.SSM_BF16, flags=ssm.SSM_FLAG_TOKEN_MAJOR)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call in range(2):
+        y = torch.full_like(tm["u"], float("nan"))
+        ls = torch.full((batch, dim, 16), float("nan"), dtype=torch.float32, device=cuda_device)
+        assert _noalloc(lib, shape, tm, y, ls, stream) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_ref) and torch.equal(ls, ls_ref), f"call {call}"
 
 
 def test_noalloc_rejects_shapes_beyond_the_static_scratch(cuda_device):
