@@ -46,7 +46,7 @@ def _load():
         i64, pd, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
         lib.oracle_fwd.argtypes = [i64] * 4 + [pd] * 9 + [ci, ci, pd, pd, ci]
         lib.oracle_fwd.restype = ci
-        lib.oracle_bwd.argtypes = [i64] * 4 + [pd] * 9 + [ci, pd] + [pd] * 9 + [ci]
+        lib.oracle_bwd.argtypes = [i64] * 4 + [pd] * 9 + [ci, ci, pd] + [pd] * 9 + [ci]
         lib.oracle_bwd.restype = ci
         _lib = lib
     return _lib
@@ -99,9 +99,10 @@ def fwd(case: dict, *, delta_softplus: bool = True, zoh_exact: bool = False,
     return {"y": y, "last_state": ls}
 
 
-def bwd(case: dict, dout, *, delta_softplus: bool = True, h0=None,
+def bwd(case: dict, dout, *, delta_softplus: bool = True, zoh_exact: bool = False, h0=None,
         want_dh0: bool = False, nthreads: int | None = None) -> dict:
-    """Gradients of sum(dout * y) with respect to every input of ``case``."""
+    """Gradients of sum(dout * y) with respect to every input of ``case``
+    (zoh_exact: for the exact zero-order-hold input term)."""
     lib = _load()
     bt, dm, L, N = case["batch"], case["dim"], case["seqlen"], case["dstate"]
     x = _inputs(case)
@@ -116,7 +117,8 @@ def bwd(case: dict, dout, *, delta_softplus: bool = True, h0=None,
     }
     rc = lib.oracle_bwd(bt, dm, L, N, _ptr(x["u"]), _ptr(x["delta"]), _ptr(x["A"]),
                         _ptr(x["B"]), _ptr(x["C"]), _ptr(x["D"]), _ptr(x["z"]),
-                        _ptr(x["delta_bias"]), _ptr(h0), int(delta_softplus), _ptr(dout),
+                        _ptr(x["delta_bias"]), _ptr(h0), int(delta_softplus), int(zoh_exact),
+                        _ptr(dout),
                         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]),
                         _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]),
                         _ptr(g["ddelta_bias"]), _ptr(g["dh0"]),

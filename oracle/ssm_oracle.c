@@ -79,6 +79,31 @@ static double bbar_scale(double dl, double a_n, int zoh_exact) {
   return expm1(dl * a_n) / a_n;
 }
 
+/* Its derivative with respect to Delta: 1 (Euler) or exp(Delta A_n) (ZOH). */
+static double bbar_scale_ddelta(double dl, double a_n, int zoh_exact) {
+  return zoh_exact ? exp(dl * a_n) : 1.0;
+}
+
+/* Its derivative with respect to A_n: 0 (Euler); for ZOH
+ *   d/dA [(e^{Delta A} - 1) / A] = (x e^x - (e^x - 1)) / A^2,  x = Delta A,
+ * which is Delta^2 sum_{k>=2} x^(k-2) (k-1) / k!  (used for |x| < 0.1, where
+ * the closed form cancels). */
+static double bbar_scale_dA(double dl, double a_n, int zoh_exact) {
+  if (!zoh_exact) return 0.0;
+  const double x = dl * a_n;
+  if (fabs(x) < 0.1) {
+    double term = 1.0, sum = 0.0;  /* term = x^m, with m = k - 2 */
+    double fact = 2.0;             /* (m + 2)! */
+    for (int m = 0; m < 12; ++m) {
+      sum += term * (double)(m + 1) / fact;
+      term *= x;
+      fact *= (double)(m + 3);
+    }
+    return dl * dl * sum;
+  }
+  return (x * exp(x) - expm1(x)) / (a_n * a_n);
+}
+
 static void *fwd_worker(void *arg) {
   job_t *j = (job_t *)arg;
   const int64_t L = j->seqlen, N = j->dstate, Dm = j->dim;
@@ -145,7 +170,7 @@ static void *bwd_worker(void *arg) {
       double acc = 0.0;
       for (int64_t n = 0; n < N; ++n) {
         const double abar = exp(dl[t] * Ad[n]);
-        const double hn = abar * hs[t * N + n] + dl[t] * Bb[t * N + n] * u[t];
+        const double hn = abar * hs[t * N + n] + bbar_scale(dl[t], Ad[n], j->zoh_exact) * Bb[t * N + n] * u[t];
         hs[(t + 1) * N + n] = hn;
         acc += Cb[t * N + n] * hn;
       }
@@ -167,12 +192,15 @@ static void *bwd_worker(void *arg) {
         const double ht = hs[(t + 1) * N + n], hp = hs[t * N + n];
         const double abar = exp(dl[t] * Ad[n]);
         const double Btn = Bb[t * N + n];
+        const double beta = bbar_scale(dl[t], Ad[n], j->zoh_exact);
         g[n] += dyy * Cb[t * N + n];            /* dL/dh_t */
         j->pdC[(b * L + t) * N + n] += dyy * ht;
-        ddl += g[n] * (Ad[n] * abar * hp + Btn * u[t]);
-        j->pdA[d * N + n] += g[n] * dl[t] * abar * hp;
-        j->pdB[(b * L + t) * N + n] += g[n] * dl[t] * u[t];
-        du += g[n] * dl[t] * Btn;
+        /* h_t = abar h_{t-1} + beta B u, abar = exp(Delta A), beta = beta(Delta, A) */
+        ddl += g[n] * (Ad[n] * abar * hp + bbar_scale_ddelta(dl[t], Ad[n], j->zoh_exact) * Btn * u[t]);
+        j->pdA[d * N + n] += g[n] * (dl[t] * abar * hp +
+                                     bbar_scale_dA(dl[t], Ad[n], j->zoh_exact) * Btn * u[t]);
+        j->pdB[(b * L + t) * N + n] += g[n] * beta * u[t];
+        du += g[n] * beta * Btn;
         g[n] *= abar;                            /* dL/dh_{t-1} via h_t */
       }
       const double ds = j->delta_softplus ? ddl * sigmoid(sv[t]) : ddl;
@@ -238,7 +266,7 @@ int oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
                const double *u, const double *delta, const double *A,
                const double *B, const double *C, const double *D,
                const double *z, const double *delta_bias, const double *h0,
-               int delta_softplus, const double *dout,
+               int delta_softplus, int zoh_exact, const double *dout,
                double *du, double *ddelta, double *dA, double *dB, double *dC,
                double *dD, double *dz, double *ddelta_bias, double *dh0,
                int nthreads) {
@@ -258,7 +286,7 @@ int oracle_bwd(int64_t batch, int64_t dim, int64_t seqlen, int64_t dstate,
   base.batch = batch; base.dim = dim; base.seqlen = seqlen; base.dstate = dstate;
   base.u = u; base.delta = delta; base.A = A; base.B = B; base.C = C; base.D = D;
   base.z = z; base.delta_bias = delta_bias; base.h0 = h0;
-  base.delta_softplus = delta_softplus; base.dout = dout;
+  base.delta_softplus = delta_softplus; base.zoh_exact = zoh_exact; base.dout = dout;
   base.du = du; base.ddelta = ddelta; base.dz = dz; base.dh0 = dh0;
   job_t *jobs = NULL;
   int nt = make_jobs(&base, nthreads, &jobs);

@@ -241,17 +241,25 @@ _GRAD_OF = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC",
             "D": "dD", "z": "dz", "delta_bias": "ddelta_bias"}
 
 
-def _objective(c, dout, softplus, h0=None):
-    return float(np.sum(dout * oracle.fwd(c, delta_softplus=softplus, h0=h0)["y"]))
+def _objective(c, dout, softplus, h0=None, zoh=False):
+    return float(np.sum(dout * oracle.fwd(c, delta_softplus=softplus, h0=h0, zoh_exact=zoh)["y"]))
 
 
+@pytest.mark.parametrize("zoh", [False, True])
 @pytest.mark.parametrize("softplus", [True, False])
-def test_backward_matches_finite_differences(softplus):
+def test_backward_matches_finite_differences(softplus, zoh):
+    # zoh: the exact zero-order-hold input term of the reading guide's "Metodo"
+    # (Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B); one A entry per channel
+    # is 0 there, so the A -> 0 limit of its derivative is checked too, and
+    # Delta A spans both sides of the oracle's series/closed-form switch
     c = _case(2, 3, 11, 3, 21, softplus=softplus)
+    if zoh:
+        c["A"] = c["A"].copy()
+        c["A"][:, 1] = 0.0
     rng = np.random.default_rng(22)
     dout = rng.standard_normal(c["u"].shape)
     h0 = rng.standard_normal((2, 3, 3)) * 0.5
-    g = oracle.bwd(c, dout, delta_softplus=softplus, h0=h0, want_dh0=True)
+    g = oracle.bwd(c, dout, delta_softplus=softplus, zoh_exact=zoh, h0=h0, want_dh0=True)
     for name, gname in _GRAD_OF.items():
         x = c[name]
         flat_idx = rng.choice(x.size, size=min(6, x.size), replace=False)
@@ -261,8 +269,8 @@ def test_backward_matches_finite_differences(softplus):
             xp, xm = x.copy(), x.copy()
             xp[idx] += eps
             xm[idx] -= eps
-            fd = (_objective(dict(c, **{name: xp}), dout, softplus, h0)
-                  - _objective(dict(c, **{name: xm}), dout, softplus, h0)) / (2 * eps)
+            fd = (_objective(dict(c, **{name: xp}), dout, softplus, h0, zoh)
+                  - _objective(dict(c, **{name: xm}), dout, softplus, h0, zoh)) / (2 * eps)
             an = g[gname][idx]
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, idx, fd, an)
     # gradient with respect to the initial state
@@ -271,21 +279,31 @@ def test_backward_matches_finite_differences(softplus):
         hp, hm = h0.copy(), h0.copy()
         hp[idx] += 1e-6
         hm[idx] -= 1e-6
-        fd = (_objective(c, dout, softplus, hp) - _objective(c, dout, softplus, hm)) / 2e-6
+        fd = (_objective(c, dout, softplus, hp, zoh) - _objective(c, dout, softplus, hm, zoh)) / 2e-6
         assert abs(fd - g["dh0"][idx]) <= 1e-6 * max(1.0, abs(fd))
+    if zoh:  # every dA entry, the A = 0 column included
+        for idx in np.ndindex(*c["A"].shape):
+            eps = 1e-6
+            xp, xm = c["A"].copy(), c["A"].copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            fd = (_objective(dict(c, A=xp), dout, softplus, h0, True)
+                  - _objective(dict(c, A=xm), dout, softplus, h0, True)) / (2 * eps)
+            assert abs(fd - g["dA"][idx]) <= 1e-6 * max(1.0, abs(fd)), (idx, fd, g["dA"][idx])
 
 
-def test_backward_adjoint_dot_product():
+@pytest.mark.parametrize("zoh", [False, True])
+def test_backward_adjoint_dot_product(zoh):
     # <J^T dout, v> == d/de f(x + e v) for a random direction over all inputs
     c = _case(2, 4, 9, 3, 31)
     rng = np.random.default_rng(32)
     dout = rng.standard_normal(c["u"].shape)
-    g = oracle.bwd(c, dout)
+    g = oracle.bwd(c, dout, zoh_exact=zoh)
     v = {k: rng.standard_normal(c[k].shape) for k in _GRAD_OF}
     eps = 1e-6
     cp = dict(c, **{k: c[k] + eps * v[k] for k in v})
     cm = dict(c, **{k: c[k] - eps * v[k] for k in v})
-    fd = (_objective(cp, dout, True) - _objective(cm, dout, True)) / (2 * eps)
+    fd = (_objective(cp, dout, True, zoh=zoh) - _objective(cm, dout, True, zoh=zoh)) / (2 * eps)
     an = sum(float(np.sum(g[_GRAD_OF[k]] * v[k])) for k in v)
     assert abs(fd - an) <= 1e-6 * max(1.0, abs(an))
 
