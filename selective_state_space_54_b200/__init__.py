@@ -234,19 +234,25 @@ def causal_conv1d_bwd(x, weight, bias, dout, *, initial_state=None, silu=True,
 
 def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,
              initial_state=None, want_dinitial_state=False, out=None, workspace=None,
-             fwd_workspace=None, stream=None):
+             fwd_workspace=None, zoh_exact=False, token_major=False, stream=None):
     """Backward of scan_fwd by recomputation; returns a dict of gradients.
     fwd_workspace: the workspace of a scan_fwd(save_states=True) call on the same
-    inputs, whose saved chunk states the backward then uses."""
+    inputs, whose saved chunk states the backward then uses.  zoh_exact: the
+    exact zero-order-hold input term.  token_major: u, delta, z, dout and the
+    du, ddelta, dz gradients are (batch, seqlen, dim)."""
     import torch
-    batch, dim, seqlen = u.shape
+    if token_major:
+        batch, seqlen, dim = u.shape
+    else:
+        batch, dim, seqlen = u.shape
     dstate = B.shape[-1]
     dt, dev, f32 = u.dtype, u.device, torch.float32
-    for name, t, shp, ty in (("u", u, (batch, dim, seqlen), dt), ("delta", delta, (batch, dim, seqlen), dt),
-                             ("z", z, (batch, dim, seqlen), dt), ("B", B, (batch, seqlen, dstate), dt),
+    act = (batch, seqlen, dim) if token_major else (batch, dim, seqlen)
+    for name, t, shp, ty in (("u", u, act, dt), ("delta", delta, act, dt),
+                             ("z", z, act, dt), ("B", B, (batch, seqlen, dstate), dt),
                              ("C", C, (batch, seqlen, dstate), dt), ("A", A, (dim, dstate), f32),
                              ("D", D, (dim,), f32), ("delta_bias", delta_bias, (dim,), f32),
-                             ("dout", dout, (batch, dim, seqlen), dt),
+                             ("dout", dout, act, dt),
                              ("initial_state", initial_state, (batch, dim, dstate), f32)):
         _check_io(name, t, shp, ty, dev)
     g = dict(out or {})
@@ -261,8 +267,9 @@ def scan_bwd(u, delta, A, B, C, D, z, delta_bias, dout, *, delta_softplus=True,
                  torch.empty((dim,), dtype=f32, device=dev) if delta_bias is not None else None)
     g.setdefault("dinitial_state",
                  torch.empty((batch, dim, dstate), dtype=f32, device=dev) if want_dinitial_state else None)
-    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u),
-                       flags=SSM_FLAG_SAVE_STATES if fwd_workspace is not None else 0)
+    flags = ((SSM_FLAG_SAVE_STATES if fwd_workspace is not None else 0)
+             | (SSM_FLAG_ZOH_EXACT if zoh_exact else 0) | (SSM_FLAG_TOKEN_MAJOR if token_major else 0))
+    shape = make_shape(batch, dim, seqlen, dstate, _io_dtype(u), flags=flags)
     nbytes = bwd_workspace_bytes(shape)
     ws = _workspace(nbytes, dev, workspace)
     rc = _lib.load().ssm_scan_bwd(

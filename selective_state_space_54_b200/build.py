@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libssmscan.so")
-SOURCES = ["ssm_api.cu", "ssm_fwd.cu", "ssm_bwd.cu", "ssm_noalloc.cu", "ssm_step.cu", "ssm_conv.cu"]
+SOURCES = ["ssm_api.cu", "ssm_fwd.cu", "ssm_bwd.cu", "ssm_bwd16.cu", "ssm_noalloc.cu", "ssm_step.cu", "ssm_conv.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -170,9 +170,34 @@ ssm_status cuda_status(cudaError_t e) {
   return SSM_ERR_CUDA;
 }
 
+// Backward workspace: header, saved states (when the backward computes its
+// own), then the per-block partial sums k_bwd_reduce adds in a fixed order.
+struct BwdLayout {
+  size_t off_ckpt, off_bc, off_a, off_d, off_bias, total;
+};
+
+BwdLayout bwd_layout(const ssm_shape *s) {
+  const int NP = fwd_np_for(s->dstate);
+  const size_t bd = (size_t)s->batch * (size_t)s->dim;
+  BwdLayout l;
+  l.off_ckpt = kHeaderBytes;
+  l.off_bc = round_up(l.off_ckpt + sizeof(float) * bwd_ckpt_floats(s->batch, s->dim, s->seqlen, NP), 256);
+  l.off_a = round_up(l.off_bc + sizeof(float) * (size_t)bwd_blocks(s->dim, NP, s->flags & SSM_FLAG_ZOH_EXACT) *
+                                    (size_t)s->seqlen * 2 * NP, 256);
+  l.off_d = round_up(l.off_a + sizeof(float) * bd * (size_t)s->dstate, 256);
+  l.off_bias = round_up(l.off_d + sizeof(float) * bd, 256);
+  l.total = round_up(l.off_bias + sizeof(float) * bd, 256);
+  return l;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
+  if (check_shape(shape) != SSM_OK) return 0;
+  return bwd_layout(shape).total;
+}
 
 const char *ssm_status_string(ssm_status s) {
   switch (s) {
@@ -250,18 +275,16 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
   p.err = reinterpret_cast<unsigned *>(ws);
   p.wait_limit_ns = kWaitLimitNs;
   p.n_segs = pl.n_segs; p.seg_chunks = pl.seg_chunks;
-  if (pl.ckpt_bytes) {
-    p.ckpt_out = reinterpret_cast<float *>(ws + kHeaderBytes);
-    p.ck_cpb = (shape->dim + kCkptChannels - 1) / kCkptChannels;
-    p.ck_K = (shape->seqlen + kCkptSteps - 1) / kCkptSteps;
-  }
+  if (pl.ckpt_bytes) p.ckpt_out = reinterpret_cast<float *>(ws + kHeaderBytes);
 
-  cudaError_t e;
+  // the error word starts clear on every path, so that ssm_scan_check reads
+  // this call's status whatever the workspace held before
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
   if (pl.path == SSM_PATH_LOOKBACK || pl.path == SSM_PATH_LOOKBACK_WS) {
     p.flags = reinterpret_cast<unsigned *>(ws + pl.off_flags);
     p.carry = reinterpret_cast<float *>(ws + pl.off_carry);
-    e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);  // error word
-    if (e == cudaSuccess) e = cudaMemsetAsync(ws + pl.off_flags, 0, pl.off_carry - pl.off_flags, s);  // flags
+    e = cudaMemsetAsync(ws + pl.off_flags, 0, pl.off_carry - pl.off_flags, s);  // flags
     if (e != cudaSuccess) return cuda_status(e);
     e = pl.path == SSM_PATH_LOOKBACK_WS ? launch_fwd_ws(shape->io_dtype, pl.NP, p, s)
                                         : launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
@@ -369,17 +392,6 @@ ssm_status ssm_causal_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int
   return cuda_status(launch_conv_bwd(io_dtype, p, s));
 }
 
-size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape) {
-  if (check_shape(shape) != SSM_OK) return 0;
-  const int NP = fwd_np_for(shape->dstate);
-  const size_t acc = sizeof(float) * (size_t)shape->batch * (size_t)shape->seqlen * NP;
-  size_t total = kHeaderBytes;
-  total = round_up(total + sizeof(float) * bwd_ckpt_floats(shape->batch, shape->dim, shape->seqlen, NP), 256);
-  total = round_up(total + acc, 256);
-  total = round_up(total + acc, 256);
-  return total;
-}
-
 ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta,
                         const float *A, const void *B, const void *C, const float *D,
                         const void *z, const float *delta_bias, int delta_softplus,
@@ -390,7 +402,10 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
                         size_t ws_bytes, ssm_stream_t stream) {
   ssm_status st = check_shape(shape);
   if (st != SSM_OK) return st;
-  if (shape->flags & (SSM_FLAG_ZOH_EXACT | SSM_FLAG_TOKEN_MAJOR))  // Euler, channel-major only
+  // token-major activations: the d_state-16 kernel (dstate 9..16), bf16, Euler, dim % 8 == 0
+  if ((shape->flags & SSM_FLAG_TOKEN_MAJOR) &&
+      (fwd_np_for(shape->dstate) != 16 || shape->io_dtype != SSM_BF16 ||
+       (shape->flags & SSM_FLAG_ZOH_EXACT) || shape->dim % 8 != 0))
     return SSM_ERR_UNSUPPORTED;
   // saved states come from a forward run with the same shape and flag
   if (fwd_workspace && (!(shape->flags & SSM_FLAG_SAVE_STATES) || !aligned(fwd_workspace, 256)))
@@ -419,14 +434,10 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
       !aligned(D, 4) || !aligned(delta_bias, 4) || !aligned(initial_state, 4) ||
       !aligned(dA, 4) || !aligned(dD, 4) || !aligned(ddelta_bias, 4) || !aligned(dinitial_state, 4))
     return SSM_ERR_INVALID_ARG;
-  const size_t need = ssm_scan_bwd_workspace_bytes(shape);
-  if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
+  const BwdLayout lay = bwd_layout(shape);
+  if (!workspace || ws_bytes < lay.total || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
   const int NP = fwd_np_for(N);
   char *ws = static_cast<char *>(workspace);
-  const size_t acc = sizeof(float) * (size_t)batch * (size_t)L * NP;
-  const size_t off_ckpt = kHeaderBytes;
-  const size_t off_dB = round_up(off_ckpt + sizeof(float) * bwd_ckpt_floats(batch, dim, L, NP), 256);
-  const size_t off_dC = round_up(off_dB + acc, 256);
 
   BwdParams p;
   memset(&p, 0, sizeof(p));
@@ -438,22 +449,22 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
     p.ckpt = reinterpret_cast<float *>(const_cast<char *>(static_cast<const char *>(fwd_workspace)) + kHeaderBytes);
     p.ckpt_given = 1;
   } else {
-    p.ckpt = reinterpret_cast<float *>(ws + off_ckpt);
+    p.ckpt = reinterpret_cast<float *>(ws + lay.off_ckpt);
   }
-  p.dB_acc = reinterpret_cast<float *>(ws + off_dB);
-  p.dC_acc = reinterpret_cast<float *>(ws + off_dC);
+  p.dBC_part = reinterpret_cast<float *>(ws + lay.off_bc);
+  p.dA_part = reinterpret_cast<float *>(ws + lay.off_a);
+  p.dD_part = D ? reinterpret_cast<float *>(ws + lay.off_d) : nullptr;
+  p.dbias_part = delta_bias ? reinterpret_cast<float *>(ws + lay.off_bias) : nullptr;
   p.dB = dB; p.dC = dC;
   p.batch = batch; p.dim = dim; p.L = L; p.N = (int)N;
   p.softplus = delta_softplus ? 1 : 0;
-  p.io_vec = ((L * (int64_t)es) % 16 == 0) && aligned(u, 16) && aligned(delta, 16) &&
-             aligned(z, 16) && aligned(dout, 16) && aligned(du, 16) && aligned(ddelta, 16) &&
-             aligned(dz, 16);
+  p.zoh = (shape->flags & SSM_FLAG_ZOH_EXACT) ? 1 : 0;
+  p.tok = (shape->flags & SSM_FLAG_TOKEN_MAJOR) ? 1 : 0;
+  const bool act16 = aligned(u, 16) && aligned(delta, 16) && aligned(z, 16) && aligned(dout, 16) &&
+                     aligned(du, 16) && aligned(ddelta, 16) && aligned(dz, 16);
+  if (p.tok && !act16) return SSM_ERR_INVALID_ARG;
+  p.io_vec = (p.tok || (L * (int64_t)es) % 16 == 0) && act16;
   p.bc_vec = (N == NP) && ((N * (int64_t)es) % 16 == 0) && aligned(B, 16) && aligned(C, 16);
-  cudaError_t e = cudaMemsetAsync(dA, 0, sizeof(float) * dim * N, s);
-  if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, sizeof(float) * dim, s);
-  if (e == cudaSuccess && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * dim, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws + off_dB, 0, (off_dC - off_dB) + acc, s);
-  if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(launch_bwd(shape->io_dtype, NP, p, s));
 }
 

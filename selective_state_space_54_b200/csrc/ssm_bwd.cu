@@ -12,24 +12,28 @@
 // Estado Ciente de Hardware": intermediate states are recomputed in the
 // backward pass instead of being stored in HBM).
 //
-// Schedule: a CTA of 4 warps owns 32 channels of one batch element; warp w
-// holds channels 8w..8w+7 with 4 lanes per channel and S = NP/4 states per
-// lane.  Phase A walks the sequence forward in 16-step chunks and stores the
-// state entering each chunk in the workspace.  Phase B walks the chunks in
-// reverse: it recomputes the chunk's 16 states into registers from the
-// checkpoint, runs the reverse recurrence over them, and reduces dB/dC over
-// the channels (registers -> warp shuffles -> the CTA's 4 warps in shared
-// memory -> vector atomics into fp32 accumulators).  A last kernel rounds
-// dB/dC to the io dtype.
+// This is the general kernel (every d_state up to 64); d_state 16 takes
+// k_bwd16 (ssm_bwd16.cu).  Schedule: a CTA of 4 warps owns 32 channels of one
+// batch element; warp w holds channels 8w..8w+7 with 4 lanes per channel and
+// S = NP/4 states per lane.  Phase A walks the sequence forward in 16-step
+// chunks and stores the state entering each chunk in the workspace (the
+// saved-state layout of ssm_common.cuh, every other 8-step entry).  Phase B
+// walks the chunks in reverse: it recomputes the chunk's 16 states into
+// registers from the checkpoint, runs the reverse recurrence over them, and
+// reduces dB/dC over the channels (registers -> the CTA's 4 warps in shared
+// memory -> one partial per 32-channel block).  k_bwd_reduce adds the
+// partials (dB/dC over channel blocks, dA/dD/ddelta_bias over the batch) in a
+// fixed order and rounds dB/dC to the io dtype: no atomics, bitwise
+// repeatable.
 #include "ssm_common.cuh"
 
 namespace ssm {
 
-constexpr int kTB = kCkptSteps;  // steps per backward chunk (the saved-state chunk)
+constexpr int kTB = 2 * kCkptSteps;  // steps per backward chunk: two saved-state chunks
 constexpr int kBW = 4;        // warps per CTA
 constexpr int kBCPW = 8;      // channels per warp
 constexpr int kBPad = 4;
-static_assert(kBW * kBCPW == kCkptChannels, "a backward CTA covers one saved-state channel block");
+static_assert(kCkptPad % (kBW * kBCPW) == 0, "saved states cover every padded channel of a CTA");
 
 // 4 consecutive io values
 template <typename T> struct Vec4;
@@ -92,6 +96,7 @@ struct __align__(16) BwdWarpSmem {
   float dlu[kBCPW][kTB + kBPad];   // Delta * u
   float dy[kBCPW][kTB + kBPad];    // dout * SiLU(z)
   float ys[kBCPW][kTB + kBPad];    // sum_n C h
+  float uu[kBCPW][kTB + kBPad];    // u (0 past L), for the exact-ZOH derivatives
   // per step, channel and lane j: (sum_n g A a h_prev, sum_n g B) partials;
   // step-major so that a warp's stores of one step are contiguous
   float2 pd[kTB][kBCPW][4];
@@ -193,7 +198,37 @@ __device__ __forceinline__ bf2 bex2(bf2 x) {
   return bpack(ex2(x0), ex2(x1));
 }
 
-template <typename T, int NP>
+// Exact zero-order hold, per half of a pair with x = x2 ln 2 = Delta A_n and
+// a = exp(x): phi = (e^x - 1) / x (the input term is Delta u phi B) and
+// psi = (x e^x - (e^x - 1)) / x^2 (its derivative in A_n is Delta^2 u psi B).
+// For |x| < 1/2 psi is its Taylor series sum_{m<8} x^m (m+1)/(m+2)!
+// (remainder below 1e-8); beyond, the closed form loses at most a few bits.
+__device__ __forceinline__ float xexpm1_over_x2(float x2, float a) {
+  const float x = x2 * kLn2;
+  float q = 2.204585537918871e-05f;        // coefficient of x^m: (m+1)/(m+2)!, m = 7
+  q = fmaf(q, x, 1.736111111111111e-04f);  // m = 6
+  q = fmaf(q, x, 1.190476190476190e-03f);  // m = 5
+  q = fmaf(q, x, 6.944444444444444e-03f);  // m = 4
+  q = fmaf(q, x, 3.333333333333333e-02f);  // m = 3
+  q = fmaf(q, x, 1.250000000000000e-01f);  // m = 2
+  q = fmaf(q, x, 3.333333333333333e-01f);  // m = 1
+  q = fmaf(q, x, 0.5f);                    // m = 0
+  return fabsf(x) < 0.5f ? q : fmaf(x, a, 1.f - a) * rcp_approx(x * x);
+}
+__device__ __forceinline__ bf2 bphi(bf2 x2, bf2 a) {
+  float x0, x1, a0, a1;
+  bunpack(x2, x0, x1);
+  bunpack(a, a0, a1);
+  return bpack(expm1_over_x(x0, a0), expm1_over_x(x1, a1));
+}
+__device__ __forceinline__ bf2 bpsi(bf2 x2, bf2 a) {
+  float x0, x1, a0, a1;
+  bunpack(x2, x0, x1);
+  bunpack(a, a0, a1);
+  return bpack(xexpm1_over_x2(x0, a0), xexpm1_over_x2(x1, a1));
+}
+
+template <typename T, int NP, bool ZOH>
 __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4 ? 3 : 2)) k_bwd(BwdParams p) {
   constexpr int S = NP / 4;              // states per lane
   constexpr int SP = S >= 2 ? S / 2 : 1; // state pairs per lane (S = 1 pads one)
@@ -203,7 +238,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
   BwdWarpSmem<NP> &ws = sm.w[warp];
   const int c = lane >> 2, j = lane & 3, q = j;   // q: this lane's 4 steps of a chunk
   const int64_t cta = blockIdx.x;
-  const int64_t b = cta / p.cpb;
+  const int64_t b = cta / p.cpb, cb = cta - b * p.cpb;
   const int64_t d = (cta - b * p.cpb) * (kBW * kBCPW) + warp * kBCPW + c;
   const bool valid = d < p.dim;
   const int64_t L = p.L, K = p.K;
@@ -234,9 +269,9 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     An[i] = bpack(a[0], a[1]);
     A2[i] = bpack(a[0] * kLog2e, a[1] * kLog2e);
   }
-  float *ck = p.ckpt + cta * K * (kBW * kBCPW) * NP;
-  const int ch = warp * kBCPW + c;   // channel within the CTA
-  auto ck_at = [&](int64_t k, int i) -> float * { return &ck[(k * (kBW * kBCPW) + ch) * NP + j * S + 2 * i]; };
+  // saved state entering 16-step chunk k = 8-step saved chunk 2k (padded channels included)
+  float *ck = p.ckpt + ckpt_offset(b, d, 0, p.dim, L, NP) + j * S;
+  auto ck_at = [&](int64_t k, int i) -> float * { return &ck[2 * k * kCkptChannels * NP + 2 * i]; };
   auto Bpair = [&](int t, int i) -> bf2 {
     if constexpr (S >= 2) return *reinterpret_cast<const bf2 *>(&sm.Bs[t][j * S + 2 * i]);
     else return bpack(sm.Bs[t][j], 0.f);
@@ -271,6 +306,17 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     }
     *reinterpret_cast<float4 *>(&ws.dl[c][4 * q]) = make_float4(dl4[0], dl4[1], dl4[2], dl4[3]);
     *reinterpret_cast<float4 *>(&ws.dlu[c][4 * q]) = make_float4(du4[0], du4[1], du4[2], du4[3]);
+    if (ZOH) {
+      float u4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) u4[i] = (valid && t0 + 4 * q + i < L) ? uu[i] : 0.f;
+      *reinterpret_cast<float4 *>(&ws.uu[c][4 * q]) = make_float4(u4[0], u4[1], u4[2], u4[3]);
+    }
+  };
+  // the input term Bbar_n u: Delta u B_n (Euler) or Delta u phi(Delta A_n) B_n (exact ZOH)
+  auto bterm = [&](bf2 du2, bf2 x, bf2 a, bf2 Bv) -> bf2 {
+    if constexpr (ZOH) return bmul(bmul(du2, bphi(x, a)), Bv);
+    else return bmul(du2, Bv);
   };
 
   // inputs of one chunk, loaded a chunk ahead of their use
@@ -332,7 +378,10 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     for (int t = 0; t < kTB; ++t) {
       const bf2 dl2 = bpack(ws.dl[c][t], ws.dl[c][t]), du2 = bpack(ws.dlu[c][t], ws.dlu[c][t]);
 #pragma unroll
-      for (int i = 0; i < SP; ++i) h[i] = bfma(bex2(bmul(dl2, A2[i])), h[i], bmul(du2, Bpair(t, i)));
+      for (int i = 0; i < SP; ++i) {
+        const bf2 x = bmul(dl2, A2[i]), a = bex2(x);
+        h[i] = bfma(a, h[i], bterm(du2, x, a, Bpair(t, i)));
+      }
     }
     __syncthreads();
   }
@@ -376,7 +425,8 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         bf2 acc = bpack(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
-          hh[i] = bfma(bex2(bmul(dl2, A2[i])), hh[i], bmul(du2, Bpair(tt, i)));
+          const bf2 x = bmul(dl2, A2[i]), a = bex2(x);
+          hh[i] = bfma(a, hh[i], bterm(du2, x, a, Bpair(tt, i)));
           acc = bfma(Cpair(tt, i), hh[i], acc);
         }
         float a0, a1;
@@ -434,8 +484,9 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         const bf2 dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
-          ag[u][i] = bex2(bmul(dl2, A2[i]));
-          hg[u][i] = bfma(ag[u][i], u == 0 ? H4[grp][i] : hg[u - 1][i], bmul(du2, Bpair(t, i)));
+          const bf2 x = bmul(dl2, A2[i]);
+          ag[u][i] = bex2(x);
+          hg[u][i] = bfma(ag[u][i], u == 0 ? H4[grp][i] : hg[u - 1][i], bterm(du2, x, ag[u][i], Bpair(t, i)));
         }
       }
 #pragma unroll
@@ -444,6 +495,12 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         const float dyv = ws.dy[c][t], dlv = ws.dl[c][t], duv = ws.dlu[c][t];
         const bf2 dy2 = bpack(dyv, dyv), dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
         bf2 ddl2 = bpack(0.f, 0.f), s12 = ddl2;
+        bf2 u2 = ddl2, ddu2 = ddl2;
+        if constexpr (ZOH) {
+          const float uv = ws.uu[c][t];
+          u2 = bpack(uv, uv);
+          ddu2 = bpack(dlv * duv, dlv * duv);
+        }
         float *pB = &ws.part[u][0][j][c * S];
         float *pC = &ws.part[u][1][j][c * S];
 #pragma unroll
@@ -454,8 +511,21 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
           const bf2 qv = bmul(ga, hp);
           dA_acc[i] = bfma(dl2, qv, dA_acc[i]);
           ddl2 = bfma(An[i], qv, ddl2);
-          s12 = bfma(g[i], Bpair(t, i), s12);
-          const bf2 vB = bmul(g[i], du2), vC = bmul(dy2, hg[u][i]);
+          bf2 vB;
+          if constexpr (ZOH) {
+            // h_t = a h_{t-1} + Delta u phi(x) B with x = Delta A: d/dDelta of the
+            // input term is a u B, d/dA is Delta^2 u psi(x) B, d/du is Delta phi B
+            const bf2 x = bmul(dl2, A2[i]);
+            const bf2 phi = bphi(x, ag[u][i]), gB = bmul(g[i], Bpair(t, i));
+            ddl2 = bfma(bmul(ga, Bpair(t, i)), u2, ddl2);
+            dA_acc[i] = bfma(bmul(gB, bpsi(x, ag[u][i])), ddu2, dA_acc[i]);
+            s12 = bfma(gB, phi, s12);
+            vB = bmul(bmul(g[i], du2), phi);
+          } else {
+            s12 = bfma(g[i], Bpair(t, i), s12);
+            vB = bmul(g[i], du2);
+          }
+          const bf2 vC = bmul(dy2, hg[u][i]);
           g[i] = ga;
           if constexpr (S >= 2) {
             *reinterpret_cast<bf2 *>(pB + 2 * i) = vB;
@@ -510,8 +580,8 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
               float4 acc;
               bunpack(acc0, acc.x, acc.y);
               bunpack(acc1, acc.z, acc.w);
-              float *dst = (which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n);
-              atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+              *reinterpret_cast<float4 *>(p.dBC_part + ((cb * p.batch + b) * L + t0 + t) * 2 * NP +
+                                          which * NP + n) = acc;
             }
           }
         }
@@ -527,7 +597,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
             for (int w = 0; w < kBW; ++w)
 #pragma unroll
               for (int cc = 0; cc < kBCPW; ++cc) acc += sm.w[w].part[tl][which][jj][cc * S + s0];
-            atomicAdd((which ? p.dC_acc : p.dB_acc) + ((b * L + t0 + t) * NP + n), acc);
+            p.dBC_part[((cb * p.batch + b) * L + t0 + t) * 2 * NP + which * NP + n] = acc;
           }
         }
         __syncthreads();  // the next group rewrites part
@@ -549,7 +619,9 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         const float s1 = (pa.y + pa.w) + (pb.y + pb.w);
         const float dl = ws.dl[c][t];
         duv[i] = fmaf(dl, s1, ws.dy[c][t] * Dd);
-        float dd = fmaf(uu[i], s1, ddl);
+        // Euler: dDelta = sum g (A a h_prev + B u); exact ZOH: the u term is
+        // already inside ddl (sum g a B u) and s1 = sum g phi B
+        float dd = ZOH ? ddl : fmaf(uu[i], s1, ddl);
         if (p.softplus) dd *= sgs[i];
         dd = (valid && t0 + t < L) ? dd : 0.f;
         ddv[i] = dd;
@@ -574,7 +646,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
       for (int h2 = 0; h2 < 2; ++h2) {
         const int s = 2 * i + h2, n = j * S + s;
         if (s < S && n < N) {
-          atomicAdd(&p.dA[d * N + n], lo[h2]);
+          p.dA_part[(b * p.dim + d) * N + n] = lo[h2];
           if (p.dh0) p.dh0[(b * p.dim + d) * N + n] = gg[h2];
         }
       }
@@ -585,21 +657,55 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
   dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 1);
   dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, 2);
   if (valid && j == 0) {
-    if (p.dD) atomicAdd(&p.dD[d], dD_acc);
-    if (p.dbias) atomicAdd(&p.dbias[d], dbias_acc);
+    if (p.dD_part) p.dD_part[b * p.dim + d] = dD_acc;
+    if (p.dbias_part) p.dbias_part[b * p.dim + d] = dbias_acc;
   }
 }
 
-// dB, dC: fp32 accumulators [batch][L][NP] -> io dtype [batch][L][N]
+// The partial sums in a fixed order (bitwise repeatable):
+//   dB[b][t][n] = sum over channel blocks cb of dBC_part[cb][b][t][n]      (io dtype)
+//   dC[b][t][n] = sum over cb of dBC_part[cb][b][t][NP + n]
+//   dA[d][n] = sum over b of dA_part[b][d][n];  dD, ddelta_bias likewise.
+// One thread per output; the sums run in index order.
 template <typename T, int NP>
-__global__ void k_bwd_finalize(BwdParams p) {
+__global__ void k_bwd_reduce(BwdParams p) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t total = p.batch * p.L * p.N;
-  if (i >= total) return;
-  const int64_t bt = i / p.N;
-  const int n = (int)(i - bt * p.N);
-  IO<T>::store1(static_cast<T *>(p.dB), i, p.dB_acc[bt * NP + n]);
-  IO<T>::store1(static_cast<T *>(p.dC), i, p.dC_acc[bt * NP + n]);
+  const int64_t n_bc = p.batch * p.L * p.N;
+  const int64_t n_a = p.dim * p.N;
+  if (i < n_bc) {
+    const int64_t bt = i / p.N;
+    const int n = (int)(i - bt * p.N);
+    const int64_t stride = p.batch * p.L * 2 * NP;
+    const float *src = p.dBC_part + bt * 2 * NP + n;
+    float sb = 0.f, sc = 0.f;
+    for (int64_t cb = 0; cb < p.n_blocks; ++cb) {
+      sb += __ldcs(src + cb * stride);
+      sc += __ldcs(src + cb * stride + NP);
+    }
+    IO<T>::store1(static_cast<T *>(p.dB), i, sb);
+    IO<T>::store1(static_cast<T *>(p.dC), i, sc);
+    return;
+  }
+  const int64_t ia = i - n_bc;
+  if (ia < n_a) {
+    float acc = 0.f;
+    for (int64_t b = 0; b < p.batch; ++b) acc += p.dA_part[b * n_a + ia];
+    p.dA[ia] = acc;
+    return;
+  }
+  const int64_t id = ia - n_a;
+  if (id < p.dim) {
+    if (p.dD) {
+      float acc = 0.f;
+      for (int64_t b = 0; b < p.batch; ++b) acc += p.dD_part[b * p.dim + id];
+      p.dD[id] = acc;
+    }
+    if (p.dbias) {
+      float acc = 0.f;
+      for (int64_t b = 0; b < p.batch; ++b) acc += p.dbias_part[b * p.dim + id];
+      p.dbias[id] = acc;
+    }
+  }
 }
 
 // ---- host side ------------------------------------------------------------------
@@ -624,29 +730,46 @@ static cudaError_t bwd_dispatch(int io_dtype, int NP, F &&f) {
 }
 
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP) {
-  const int64_t cpb = (dim + kBW * kBCPW - 1) / (kBW * kBCPW);
-  const int64_t K = (L + kTB - 1) / kTB;
-  return (size_t)(batch * cpb) * (size_t)K * (kBW * kBCPW) * NP;
+  return (size_t)batch * (size_t)ckpt_groups(dim) * (size_t)ckpt_chunks(L) * kCkptChannels * NP;
+}
+
+size_t bwd16_smem_bytes(int io_dtype);
+int64_t bwd16_blocks(int64_t dim);
+cudaError_t launch_bwd16(int io_dtype, BwdParams &p, cudaStream_t s);
+
+// Channel blocks of the dB/dC partials: 64-channel CTAs of k_bwd16 for
+// d_state 16 with the Euler term, 32-channel CTAs of k_bwd otherwise.
+bool bwd_uses_bwd16(int NP, int zoh) { return NP == 16 && !zoh; }
+
+int64_t bwd_blocks(int64_t dim, int NP, int zoh) {
+  return bwd_uses_bwd16(NP, zoh) ? bwd16_blocks(dim) : (dim + kBW * kBCPW - 1) / (kBW * kBCPW);
 }
 
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s) {
-  p.cpb = (p.dim + kBW * kBCPW - 1) / (kBW * kBCPW);
-  p.K = (p.L + kTB - 1) / kTB;
+  p.n_blocks = bwd_blocks(p.dim, NP, p.zoh);
   return bwd_dispatch(io_dtype, NP, [&](auto tt, auto np) -> cudaError_t {
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value;
-    const size_t smem = sizeof(BwdSmem<kNP>);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(k_bwd<T, kNP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
+    cudaError_t e;
+    auto general = [&](auto kern) -> cudaError_t {
+      p.cpb = (p.dim + kBW * kBCPW - 1) / (kBW * kBCPW);
+      p.K = (p.L + kTB - 1) / kTB;
+      const size_t smem = sizeof(BwdSmem<kNP>);
+      if (smem > 48 * 1024) {
+        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e2 != cudaSuccess) return e2;
+      }
+      kern<<<(unsigned)(p.batch * p.cpb), kBW * 32, smem, s>>>(p);
+      return cudaGetLastError();
+    };
+    if constexpr (kNP == 16) {
+      e = p.zoh ? general(k_bwd<T, kNP, true>) : launch_bwd16(io_dtype, p, s);
+    } else {
+      e = p.zoh ? general(k_bwd<T, kNP, true>) : general(k_bwd<T, kNP, false>);
     }
-    const int64_t ctas = p.batch * p.cpb;
-    k_bwd<T, kNP><<<(unsigned)ctas, kBW * 32, smem, s>>>(p);
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t total = p.batch * p.L * p.N;
-    k_bwd_finalize<T, kNP><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(p);
+    const int64_t total = p.batch * p.L * p.N + p.dim * p.N + p.dim;
+    k_bwd_reduce<T, kNP><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(p);
     return cudaGetLastError();
   });
 }

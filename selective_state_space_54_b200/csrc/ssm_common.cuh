@@ -23,10 +23,24 @@ constexpr int kRowPad = 4;       // smem row padding (floats) against bank confl
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Saved-state layout shared by the forward (writer) and the backward (reader):
-// the state entering every kCkptSteps-step chunk, per block of kCkptChannels
-// channels of one batch element.
-constexpr int kCkptSteps = 16;
-constexpr int kCkptChannels = 32;
+// the state entering every kCkptSteps-step chunk, laid out
+// [batch][channel group of kCkptChannels][chunk][kCkptChannels][NP] fp32, with
+// the channel count padded to a multiple of kCkptPad (see ckpt_groups).
+constexpr int kCkptSteps = 8;
+constexpr int kCkptChannels = 16;
+constexpr int kCkptPad = 64;
+__host__ __device__ __forceinline__ int64_t ckpt_groups(int64_t dim) {
+  return (dim + kCkptPad - 1) / kCkptPad * (kCkptPad / kCkptChannels);
+}
+__host__ __device__ __forceinline__ int64_t ckpt_chunks(int64_t L) {
+  return (L + kCkptSteps - 1) / kCkptSteps;
+}
+// Offset (in floats) of the saved state of channel d of batch b entering chunk k.
+__host__ __device__ __forceinline__ int64_t ckpt_offset(int64_t b, int64_t d, int64_t k, int64_t dim,
+                                                        int64_t L, int NP) {
+  return (((b * ckpt_groups(dim) + d / kCkptChannels) * ckpt_chunks(L) + k) * kCkptChannels +
+          d % kCkptChannels) * NP;
+}
 
 // Workspace header: byte 0 holds the device error word.
 constexpr size_t kHeaderBytes = 256;
@@ -61,10 +75,8 @@ struct FwdParams {
   // split-L schedule
   int64_t n_segs, seg_chunks;
   // saved states for the backward (nullable): the state entering every
-  // kCkptSteps-step chunk, laid out [cta][chunk][kCkptChannels][NP] with
-  // cta = b * ck_cpb + d / kCkptChannels (the backward's own layout)
+  // kCkptSteps-step chunk, at ckpt_offset(b, d, chunk, dim, L, NP)
   float *ckpt_out;
-  int64_t ck_cpb, ck_K;
   float *seg_h;       // [n_groups * n_segs][32/LPC][NP] segment end state from zero
   float *seg_dsum;    // [n_groups * n_segs][32/LPC]     sum of Delta over the segment
   float *seg_carry;   // [n_groups * n_segs][32/LPC][NP] state entering the segment
@@ -108,23 +120,29 @@ struct ConvBwdParams {
   int vec;                             // 16-byte aligned rows
 };
 
-// Backward parameters (ssm_bwd.cu).
+// Backward parameters (ssm_bwd.cu, ssm_bwd16.cu).
 struct BwdParams {
   const void *u, *delta, *z, *B, *C, *dout;
   const float *A, *D, *bias, *h0;
   void *du, *ddelta, *dz;
-  float *dA, *dD, *dbias, *dh0;
-  float *dB_acc, *dC_acc;     // [batch][L][NP] fp32
-  float *ckpt;                // [cta][K][32][NP]
-  int ckpt_given;             // ckpt holds states saved by the forward: skip the checkpoint pass
-  void *dB, *dC;              // [batch][L][N] io dtype (finalize)
+  float *dA, *dD, *dbias, *dh0;     // final gradients (k_bwd_reduce)
+  float *ckpt;                      // saved states, at ckpt_offset(...)
+  int ckpt_given;                   // ckpt holds states saved by the forward: skip the checkpoint pass
+  void *dB, *dC;                    // [batch][L][N] io dtype (k_bwd_reduce)
+  // per-block partial sums, added in a fixed order by k_bwd_reduce
+  float *dBC_part;                  // [channel block][batch][L][2 * NP] (dB states, then dC states)
+  float *dA_part;                   // [batch][dim][N]
+  float *dD_part, *dbias_part;      // [batch][dim] (nullable with D / delta_bias)
+  int64_t n_blocks;                 // channel blocks of dBC_part
   int64_t batch, dim, L;
   int N;
   int softplus;
+  int zoh;                          // exact zero-order-hold input term (general kernel)
+  int tok;                          // u/delta/z/dout/du/ddelta/dz laid out [batch][L][dim] (k_bwd16)
   int io_vec;
-  int bc_vec;                 // B/C rows 16-byte aligned and N == NP
-  int64_t cpb;                // CTAs per batch element
-  int64_t K;                  // backward chunks
+  int bc_vec;                       // B/C rows 16-byte aligned and N == NP
+  int64_t cpb;                      // CTAs per batch element
+  int64_t K;                        // backward chunks
 };
 
 // ---- io helpers ---------------------------------------------------------------
@@ -204,6 +222,36 @@ template <> struct IO<float> {
   }
   __device__ __forceinline__ static void store1(float *p, int64_t i, float v) { p[i] = v; }
 };
+
+// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) -----------------------------
+// A pair of fp32 values in one 64-bit register pair; the packed add, multiply
+// and fused multiply-add issue once for both halves.
+typedef unsigned long long f2;
+
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 splat2(float v) { return pack2(v, v); }
 
 // ---- math helpers -------------------------------------------------------------
 // 2^x on the special-function unit (flush-to-zero; 2^-big == 0 exactly).
@@ -314,6 +362,7 @@ int fwd_ws_pairs();
 cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm);
 cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
+int64_t bwd_blocks(int64_t dim, int NP, int zoh);
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);
 cudaError_t launch_step(int io_dtype, const StepParams &p, cudaStream_t s);
 cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s);

@@ -32,37 +32,8 @@
 
 namespace ssm {
 
-// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) -----------------------------
-typedef unsigned long long f2;
-
-__device__ __forceinline__ f2 pack2(float lo, float hi) {
-  f2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void unpack2(f2 v, float &lo, float &hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
-  f2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-  f2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
-  f2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-
 // The same two functions on a pair of values, the polynomial and the
 // products in packed fp32 pairs.
-__device__ __forceinline__ f2 splat2(float v) { return pack2(v, v); }
 __device__ __forceinline__ f2 softplus2(f2 s) {
   float s0, s1;
   unpack2(s, s0, s1);
@@ -632,7 +603,7 @@ __global__ void k_wait_probe(unsigned *flag, unsigned *err, unsigned long long l
 // full" (producer -> consumer) and "sums ready" (consumer -> producer) per
 // pair and stage.
 constexpr int kTW = 16;
-static_assert(kTW == kCkptSteps, "the saved states are written at warp-specialised chunk starts");
+static_assert(kTW == 2 * kCkptSteps, "the saved states are written at the start and the middle of each chunk");
 constexpr int kPairs = 4;
 constexpr int kWSThreads = 2 * kPairs * 32;
 
@@ -732,28 +703,30 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
     f2 hp[S / 2];
 #pragma unroll
     for (int s = 0; s < S; s += 2) hp[s / 2] = pack2(h[s], h[s + 1]);
-    // saved states for the backward: this lane's S states of the channel
+    // saved states for the backward: this lane's S states of the channel,
+    // entering every kCkptSteps-step chunk (two per kTW-step chunk here)
     float *ck = nullptr;
-    if (p.ckpt_out && ln.valid)
-      ck = p.ckpt_out + ((ln.b * p.ck_cpb + ln.d / kCkptChannels) * p.ck_K * kCkptChannels +
-                         ln.d % kCkptChannels) * NP + j * S;
+    const int64_t ck_K = ckpt_chunks(p.L);
+    if (p.ckpt_out && ln.valid) ck = p.ckpt_out + ckpt_offset(ln.b, ln.d, 0, p.dim, p.L, NP) + j * S;
+    auto save_state = [&](int64_t k8) {
+      float *dst = ck + k8 * kCkptChannels * NP;
+      if constexpr (S % 4 == 0) {
+#pragma unroll
+        for (int s = 0; s < S; s += 4)
+          __stcg(reinterpret_cast<ulonglong2 *>(dst + s), make_ulonglong2(hp[s / 2], hp[s / 2 + 1]));
+      } else {
+#pragma unroll
+        for (int s = 0; s < S; s += 2) __stcg(reinterpret_cast<unsigned long long *>(dst + s), hp[s / 2]);
+      }
+    };
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = (int)(it & 1);
       WSStage<NP> &st = sm.st[stage];
-      if (ck) {  // the state entering chunk k
-        float *dst = ck + k * kCkptChannels * NP;
-        if constexpr (S % 4 == 0) {
-#pragma unroll
-          for (int s = 0; s < S; s += 4)
-            __stcg(reinterpret_cast<ulonglong2 *>(dst + s), make_ulonglong2(hp[s / 2], hp[s / 2 + 1]));
-        } else {
-#pragma unroll
-          for (int s = 0; s < S; s += 2) __stcg(reinterpret_cast<unsigned long long *>(dst + s), hp[s / 2]);
-        }
-      }
+      if (ck) save_state(2 * k);  // the state entering step kTW * k
       bar_sync_n(bar_full + stage, 64);
 #pragma unroll
       for (int tt = 0; tt < kTW; tt += 4) {
+        if (tt == kCkptSteps && ck && 2 * k + 1 < ck_K) save_state(2 * k + 1);  // entering step kTW k + 8
         const float4 d4 = *reinterpret_cast<const float4 *>(&st.dl[c][tt]);
         const float4 u4 = *reinterpret_cast<const float4 *>(&st.dlu[c][tt]);
         const float dls[4] = {d4.x, d4.y, d4.z, d4.w};

@@ -36,10 +36,11 @@ int main(void) {
          SSM_ERR_INVALID_ARG);
   expect("conv width 9", ssm_causal_conv1d(2, 16, 64, 9, SSM_BF16, p, f, NULL, NULL, 1, p, NULL, NULL),
          SSM_ERR_UNSUPPORTED);
-  ssm_shape zoh = s;
-  zoh.flags = SSM_FLAG_ZOH_EXACT;
-  expect("zoh backward", ssm_scan_bwd(&zoh, p, p, f, p, p, NULL, NULL, NULL, 1, NULL, p, NULL, p, p, f, p, p,
-                                      NULL, NULL, NULL, NULL, p, 1 << 20, NULL),
+  ssm_shape tokf = s;
+  tokf.flags = SSM_FLAG_TOKEN_MAJOR;
+  tokf.io_dtype = SSM_F32;
+  expect("fp32 token-major backward", ssm_scan_bwd(&tokf, p, p, f, p, p, NULL, NULL, NULL, 1, NULL, p, NULL, p, p,
+                                                   f, p, p, NULL, NULL, NULL, NULL, p, 1 << 20, NULL),
          SSM_ERR_UNSUPPORTED);
   ssm_shape empty = s;
   empty.batch = 0;

@@ -242,8 +242,9 @@ def test_flags_checked_before_launch(lib):
             _lib.SSM_ERR_UNSUPPORTED
         assert lib.ssm_scan_fwd_workspace_bytes(
             ctypes.byref(_shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path))) == 0
-    # the backward is Euler only
-    assert _bwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED
+    # the backward takes both input terms: exact ZOH passes the argument checks
+    # (and stops only at the missing workspace here)
+    assert _bwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_WORKSPACE
 
 
 def test_saved_states_flag_checked_before_launch(lib):
@@ -264,7 +265,15 @@ def test_token_major_flag_checked_before_launch(lib):
     assert _fwd(lib, _shape(flags=tok, dim=20)) == _lib.SSM_ERR_UNSUPPORTED
     assert _fwd(lib, _shape(flags=tok | _lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED
     assert _fwd(lib, _shape(flags=tok, path=_lib.SSM_PATH_LOOKBACK)) == _lib.SSM_ERR_UNSUPPORTED
-    assert _bwd(lib, _shape(flags=tok)) == _lib.SSM_ERR_UNSUPPORTED
+    # the backward takes token-major activations on its d_state-16 kernel (dstate
+    # 9..16), bf16, Euler, dim % 8 == 0
+    assert _bwd(lib, _shape(flags=tok)) == _lib.SSM_ERR_WORKSPACE
+    assert _bwd(lib, _shape(flags=tok, dstate=12)) == _lib.SSM_ERR_WORKSPACE
+    assert _bwd(lib, _shape(flags=tok, dstate=32)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _bwd(lib, _shape(flags=tok, dstate=8)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _bwd(lib, _shape(flags=tok, io_dtype=_lib.SSM_F32)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _bwd(lib, _shape(flags=tok, dim=20)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _bwd(lib, _shape(flags=tok | _lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_UNSUPPORTED
 
 
 def test_c_program_against_the_header(lib, tmp_path):

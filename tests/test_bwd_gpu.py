@@ -18,21 +18,22 @@ GRADS = ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias")
 IO_GRADS = ("du", "ddelta", "dB", "dC", "dz")
 
 
-def _bwd(case, device, softplus=True, h0=None, want_dh0=False):
+def _bwd(case, device, softplus=True, h0=None, want_dh0=False, zoh=False):
     import torch
     import selective_state_space_54_b200 as ssm
     g = upload(case, device)
     h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
     out = ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
                        g["delta_bias"], g["dy"], delta_softplus=softplus, initial_state=h0_t,
-                       want_dinitial_state=want_dh0)
+                       want_dinitial_state=want_dh0, zoh_exact=zoh)
     torch.cuda.synchronize()
     return {k: (None if v is None else to_f64(v)) for k, v in out.items()}
 
 
-def _check(case, device, softplus=True, h0=None):
-    ref = oracle.bwd(case, case["dy"], delta_softplus=softplus, h0=h0, want_dh0=h0 is not None)
-    got = _bwd(case, device, softplus, h0, want_dh0=h0 is not None)
+def _check(case, device, softplus=True, h0=None, zoh=False):
+    ref = oracle.bwd(case, case["dy"], delta_softplus=softplus, h0=h0, want_dh0=h0 is not None,
+                     zoh_exact=zoh)
+    got = _bwd(case, device, softplus, h0, want_dh0=h0 is not None, zoh=zoh)
     stats = {}
     for k in GRADS:
         if ref.get(k) is None or (k == "dD" and case.get("D") is None) or \
@@ -53,7 +54,7 @@ def _case(batch, dim, L, N, dtype, seed, **kw):
 
 
 @pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
-@pytest.mark.parametrize("N", [1, 4, 8, 16, 32])
+@pytest.mark.parametrize("N", [1, 4, 8, 12, 16, 32, 64])
 def test_bwd_dstate_sizes(cuda_device, dtype, N):
     _check(_case(2, 40, 150, N, dtype, 200 + N), cuda_device)
 
@@ -81,12 +82,16 @@ def test_bwd_initial_state_gradient(cuda_device):
     _check(case, cuda_device, h0=h0)
 
 
-def test_bwd_deterministic_per_channel_outputs(cuda_device):
-    # du, ddelta, dz involve no cross-channel sums: bitwise repeatable
-    case = _case(2, 64, 512, 16, synth.BF16, 7)
-    a = _bwd(case, cuda_device)
-    b = _bwd(case, cuda_device)
-    for k in ("du", "ddelta", "dz"):
+@pytest.mark.parametrize("N", [16, 8])
+def test_bwd_bitwise_repeatable(cuda_device, N):
+    # every sum over channels, steps or the batch is formed in a fixed order
+    # (per-block partials added by a separate pass, no atomics): two runs give
+    # bitwise-equal gradients, the cross-channel ones included
+    case = _case(3, 200, 777, N, synth.BF16, 7)
+    h0 = np.random.default_rng(8).standard_normal((3, 200, N)).astype(np.float32)
+    a = _bwd(case, cuda_device, h0=h0, want_dh0=True)
+    b = _bwd(case, cuda_device, h0=h0, want_dh0=True)
+    for k in GRADS + ("dinitial_state",):
         assert np.array_equal(a[k], b[k]), k
 
 
@@ -123,7 +128,7 @@ def _bwd_saved(case, device, h0=None):
 
 
 @pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
-@pytest.mark.parametrize("N", [4, 16, 32])
+@pytest.mark.parametrize("N", [4, 12, 16, 32])
 def test_bwd_with_saved_states(cuda_device, dtype, N):
     # 40 channels: a partial 32-channel block; 333 steps: a partial 16-step chunk
     case = _case(2, 40, 333, N, dtype, 600 + N)
@@ -151,3 +156,69 @@ def test_bwd_full_mamba_1p4b_layer_with_saved_states(cuda_device):
     _, got = _bwd_saved(case, cuda_device)
     for k in GRADS:
         assert_close(got[k], ref[k], case["dtype"], k, stored_bf16=k in IO_GRADS)
+
+
+# ---- the exact zero-order-hold input term (reading guide, "Metodo") ----------
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("N", [1, 4, 16, 32])
+def test_bwd_zoh_exact(cuda_device, dtype, N):
+    # 40 channels (a partial block), 333 steps (a partial chunk), an initial state
+    case = _case(2, 40, 333, N, dtype, 650 + N)
+    h0 = np.random.default_rng(N + 1).standard_normal((2, 40, N)).astype(np.float32)
+    _check(case, cuda_device, h0=h0, zoh=True)
+
+
+def test_bwd_zoh_exact_large_and_zero_steps(cuda_device):
+    # Delta A on both sides of the series / closed-form switch, and A_n = 0
+    case = _case(1, 32, 200, 16, synth.F32, 660)
+    case["delta_bias"] = np.linspace(-6.0, 2.0, 32).astype(np.float32)
+    case["A"] = case["A"].copy()
+    case["A"][:, 3] = 0.0
+    _check(case, cuda_device, zoh=True)
+
+
+# ---- token-major activations (batch, seqlen, dim), as a projection writes them ----
+@pytest.mark.parametrize("batch,dim,L", [(2, 64, 256), (1, 40, 333), (3, 8, 17), (2, 1024, 1000)])
+def test_bwd_token_major(cuda_device, batch, dim, L):
+    import torch
+    import selective_state_space_54_b200 as ssm
+    case = _case(batch, dim, L, 16, synth.BF16, 700 + dim)
+    g = upload(case, cuda_device)
+    cm = ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                      g["delta_bias"], g["dy"])
+    tm = {k: g[k].transpose(1, 2).contiguous() for k in ("u", "delta", "z", "dy")}
+    tk = ssm.scan_bwd(tm["u"], tm["delta"], g["A"], g["B"], g["C"], g["D"], tm["z"],
+                      g["delta_bias"], tm["dy"], token_major=True)
+    torch.cuda.synchronize()
+    # the same arithmetic in the same order: only the loads and stores move
+    for k in ("du", "ddelta", "dz"):
+        assert torch.equal(tk[k].transpose(1, 2), cm[k]), k
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        assert torch.equal(tk[k], cm[k]), k
+    ref = oracle.bwd(case, case["dy"])
+    for k in GRADS:
+        got = tk[k].transpose(1, 2) if k in ("du", "ddelta", "dz") else tk[k]
+        assert_close(to_f64(got), ref[k], synth.BF16, k, stored_bf16=k in IO_GRADS)
+
+
+def test_bwd_token_major_with_saved_states(cuda_device):
+    # the training step on projection-layout activations: the token-major
+    # forward saves the chunk states, the token-major backward starts from them
+    import torch
+    import selective_state_space_54_b200 as ssm
+    batch, dim, L = 2, 128, 500
+    case = _case(batch, dim, L, 16, synth.BF16, 710)
+    g = upload(case, cuda_device)
+    tm = {k: g[k].transpose(1, 2).contiguous() for k in ("u", "delta", "z", "dy")}
+    shape = ssm.make_shape(batch, dim, L, 16, ssm.SSM_BF16,
+                           flags=ssm.SSM_FLAG_SAVE_STATES | ssm.SSM_FLAG_TOKEN_MAJOR)
+    ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=cuda_device)
+    ssm.scan_fwd(tm["u"], tm["delta"], g["A"], g["B"], g["C"], g["D"], tm["z"], g["delta_bias"],
+                 workspace=ws, save_states=True, token_major=True)
+    got = ssm.scan_bwd(tm["u"], tm["delta"], g["A"], g["B"], g["C"], g["D"], tm["z"],
+                       g["delta_bias"], tm["dy"], fwd_workspace=ws, token_major=True)
+    torch.cuda.synchronize()
+    ref = oracle.bwd(case, case["dy"])
+    for k in GRADS:
+        v = got[k].transpose(1, 2) if k in ("du", "ddelta", "dz") else got[k]
+        assert_close(to_f64(v), ref[k], synth.BF16, k, stored_bf16=k in IO_GRADS)
