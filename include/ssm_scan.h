@@ -106,40 +106,43 @@ typedef struct {
  *                      guide's "Metodo" formula Bbar = (Delta A)^-1
  *                      (exp(Delta A) - I) Delta B, i.e. per state
  *                      Bbar_n = (exp(Delta A_n) - 1) / A_n * B_n (Delta * B_n
- *                      where A_n = 0).  Forward on path LOOKBACK (AUTO
- *                      picks it; other explicit paths return
- *                      SSM_ERR_UNSUPPORTED) and ssm_scan_step; ssm_scan_bwd
- *                      returns SSM_ERR_UNSUPPORTED for it. */
+ *                      where A_n = 0).  Forward on paths LOOKBACK and
+ *                      LOOKBACK_WS (AUTO picks one of them; SPLIT_L and
+ *                      PER_GROUP return SSM_ERR_UNSUPPORTED), ssm_scan_step,
+ *                      and ssm_scan_bwd (channel-major activations). */
 typedef enum {
   SSM_FLAG_ZOH_EXACT = 1,
   SSM_FLAG_SAVE_STATES = 2,
   SSM_FLAG_TOKEN_MAJOR = 4
 } ssm_flags;
 
-/* SSM_FLAG_TOKEN_MAJOR (forward): u, delta, z and y are laid out
- * [batch][seqlen][dim] (dim contiguous), as a projection produces them, instead
- * of [batch][dim][seqlen]; B and C keep their layout.  bf16 only, dim % 8 == 0,
- * u/delta/z/y 16-byte aligned; path AUTO or LOOKBACK_WS with the Euler term
- * (SSM_ERR_UNSUPPORTED otherwise, SSM_ERR_INVALID_ARG for misaligned
- * pointers).  ssm_scan_bwd returns SSM_ERR_UNSUPPORTED for it; ssm_scan_step
- * ignores it (one token has no time axis). */
+/* SSM_FLAG_TOKEN_MAJOR: u, delta, z and y (and, in ssm_scan_bwd, dout, du,
+ * ddelta and dz) are laid out [batch][seqlen][dim] (dim contiguous), as a
+ * projection produces them, instead of [batch][dim][seqlen]; B and C keep
+ * their layout.  bf16 only, dim % 8 == 0, those activations 16-byte aligned,
+ * the Euler term (SSM_ERR_UNSUPPORTED otherwise, SSM_ERR_INVALID_ARG for
+ * misaligned pointers).  Forward on path AUTO or LOOKBACK_WS; backward for
+ * dstate 9..16 (the d_state-16 kernel).  ssm_scan_step ignores it (one token
+ * has no time axis). */
 
-/* SSM_FLAG_SAVE_STATES (forward, with the Euler term): besides y, the forward
- * writes into its workspace the state entering every 16-step chunk of every
- * channel (fp32, 4 * batch * ceil(dim/32) * 32 * ceil(seqlen/16) * NP bytes,
- * NP = dstate rounded up to a power of two >= 4; ssm_scan_fwd_workspace_bytes
- * counts them).  Passing that workspace as fwd_workspace to ssm_scan_bwd, with
- * the same shape and flag, lets the backward skip its own forward pass over
- * the chunks.  It runs on path LOOKBACK_WS (AUTO picks it; other explicit
- * paths, lanes = 4 and SSM_FLAG_ZOH_EXACT return SSM_ERR_UNSUPPORTED). */
+/* SSM_FLAG_SAVE_STATES (forward): besides y, the forward writes into its
+ * workspace the state entering every 8-step chunk of every channel (fp32,
+ * 4 * batch * G * ceil(seqlen/8) * 16 * NP bytes with G = 4 * ceil(dim/64)
+ * groups of 16 channels and NP = dstate rounded up to a power of two >= 4;
+ * ssm_scan_fwd_workspace_bytes counts them).  Passing that workspace as
+ * fwd_workspace to ssm_scan_bwd, with the same shape and flags, lets the
+ * backward skip its own forward pass over the chunks.  It runs on path
+ * LOOKBACK_WS (AUTO picks it; other explicit paths and lanes = 4 return
+ * SSM_ERR_UNSUPPORTED). */
 
 /* Bytes of workspace ssm_scan_fwd needs for `shape` on the current device
  * (at least 256: the header holding the device error word).  Returns 0 for
  * an invalid shape. */
 size_t ssm_scan_fwd_workspace_bytes(const ssm_shape *shape);
 
-/* Bytes of workspace ssm_scan_bwd needs (state checkpoints of the forward
- * recomputation, fp32 dB/dC accumulators, header).  0 for an invalid shape. */
+/* Bytes of workspace ssm_scan_bwd needs (header, state checkpoints of the
+ * forward recomputation, fp32 per-block partial sums of dB/dC, dA, dD and
+ * ddelta_bias).  0 for an invalid shape. */
 size_t ssm_scan_bwd_workspace_bytes(const ssm_shape *shape);
 
 /* Forward selective scan (the operation above).
@@ -158,12 +161,12 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
                         void *y, float *last_state,
                         void *workspace, size_t ws_bytes, ssm_stream_t stream);
 
-/* Backward of ssm_scan_fwd by recomputation: the states inside each 16-step
- * chunk are recomputed from the inputs, reading guide, "Expansao de Estado
- * Ciente de Hardware"; only the state entering each chunk may come from the
+/* Backward of ssm_scan_fwd by recomputation: the states inside each chunk
+ * are recomputed from the inputs, reading guide, "Expansao de Estado Ciente
+ * de Hardware"; only the state entering each 8-step chunk may come from the
  * forward (fwd_workspace, nullable: a workspace that ssm_scan_fwd filled with
- * SSM_FLAG_SAVE_STATES for the same shape, inputs and initial state; the
- * shape passed here must carry that flag too).  Without it the backward
+ * SSM_FLAG_SAVE_STATES for the same shape, flags, inputs and initial state;
+ * the shape passed here must carry that flag too).  Without it the backward
  * first recomputes those chunk states itself.  Gradients of sum(dout * y):
  *  du, ddelta, dz          [batch][dim][seqlen] io dtype (ddelta is with
  *                          respect to the raw delta argument)
@@ -172,7 +175,11 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
  *  dD, ddelta_bias         [dim] fp32, summed over batch and seqlen
  *  dinitial_state          [batch][dim][dstate] fp32 (nullable)
  * dz must be given exactly when z is, dD exactly when D is, ddelta_bias when
- * delta_bias is (else NULL).  Outputs are overwritten, not accumulated. */
+ * delta_bias is (else NULL).  Outputs are overwritten, not accumulated.
+ * Every sum over channels, steps or the batch is formed per block and the
+ * blocks are added in a fixed order (no atomics): a call repeated on the
+ * same inputs gives bitwise-equal gradients.  The workspace holds those
+ * per-block partial sums (ssm_scan_bwd_workspace_bytes). */
 ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta,
                         const float *A, const void *B, const void *C,
                         const float *D, const void *z, const float *delta_bias,

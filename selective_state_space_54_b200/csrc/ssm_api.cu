@@ -38,12 +38,13 @@ ssm_status check_shape(const ssm_shape *s) {
       (s->io_dtype != SSM_BF16 || s->dim % 8 != 0 || (s->flags & SSM_FLAG_ZOH_EXACT) ||
        (s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK_WS) || s->lanes == 4))
     return SSM_ERR_UNSUPPORTED;
-  if ((s->flags & SSM_FLAG_ZOH_EXACT) && s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK)
+  // the exact-ZOH input term is built into the two look-back kernels
+  if ((s->flags & SSM_FLAG_ZOH_EXACT) && s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK &&
+      s->path != SSM_PATH_LOOKBACK_WS)
     return SSM_ERR_UNSUPPORTED;
-  // saved states are written by the warp-specialised kernel, which is Euler only
+  // saved states are written by the warp-specialised kernel
   if ((s->flags & SSM_FLAG_SAVE_STATES) &&
-      ((s->flags & SSM_FLAG_ZOH_EXACT) || (s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK_WS) ||
-       s->lanes == 4))
+      ((s->path != SSM_PATH_AUTO && s->path != SSM_PATH_LOOKBACK_WS) || s->lanes == 4))
     return SSM_ERR_UNSUPPORTED;
   // index arithmetic is int64; keep every flat index well inside it
   const double elems = (double)s->batch * (double)s->dim * (double)s->seqlen;
@@ -107,8 +108,8 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   // the exact-ZOH input term is built into the look-back kernel only
   const bool zoh = (s->flags & SSM_FLAG_ZOH_EXACT) != 0;
   if (path == SSM_PATH_AUTO) {
-    if (zoh) path = SSM_PATH_LOOKBACK;
-    else if (G >= unit) path = lpc == 2 ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
+    if (G >= unit) path = lpc == 2 ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
+    else if (zoh) path = SSM_PATH_LOOKBACK;  // split-L and per-group are Euler only
     else if (p.K >= 64) path = SSM_PATH_SPLIT_L;
     else path = SSM_PATH_PER_GROUP;
   }
@@ -182,8 +183,9 @@ BwdLayout bwd_layout(const ssm_shape *s) {
   BwdLayout l;
   l.off_ckpt = kHeaderBytes;
   l.off_bc = round_up(l.off_ckpt + sizeof(float) * bwd_ckpt_floats(s->batch, s->dim, s->seqlen, NP), 256);
-  l.off_a = round_up(l.off_bc + sizeof(float) * (size_t)bwd_blocks(s->dim, NP, s->flags & SSM_FLAG_ZOH_EXACT) *
-                                    (size_t)s->seqlen * 2 * NP, 256);
+  // dB/dC partials: [channel block][batch][seqlen][2 * NP]
+  const size_t blocks = (size_t)bwd_blocks(s->dim, NP, s->flags & SSM_FLAG_ZOH_EXACT);
+  l.off_a = round_up(l.off_bc + sizeof(float) * blocks * (size_t)s->batch * (size_t)s->seqlen * 2 * NP, 256);
   l.off_d = round_up(l.off_a + sizeof(float) * bd * (size_t)s->dstate, 256);
   l.off_bias = round_up(l.off_d + sizeof(float) * bd, 256);
   l.total = round_up(l.off_bias + sizeof(float) * bd, 256);

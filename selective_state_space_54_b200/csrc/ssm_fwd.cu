@@ -48,11 +48,30 @@ __device__ __forceinline__ f2 softplus2(f2 s) {
   q = fma2(q, x, splat2(9.999999404e-01f));
   return fma2(x, q, pack2(fmaxf(s0, 0.f), fmaxf(s1, 0.f)));
 }
+// 1/d for a pair d in [1, inf) on the FMA pipe, keeping the special-function
+// unit for the recurrence's exponentials.  Seed: the bit pattern
+// kRcpSeed - bits(d), which is 2^-e (2 - m) - like for d = 2^e m and whose
+// constant minimises the seed's maximum relative error over a binade (5.1 %,
+// found by a direct search over the constant); then three Newton-Raphson
+// steps y <- y + y (1 - d y), each squaring the relative error
+// (5.1e-2 -> 2.6e-3 -> 6.5e-6 -> below fp32 rounding).  d is clamped to
+// 2^64 first (SiLU's 1/(1 + e^-z) is below 1e-19 there either way).
+constexpr int kRcpSeed = 0x7EF311C2;
+__device__ __forceinline__ f2 rcp2_newton(f2 d) {
+  float d0, d1;
+  unpack2(d, d0, d1);
+  d0 = fminf(d0, 1.8446744e19f);
+  d1 = fminf(d1, 1.8446744e19f);
+  f2 y = pack2(__int_as_float(kRcpSeed - __float_as_int(d0)), __int_as_float(kRcpSeed - __float_as_int(d1)));
+  const f2 nd = pack2(-d0, -d1), one = splat2(1.f);
+#pragma unroll
+  for (int k = 0; k < 3; ++k) y = fma2(y, fma2(nd, y, one), y);
+  return y;
+}
 __device__ __forceinline__ f2 silu2(f2 z) {
-  float e0, e1, d0, d1;
+  float e0, e1;
   unpack2(mul2(z, splat2(-kLog2e)), e0, e1);
-  unpack2(add2(pack2(ex2(e0), ex2(e1)), splat2(1.f)), d0, d1);
-  return mul2(z, pack2(rcp_approx(d0), rcp_approx(d1)));
+  return mul2(z, rcp2_newton(add2(pack2(ex2(e0), ex2(e1)), splat2(1.f))));
 }
 
 // ---- raw io vectors of 8 values ------------------------------------------------
@@ -674,7 +693,7 @@ struct Share {
   }
 };
 
-template <typename T, int NP>
+template <typename T, int NP, bool ZOH>
 __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &sm, int64_t w,
                                             const Share &sh, unsigned bar_full, unsigned bar_ys) {
   constexpr int S = NP / 2, CPW = 16;
@@ -737,7 +756,7 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
           const float *Brow = &st.Bs[tt + i][j * S];
           const float *Crow = &st.Cs[tt + i][j * S];
           const f2 dl2 = pack2(dls[i], dls[i]), du2 = pack2(dus[i], dus[i]);
-          f2 acc[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};  // two chains
+          f2 acc = 0;  // sum_n C h as a pair of partial sums
 #pragma unroll
           for (int s = 0; s < S; s += 2) {
             f2 bv, cv;
@@ -752,12 +771,17 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
             }
             float x0, x1;
             unpack2(mul2(dl2, A2p[s / 2]), x0, x1);
-            const f2 a = pack2(ex2(x0), ex2(x1));
-            hp[s / 2] = fma2(a, hp[s / 2], mul2(du2, bv));
-            acc[(s / 2) & 1] = fma2(cv, hp[s / 2], acc[(s / 2) & 1]);
+            const float a0 = ex2(x0), a1 = ex2(x1);
+            const f2 a = pack2(a0, a1);
+            if constexpr (ZOH)  // exact zero-order hold: Delta u (e^x - 1)/x B, x = Delta A_n
+              hp[s / 2] = fma2(a, hp[s / 2],
+                               mul2(mul2(du2, pack2(expm1_over_x(x0, a0), expm1_over_x(x1, a1))), bv));
+            else
+              hp[s / 2] = fma2(a, hp[s / 2], mul2(du2, bv));
+            acc = s == 0 ? mul2(cv, hp[0]) : fma2(cv, hp[s / 2], acc);
           }
           float a0, a1;
-          unpack2(add2(acc[0], acc[1]), a0, a1);
+          unpack2(acc, a0, a1);
           yp[i] = a0 + a1;
         }
         // this lane's half of the channel's C.h; the producer adds the halves
@@ -1109,7 +1133,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   cp_async_wait<0>();
 }
 
-template <typename T, int NP, bool TOK>
+template <typename T, int NP, bool TOK, bool ZOH>
 __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
@@ -1121,7 +1145,7 @@ __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   const Share sh(w, p.n_workers, p.n_groups, p.n_chunks);
   const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
   if (producer) ws_producer<T, NP, TOK>(p, sm, sh, bar_full, bar_ys);
-  else ws_consumer<T, NP>(p, sm, w, sh, bar_full, bar_ys);
+  else ws_consumer<T, NP, ZOH>(p, sm, w, sh, bar_full, bar_ys);
 }
 
 // ---- host side ------------------------------------------------------------------
@@ -1216,9 +1240,9 @@ cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm) {
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value;
     const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
-    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false>, smem);
+    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false, false>, smem);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP, false>, kWSThreads,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP, false, false>, kWSThreads,
                                                          smem);
   });
 }
@@ -1231,17 +1255,18 @@ cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t
     const unsigned grid = (unsigned)((p.n_workers + kPairs - 1) / kPairs);
     if (p.tok) {  // token-major tiles: bf16 only (the API checks)
       if constexpr (sizeof(T) == 2) {
-        cudaError_t e = allow_smem(k_fwd_ws<T, kNP, true>, smem);
+        cudaError_t e = allow_smem(k_fwd_ws<T, kNP, true, false>, smem);
         if (e != cudaSuccess) return e;
-        k_fwd_ws<T, kNP, true><<<grid, kWSThreads, smem, s>>>(p);
+        k_fwd_ws<T, kNP, true, false><<<grid, kWSThreads, smem, s>>>(p);
         return cudaGetLastError();
       } else {
         return cudaErrorInvalidValue;
       }
     }
-    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false>, smem);
+    auto kern = p.zoh ? k_fwd_ws<T, kNP, false, true> : k_fwd_ws<T, kNP, false, false>;
+    cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    k_fwd_ws<T, kNP, false><<<grid, kWSThreads, smem, s>>>(p);
+    kern<<<grid, kWSThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }

@@ -65,6 +65,10 @@ def _fwd(lib, shape, ptrs=None, ws=None, ws_bytes=0):
                             v(p["bias"]), 1, v(p["h0"]), v(p["y"]), v(p["ls"]), v(ws), ws_bytes, None)
 
 
+# argument checks passed: no workspace given (a GPU machine) or no device (here)
+ACCEPTED = (_lib.SSM_ERR_WORKSPACE, _lib.SSM_ERR_CUDA)
+
+
 def test_null_shape_rejected(lib):
     assert _fwd(lib, None) == _lib.SSM_ERR_INVALID_ARG
     assert lib.ssm_scan_fwd_workspace_bytes(None) == 0
@@ -236,8 +240,10 @@ def test_conv_empty_problem_is_a_noop(lib):
 
 def test_flags_checked_before_launch(lib):
     assert _fwd(lib, _shape(flags=8)) == _lib.SSM_ERR_INVALID_ARG  # an unknown bit
-    # exact ZOH runs on the look-back path only; other explicit paths are refused
-    for path in (_lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP, _lib.SSM_PATH_LOOKBACK_WS):
+    # exact ZOH runs on the two look-back paths; the others are refused
+    for path in (_lib.SSM_PATH_LOOKBACK, _lib.SSM_PATH_LOOKBACK_WS):
+        assert _fwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path)) in ACCEPTED
+    for path in (_lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP):
         assert _fwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT, path=path)) == \
             _lib.SSM_ERR_UNSUPPORTED
         assert lib.ssm_scan_fwd_workspace_bytes(
@@ -249,8 +255,8 @@ def test_flags_checked_before_launch(lib):
 
 def test_saved_states_flag_checked_before_launch(lib):
     save, zoh = _lib.SSM_FLAG_SAVE_STATES, _lib.SSM_FLAG_ZOH_EXACT
-    # written by the warp-specialised kernel only: Euler, 2 lanes, AUTO or LOOKBACK_WS
-    assert _fwd(lib, _shape(flags=save | zoh)) == _lib.SSM_ERR_UNSUPPORTED
+    # written by the warp-specialised kernel only: 2 lanes, AUTO or LOOKBACK_WS
+    assert _fwd(lib, _shape(flags=save | zoh)) in ACCEPTED
     for path in (_lib.SSM_PATH_LOOKBACK, _lib.SSM_PATH_SPLIT_L, _lib.SSM_PATH_PER_GROUP):
         assert _fwd(lib, _shape(flags=save, path=path)) == _lib.SSM_ERR_UNSUPPORTED
     assert _fwd(lib, _shape(flags=save, lanes=4)) == _lib.SSM_ERR_UNSUPPORTED
@@ -304,3 +310,18 @@ def test_conv_bwd_rejects_bad_arguments_before_launch(lib):
     assert call(bias=16) == _lib.SSM_ERR_INVALID_ARG          # dbias missing
     assert call(dw=None) == _lib.SSM_ERR_INVALID_ARG
     assert call(w=6) == _lib.SSM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dstate,blk", [(16, 64), (8, 32), (4, 32)])
+def test_bwd_workspace_holds_every_partial(lib, dstate, blk):
+    # the backward's workspace must hold, besides the header and the saved
+    # states, one dB/dC partial per channel block, batch element, step and
+    # (padded) state, and the dA/dD/ddelta_bias partials of every batch
+    # element: it grows with the batch (a missing factor here once sent the
+    # partial sums past the end of the workspace)
+    for batch, dim, L in ((1, 100, 50), (3, 100, 50), (2, 4096, 2048)):
+        sh = _shape(batch=batch, dim=dim, seqlen=L, dstate=dstate)
+        np_ = 16 if dstate > 8 else (8 if dstate > 4 else 4)
+        ckpt = 4 * batch * (4 * -(-dim // 64)) * -(-L // 8) * 16 * np_
+        parts = 4 * (-(-dim // blk) * batch * L * 2 * np_ + batch * dim * dstate + 2 * batch * dim)
+        assert lib.ssm_scan_bwd_workspace_bytes(ctypes.byref(sh)) >= 256 + ckpt + parts

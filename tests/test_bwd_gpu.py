@@ -109,20 +109,20 @@ def test_bwd_single_step_and_single_channel(cuda_device):
 
 
 # ---- states saved by the forward (the chunk checkpoints of the training step) ----
-def _bwd_saved(case, device, h0=None):
+def _bwd_saved(case, device, h0=None, zoh=False):
     import torch
     import selective_state_space_54_b200 as ssm
     g = upload(case, device)
     h0_t = None if h0 is None else torch.from_numpy(np.asarray(h0, np.float32)).to(device)
     shape = ssm.make_shape(case["batch"], case["dim"], case["seqlen"], case["dstate"],
                            ssm.SSM_BF16 if case["dtype"] == synth.BF16 else ssm.SSM_F32,
-                           flags=ssm.SSM_FLAG_SAVE_STATES)
+                           flags=ssm.SSM_FLAG_SAVE_STATES | (ssm.SSM_FLAG_ZOH_EXACT if zoh else 0))
     ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=device)
     y = ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                     initial_state=h0_t, workspace=ws, save_states=True)
+                     initial_state=h0_t, workspace=ws, save_states=True, zoh_exact=zoh)
     out = ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
                        g["delta_bias"], g["dy"], initial_state=h0_t, fwd_workspace=ws,
-                       want_dinitial_state=h0 is not None)
+                       want_dinitial_state=h0 is not None, zoh_exact=zoh)
     torch.cuda.synchronize()
     return to_f64(y), {k: (None if v is None else to_f64(v)) for k, v in out.items()}
 
@@ -166,6 +166,20 @@ def test_bwd_zoh_exact(cuda_device, dtype, N):
     case = _case(2, 40, 333, N, dtype, 650 + N)
     h0 = np.random.default_rng(N + 1).standard_normal((2, 40, N)).astype(np.float32)
     _check(case, cuda_device, h0=h0, zoh=True)
+
+
+@pytest.mark.parametrize("N", [16, 8])
+def test_bwd_zoh_exact_with_saved_states(cuda_device, N):
+    # the exact-ZOH training step: the warp-specialised forward saves the chunk
+    # states, the backward starts from them
+    case = _case(2, 40, 333, N, synth.BF16, 670 + N)
+    h0 = np.random.default_rng(N + 2).standard_normal((2, 40, N)).astype(np.float32)
+    ref = oracle.bwd(case, case["dy"], h0=h0, want_dh0=True, zoh_exact=True)
+    y, got = _bwd_saved(case, cuda_device, h0, zoh=True)
+    assert_close(y, oracle.fwd(case, h0=h0, zoh_exact=True)["y"], synth.BF16, "y")
+    for k in GRADS:
+        assert_close(got[k], ref[k], synth.BF16, k, stored_bf16=k in IO_GRADS)
+    assert_close(got["dinitial_state"], ref["dh0"], synth.BF16, "dh0", stored_bf16=False)
 
 
 def test_bwd_zoh_exact_large_and_zero_steps(cuda_device):
@@ -222,3 +236,42 @@ def test_bwd_token_major_with_saved_states(cuda_device):
     for k in GRADS:
         v = got[k].transpose(1, 2) if k in ("du", "ddelta", "dz") else got[k]
         assert_close(to_f64(v), ref[k], synth.BF16, k, stored_bf16=k in IO_GRADS)
+
+
+def test_bwd_writes_only_its_outputs_and_workspace(cuda_device):
+    # outputs and the workspace sit inside larger buffers whose margins hold a
+    # NaN pattern; the backward must touch none of them (a bounds check
+    # without a sanitizer), on both kernels and with saved states
+    import torch
+    import selective_state_space_54_b200 as ssm
+    pad = 4096
+    for N, saved in ((16, False), (16, True), (8, False)):
+        case = _case(3, 70, 301, N, synth.BF16, 720 + N)
+        g = upload(case, cuda_device)
+        shape = ssm.make_shape(3, 70, 301, N, ssm.SSM_BF16,
+                               flags=ssm.SSM_FLAG_SAVE_STATES if saved else 0)
+        fws = None
+        if saved:
+            fws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=cuda_device)
+            ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                         workspace=fws, save_states=True)
+        nws = ssm.bwd_workspace_bytes(shape)
+        wbuf = torch.full((nws + 2 * pad,), 0x7F, dtype=torch.uint8, device=cuda_device)
+        ws = wbuf[pad:pad + nws]
+        bufs, out = {}, {}
+        for k, like in (("du", g["u"]), ("ddelta", g["u"]), ("dz", g["u"]), ("dB", g["B"]), ("dC", g["C"])):
+            bufs[k] = torch.full((like.numel() + 2 * pad,), float("nan"), dtype=like.dtype, device=cuda_device)
+            out[k] = bufs[k][pad:pad + like.numel()].view(like.shape)
+        for k, n in (("dA", 70 * N), ("dD", 70), ("ddelta_bias", 70)):
+            bufs[k] = torch.full((n + 2 * pad,), float("nan"), dtype=torch.float32, device=cuda_device)
+            out[k] = bufs[k][pad:pad + n].view((70, N) if k == "dA" else (70,))
+        ssm.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                     g["dy"], out=out, workspace=ws, fwd_workspace=fws)
+        torch.cuda.synchronize()
+        assert (wbuf[:pad] == 0x7F).all() and (wbuf[pad + nws:] == 0x7F).all(), (N, saved, "workspace")
+        for k, buf in bufs.items():
+            n = out[k].numel()
+            assert torch.isnan(buf[:pad].float()).all() and torch.isnan(buf[pad + n:].float()).all(), (N, saved, k)
+        ref = oracle.bwd(case, case["dy"])
+        for k in GRADS:
+            assert_close(to_f64(out[k]), ref[k], synth.BF16, k, stored_bf16=k in IO_GRADS)

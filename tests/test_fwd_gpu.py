@@ -316,6 +316,31 @@ def test_zoh_exact_matches_oracle(cuda_device, dtype, N, lanes):
     assert_close(ls, ref["last_state"], dtype, "last_state", stored_bf16=False)
 
 
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("N", [4, 16, 64])
+def test_zoh_exact_warp_specialised(cuda_device, dtype, N):
+    # the warp-specialised look-back kernel with the exact input term, on a
+    # ragged shape (partial 16-channel group, partial chunk) with an initial state
+    case = synth.make_case(2, 40, 333, N, dtype, seed=420 + N)
+    h0 = np.random.default_rng(N).standard_normal((2, 40, N)).astype(np.float32)
+    ref = oracle.fwd(case, zoh_exact=True, h0=h0)
+    y, ls = _run_zoh(case, cuda_device, "lookback_ws", 2, h0=h0)
+    assert_close(y, ref["y"], dtype, "y")
+    assert_close(ls, ref["last_state"], dtype, "last_state", stored_bf16=False)
+
+
+def test_zoh_exact_auto_picks_warp_specialised(cuda_device):
+    # a Mamba-layer-like shape: AUTO takes the warp-specialised kernel for ZOH too
+    import selective_state_space_54_b200 as ssm
+    case = synth.make_case(4, 5120, 160, 16, synth.BF16, seed=430)
+    shape = ssm.make_shape(4, 5120, 160, 16, ssm.SSM_BF16, flags=ssm.SSM_FLAG_ZOH_EXACT)
+    assert ssm.fwd_path(shape) == "lookback_ws"
+    ref = oracle.fwd(case, zoh_exact=True)
+    y, ls = _run_zoh(case, cuda_device)
+    assert_close(y, ref["y"], synth.BF16, "y")
+    assert_close(ls, ref["last_state"], synth.BF16, "last_state", stored_bf16=False)
+
+
 def test_zoh_exact_with_initial_state_and_large_steps(cuda_device):
     # Delta A spans both branches of (e^x - 1) / x (|x| < 1/2 and beyond)
     case = synth.make_case(1, 64, 200, 16, synth.F32, seed=410)
