@@ -132,7 +132,8 @@ typedef enum {
  * ssm_scan_fwd_workspace_bytes counts them).  Passing that workspace as
  * fwd_workspace to ssm_scan_bwd, with the same shape and flags, lets the
  * backward skip its own forward pass over the chunks.  It runs on path
- * LOOKBACK_WS (AUTO picks it; other explicit paths and lanes = 4 return
+ * LOOKBACK_WS (AUTO picks it; other explicit paths, lanes = 4, and fp32 with
+ * dstate > 32, whose tiles do not fit that kernel's shared memory, return
  * SSM_ERR_UNSUPPORTED). */
 
 /* Bytes of workspace ssm_scan_fwd needs for `shape` on the current device

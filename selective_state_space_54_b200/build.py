@@ -39,21 +39,45 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def _compile(args):
+    cmd, src = args
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    return src, r.returncode, r.stdout + r.stderr
+
+
 def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
+    """Compile every source to an object in parallel, then link the library."""
     if not force and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-shared",
-           "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    from concurrent.futures import ThreadPoolExecutor
+    tmpdir = os.path.join(PKG, f"_build{os.getpid()}")
+    os.makedirs(tmpdir, exist_ok=True)
+    base = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
+            "-I", INCLUDE, "-I", CSRC, "-c"]
     if ptxas_verbose:
-        cmd += ["-Xptxas", "-v"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libssmscan.so")
-    if ptxas_verbose or not quiet:
-        sys.stderr.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
+        base += ["-Xptxas", "-v"]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+        jobs.append((base + ["-o", obj, src], src))
+    try:
+        with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+            results = list(ex.map(_compile, jobs))
+        log = "".join(out for _, _, out in results)
+        if any(rc != 0 for _, rc, _ in results):
+            sys.stderr.write(log)
+            raise RuntimeError("nvcc failed building libssmscan.so")
+        tmp = LIB + f".tmp{os.getpid()}"
+        objs = [os.path.join(tmpdir, os.path.basename(src) + ".o") for src in sources()]
+        r = subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], capture_output=True, text=True)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise RuntimeError("nvcc failed linking libssmscan.so")
+        if ptxas_verbose or not quiet:
+            sys.stderr.write(log)
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(tmpdir, ignore_errors=True)
     return LIB
 
 

@@ -114,8 +114,23 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
     else path = SSM_PATH_PER_GROUP;
   }
   int occ = 0;
-  cudaError_t oe = path == SSM_PATH_LOOKBACK_WS ? fwd_ws_occupancy(s->io_dtype, p.NP, &occ)
-                                                : fwd_occupancy(s->io_dtype, p.NP, lpc, zoh, &occ);
+  cudaError_t oe = cudaSuccess;
+  if (path == SSM_PATH_LOOKBACK_WS) {
+    oe = fwd_ws_occupancy(s->io_dtype, p.NP, &occ);
+    // the warp-specialised kernel's shared memory does not fit every dtype and
+    // state count (fp32 with 64 states needs more than a CTA may have, which
+    // the occupancy query reports as an error): AUTO falls back to the plain
+    // look-back kernel; an explicit request, saved states or token-major
+    // activations (which need it) are refused
+    if (oe != cudaSuccess || occ <= 0) {
+      cudaGetLastError();
+      oe = cudaSuccess;
+      occ = 0;
+      if (s->path != SSM_PATH_AUTO || save || (s->flags & SSM_FLAG_TOKEN_MAJOR)) return SSM_ERR_UNSUPPORTED;
+      path = SSM_PATH_LOOKBACK;
+    }
+  }
+  if (path != SSM_PATH_LOOKBACK_WS) oe = fwd_occupancy(s->io_dtype, p.NP, lpc, zoh, &occ);
   if (oe != cudaSuccess || occ <= 0) {
     cudaGetLastError();
     return SSM_ERR_CUDA;

@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kQThreads, 4) k_bwd16(BwdParams p) {
         float yss = my_c ? k1 : k0;
         yss += __shfl_xor_sync(0xffffffffu, my_c ? k0 : k1, 1);
         const int t = tg + my_s, ch = ch0 + my_c;
-        yss = fmaf(Dd[my_c], st.uu[t][ch], yss);
+        yss = fmaf(my_c ? Dd[1] : Dd[0], st.uu[t][ch], yss);
         q_put(raw.act[2][at<TOK>(ch, t)], yss * st.fz[t][ch]);
       }
       // the reverse recurrence over the group's 2 steps
@@ -486,7 +486,7 @@ __global__ void __launch_bounds__(kQThreads, 4) k_bwd16(BwdParams p) {
         float dlv, dlv_hi, dyv, dyv_hi;
         unpack2(st.dl2[t][ch], dlv, dlv_hi);
         unpack2(st.dy2[t][ch], dyv, dyv_hi);
-        const float du_v = fmaf(dlv, s1sum, dyv * Dd[my_c]);
+        const float du_v = fmaf(dlv, s1sum, dyv * (my_c ? Dd[1] : Dd[0]));
         const float ddl = st.sg[t][ch] * fmaf(st.uu[t][ch], s1sum, kLn2f * ddsum);
         q_put(raw.act[0][at<TOK>(ch, t)], du_v);
         q_put(raw.act[1][at<TOK>(ch, t)], ddl);

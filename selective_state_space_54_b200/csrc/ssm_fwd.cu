@@ -693,7 +693,7 @@ struct Share {
   }
 };
 
-template <typename T, int NP, bool ZOH>
+template <typename T, int NP, bool ZOH, bool SAVE>
 __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &sm, int64_t w,
                                             const Share &sh, unsigned bar_full, unsigned bar_ys) {
   constexpr int S = NP / 2, CPW = 16;
@@ -726,7 +726,7 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
     // entering every kCkptSteps-step chunk (two per kTW-step chunk here)
     float *ck = nullptr;
     const int64_t ck_K = ckpt_chunks(p.L);
-    if (p.ckpt_out && ln.valid) ck = p.ckpt_out + ckpt_offset(ln.b, ln.d, 0, p.dim, p.L, NP) + j * S;
+    if (SAVE && ln.valid) ck = p.ckpt_out + ckpt_offset(ln.b, ln.d, 0, p.dim, p.L, NP) + j * S;
     auto save_state = [&](int64_t k8) {
       float *dst = ck + k8 * kCkptChannels * NP;
       if constexpr (S % 4 == 0) {
@@ -741,11 +741,11 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = (int)(it & 1);
       WSStage<NP> &st = sm.st[stage];
-      if (ck) save_state(2 * k);  // the state entering step kTW * k
+      if (SAVE && ck) save_state(2 * k);  // the state entering step kTW * k
       bar_sync_n(bar_full + stage, 64);
 #pragma unroll
       for (int tt = 0; tt < kTW; tt += 4) {
-        if (tt == kCkptSteps && ck && 2 * k + 1 < ck_K) save_state(2 * k + 1);  // entering step kTW k + 8
+        if (SAVE && tt == kCkptSteps && ck && 2 * k + 1 < ck_K) save_state(2 * k + 1);  // entering step kTW k + 8
         const float4 d4 = *reinterpret_cast<const float4 *>(&st.dl[c][tt]);
         const float4 u4 = *reinterpret_cast<const float4 *>(&st.dlu[c][tt]);
         const float dls[4] = {d4.x, d4.y, d4.z, d4.w};
@@ -1133,7 +1133,10 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   cp_async_wait<0>();
 }
 
-template <typename T, int NP, bool TOK, bool ZOH>
+// TOK: token-major activations; ZOH: the exact input term; SAVE: the chunk
+// states for the backward are written (separate instantiations, so that the
+// plain forward carries none of that code)
+template <typename T, int NP, bool TOK, bool ZOH, bool SAVE>
 __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
@@ -1145,7 +1148,7 @@ __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   const Share sh(w, p.n_workers, p.n_groups, p.n_chunks);
   const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
   if (producer) ws_producer<T, NP, TOK>(p, sm, sh, bar_full, bar_ys);
-  else ws_consumer<T, NP, ZOH>(p, sm, w, sh, bar_full, bar_ys);
+  else ws_consumer<T, NP, ZOH, SAVE>(p, sm, w, sh, bar_full, bar_ys);
 }
 
 // ---- host side ------------------------------------------------------------------
@@ -1240,9 +1243,9 @@ cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm) {
     using T = typename decltype(tt)::type;
     constexpr int kNP = decltype(np)::value;
     const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
-    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false, false>, smem);
+    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false, false, false>, smem);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP, false, false>, kWSThreads,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP, false, false, false>, kWSThreads,
                                                          smem);
   });
 }
@@ -1253,17 +1256,20 @@ cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t
     constexpr int kNP = decltype(np)::value;
     const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
     const unsigned grid = (unsigned)((p.n_workers + kPairs - 1) / kPairs);
-    if (p.tok) {  // token-major tiles: bf16 only (the API checks)
+    const bool save = p.ckpt_out != nullptr;
+    if (p.tok) {  // token-major tiles: bf16, Euler only (the API checks)
       if constexpr (sizeof(T) == 2) {
-        cudaError_t e = allow_smem(k_fwd_ws<T, kNP, true, false>, smem);
+        auto kern = save ? k_fwd_ws<T, kNP, true, false, true> : k_fwd_ws<T, kNP, true, false, false>;
+        cudaError_t e = allow_smem(kern, smem);
         if (e != cudaSuccess) return e;
-        k_fwd_ws<T, kNP, true, false><<<grid, kWSThreads, smem, s>>>(p);
+        kern<<<grid, kWSThreads, smem, s>>>(p);
         return cudaGetLastError();
       } else {
         return cudaErrorInvalidValue;
       }
     }
-    auto kern = p.zoh ? k_fwd_ws<T, kNP, false, true> : k_fwd_ws<T, kNP, false, false>;
+    auto kern = p.zoh ? (save ? k_fwd_ws<T, kNP, false, true, true> : k_fwd_ws<T, kNP, false, true, false>)
+                      : (save ? k_fwd_ws<T, kNP, false, false, true> : k_fwd_ws<T, kNP, false, false, false>);
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kWSThreads, smem, s>>>(p);

@@ -316,8 +316,8 @@ def test_zoh_exact_matches_oracle(cuda_device, dtype, N, lanes):
     assert_close(ls, ref["last_state"], dtype, "last_state", stored_bf16=False)
 
 
-@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
-@pytest.mark.parametrize("N", [4, 16, 64])
+@pytest.mark.parametrize("dtype,N", [(synth.F32, 4), (synth.F32, 16), (synth.BF16, 4),
+                                     (synth.BF16, 16), (synth.BF16, 64)])
 def test_zoh_exact_warp_specialised(cuda_device, dtype, N):
     # the warp-specialised look-back kernel with the exact input term, on a
     # ragged shape (partial 16-channel group, partial chunk) with an initial state
@@ -339,6 +339,23 @@ def test_zoh_exact_auto_picks_warp_specialised(cuda_device):
     y, ls = _run_zoh(case, cuda_device)
     assert_close(y, ref["y"], synth.BF16, "y")
     assert_close(ls, ref["last_state"], synth.BF16, "last_state", stored_bf16=False)
+
+
+def test_warp_specialised_capacity_fallback(cuda_device):
+    # fp32 with 64 states does not fit the warp-specialised kernel's shared
+    # memory: an explicit request is refused, AUTO takes the plain look-back
+    # kernel on a shape where it would otherwise pick the specialised one
+    import selective_state_space_54_b200 as ssm
+    explicit = ssm.make_shape(4, 5120, 64, 64, ssm.SSM_F32, ssm.SSM_PATH_LOOKBACK_WS)
+    assert ssm.fwd_workspace_bytes(explicit) == 0
+    auto = ssm.make_shape(4, 5120, 64, 64, ssm.SSM_F32)
+    assert ssm.fwd_path(auto) == "lookback"
+    assert ssm.fwd_path(ssm.make_shape(4, 5120, 64, 64, ssm.SSM_BF16)) == "lookback_ws"
+    case = synth.make_case(4, 5120, 64, 64, synth.F32, seed=440)
+    ref = oracle.fwd(case)
+    y, ls = _run(case, cuda_device)
+    assert_close(y, ref["y"], synth.F32, "y")
+    assert_close(ls, ref["last_state"], synth.F32, "last_state")
 
 
 def test_zoh_exact_with_initial_state_and_large_steps(cuda_device):
