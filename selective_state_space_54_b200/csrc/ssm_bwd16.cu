@@ -445,12 +445,13 @@ __global__ void __launch_bounds__(kQThreads, 4) k_bwd16(BwdParams p) {
           for (int q = 0; q < 2; ++q) {
             g[c][q] = fma2(dy[c], C[q], g[c][q]);
             dCp[q] = c ? fma2(dy[c], hs[s][c][q], dCp[q]) : mul2(dy[c], hs[s][c][q]);
-            const f2 qv = mul2(g[c][q], mul2(as[s][c][q], s ? hs[0][c][q] : he[c][q]));
-            dA[c][q] = fma2(dl[c], qv, dA[c][q]);
-            dd = q ? fma2(A2[c][q], qv, dd) : mul2(A2[c][q], qv);
             s1 = q ? fma2(g[c][q], B[q], s1) : mul2(g[c][q], B[q]);
             dBp[q] = c ? fma2(g[c][q], du[c], dBp[q]) : mul2(g[c][q], du[c]);
+            // g a_t is both dL/dh_{t-1} and the factor of h_{t-1} in dA and dDelta
             g[c][q] = mul2(g[c][q], as[s][c][q]);
+            const f2 qv = mul2(g[c][q], s ? hs[0][c][q] : he[c][q]);  // g a_t h_{t-1}
+            dA[c][q] = fma2(dl[c], qv, dA[c][q]);
+            dd = q ? fma2(A2[c][q], qv, dd) : mul2(A2[c][q], qv);
           }
           float lo, hi;
           unpack2(dd, lo, hi);
