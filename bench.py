@@ -342,18 +342,19 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     ms_b = max_over_ranks(t_b / steps)
     # The roofline counts the method's own special-function work: one exp2
     # per (b, t, d, n) element (the decay exp(Delta A) the backward must
-    # recompute).  The kernel's own count is reported beside it: it
-    # exponentiates each element twice (once to recompute the 16-step chunk's
-    # sums, once for the 4-step group whose decays the reverse pass reuses).
+    # recompute).  The kernel's own count is reported beside it: the d_state-16
+    # backward exponentiates 6 of every 8 steps to rebuild the 2-step group
+    # entry states of a chunk, then every step again for the group whose
+    # decays the reverse pass uses (1.75 per element).
     ex2_per_element = 1
-    kernel_ex2 = 2
+    kernel_ex2 = 1.75
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
     bwd_achieved = ex2_per_element * w.bldn / (ms_b * 1e-3)
     bwd_roofline = {"bound": "alu", "achieved": bwd_achieved / 1e12, "peak": ex2_peak / 1e12,
                     "unit": "Tex2/s", "frac": bwd_achieved / ex2_peak, "traffic": None,
-                    "kernel": "k_bwd", "ex2_per_element": ex2_per_element,
+                    "kernel": "k_bwd16", "ex2_per_element": ex2_per_element,
                     "kernel_ex2_per_element": kernel_ex2,
                     "kernel_mufu_frac": kernel_ex2 * w.bldn / (ms_b * 1e-3) / ex2_peak,
                     "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "

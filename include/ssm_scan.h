@@ -196,7 +196,7 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
  * one on the execute path, or real-time loops that allocate nothing after
  * start-up.  The pages have no counterpart of this: it is a deployment
  * convenience.  Same arguments and results as ssm_scan_fwd, without the
- * workspace: the scratch lives in one 4 MiB device array inside the library
+ * workspace: the scratch lives in one 16 MiB device array inside the library
  * (held on every GPU that loads it until the process exits).
  *  - path AUTO keeps ssm_scan_fwd's own choice when that is LOOKBACK,
  *    LOOKBACK_WS (the default for Mamba layer shapes, token-major included)

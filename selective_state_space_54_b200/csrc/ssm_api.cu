@@ -60,6 +60,7 @@ struct FwdPlan {
   int64_t P = 0;                     // look-back warps
   int64_t n_segs = 1, seg_chunks = 0;
   size_t off_flags = 0, off_carry = 0, off_seg_h = 0, off_seg_dsum = 0, off_seg_carry = 0;
+  size_t off_bcf = 0;                // fp32 B and C (warp-specialised schedule)
   size_t ckpt_bytes = 0;             // saved states, right after the header
   size_t total = kHeaderBytes;
 };
@@ -157,6 +158,10 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
     p.off_flags = round_up(kHeaderBytes + p.ckpt_bytes, 256);
     p.off_carry = round_up(p.off_flags + sizeof(unsigned) * (size_t)p.P, 256);
     p.total = round_up(p.off_carry + sizeof(float) * (size_t)p.P * cpw * p.NP, 256);
+    if (path == SSM_PATH_LOOKBACK_WS) {  // fp32 B and C, [batch][L][NP] each
+      p.off_bcf = p.total;
+      p.total = round_up(p.off_bcf + 2 * sizeof(float) * (size_t)s->batch * (size_t)s->seqlen * p.NP, 256);
+    }
   } else if (path == SSM_PATH_SPLIT_L) {
     // about two waves of resident warps; segments of at least 4 chunks
     int64_t target = 2 * slots;
@@ -303,6 +308,14 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
     p.carry = reinterpret_cast<float *>(ws + pl.off_carry);
     e = cudaMemsetAsync(ws + pl.off_flags, 0, pl.off_carry - pl.off_flags, s);  // flags
     if (e != cudaSuccess) return cuda_status(e);
+    if (pl.path == SSM_PATH_LOOKBACK_WS) {
+      float *Bf = reinterpret_cast<float *>(ws + pl.off_bcf);
+      float *Cf = Bf + (size_t)shape->batch * (size_t)shape->seqlen * pl.NP;
+      p.Bf = Bf;
+      p.Cf = Cf;
+      e = launch_widen_bc(shape->io_dtype, B, C, Bf, Cf, shape->batch * shape->seqlen, (int)shape->dstate, pl.NP, s);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
     e = pl.path == SSM_PATH_LOOKBACK_WS ? launch_fwd_ws(shape->io_dtype, pl.NP, p, s)
                                         : launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
   } else {

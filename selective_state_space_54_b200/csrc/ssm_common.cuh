@@ -77,6 +77,8 @@ struct FwdParams {
   // saved states for the backward (nullable): the state entering every
   // kCkptSteps-step chunk, at ckpt_offset(b, d, chunk, dim, L, NP)
   float *ckpt_out;
+  // B and C as fp32 [batch][L][NP] (warp-specialised schedule; k_widen_bc)
+  const float *Bf, *Cf;
   float *seg_h;       // [n_groups * n_segs][32/LPC][NP] segment end state from zero
   float *seg_dsum;    // [n_groups * n_segs][32/LPC]     sum of Delta over the segment
   float *seg_carry;   // [n_groups * n_segs][32/LPC][NP] state entering the segment
@@ -361,6 +363,8 @@ int fwd_ws_chunk();
 int fwd_ws_pairs();
 cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm);
 cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
+cudaError_t launch_widen_bc(int io_dtype, const void *B, const void *C, float *Bf, float *Cf, int64_t rows,
+                            int N, int NP, cudaStream_t s);
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);
 int64_t bwd_blocks(int64_t dim, int NP, int zoh);
 cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s);

@@ -616,11 +616,12 @@ __global__ void k_wait_probe(unsigned *flag, unsigned *err, unsigned long long l
 // consumer runs only the recurrence: per element one MUFU ex2 and two packed
 // fp32 pair operations, so the special-function unit is kept busy.  The
 // producer does everything else for the same chunks: the input copies
-// (cp.async into a ring of raw chunks, three chunks ahead), softplus,
-// Delta*u, the B/C widening, the gate, and the output epilogue of the chunk
-// before.  Two shared-memory stages alternate; named barriers carry "stage
-// full" (producer -> consumer) and "sums ready" (consumer -> producer) per
-// pair and stage.
+// (cp.async into a ring of raw chunks, three chunks ahead; B and C from the
+// fp32 copy k_widen_bc makes before the scan, into a ring of its own that
+// the consumer reads directly), softplus, Delta*u, the gate, and the output
+// epilogue of the chunk before.  Two shared-memory stages alternate; named
+// barriers carry "stage full" (producer -> consumer) and "sums ready"
+// (consumer -> producer) per pair and stage.
 constexpr int kTW = 16;
 static_assert(kTW == 2 * kCkptSteps, "the saved states are written at the start and the middle of each chunk");
 constexpr int kPairs = 4;
@@ -631,21 +632,28 @@ struct __align__(16) WSStage {
   float dl[16][kTW + 4];
   float dlu[16][kTW + 4];
   float ys[2][16][kTW + 4];  // C.h partial sums of a channel's two lanes
-  float Bs[kTW][NP];
-  float Cs[kTW][NP];
 };
-constexpr int kSlots = 4;  // raw-input ring: chunks k+1..k+3 in flight while k is processed
+constexpr int kSlots = 4;    // raw-input ring: chunks k+1..k+3 in flight while k is processed
+constexpr int kBCSlots = 5;  // B/C ring: a chunk's B and C stay until the consumer is done with it
 
-template <typename T, int NP>
+template <typename T>
 struct __align__(16) WSRaw {
   T u[16][kTW], d[16][kTW], z[16][kTW];  // [channel][step], io dtype
-  T B[kTW][NP], C[kTW][NP];              // [step][state], io dtype
+};
+
+// B and C of one chunk in fp32 ([step][state], zero padded), copied straight
+// from the fp32 copy k_widen_bc makes before the scan: the consumer reads
+// them from the ring, so nobody widens them inside the scan.
+template <int NP>
+struct __align__(16) WSBC {
+  float B[kTW][NP], C[kTW][NP];
 };
 
 template <typename T, int NP>
 struct __align__(16) WSPair {
   WSStage<NP> st[2];
-  WSRaw<T, NP> raw[kSlots];
+  WSRaw<T> raw[kSlots];
+  WSBC<NP> bc[kBCSlots];
 };
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
@@ -698,6 +706,7 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
                                             const Share &sh, unsigned bar_full, unsigned bar_ys) {
   constexpr int S = NP / 2, CPW = 16;
   int64_t it = 0;
+  int bc_slot = 0;  // B/C ring slot of the chunk being processed
   for (int64_t r = 0; r < sh.n_runs; ++r) {
     int64_t g, k0, k1;
     sh.get(r, g, k0, k1);
@@ -741,6 +750,8 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = (int)(it & 1);
       WSStage<NP> &st = sm.st[stage];
+      const WSBC<NP> &bcs = sm.bc[bc_slot];
+      bc_slot = bc_slot + 1 == kBCSlots ? 0 : bc_slot + 1;
       if (SAVE && ck) save_state(2 * k);  // the state entering step kTW * k
       bar_sync_n(bar_full + stage, 64);
 #pragma unroll
@@ -753,8 +764,8 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
         float yp[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float *Brow = &st.Bs[tt + i][j * S];
-          const float *Crow = &st.Cs[tt + i][j * S];
+          const float *Brow = &bcs.B[tt + i][j * S];
+          const float *Crow = &bcs.C[tt + i][j * S];
           const f2 dl2 = pack2(dls[i], dls[i]), du2 = pack2(dus[i], dus[i]);
           f2 acc = 0;  // sum_n C h as a pair of partial sums
 #pragma unroll
@@ -807,11 +818,12 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
 // Producer lanes take channel c = lane % 16 and steps [8j, 8j+8) of every
 // chunk with j = lane / 16, so that a quarter warp's 16-byte row accesses fall
 // in distinct shared-memory banks.  The u/delta/z/y pointers already point at
-// step 8j of the channel's row; B/C at this lane's first 16-byte piece.
+// step 8j of the channel's row; the fp32 B/C at this lane's first 16-byte piece.
 template <typename T, int NP>
 struct RunRows {
   static constexpr int EPP = 16 / (int)sizeof(T);  // elements per 16-byte piece
-  const T *u, *dr, *z, *Bb, *Cb, *Bl, *Cl;
+  const T *u, *dr, *z;
+  const float *Bl, *Cl;  // this lane's first 16-byte piece of the fp32 B/C rows of the batch element
   T *y;
   float bias, Dd;
   bool valid;
@@ -830,10 +842,8 @@ struct RunRows {
     dr = static_cast<const T *>(p.delta) + row;
     z = p.z ? static_cast<const T *>(p.z) + row : nullptr;
     y = static_cast<T *>(p.y) + row;
-    Bb = static_cast<const T *>(p.B) + b * p.L * p.N;
-    Cb = static_cast<const T *>(p.C) + b * p.L * p.N;
-    Bl = Bb + lane * EPP;
-    Cl = Cb + lane * EPP;
+    Bl = p.Bf + b * p.L * NP + lane * 4;
+    Cl = p.Cf + b * p.L * NP + lane * 4;
     bias = (p.bias && valid) ? p.bias[d] : 0.f;
     Dd = (p.D && valid) ? p.D[d] : 0.f;
     tok_c0 = (g - b * p.gpb) * 16;
@@ -847,10 +857,10 @@ struct RunRows {
 // unaligned rows take the checked one (zero fill past L).  Every lane later
 // reads only the pieces it copied itself.
 template <typename T, int NP, bool TOK>
-__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, const RunRows<T, NP> &rr,
-                                         int64_t k, int lane) {
+__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T> &raw, WSBC<NP> &bc,
+                                         const RunRows<T, NP> &rr, int64_t k, int lane) {
   constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
-  constexpr int NV = kTW * NP / EPP;  // B/C pieces per chunk
+  constexpr int NVF = kTW * NP / 4;  // fp32 B/C pieces per chunk and tensor
   const int c = lane & 15, j8 = (lane >> 4) * 8;
   const int64_t L = p.L, t0 = k * kTW;
   const bool whole = t0 + kTW <= L;
@@ -900,25 +910,17 @@ __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, NP> &raw, 
       if (rr.z) raw.z[c][j8 + i] = in ? rr.z[t0 + i] : T(0);
     }
   }
-  if (p.bc_vec && NP % EPP == 0) {
-    T *rB = &raw.B[0][0], *rC = &raw.C[0][0];
+  // fp32 B/C pieces lane, lane + 32, ... of the chunk (a piece is 4 states of one step)
+  float *rB = &bc.B[0][0], *rC = &bc.C[0][0];
 #pragma unroll
-    for (int q = 0; q < (NV + 31) / 32; ++q) {
-      const int v = lane + 32 * q;
-      if (NV % 32 == 0 || v < NV) {
-        const int e = v * EPP;
-        const bool in = whole || t0 + e / NP < L;
-        const int64_t off = in ? t0 * NP + q * 32 * EPP : -(int64_t)lane * EPP;
-        cp_async16(rB + e, rr.Bl + off, in ? 16 : 0);
-        cp_async16(rC + e, rr.Cl + off, in ? 16 : 0);
-      }
-    }
-  } else {
-    for (int e = lane; e < kTW * NP; e += 32) {
-      const int t = e / NP, n = e - t * NP;
-      const bool in = n < p.N && t0 + t < L;
-      raw.B[t][n] = in ? rr.Bb[(t0 + t) * p.N + n] : T(0);
-      raw.C[t][n] = in ? rr.Cb[(t0 + t) * p.N + n] : T(0);
+  for (int q = 0; q < (NVF + 31) / 32; ++q) {
+    const int v = lane + 32 * q;
+    if (NVF % 32 == 0 || v < NVF) {
+      const int e = v * 4;
+      const bool in = whole || t0 + e / NP < L;
+      const int64_t off = in ? t0 * NP + q * 32 * 4 : -(int64_t)lane * 4;  // the row start when nothing is read
+      cp_async16(rB + e, rr.Bl + off, in ? 16 : 0);
+      cp_async16(rC + e, rr.Cl + off, in ? 16 : 0);
     }
   }
 }
@@ -929,8 +931,6 @@ __device__ __forceinline__ float io_to_f(float v) { return v; }
 template <typename T, int NP, bool TOK>
 __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &sm, const Share &sh,
                                             unsigned bar_full, unsigned bar_ys) {
-  constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
-  constexpr int NV = kTW * NP / EPP;
   const int64_t L = p.L;
   const int lane = threadIdx.x & 31;
   const int c = lane & 15, j8 = (lane >> 4) * 8;
@@ -962,15 +962,18 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
       }
     }
   };
-  int it_f = 0;  // chunks fetched (slot cursor)
-  for (int i = 0; i < kSlots - 1; ++i) {
+  int it_f = 0;     // chunks fetched (raw slot cursor)
+  int bc_f = 0;     // B/C ring slot of the next chunk fetched
+  auto fetch_next = [&]() {
     if (pf_live) {
-      ws_fetch<T, NP, TOK>(p, sm.raw[it_f % kSlots], pf, pk, lane);
+      ws_fetch<T, NP, TOK>(p, sm.raw[it_f % kSlots], sm.bc[bc_f], pf, pk, lane);
       advance();
     }
     cp_async_commit();
     ++it_f;
-  }
+    bc_f = bc_f + 1 == kBCSlots ? 0 : bc_f + 1;
+  };
+  for (int i = 0; i < kSlots - 1; ++i) fetch_next();
 
   int it = 0;
   for (int64_t r = 0; r < sh.n_runs; ++r) {
@@ -981,12 +984,12 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = it & 1;
       WSStage<NP> &st = sm.st[stage];
-      WSRaw<T, NP> &raw = sm.raw[it % kSlots];
+      WSRaw<T> &raw = sm.raw[it % kSlots];
       const int64_t t0 = k * kTW;
       const bool whole = cur.valid && t0 + kTW <= L;
       cp_async_wait<kSlots - 2>();  // this chunk's copies have landed
       if constexpr (tok) __syncwarp();  // token-major tiles hold other lanes' copies
-      // ---- pre-pass of chunk k into the stage: Delta, Delta*u, B/C in fp32 ----
+      // ---- pre-pass of chunk k into the stage: Delta, Delta*u ----
       float u8[8], s8[8];
       if constexpr (tok) {  // [step][channel] tile: this lane's channel c at steps j8..j8+7
 #pragma unroll
@@ -1028,32 +1031,10 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
         *reinterpret_cast<ulonglong2 *>(pu) = make_ulonglong2(dlu2[0], dlu2[1]);
         *reinterpret_cast<ulonglong2 *>(pu + 4) = make_ulonglong2(dlu2[2], dlu2[3]);
       }
-      // widen this lane's B/C pieces (the ones it fetched) to fp32
-      if (p.bc_vec && NP % EPP == 0) {
-#pragma unroll
-        for (int q = 0; q < (NV + 31) / 32; ++q) {
-          const int v = lane + 32 * q;
-          if (NV % 32 == 0 || v < NV) {
-            const int e = v * EPP;
-            bc_store_vec<T, NP>(st.Bs, *reinterpret_cast<const uint4 *>(&raw.B[0][0] + e), v);
-            bc_store_vec<T, NP>(st.Cs, *reinterpret_cast<const uint4 *>(&raw.C[0][0] + e), v);
-          }
-        }
-      } else {
-        for (int e = lane; e < kTW * NP; e += 32) {
-          const int t = e / NP, n = e - t * NP;
-          st.Bs[t][n] = io_to_f(raw.B[t][n]);
-          st.Cs[t][n] = io_to_f(raw.C[t][n]);
-        }
-      }
       bar_arrive_n(bar_full + stage, 64);
-      // ---- copies of the chunk kSlots-1 ahead, into the slot of chunk k-1 ----
-      if (pf_live) {
-        ws_fetch<T, NP, TOK>(p, sm.raw[it_f % kSlots], pf, pk, lane);
-        advance();
-      }
-      cp_async_commit();
-      ++it_f;
+      // ---- copies of the chunk kSlots-1 ahead: raw slot of chunk k-1; B/C slot
+      // of chunk k-2, which the consumer released before this stage was filled ----
+      fetch_next();
       // ---- epilogue of chunk k-1: y = (C.h + D*u) * SiLU(z) ----
       if (pend) {
         bar_sync_n(bar_ys + pstage, 64);
@@ -1149,6 +1130,38 @@ __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
   if (producer) ws_producer<T, NP, TOK>(p, sm, sh, bar_full, bar_ys);
   else ws_consumer<T, NP, ZOH, SAVE>(p, sm, w, sh, bar_full, bar_ys);
+}
+
+// B and C as fp32 [batch][L][NP], zero padded past N: the warp-specialised
+// kernel copies them into its B/C ring as they are, so that no warp widens
+// them inside the scan (4 MB at the Mamba-2.8B layer shape, against 1.3 GB
+// the scan streams).
+template <typename T>
+__global__ void k_widen_bc(const T *__restrict__ B, const T *__restrict__ C, float *__restrict__ Bf,
+                           float *__restrict__ Cf, int64_t rows, int N, int NP) {
+  const int64_t total = rows * NP;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / NP;
+    const int n = (int)(i - r * NP);
+    Bf[i] = n < N ? io_to_f(B[r * N + n]) : 0.f;
+    Cf[i] = n < N ? io_to_f(C[r * N + n]) : 0.f;
+  }
+}
+
+cudaError_t launch_widen_bc(int io_dtype, const void *B, const void *C, float *Bf, float *Cf, int64_t rows,
+                            int N, int NP, cudaStream_t s) {
+  const int64_t total = rows * NP;
+  if (total == 0) return cudaSuccess;
+  const int64_t want = (total + 255) / 256;
+  const unsigned grid = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+  if (io_dtype == 1)
+    k_widen_bc<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(B), static_cast<const uint16_t *>(C),
+                                              Bf, Cf, rows, N, NP);
+  else
+    k_widen_bc<float><<<grid, 256, 0, s>>>(static_cast<const float *>(B), static_cast<const float *>(C), Bf, Cf,
+                                           rows, N, NP);
+  return cudaGetLastError();
 }
 
 // ---- host side ------------------------------------------------------------------

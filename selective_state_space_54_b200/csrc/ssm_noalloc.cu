@@ -9,7 +9,7 @@
 // and the error word) in one fixed device array that lives in this library.
 //
 // Costs and limits, for a user of this library:
-//  - the array holds kStaticScratchBytes (4 MiB) on every GPU that loads the
+//  - the array holds kStaticScratchBytes (16 MiB) on every GPU that loads the
 //    library, from load until the process exits;
 //  - shapes whose scratch would exceed it are rejected (SSM_ERR_UNSUPPORTED,
 //    with a message on stderr) before anything is launched;
@@ -30,7 +30,7 @@
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(4) << 20;
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
 
 // The scratch itself.  Host code may not use the symbol as an address: it is
 // a host-side stand-in, so the device address is looked up on every call.
