@@ -544,11 +544,11 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         ws.pd[t][c][j] = make_float2(d0 + d1, s0 + s1v);
       }
       __syncthreads();
-      // dB, dC of this group: sums over the 4 warps x 8 channels, added to
-      // the fp32 accumulators (16-byte vector atomics when S >= 4)
+      // dB, dC of this group: sums over the 4 warps x 8 channels, stored as
+      // this 32-channel block's partial (16-byte stores when S >= 4)
       if constexpr (S >= 4) {
         // every warp sums its own 8 channels for each output; warp 0 then
-        // adds the 4 warps' sums and issues the atomics
+        // adds the 4 warps' sums in order and stores them
         for (int o = lane; o < kRedOutputs; o += 32) {
           const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
           const int which = r4 / NP, n = r4 - which * NP;

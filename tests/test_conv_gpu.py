@@ -165,3 +165,4 @@ def test_conv_bwd_full_mamba_2p8b_layer(cuda_device):
     assert_close(got["dx"], ref["dx"], synth.BF16, "dx")
     assert_close(got["dweight"], ref["dweight"], synth.BF16, "dweight", stored_bf16=False)
     assert_close(got["dbias"], ref["dbias"], synth.BF16, "dbias", stored_bf16=False)
+
