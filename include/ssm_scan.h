@@ -75,11 +75,16 @@ typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
  *            a sequential carry over segments, then the output pass);
  *            for long sequences with few channels;
  *  PER_GROUP one warp per channel group over the whole sequence;
- *  LOOKBACK_WS  the look-back schedule with warp specialisation (2 lanes per
- *            channel): producer warps load inputs and compute softplus, the
- *            gate and the output epilogue on the FMA pipe, consumer warps run
- *            only the recurrence; AUTO picks it when it picks LOOKBACK with
- *            2 lanes per channel. */
+ *  LOOKBACK_WS  the look-back schedule (16-step chunks) with warp
+ *            specialisation: producer warps load inputs and compute softplus,
+ *            the gate and the output epilogue on the FMA pipe, consumer warps
+ *            run only the recurrence.  2 lanes per channel (16-channel groups;
+ *            the default when lanes = 0) or 4 (8-channel groups, dstate 5..16,
+ *            channel-major, no saved states; SSM_ERR_UNSUPPORTED otherwise).
+ *            AUTO picks it with 2 lanes once batch * ceil(dim/16) reaches 3/4
+ *            of the device's SM sub-partitions (4 per SM), with 4 lanes when
+ *            batch * ceil(dim/8) reaches them, and falls back to LOOKBACK
+ *            where its shared memory does not fit (fp32, dstate > 32). */
 typedef enum {
   SSM_PATH_AUTO = 0,
   SSM_PATH_LOOKBACK = 1,
@@ -95,7 +100,7 @@ typedef struct {
   int64_t dstate;   /* N, 1..64 */
   int32_t io_dtype; /* ssm_dtype */
   int32_t path;     /* ssm_path (forward only; ignored by the backward) */
-  int32_t lanes;    /* lanes per channel in the forward: 0 = auto, 2 or 4 */
+  int32_t lanes;    /* lanes per channel in the forward: 0 = auto, 2 or 4 (see LOOKBACK_WS) */
   int32_t flags;    /* ssm_flags bits; others must be 0 */
 } ssm_shape;
 

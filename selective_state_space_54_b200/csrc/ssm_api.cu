@@ -29,7 +29,9 @@ ssm_status check_shape(const ssm_shape *s) {
   if (s->dstate > 64) return SSM_ERR_UNSUPPORTED;
   if (s->io_dtype != SSM_F32 && s->io_dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
   if (s->path < SSM_PATH_AUTO || s->path > SSM_PATH_LOOKBACK_WS) return SSM_ERR_UNSUPPORTED;
-  if (s->path == SSM_PATH_LOOKBACK_WS && s->lanes == 4) return SSM_ERR_UNSUPPORTED;
+  // the warp-specialised kernel takes 4 lanes per channel for 5..16 states only
+  if (s->path == SSM_PATH_LOOKBACK_WS && s->lanes == 4 && (s->dstate < 5 || s->dstate > 16))
+    return SSM_ERR_UNSUPPORTED;
   if (s->lanes != 0 && s->lanes != 2 && s->lanes != 4) return SSM_ERR_UNSUPPORTED;
   if (s->flags & ~(SSM_FLAG_ZOH_EXACT | SSM_FLAG_SAVE_STATES | SSM_FLAG_TOKEN_MAJOR))
     return SSM_ERR_INVALID_ARG;
@@ -72,10 +74,17 @@ int64_t groups_for(const ssm_shape *s, int lpc) {
 
 // Schedule choice.  The look-back schedule needs at least one channel group
 // per warp slot it uses (P <= groups) and balances work exactly, so it is
-// preferred whenever the problem has enough channel groups; two lanes per
-// channel (fewer instructions per element) when that still leaves two warps
-// per SM sub-partition, else four.  Long sequences with few channels take the
-// two-pass split-L schedule; tiny problems one warp per group.
+// preferred whenever the problem has enough channel groups.  AUTO takes the
+// warp-specialised kernel with 16-channel groups (2 lanes per channel) once
+// there are 3/4 as many such groups as SM sub-partitions: even with a single
+// producer / consumer pair on most sub-partitions it beats every other
+// schedule there (measured on B200: 0.137 ms against 0.172 ms with 8-channel
+// groups and 0.236 ms for the plain kernel at batch 8, d_inner 1024, L 2048).
+// With fewer, the 8-channel-group version (4 lanes per channel) once those
+// groups fill the sub-partitions (0.250 against 0.260 and 0.347 ms at batch 4,
+// d_inner 1536, L 4096), the plain look-back kernel where the state count has
+// no such version.  Long sequences with few channels take the two-pass
+// split-L schedule; tiny problems one warp per group.
 ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   ssm_status st = check_shape(s);
   if (st != SSM_OK) return st;
@@ -98,18 +107,22 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
     lpc = 2;
   }
   if (save) p.ckpt_bytes = sizeof(float) * bwd_ckpt_floats(s->batch, s->dim, s->seqlen, p.NP);
+  // the warp-specialised kernel with 4 lanes per channel exists for 8 and 16 padded states
+  const bool ws4 = p.NP == 8 || p.NP == 16;
   if (lpc == 0) {
     if (path == SSM_PATH_SPLIT_L || path == SSM_PATH_LOOKBACK_WS) lpc = 2;
     else if (path == SSM_PATH_PER_GROUP) lpc = 4;
+    else if (path == SSM_PATH_AUTO && 4 * g2 >= 3 * unit) lpc = 2;  // the warp-specialised kernel
     else if (g2 >= 2 * unit) lpc = 2;
     else if (g4 >= unit || path == SSM_PATH_LOOKBACK) lpc = 4;
     else lpc = p.K >= 64 ? 2 : 4;
   }
-  const int64_t G = lpc == 2 ? g2 : g4;
-  // the exact-ZOH input term is built into the look-back kernel only
+  int64_t G = lpc == 2 ? g2 : g4;
+  // the exact-ZOH input term is built into the look-back kernels only
   const bool zoh = (s->flags & SSM_FLAG_ZOH_EXACT) != 0;
   if (path == SSM_PATH_AUTO) {
-    if (G >= unit) path = lpc == 2 ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
+    if (lpc == 2 && 4 * G >= 3 * unit) path = SSM_PATH_LOOKBACK_WS;
+    else if (G >= unit) path = (lpc == 2 || ws4) ? SSM_PATH_LOOKBACK_WS : SSM_PATH_LOOKBACK;
     else if (zoh) path = SSM_PATH_LOOKBACK;  // split-L and per-group are Euler only
     else if (p.K >= 64) path = SSM_PATH_SPLIT_L;
     else path = SSM_PATH_PER_GROUP;
@@ -117,7 +130,7 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   int occ = 0;
   cudaError_t oe = cudaSuccess;
   if (path == SSM_PATH_LOOKBACK_WS) {
-    oe = fwd_ws_occupancy(s->io_dtype, p.NP, &occ);
+    oe = fwd_ws_occupancy(s->io_dtype, p.NP, lpc, &occ);
     // the warp-specialised kernel's shared memory does not fit every dtype and
     // state count (fp32 with 64 states needs more than a CTA may have, which
     // the occupancy query reports as an error): AUTO falls back to the plain
@@ -129,6 +142,10 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
       occ = 0;
       if (s->path != SSM_PATH_AUTO || save || (s->flags & SSM_FLAG_TOKEN_MAJOR)) return SSM_ERR_UNSUPPORTED;
       path = SSM_PATH_LOOKBACK;
+      if (s->lanes == 0 && g2 < 2 * unit && g4 >= unit) {  // the plain kernel's own lane choice
+        lpc = 4;
+        G = g4;
+      }
     }
   }
   if (path != SSM_PATH_LOOKBACK_WS) oe = fwd_occupancy(s->io_dtype, p.NP, lpc, zoh, &occ);
@@ -316,7 +333,7 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
       e = launch_widen_bc(shape->io_dtype, B, C, Bf, Cf, shape->batch * shape->seqlen, (int)shape->dstate, pl.NP, s);
       if (e != cudaSuccess) return cuda_status(e);
     }
-    e = pl.path == SSM_PATH_LOOKBACK_WS ? launch_fwd_ws(shape->io_dtype, pl.NP, p, s)
+    e = pl.path == SSM_PATH_LOOKBACK_WS ? launch_fwd_ws(shape->io_dtype, pl.NP, pl.LPC, p, s)
                                         : launch_fwd_lookback(shape->io_dtype, pl.NP, pl.LPC, p, s);
   } else {
     if (pl.n_segs > 1) {

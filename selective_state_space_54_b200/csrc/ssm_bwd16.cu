@@ -42,7 +42,11 @@
 
 namespace ssm {
 
-constexpr int kQW = 4;             // warps per CTA
+#ifndef SSM_BWD16_WARPS
+#define SSM_BWD16_WARPS 4
+#endif
+constexpr int kQW = SSM_BWD16_WARPS;  // warps per CTA (1, 2 or 4)
+static_assert(kQW == 1 || kQW == 2 || kQW == 4, "1, 2 or 4 warps per CTA");
 constexpr int kQC = 16 * kQW;      // channels per CTA
 constexpr int kQT = kCkptSteps;    // steps per chunk
 constexpr int kQThreads = 32 * kQW;
@@ -217,11 +221,11 @@ __device__ __forceinline__ float q_prepass(const BwdParams &p, QRaw<T> &raw, QSt
       dD = fmaf(dy, u, dD);
     }
   }
-  // B (and C) widened to fp32 by the first 64 threads
-  if (tid < (FULL ? 64 : 32)) {
-    const int e = (tid & 31) * 4, t = e >> 4, n = e & 15;
-    const T *src = (tid >> 5) ? &raw.C[t][n] : &raw.B[t][n];
-    float *dst = (tid >> 5) ? &st.Cs[t][n] : &st.Bs[t][n];
+  // B (and C) widened to fp32, 4 values per thread
+  for (int v = tid; v < (FULL ? 64 : 32); v += kQThreads) {
+    const int e = (v & 31) * 4, t = e >> 4, n = e & 15;
+    const T *src = (v >> 5) ? &raw.C[t][n] : &raw.B[t][n];
+    float *dst = (v >> 5) ? &st.Cs[t][n] : &st.Bs[t][n];
     *reinterpret_cast<float4 *>(dst) = make_float4(q_f(src[0]), q_f(src[1]), q_f(src[2]), q_f(src[3]));
   }
   (void)Dd;
@@ -229,7 +233,7 @@ __device__ __forceinline__ float q_prepass(const BwdParams &p, QRaw<T> &raw, QSt
 }
 
 template <typename T, bool TOK>
-__global__ void __launch_bounds__(kQThreads, 4) k_bwd16(BwdParams p) {
+__global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   QSmem<T> &sm = *reinterpret_cast<QSmem<T> *>(smem_raw);
   QStage &st = sm.st;
@@ -495,12 +499,14 @@ __global__ void __launch_bounds__(kQThreads, 4) k_bwd16(BwdParams p) {
       }
     }
     __syncthreads();
-    // dB/dC of the chunk: the 4 warps' sums, one partial per 64-channel block
+    // dB/dC of the chunk: the warps' sums, one partial per block of kQC channels
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int t = (tid >> 5) + 4 * r, out = tid & 31;
+    for (int r = 0; r < kQT / kQW; ++r) {
+      const int t = warp + kQW * r, out = lane;
       if (t0 + t < L) {
-        const float v = (sm.red[t][0][out] + sm.red[t][1][out]) + (sm.red[t][2][out] + sm.red[t][3][out]);
+        float v = sm.red[t][0][out];
+        if constexpr (kQW == 2) v += sm.red[t][1][out];
+        if constexpr (kQW == 4) v = (v + sm.red[t][1][out]) + (sm.red[t][2][out] + sm.red[t][3][out]);
         p.dBC_part[((cb * p.batch + b) * L + t0 + t) * 32 + out] = v;
       }
     }

@@ -191,6 +191,17 @@ template <> struct IO<uint16_t> {
         }
     }
   }
+  // 4 consecutive values row[t..t+4), those at or past L dropped
+  __device__ __forceinline__ static void store4(uint16_t *row, int64_t t, int64_t L, bool vec,
+                                                const float (&v)[4]) {
+    if (vec && t + 4 <= L) {
+      *reinterpret_cast<uint2 *>(row + t) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (t + i < L) store1(row, t + i, v[i]);
+    }
+  }
   __device__ __forceinline__ static void store1(uint16_t *p, int64_t i, float v) {
     __nv_bfloat16 b = __float2bfloat16_rn(v);
     p[i] = *reinterpret_cast<uint16_t *>(&b);
@@ -219,6 +230,16 @@ template <> struct IO<float> {
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
+        if (t + i < L) row[t + i] = v[i];
+    }
+  }
+  __device__ __forceinline__ static void store4(float *row, int64_t t, int64_t L, bool vec,
+                                                const float (&v)[4]) {
+    if (vec && t + 4 <= L) {
+      *reinterpret_cast<float4 *>(row + t) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
         if (t + i < L) row[t + i] = v[i];
     }
   }
@@ -361,8 +382,8 @@ cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &
 cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 int fwd_ws_chunk();
 int fwd_ws_pairs();
-cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm);
-cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s);
+cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm);
+cudaError_t launch_fwd_ws(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 cudaError_t launch_widen_bc(int io_dtype, const void *B, const void *C, float *Bf, float *Cf, int64_t rows,
                             int N, int NP, cudaStream_t s);
 size_t bwd_ckpt_floats(int64_t batch, int64_t dim, int64_t L, int NP);

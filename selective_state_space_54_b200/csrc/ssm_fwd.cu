@@ -609,10 +609,13 @@ __global__ void k_wait_probe(unsigned *flag, unsigned *err, unsigned long long l
   warp_wait_flag(flag, err, limit_ns);
 }
 
-// ---- warp-specialised look-back forward (2 lanes per channel) -------------------
+// ---- warp-specialised look-back forward ------------------------------------------
 // A CTA holds kPairs producer warps (0..kPairs-1) and kPairs consumer warps
 // (kPairs..2*kPairs-1).  Producer i and consumer i form a pair that walks one
-// look-back share (same items as k_fwd_lookback, 16-step chunks).  The
+// look-back share (same items as k_fwd_lookback, 16-step chunks) of channel
+// groups of 32/LPC channels: LPC = 2 lanes per channel (16 channels, NP/2
+// states per consumer lane) where the problem has enough such groups, else
+// LPC = 4 (8 channels, NP/4 states per lane), which doubles the groups.  The
 // consumer runs only the recurrence: per element one MUFU ex2 and two packed
 // fp32 pair operations, so the special-function unit is kept busy.  The
 // producer does everything else for the same chunks: the input copies
@@ -627,18 +630,26 @@ static_assert(kTW == 2 * kCkptSteps, "the saved states are written at the start 
 constexpr int kPairs = 4;
 constexpr int kWSThreads = 2 * kPairs * 32;
 
-template <int NP>
+template <int NP, int LPC>
 struct __align__(16) WSStage {
-  float dl[16][kTW + 4];
-  float dlu[16][kTW + 4];
-  float ys[2][16][kTW + 4];  // C.h partial sums of a channel's two lanes
+  static constexpr int CPW = 32 / LPC;
+  // lane-j stride of the partial sums; with 4 lanes per channel it is padded
+  // so that a channel's 4 lanes store into different banks
+  static constexpr int YS = CPW * (kTW + 4) + (LPC == 4 ? 8 : 0);
+  float dl[CPW][kTW + 4];
+  float dlu[CPW][kTW + 4];
+  float ys[LPC * YS];  // C.h partial sums of a channel's LPC lanes: [lane j][channel][step]
+  __device__ __forceinline__ float *ys_at(int j, int c, int t) { return ys + j * YS + c * (kTW + 4) + t; }
+  __device__ __forceinline__ const float *ys_at(int j, int c, int t) const {
+    return ys + j * YS + c * (kTW + 4) + t;
+  }
 };
 constexpr int kSlots = 4;    // raw-input ring: chunks k+1..k+3 in flight while k is processed
 constexpr int kBCSlots = 5;  // B/C ring: a chunk's B and C stay until the consumer is done with it
 
-template <typename T>
+template <typename T, int LPC>
 struct __align__(16) WSRaw {
-  T u[16][kTW], d[16][kTW], z[16][kTW];  // [channel][step], io dtype
+  T u[32 / LPC][kTW], d[32 / LPC][kTW], z[32 / LPC][kTW];  // [channel][step], io dtype
 };
 
 // B and C of one chunk in fp32 ([step][state], zero padded), copied straight
@@ -649,10 +660,10 @@ struct __align__(16) WSBC {
   float B[kTW][NP], C[kTW][NP];
 };
 
-template <typename T, int NP>
+template <typename T, int NP, int LPC>
 struct __align__(16) WSPair {
-  WSStage<NP> st[2];
-  WSRaw<T> raw[kSlots];
+  WSStage<NP, LPC> st[2];
+  WSRaw<T, LPC> raw[kSlots];
   WSBC<NP> bc[kBCSlots];
 };
 
@@ -660,6 +671,18 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src
   const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem), "r"(src_bytes)
                : "memory");
+}
+// 8-byte copies go through L1 (.ca): the L2-only form takes 16-byte copies only
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem, int src_bytes) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(sa), "l"(gmem), "r"(src_bytes)
+               : "memory");
+}
+template <int PB>
+__device__ __forceinline__ void cp_async_piece(void *smem, const void *gmem, int src_bytes) {
+  static_assert(PB == 8 || PB == 16, "8- or 16-byte pieces");
+  if constexpr (PB == 16) cp_async16(smem, gmem, src_bytes);
+  else cp_async8(smem, gmem, src_bytes);
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -701,16 +724,17 @@ struct Share {
   }
 };
 
-template <typename T, int NP, bool ZOH, bool SAVE>
-__device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &sm, int64_t w,
+template <typename T, int NP, int LPC, bool ZOH, bool SAVE>
+__device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP, LPC> &sm, int64_t w,
                                             const Share &sh, unsigned bar_full, unsigned bar_ys) {
-  constexpr int S = NP / 2, CPW = 16;
+  constexpr int S = NP / LPC, CPW = 32 / LPC;
+  static_assert(S >= 2 && S % 2 == 0, "a consumer lane holds its states as fp32 pairs");
   int64_t it = 0;
   int bc_slot = 0;  // B/C ring slot of the chunk being processed
   for (int64_t r = 0; r < sh.n_runs; ++r) {
     int64_t g, k0, k1;
     sh.get(r, g, k0, k1);
-    const Lane ln = lane_of<2>(p, g);
+    const Lane ln = lane_of<LPC>(p, g);
     const int c = ln.c, j = ln.j;
     f2 A2p[S / 2];
 #pragma unroll
@@ -726,7 +750,7 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
 #pragma unroll
       for (int s = 0; s < S; ++s) h[s] = __ldcg(&p.carry[((w - 1) * CPW + c) * NP + j * S + s]);
     } else {
-      init_state<NP, 2>(p, ln, h);
+      init_state<NP, LPC>(p, ln, h);
     }
     f2 hp[S / 2];
 #pragma unroll
@@ -749,7 +773,7 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
     };
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = (int)(it & 1);
-      WSStage<NP> &st = sm.st[stage];
+      WSStage<NP, LPC> &st = sm.st[stage];
       const WSBC<NP> &bcs = sm.bc[bc_slot];
       bc_slot = bc_slot + 1 == kBCSlots ? 0 : bc_slot + 1;
       if (SAVE && ck) save_state(2 * k);  // the state entering step kTW * k
@@ -795,8 +819,8 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
           unpack2(acc, a0, a1);
           yp[i] = a0 + a1;
         }
-        // this lane's half of the channel's C.h; the producer adds the halves
-        *reinterpret_cast<float4 *>(&st.ys[j][c][tt]) = make_float4(yp[0], yp[1], yp[2], yp[3]);
+        // this lane's part of the channel's C.h; the producer adds the LPC parts
+        *reinterpret_cast<float4 *>(st.ys_at(j, c, tt)) = make_float4(yp[0], yp[1], yp[2], yp[3]);
       }
       bar_arrive_n(bar_ys + stage, 64);
     }
@@ -809,19 +833,19 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP> &s
       __syncwarp();
       if (ln.lane == 0) st_release(&p.flags[w], 1u);
     } else {
-      write_last_state<NP, 2>(p, ln, h);
+      write_last_state<NP, LPC>(p, ln, h);
     }
   }
 }
-
 // Row pointers and per-channel constants of one run, computed once per run.
-// Producer lanes take channel c = lane % 16 and steps [8j, 8j+8) of every
-// chunk with j = lane / 16, so that a quarter warp's 16-byte row accesses fall
-// in distinct shared-memory banks.  The u/delta/z/y pointers already point at
-// step 8j of the channel's row; the fp32 B/C at this lane's first 16-byte piece.
-template <typename T, int NP>
+// Producer lanes take channel c = lane % CPW and steps [VPL j, VPL j + VPL)
+// of every chunk with j = lane / CPW (VPL = kTW / LPC), so that a quarter
+// warp's row accesses fall in distinct shared-memory banks.  The
+// u/delta/z/y pointers already point at step VPL j of the channel's row; the
+// fp32 B/C at this lane's first 16-byte piece.
+template <typename T, int NP, int LPC>
 struct RunRows {
-  static constexpr int EPP = 16 / (int)sizeof(T);  // elements per 16-byte piece
+  static constexpr int CPW = 32 / LPC, VPL = kTW / LPC;
   const T *u, *dr, *z;
   const float *Bl, *Cl;  // this lane's first 16-byte piece of the fp32 B/C rows of the batch element
   T *y;
@@ -830,14 +854,14 @@ struct RunRows {
   int64_t tok_c0;  // token-major: the group's first channel
   template <bool TOK>
   __device__ __forceinline__ void set(const FwdParams &p, int64_t g, int lane) {
-    const int c = lane & 15, j = lane >> 4;
+    const int c = lane % CPW, j = lane / CPW;
     const int64_t b = g / p.gpb;
-    const int64_t d = (g - b * p.gpb) * 16 + c;
+    const int64_t d = (g - b * p.gpb) * CPW + c;
     valid = d < p.dim;
-    // channel-major: this lane's row at step 8j; token-major: the group's
+    // channel-major: this lane's row at step VPL j; token-major: the group's
     // first channel at step 0 (time stride dim)
-    const int64_t row = TOK ? b * p.L * p.dim + (g - b * p.gpb) * 16
-                            : (b * p.dim + (valid ? d : 0)) * p.L + j * 8;
+    const int64_t row = TOK ? b * p.L * p.dim + (g - b * p.gpb) * CPW
+                            : (b * p.dim + (valid ? d : 0)) * p.L + j * VPL;
     u = static_cast<const T *>(p.u) + row;
     dr = static_cast<const T *>(p.delta) + row;
     z = p.z ? static_cast<const T *>(p.z) + row : nullptr;
@@ -846,22 +870,26 @@ struct RunRows {
     Cl = p.Cf + b * p.L * NP + lane * 4;
     bias = (p.bias && valid) ? p.bias[d] : 0.f;
     Dd = (p.D && valid) ? p.D[d] : 0.f;
-    tok_c0 = (g - b * p.gpb) * 16;
+    tok_c0 = (g - b * p.gpb) * CPW;
   }
 };
 
 // Copy this lane's pieces of chunk k of run `rr` into raw slot `slot`:
-// u/delta/z steps [8j, 8j+8) of channel c, and the B/C 16-byte pieces lane,
-// lane+32, ...  Whole chunks of valid channels with 16-byte aligned rows take
-// the short path; the last chunk of a ragged L, padded channels and
-// unaligned rows take the checked one (zero fill past L).  Every lane later
-// reads only the pieces it copied itself.
-template <typename T, int NP, bool TOK>
-__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T> &raw, WSBC<NP> &bc,
-                                         const RunRows<T, NP> &rr, int64_t k, int lane) {
-  constexpr int ES = (int)sizeof(T), EPP = 16 / ES;
-  constexpr int NVF = kTW * NP / 4;  // fp32 B/C pieces per chunk and tensor
-  const int c = lane & 15, j8 = (lane >> 4) * 8;
+// u/delta/z steps [VPL j, VPL j + VPL) of channel c, and the B/C 16-byte
+// pieces lane, lane+32, ...  Whole chunks of valid channels with 16-byte
+// aligned rows take the short path; the last chunk of a ragged L, padded
+// channels and unaligned rows take the checked one (zero fill past L).
+// Every lane later reads only the u/delta/z pieces it copied itself.
+template <typename T, int NP, int LPC, bool TOK>
+__device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T, LPC> &raw, WSBC<NP> &bc,
+                                         const RunRows<T, NP, LPC> &rr, int64_t k, int lane) {
+  constexpr int ES = (int)sizeof(T), CPW = 32 / LPC, VPL = kTW / LPC;
+  constexpr int PB = VPL * ES >= 16 ? 16 : VPL * ES;  // bytes per copied piece (8 or 16)
+  constexpr int EPC = PB / ES;                        // elements per piece
+  constexpr int NPC = VPL / EPC;                      // pieces per lane and tensor
+  constexpr int NVF = kTW * NP / 4;                   // fp32 B/C pieces per chunk and tensor
+  static_assert(!TOK || LPC == 2, "token-major tiles are laid out for 16-channel groups");
+  const int c = lane % CPW, jv = (lane / CPW) * VPL;
   const int64_t L = p.L, t0 = k * kTW;
   const bool whole = t0 + kTW <= L;
   bool tok_done = false;
@@ -885,29 +913,29 @@ __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T> &raw, WSBC
   if (tok_done) {
   } else if (whole && rr.valid && p.io_vec) {
 #pragma unroll
-    for (int q = 0; q < 8 / EPP; ++q) {
-      cp_async16(&raw.u[c][j8 + q * EPP], rr.u + t0 + q * EPP, 16);
-      cp_async16(&raw.d[c][j8 + q * EPP], rr.dr + t0 + q * EPP, 16);
-      if (rr.z) cp_async16(&raw.z[c][j8 + q * EPP], rr.z + t0 + q * EPP, 16);
+    for (int q = 0; q < NPC; ++q) {
+      cp_async_piece<PB>(&raw.u[c][jv + q * EPC], rr.u + t0 + q * EPC, PB);
+      cp_async_piece<PB>(&raw.d[c][jv + q * EPC], rr.dr + t0 + q * EPC, PB);
+      if (rr.z) cp_async_piece<PB>(&raw.z[c][jv + q * EPC], rr.z + t0 + q * EPC, PB);
     }
   } else if (p.io_vec) {
 #pragma unroll
-    for (int q = 0; q < 8 / EPP; ++q) {
-      const int64_t t = t0 + j8 + q * EPP;
+    for (int q = 0; q < NPC; ++q) {
+      const int64_t t = t0 + jv + q * EPC;
       const int64_t left = rr.valid ? L - t : 0;
-      const int bytes = left >= EPP ? 16 : (left > 0 ? (int)left * ES : 0);
-      const int64_t off = bytes > 0 ? t0 + q * EPP : -j8;  // row start when nothing is read
-      cp_async16(&raw.u[c][j8 + q * EPP], rr.u + off, bytes);
-      cp_async16(&raw.d[c][j8 + q * EPP], rr.dr + off, bytes);
-      if (rr.z) cp_async16(&raw.z[c][j8 + q * EPP], rr.z + off, bytes);
+      const int bytes = left >= EPC ? PB : (left > 0 ? (int)left * ES : 0);
+      const int64_t off = bytes > 0 ? t0 + q * EPC : -jv;  // row start when nothing is read
+      cp_async_piece<PB>(&raw.u[c][jv + q * EPC], rr.u + off, bytes);
+      cp_async_piece<PB>(&raw.d[c][jv + q * EPC], rr.dr + off, bytes);
+      if (rr.z) cp_async_piece<PB>(&raw.z[c][jv + q * EPC], rr.z + off, bytes);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool in = rr.valid && t0 + j8 + i < L;
-      raw.u[c][j8 + i] = in ? rr.u[t0 + i] : T(0);
-      raw.d[c][j8 + i] = in ? rr.dr[t0 + i] : T(0);
-      if (rr.z) raw.z[c][j8 + i] = in ? rr.z[t0 + i] : T(0);
+    for (int i = 0; i < VPL; ++i) {
+      const bool in = rr.valid && t0 + jv + i < L;
+      raw.u[c][jv + i] = in ? rr.u[t0 + i] : T(0);
+      raw.d[c][jv + i] = in ? rr.dr[t0 + i] : T(0);
+      if (rr.z) raw.z[c][jv + i] = in ? rr.z[t0 + i] : T(0);
     }
   }
   // fp32 B/C pieces lane, lane + 32, ... of the chunk (a piece is 4 states of one step)
@@ -928,12 +956,41 @@ __device__ __forceinline__ void ws_fetch(const FwdParams &p, WSRaw<T> &raw, WSBC
 __device__ __forceinline__ float io_to_f(uint16_t v) { return bf16_to_f(v); }
 __device__ __forceinline__ float io_to_f(float v) { return v; }
 
-template <typename T, int NP, bool TOK>
-__device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &sm, const Share &sh,
+// V consecutive io values from shared memory, widened (V = 4 or 8; the
+// address is 2V- or 4V-byte aligned)
+template <int V>
+__device__ __forceinline__ void load_row(const uint16_t *p, float (&o)[V]) {
+  if constexpr (V == 8) {
+    Vec8<uint16_t> v;
+    v.load_shared(p);
+    v.unpack(o);
+  } else {
+    static_assert(V == 4, "4 or 8 values");
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    o[0] = bf16_lo(v.x); o[1] = bf16_hi(v.x); o[2] = bf16_lo(v.y); o[3] = bf16_hi(v.y);
+  }
+}
+template <int V>
+__device__ __forceinline__ void load_row(const float *p, float (&o)[V]) {
+  if constexpr (V == 8) {
+    Vec8<float> v;
+    v.load_shared(p);
+    v.unpack(o);
+  } else {
+    static_assert(V == 4, "4 or 8 values");
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  }
+}
+
+template <typename T, int NP, int LPC, bool TOK>
+__device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP, LPC> &sm, const Share &sh,
                                             unsigned bar_full, unsigned bar_ys) {
+  constexpr int CPW = 32 / LPC, VPL = kTW / LPC, HP = VPL / 2;
+  static_assert(VPL == 4 || VPL == 8, "4 or 8 steps per producer lane");
   const int64_t L = p.L;
   const int lane = threadIdx.x & 31;
-  const int c = lane & 15, j8 = (lane >> 4) * 8;
+  const int c = lane % CPW, jv = (lane / CPW) * VPL;
   const bool io_vec = p.io_vec != 0;
   const bool has_z = p.z != nullptr;
   constexpr bool tok = TOK;  // u/delta/z/y laid out [batch][seqlen][dim]
@@ -942,11 +999,11 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   int pstage = 0;
   T *py = nullptr;
   int64_t pt = 0;
-  f2 gate2[4], du2[4];
+  f2 gate2[HP], du2[HP];
 
   // prefetch cursor: the item kSlots-1 chunks ahead of the one processed
   int64_t pr = 0, pk = 0, pk1 = 0, pg = 0;
-  RunRows<T, NP> pf;
+  RunRows<T, NP, LPC> pf;
   bool pf_live = sh.n_runs > 0;
   if (pf_live) {
     sh.get(0, pg, pk, pk1);
@@ -966,7 +1023,7 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   int bc_f = 0;     // B/C ring slot of the next chunk fetched
   auto fetch_next = [&]() {
     if (pf_live) {
-      ws_fetch<T, NP, TOK>(p, sm.raw[it_f % kSlots], sm.bc[bc_f], pf, pk, lane);
+      ws_fetch<T, NP, LPC, TOK>(p, sm.raw[it_f % kSlots], sm.bc[bc_f], pf, pk, lane);
       advance();
     }
     cp_async_commit();
@@ -975,109 +1032,118 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
   };
   for (int i = 0; i < kSlots - 1; ++i) fetch_next();
 
+  // y = (C.h + D*u) * SiLU(z) of the pending chunk, once its sums are ready
+  auto epilogue = [&]() {
+    bar_sync_n(bar_ys + pstage, 64);
+    if (!pvalid) return;
+    const WSStage<NP, LPC> &ps = sm.st[pstage];
+    f2 ya[HP];
+#pragma unroll
+    for (int q = 0; q < VPL / 4; ++q) {
+      const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(ps.ys_at(0, c, jv + 4 * q));
+      ya[2 * q] = v.x;
+      ya[2 * q + 1] = v.y;
+    }
+#pragma unroll
+    for (int jj = 1; jj < LPC; ++jj)
+#pragma unroll
+      for (int q = 0; q < VPL / 4; ++q) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(ps.ys_at(jj, c, jv + 4 * q));
+        ya[2 * q] = add2(ya[2 * q], v.x);
+        ya[2 * q + 1] = add2(ya[2 * q + 1], v.y);
+      }
+    float o[VPL];
+#pragma unroll
+    for (int i = 0; i < HP; ++i) unpack2(mul2(add2(ya[i], du2[i]), gate2[i]), o[2 * i], o[2 * i + 1]);
+    if constexpr (tok) {  // time stride dim; a warp's 16 channels of a step are contiguous
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (pt + jv + i < L) IO<T>::store1(py, (pt + jv + i) * p.dim + c, o[i]);
+    } else if constexpr (VPL == 8) {
+      IO<T>::store8(py, pt, L - jv, io_vec, o);
+    } else {
+      IO<T>::store4(py, pt, L - jv, io_vec, o);
+    }
+  };
+
   int it = 0;
   for (int64_t r = 0; r < sh.n_runs; ++r) {
     int64_t g, k0, k1;
     sh.get(r, g, k0, k1);
-    RunRows<T, NP> cur;
+    RunRows<T, NP, LPC> cur;
     cur.template set<TOK>(p, g, lane);
     for (int64_t k = k0; k < k1; ++k, ++it) {
       const int stage = it & 1;
-      WSStage<NP> &st = sm.st[stage];
-      WSRaw<T> &raw = sm.raw[it % kSlots];
+      WSStage<NP, LPC> &st = sm.st[stage];
+      WSRaw<T, LPC> &raw = sm.raw[it % kSlots];
       const int64_t t0 = k * kTW;
       const bool whole = cur.valid && t0 + kTW <= L;
       cp_async_wait<kSlots - 2>();  // this chunk's copies have landed
       if constexpr (tok) __syncwarp();  // token-major tiles hold other lanes' copies
       // ---- pre-pass of chunk k into the stage: Delta, Delta*u ----
-      float u8[8], s8[8];
-      if constexpr (tok) {  // [step][channel] tile: this lane's channel c at steps j8..j8+7
+      float u8[VPL], s8[VPL];
+      if constexpr (tok) {  // [step][channel] tile: this lane's channel c at steps jv..jv+VPL-1
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          u8[i] = io_to_f((&raw.u[0][0])[(j8 + i) * 16 + c]);
-          s8[i] = io_to_f((&raw.d[0][0])[(j8 + i) * 16 + c]);
+        for (int i = 0; i < VPL; ++i) {
+          u8[i] = io_to_f((&raw.u[0][0])[(jv + i) * 16 + c]);
+          s8[i] = io_to_f((&raw.d[0][0])[(jv + i) * 16 + c]);
         }
       } else {
-        Vec8<T> vu, vd;
-        vu.load_shared(&raw.u[c][j8]);
-        vd.load_shared(&raw.d[c][j8]);
-        vu.unpack(u8);
-        vd.unpack(s8);
+        load_row<VPL>(&raw.u[c][jv], u8);
+        load_row<VPL>(&raw.d[c][jv], s8);
       }
-      f2 dl2[4], dlu2[4];
+      f2 dl2[HP], dlu2[HP];
       const f2 bias2 = pack2(cur.bias, cur.bias);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < HP; ++i) {
         const f2 s = add2(pack2(s8[2 * i], s8[2 * i + 1]), bias2);
         dl2[i] = p.softplus ? softplus2(s) : s;
       }
       if (!whole) {  // zero Delta past L and on padded channels: the state holds
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < HP; ++i) {
           float a, b;
           unpack2(dl2[i], a, b);
-          a = (cur.valid && t0 + j8 + 2 * i < L) ? a : 0.f;
-          b = (cur.valid && t0 + j8 + 2 * i + 1 < L) ? b : 0.f;
+          a = (cur.valid && t0 + jv + 2 * i < L) ? a : 0.f;
+          b = (cur.valid && t0 + jv + 2 * i + 1 < L) ? b : 0.f;
           dl2[i] = pack2(a, b);
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) dlu2[i] = mul2(dl2[i], pack2(u8[2 * i], u8[2 * i + 1]));
+      for (int i = 0; i < HP; ++i) dlu2[i] = mul2(dl2[i], pack2(u8[2 * i], u8[2 * i + 1]));
       {
-        float *pd = &st.dl[c][j8];
-        float *pu = &st.dlu[c][j8];
-        *reinterpret_cast<ulonglong2 *>(pd) = make_ulonglong2(dl2[0], dl2[1]);
-        *reinterpret_cast<ulonglong2 *>(pd + 4) = make_ulonglong2(dl2[2], dl2[3]);
-        *reinterpret_cast<ulonglong2 *>(pu) = make_ulonglong2(dlu2[0], dlu2[1]);
-        *reinterpret_cast<ulonglong2 *>(pu + 4) = make_ulonglong2(dlu2[2], dlu2[3]);
+        float *pd = &st.dl[c][jv];
+        float *pu = &st.dlu[c][jv];
+#pragma unroll
+        for (int i = 0; i < HP; i += 2) {
+          *reinterpret_cast<ulonglong2 *>(pd + 2 * i) = make_ulonglong2(dl2[i], dl2[i + 1]);
+          *reinterpret_cast<ulonglong2 *>(pu + 2 * i) = make_ulonglong2(dlu2[i], dlu2[i + 1]);
+        }
       }
       bar_arrive_n(bar_full + stage, 64);
       // ---- copies of the chunk kSlots-1 ahead: raw slot of chunk k-1; B/C slot
       // of chunk k-2, which the consumer released before this stage was filled ----
       fetch_next();
-      // ---- epilogue of chunk k-1: y = (C.h + D*u) * SiLU(z) ----
-      if (pend) {
-        bar_sync_n(bar_ys + pstage, 64);
-        if (pvalid) {
-          const WSStage<NP> &ps = sm.st[pstage];
-          const ulonglong2 a0 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[0][c][j8]);
-          const ulonglong2 a1 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[0][c][j8 + 4]);
-          const ulonglong2 b0 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[1][c][j8]);
-          const ulonglong2 b1 = *reinterpret_cast<const ulonglong2 *>(&ps.ys[1][c][j8 + 4]);
-          const f2 ya[4] = {a0.x, a0.y, a1.x, a1.y}, yb[4] = {b0.x, b0.y, b1.x, b1.y};
-          float o[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            unpack2(mul2(add2(add2(ya[i], yb[i]), du2[i]), gate2[i]), o[2 * i], o[2 * i + 1]);
-          if constexpr (tok) {  // time stride dim; a warp's 16 channels of a step are contiguous
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              if (pt + j8 + i < L) IO<T>::store1(py, (pt + j8 + i) * p.dim + c, o[i]);
-          } else {
-            IO<T>::store8(py, pt, L - j8, io_vec, o);
-          }
-        }
-      }
+      // ---- epilogue of chunk k-1 ----
+      if (pend) epilogue();
       // ---- gate and D*u of chunk k, for its epilogue in the next iteration ----
       {
         const f2 D2 = pack2(cur.Dd, cur.Dd);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) du2[i] = mul2(D2, pack2(u8[2 * i], u8[2 * i + 1]));
+        for (int i = 0; i < HP; ++i) du2[i] = mul2(D2, pack2(u8[2 * i], u8[2 * i + 1]));
         if (has_z) {
-          float z8[8];
+          float z8[VPL];
           if constexpr (tok) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) z8[i] = io_to_f((&raw.z[0][0])[(j8 + i) * 16 + c]);
+            for (int i = 0; i < VPL; ++i) z8[i] = io_to_f((&raw.z[0][0])[(jv + i) * 16 + c]);
           } else {
-            Vec8<T> vz;
-            vz.load_shared(&raw.z[c][j8]);
-            vz.unpack(z8);
+            load_row<VPL>(&raw.z[c][jv], z8);
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) gate2[i] = silu2(pack2(z8[2 * i], z8[2 * i + 1]));
+          for (int i = 0; i < HP; ++i) gate2[i] = silu2(pack2(z8[2 * i], z8[2 * i + 1]));
         } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) gate2[i] = pack2(1.f, 1.f);
+          for (int i = 0; i < HP; ++i) gate2[i] = pack2(1.f, 1.f);
         }
       }
       pend = true;
@@ -1087,49 +1153,26 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP> &s
       pvalid = cur.valid;
     }
   }
-  if (pend) {
-    bar_sync_n(bar_ys + pstage, 64);
-    if (pvalid) {
-      const WSStage<NP> &ps = sm.st[pstage];
-      float o[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = ps.ys[0][c][j8 + i] + ps.ys[1][c][j8 + i];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float d0, d1, g0, g1;
-        unpack2(du2[i], d0, d1);
-        unpack2(gate2[i], g0, g1);
-        o[2 * i] = (o[2 * i] + d0) * g0;
-        o[2 * i + 1] = (o[2 * i + 1] + d1) * g1;
-      }
-      if constexpr (tok) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (pt + j8 + i < L) IO<T>::store1(py, (pt + j8 + i) * p.dim + c, o[i]);
-      } else {
-        IO<T>::store8(py, pt, L - j8, io_vec, o);
-      }
-    }
-  }
+  if (pend) epilogue();
   cp_async_wait<0>();
 }
 
 // TOK: token-major activations; ZOH: the exact input term; SAVE: the chunk
 // states for the backward are written (separate instantiations, so that the
 // plain forward carries none of that code)
-template <typename T, int NP, bool TOK, bool ZOH, bool SAVE>
+template <typename T, int NP, int LPC, bool TOK, bool ZOH, bool SAVE>
 __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
   const bool producer = warp < kPairs;
   const int pair = producer ? warp : warp - kPairs;
-  WSPair<T, NP> &sm = reinterpret_cast<WSPair<T, NP> *>(smem_raw)[pair];
+  WSPair<T, NP, LPC> &sm = reinterpret_cast<WSPair<T, NP, LPC> *>(smem_raw)[pair];
   const int64_t w = (int64_t)blockIdx.x * kPairs + pair;
   if (w >= p.n_workers) return;  // both warps of a pair leave together
   const Share sh(w, p.n_workers, p.n_groups, p.n_chunks);
   const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
-  if (producer) ws_producer<T, NP, TOK>(p, sm, sh, bar_full, bar_ys);
-  else ws_consumer<T, NP, ZOH, SAVE>(p, sm, w, sh, bar_full, bar_ys);
+  if (producer) ws_producer<T, NP, LPC, TOK>(p, sm, sh, bar_full, bar_ys);
+  else ws_consumer<T, NP, LPC, ZOH, SAVE>(p, sm, w, sh, bar_full, bar_ys);
 }
 
 // B and C as fp32 [batch][L][NP], zero padded past N: the warp-specialised
@@ -1251,42 +1294,58 @@ cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p,
 int fwd_ws_chunk() { return kTW; }
 int fwd_ws_pairs() { return kPairs; }
 
-cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int *ctas_per_sm) {
-  return dispatch(io_dtype, NP, 2, [&](auto tt, auto np, auto) -> cudaError_t {
+// The warp-specialised kernel with 4 lanes per channel is built for 8 and 16
+// states (2 or 4 per lane), channel-major activations and no saved states.
+template <int NP, int LPC, bool TOK, bool SAVE>
+constexpr bool ws_built() {
+  return LPC == 2 || (LPC == 4 && (NP == 8 || NP == 16) && !TOK && !SAVE);
+}
+
+cudaError_t fwd_ws_occupancy(int io_dtype, int NP, int LPC, int *ctas_per_sm) {
+  return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
-    constexpr int kNP = decltype(np)::value;
-    const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
-    cudaError_t e = allow_smem(k_fwd_ws<T, kNP, false, false, false>, smem);
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k_fwd_ws<T, kNP, false, false, false>, kWSThreads,
-                                                         smem);
+    constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
+    if constexpr (!ws_built<kNP, kLPC, false, false>()) {
+      return cudaErrorInvalidValue;
+    } else {
+      const size_t smem = kPairs * sizeof(WSPair<T, kNP, kLPC>);
+      auto kern = k_fwd_ws<T, kNP, kLPC, false, false, false>;
+      cudaError_t e = allow_smem(kern, smem);
+      if (e != cudaSuccess) return e;
+      return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, kern, kWSThreads, smem);
+    }
   });
 }
 
-cudaError_t launch_fwd_ws(int io_dtype, int NP, const FwdParams &p, cudaStream_t s) {
-  return dispatch(io_dtype, NP, 2, [&](auto tt, auto np, auto) -> cudaError_t {
+cudaError_t launch_fwd_ws(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s) {
+  return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
-    constexpr int kNP = decltype(np)::value;
-    const size_t smem = kPairs * sizeof(WSPair<T, kNP>);
+    constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
+    const size_t smem = kPairs * sizeof(WSPair<T, kNP, kLPC>);
     const unsigned grid = (unsigned)((p.n_workers + kPairs - 1) / kPairs);
     const bool save = p.ckpt_out != nullptr;
+    auto go = [&](auto kern) -> cudaError_t {
+      cudaError_t e = allow_smem(kern, smem);
+      if (e != cudaSuccess) return e;
+      kern<<<grid, kWSThreads, smem, s>>>(p);
+      return cudaGetLastError();
+    };
     if (p.tok) {  // token-major tiles: bf16, Euler only (the API checks)
-      if constexpr (sizeof(T) == 2) {
-        auto kern = save ? k_fwd_ws<T, kNP, true, false, true> : k_fwd_ws<T, kNP, true, false, false>;
-        cudaError_t e = allow_smem(kern, smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kWSThreads, smem, s>>>(p);
-        return cudaGetLastError();
+      if constexpr (sizeof(T) == 2 && ws_built<kNP, kLPC, true, false>()) {
+        return save ? go(k_fwd_ws<T, kNP, kLPC, true, false, true>) : go(k_fwd_ws<T, kNP, kLPC, true, false, false>);
       } else {
         return cudaErrorInvalidValue;
       }
     }
-    auto kern = p.zoh ? (save ? k_fwd_ws<T, kNP, false, true, true> : k_fwd_ws<T, kNP, false, true, false>)
-                      : (save ? k_fwd_ws<T, kNP, false, false, true> : k_fwd_ws<T, kNP, false, false, false>);
-    cudaError_t e = allow_smem(kern, smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, kWSThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    if constexpr (ws_built<kNP, kLPC, false, true>()) {
+      if (save)
+        return p.zoh ? go(k_fwd_ws<T, kNP, kLPC, false, true, true>) : go(k_fwd_ws<T, kNP, kLPC, false, false, true>);
+    }
+    if constexpr (ws_built<kNP, kLPC, false, false>()) {
+      if (!save)
+        return p.zoh ? go(k_fwd_ws<T, kNP, kLPC, false, true, false>) : go(k_fwd_ws<T, kNP, kLPC, false, false, false>);
+    }
+    return cudaErrorInvalidValue;
   });
 }
 

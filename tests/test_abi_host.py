@@ -253,6 +253,20 @@ def test_flags_checked_before_launch(lib):
     assert _bwd(lib, _shape(flags=_lib.SSM_FLAG_ZOH_EXACT)) == _lib.SSM_ERR_WORKSPACE
 
 
+def test_warp_specialised_lanes_checked_before_launch(lib):
+    # 4 lanes per channel in the warp-specialised kernel: 5..16 states,
+    # channel-major, no saved states
+    ws = _lib.SSM_PATH_LOOKBACK_WS
+    for N in (1, 4, 17, 32, 64):
+        assert _fwd(lib, _shape(path=ws, lanes=4, dstate=N)) == _lib.SSM_ERR_UNSUPPORTED, N
+        assert lib.ssm_scan_fwd_workspace_bytes(ctypes.byref(_shape(path=ws, lanes=4, dstate=N))) == 0
+    for N in (5, 8, 12, 16):
+        assert _fwd(lib, _shape(path=ws, lanes=4, dstate=N)) in ACCEPTED, N
+        assert _fwd(lib, _shape(path=ws, lanes=4, dstate=N, flags=_lib.SSM_FLAG_ZOH_EXACT)) in ACCEPTED, N
+    assert _fwd(lib, _shape(path=ws, lanes=4, flags=_lib.SSM_FLAG_TOKEN_MAJOR)) == _lib.SSM_ERR_UNSUPPORTED
+    assert _fwd(lib, _shape(path=ws, lanes=4, flags=_lib.SSM_FLAG_SAVE_STATES)) == _lib.SSM_ERR_UNSUPPORTED
+
+
 def test_saved_states_flag_checked_before_launch(lib):
     save, zoh = _lib.SSM_FLAG_SAVE_STATES, _lib.SSM_FLAG_ZOH_EXACT
     # written by the warp-specialised kernel only: 2 lanes, AUTO or LOOKBACK_WS

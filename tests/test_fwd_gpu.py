@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 PATHS = {"auto": 0, "lookback": 1, "split_l": 2, "per_group": 3, "lookback_ws": 4}
 # every schedule with every lane split it supports
 PATH_LANES = [("lookback", 2), ("lookback", 4), ("split_l", 2), ("split_l", 4),
-              ("per_group", 2), ("per_group", 4), ("lookback_ws", 2)]
+              ("per_group", 2), ("per_group", 4), ("lookback_ws", 2), ("lookback_ws", 4)]
 
 
 def _run(case, device, path="auto", softplus=True, h0=None, last=True, y_out=None, lanes=0,
@@ -175,11 +175,11 @@ def test_softplus_accuracy_through_the_kernel(cuda_device):
         assert np.all(rel <= bound), (lanes, float(rel.max()), float(s[np.argmax(rel / bound)]))
 
 
-@pytest.mark.parametrize("path", ["lookback", "lookback_ws"])
-def test_deterministic(cuda_device, path):
+@pytest.mark.parametrize("path,lanes", [("lookback", 0), ("lookback_ws", 2), ("lookback_ws", 4)])
+def test_deterministic(cuda_device, path, lanes):
     case = synth.make_case(2, 64, 1024, 16, synth.BF16, seed=41)
-    a = _run(case, cuda_device, path)
-    b = _run(case, cuda_device, path)
+    a = _run(case, cuda_device, path, lanes=lanes)
+    b = _run(case, cuda_device, path, lanes=lanes)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
@@ -189,10 +189,10 @@ def test_lookback_splits_groups_between_warps(cuda_device):
     # end inside groups, so the carried states are exercised on both paths
     case = synth.make_case(8, 1536, 1000, 16, synth.BF16, seed=61)
     ref = oracle.fwd(case)
-    for path in ("lookback", "lookback_ws"):
-        y, ls = _run(case, cuda_device, path)
-        assert_close(y, ref["y"], case["dtype"], path)
-        assert_close(ls, ref["last_state"], case["dtype"], path, stored_bf16=False)
+    for path, lanes in (("lookback", 0), ("lookback_ws", 2), ("lookback_ws", 4)):
+        y, ls = _run(case, cuda_device, path, lanes=lanes)
+        assert_close(y, ref["y"], case["dtype"], f"{path}/{lanes}")
+        assert_close(ls, ref["last_state"], case["dtype"], f"{path}/{lanes}", stored_bf16=False)
 
 
 def test_guard_bands_untouched(cuda_device):
@@ -327,6 +327,30 @@ def test_zoh_exact_warp_specialised(cuda_device, dtype, N):
     y, ls = _run_zoh(case, cuda_device, "lookback_ws", 2, h0=h0)
     assert_close(y, ref["y"], dtype, "y")
     assert_close(ls, ref["last_state"], dtype, "last_state", stored_bf16=False)
+
+
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+@pytest.mark.parametrize("N", [5, 8, 12, 16])
+def test_warp_specialised_four_lanes(cuda_device, dtype, N):
+    # 8-channel groups, 4 lanes per channel (2 or 4 states each): ragged
+    # channel group (dim 44), ragged chunk, initial state; Euler and exact ZOH
+    case = synth.make_case(2, 44, 333, N, dtype, seed=450 + N)
+    h0 = np.random.default_rng(N).standard_normal((2, 44, N)).astype(np.float32)
+    for zoh in (False, True):
+        ref = oracle.fwd(case, zoh_exact=zoh, h0=h0)
+        y, ls = _run(case, cuda_device, "lookback_ws", h0=h0, lanes=4, zoh=zoh)
+        assert_close(y, ref["y"], dtype, f"y zoh={zoh}")
+        assert_close(ls, ref["last_state"], dtype, f"last_state zoh={zoh}", stored_bf16=False)
+
+
+def test_warp_specialised_four_lanes_limits(cuda_device):
+    # 4 lanes per channel in the warp-specialised kernel: 5..16 states only,
+    # and AUTO takes it where 16-channel groups are too few (the Mamba-130M layer)
+    import selective_state_space_54_b200 as ssm
+    for N, ok in ((4, False), (5, True), (16, True), (17, False), (64, False)):
+        shape = ssm.make_shape(2, 64, 256, N, ssm.SSM_BF16, ssm.SSM_PATH_LOOKBACK_WS, 4)
+        assert (ssm.fwd_workspace_bytes(shape) > 0) == ok, N
+    assert ssm.fwd_path(ssm.make_shape(8, 1536, 2048, 16, ssm.SSM_BF16)) == "lookback_ws"
 
 
 def test_zoh_exact_auto_picks_warp_specialised(cuda_device):
