@@ -42,10 +42,12 @@
 
 namespace ssm {
 
-#ifndef SSM_BWD16_WARPS
-#define SSM_BWD16_WARPS 4
-#endif
-constexpr int kQW = SSM_BWD16_WARPS;  // warps per CTA (1, 2 or 4)
+// Warps per CTA (the code takes 1, 2 or 4).  At the Mamba-1.4B training shape
+// (512 CTAs of 4 warps, 3 or 4 per SM) 2-warp CTAs even out the warps per SM
+// but measured only 1.3 % faster on B200 (1.874 against 1.899 ms) while
+// doubling the dB/dC partials, and 1-warp CTAs 1.9 % slower: the kernel is
+// bound by its instruction latency, not by the uneven spread.
+constexpr int kQW = 4;
 static_assert(kQW == 1 || kQW == 2 || kQW == 4, "1, 2 or 4 warps per CTA");
 constexpr int kQC = 16 * kQW;      // channels per CTA
 constexpr int kQT = kCkptSteps;    // steps per chunk

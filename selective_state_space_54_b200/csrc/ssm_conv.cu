@@ -8,9 +8,9 @@
 // with x_t for t < 0 taken from the caller's initial state (zeros if none).
 //
 // Design (B200): 2 bytes in and 2 out per (b, d, t) in bf16, a few FMAs:
-// bound by HBM.  A warp takes 1024 consecutive steps of one (b, d) row in 4
+// bound by HBM.  A warp takes 2048 consecutive steps of one (b, d) row in 8
 // passes; a lane takes 8 steps per pass with one 16-byte load and store,
-// all 4 loads issued before the first pass computes.  The K-1 steps before a
+// all 8 loads issued before the first pass computes.  The K-1 steps before a
 // lane's chunk come from neighbouring lanes by shuffles, so every input byte
 // is read once.  Input and output are streamed with evict-first hints.
 #include "ssm_common.cuh"
@@ -20,8 +20,41 @@ namespace ssm {
 constexpr int kConvThreads = 256;
 
 constexpr int kConvW = 8;                  // steps per lane and pass
-constexpr int kConvR = 4;                  // passes per warp, all loads issued first
-constexpr int kConvSeg = 32 * kConvW * kConvR;  // steps per warp
+// Passes per warp, all loads issued first: 8 in the forward, i.e. 8 16-byte
+// loads in flight per lane, with the bf16 kernel held to 64 registers for 4
+// CTAs (32 warps) per SM.  Measured on B200 at the Mamba-2.8B shape (bf16,
+// width 4): 0.123 ms, against 0.133 ms at 3 CTAs per SM, 0.132 ms with 7
+// passes and 0.140 ms with 4; 9, 10, 12 or 16 passes cost registers (fewer
+// resident CTAs) and leave a ragged last segment (0.148-0.169 ms).  4 in the
+// backward, whose two input streams and register cap leave no room for more
+// (8 passes spill or halve the resident CTAs: 0.280 against 0.261 ms).
+constexpr int kConvR = 8;
+constexpr int kConvSeg = 32 * kConvW * kConvR;  // steps per forward warp
+constexpr int kConvBR = 4;
+constexpr int kConvBSeg = 32 * kConvW * kConvBR;  // steps per backward warp
+
+// (row, segment, channel) of this warp; 32-bit divisions when the grid's
+// warp count fits (the launcher checks), 64-bit otherwise
+struct ConvWarp {
+  int64_t row, seg, d;
+  bool live;
+  __device__ __forceinline__ ConvWarp(int64_t segs, int64_t rows, int64_t dim, bool narrow) {
+    if (narrow) {
+      const unsigned w = (blockIdx.x * (unsigned)kConvThreads + threadIdx.x) >> 5;
+      const unsigned r = w / (unsigned)segs;
+      live = r < (unsigned)rows;
+      row = r;
+      seg = w - r * (unsigned)segs;
+      d = r % (unsigned)dim;
+    } else {
+      const int64_t w = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
+      row = w / segs;
+      live = row < rows;
+      seg = w - row * segs;
+      d = row % dim;
+    }
+  }
+};
 
 // raw io vector of 8 values, kept packed until used
 template <typename T> struct Raw8;
@@ -70,16 +103,15 @@ template <> struct Raw8<float> {
 // kConvR 16-byte loads in flight.  The K-1 steps before a lane's chunk come
 // from the previous lane (shuffle up), or for lane 0 from lane 31 of the
 // previous pass; only the warp's first pass reads them from memory.
-template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads) k_conv(ConvParams p) {
+// NARROW: the grid's thread count fits 32 bits (a separate instantiation:
+// a run-time choice of the index width measured 5 % slower)
+template <typename T, int K, bool NARROW>
+__global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 : 1) k_conv(ConvParams p) {
   const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
   const int64_t L = p.L;
-  const int64_t segs = (L + kConvSeg - 1) / kConvSeg;
-  const int64_t row = warp / segs;
-  if (row >= p.batch * p.dim) return;  // whole warps leave together
-  const int64_t seg = warp - row * segs;
-  const int64_t d = row % p.dim;
+  const ConvWarp cw((L + kConvSeg - 1) / kConvSeg, p.batch * p.dim, p.dim, NARROW);
+  if (!cw.live) return;  // whole warps leave together
+  const int64_t row = cw.row, seg = cw.seg, d = cw.d;
   const T *xr = static_cast<const T *>(p.x) + row * L;
   T *orow = static_cast<T *>(p.out) + row * L;
   const bool vec = p.vec != 0;
@@ -174,7 +206,8 @@ __global__ void __launch_bounds__(kConvThreads) k_conv(ConvParams p) {
 // the forward: a warp recomputes a and da pass by pass, accumulates its dw and
 // dbias partials, and writes dx of the pass before once it has the next pass's
 // first K-1 values of da (a shuffle from lane 0).  The warp's last pass takes
-// them from the next segment, recomputed by lane 31 from memory.
+// them from the next segment, recomputed by lane 31 from memory.  A backward
+// warp takes 4 passes (1024 steps).
 template <typename T, int K>
 __device__ __forceinline__ float conv_act_grad(float a, float g, bool silu) {
   if (!silu) return g;
@@ -185,22 +218,21 @@ __device__ __forceinline__ float conv_act_grad(float a, float g, bool silu) {
 template <typename T, int K>
 __global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 : 1) k_conv_bwd(ConvBwdParams p) {
   const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
   const int64_t L = p.L;
-  const int64_t segs = (L + kConvSeg - 1) / kConvSeg;
-  const int64_t row = warp / segs;
-  if (row >= p.batch * p.dim) return;  // whole warps leave together
-  const int64_t seg = warp - row * segs;
-  const int64_t d = row % p.dim;
+  // 64-bit index math: the 32-bit form gained nothing here and its extra
+  // registers spill under the 64-register cap
+  const ConvWarp cw((L + kConvBSeg - 1) / kConvBSeg, p.batch * p.dim, p.dim, false);
+  if (!cw.live) return;  // whole warps leave together
+  const int64_t row = cw.row, seg = cw.seg, d = cw.d;
   const T *xr = static_cast<const T *>(p.x) + row * L;
   const T *gr = static_cast<const T *>(p.dout) + row * L;
   T *dxr = static_cast<T *>(p.dx) + row * L;
   const bool vec = p.vec != 0;
   const bool silu = p.silu != 0;
-  Raw8<T> rx[kConvR], rg[kConvR];
+  Raw8<T> rx[kConvBR], rg[kConvBR];
 #pragma unroll
-  for (int r = 0; r < kConvR; ++r) {
-    const int64_t t0 = seg * kConvSeg + r * 32 * kConvW + lane * kConvW;
+  for (int r = 0; r < kConvBR; ++r) {
+    const int64_t t0 = seg * kConvBSeg + r * 32 * kConvW + lane * kConvW;
     rx[r].load(xr, t0, L, vec);
     rg[r].load(gr, t0, L, vec);
   }
@@ -235,9 +267,9 @@ __global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 :
     if (t0 < L) IO<T>::store8(dxr, t0, L, vec, o);
   };
 #pragma unroll
-  for (int r = 0; r < kConvR; ++r) {
-    const int64_t t0 = seg * kConvSeg + r * 32 * kConvW + lane * kConvW;
-    const bool live = seg * kConvSeg + r * 32 * kConvW < L;  // warp-uniform
+  for (int r = 0; r < kConvBR; ++r) {
+    const int64_t t0 = seg * kConvBSeg + r * 32 * kConvW + lane * kConvW;
+    const bool live = seg * kConvBSeg + r * 32 * kConvW < L;  // warp-uniform
     float v[kConvW], gv[kConvW];
     rx[r].unpack(v);
     rg[r].unpack(gv);
@@ -362,6 +394,22 @@ __global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 :
   }
 }
 
+template <typename T, bool NARROW>
+static cudaError_t launch_conv_k(const ConvParams &p, unsigned g, cudaStream_t s) {
+  switch (p.K) {
+    case 1: k_conv<T, 1, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 2: k_conv<T, 2, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 3: k_conv<T, 3, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 4: k_conv<T, 4, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 5: k_conv<T, 5, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 6: k_conv<T, 6, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 7: k_conv<T, 7, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    case 8: k_conv<T, 8, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
   const int64_t segs = (p.L + kConvSeg - 1) / kConvSeg;
@@ -369,18 +417,7 @@ static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
   const int64_t blocks = (warps * 32 + kConvThreads - 1) / kConvThreads;
   if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
   const unsigned g = (unsigned)blocks;
-  switch (p.K) {
-    case 1: k_conv<T, 1><<<g, kConvThreads, 0, s>>>(p); break;
-    case 2: k_conv<T, 2><<<g, kConvThreads, 0, s>>>(p); break;
-    case 3: k_conv<T, 3><<<g, kConvThreads, 0, s>>>(p); break;
-    case 4: k_conv<T, 4><<<g, kConvThreads, 0, s>>>(p); break;
-    case 5: k_conv<T, 5><<<g, kConvThreads, 0, s>>>(p); break;
-    case 6: k_conv<T, 6><<<g, kConvThreads, 0, s>>>(p); break;
-    case 7: k_conv<T, 7><<<g, kConvThreads, 0, s>>>(p); break;
-    case 8: k_conv<T, 8><<<g, kConvThreads, 0, s>>>(p); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  return blocks * kConvThreads <= 0xffffffffll ? launch_conv_k<T, true>(p, g, s) : launch_conv_k<T, false>(p, g, s);
 }
 
 cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s) {
@@ -389,7 +426,7 @@ cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s) {
 
 template <typename T>
 static cudaError_t launch_conv_bwd_t(const ConvBwdParams &p, cudaStream_t s) {
-  const int64_t segs = (p.L + kConvSeg - 1) / kConvSeg;
+  const int64_t segs = (p.L + kConvBSeg - 1) / kConvBSeg;
   const int64_t warps = p.batch * p.dim * segs;
   const int64_t blocks = (warps * 32 + kConvThreads - 1) / kConvThreads;
   if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
