@@ -359,14 +359,78 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
                     "kernel_mufu_frac": kernel_ex2 * w.bldn / (ms_b * 1e-3) / ex2_peak,
                     "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                                   f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
+    variants = measure_training_variants(ssm, torch, dev, g, y, out, w, steps, barrier, max_over_ranks)
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
             "d_state": w.dstate, "io_dtype": w.dtype, "steps": steps,
             "fwd_path": ssm.fwd_path(shape), "saved_states": True, "fwd_ms": ms_f, "bwd_ms": ms_b,
+            **variants,
             "bwd_roofline": bwd_roofline,
             "value": aggregate_value(world, w.bld, (ms_f + ms_b) * 1e-3), "unit": UNIT + " (fwd+bwd)",
             "bwd_value": aggregate_value(world, w.bld, ms_b * 1e-3),
             "bwd_ex2_per_element": ex2_per_element, "bwd_kernel_ex2_per_element": kernel_ex2,
             "bwd_kernels_per_step": 2}
+
+
+def measure_training_variants(ssm, torch, dev, g, y, out, w, steps, barrier, max_over_ranks):
+    """The same training step (forward saving chunk states, backward from them)
+    with the exact zero-order-hold input term (the general backward kernel)
+    and with token-major activations ([batch][seqlen][d_inner] u, delta, z,
+    dout and their gradients; the d_state-16 kernel)."""
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    tm = None
+    if w.dtype == synth.BF16 and w.dim % 8 == 0:
+        tm = {k: g[k].transpose(1, 2).contiguous() for k in ("u", "delta", "z", "dy")}
+        tm_out = dict(out, du=torch.empty_like(tm["u"]), ddelta=torch.empty_like(tm["u"]),
+                      dz=torch.empty_like(tm["u"]))
+        y_tm = torch.empty_like(tm["u"])
+    for name, flags in (("zoh_exact", ssm.SSM_FLAG_ZOH_EXACT), ("token_major", ssm.SSM_FLAG_TOKEN_MAJOR)):
+        tok = name == "token_major"
+        if tok and tm is None:
+            continue
+        shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
+                               ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32,
+                               flags=ssm.SSM_FLAG_SAVE_STATES | flags)
+        ws_f = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+        ws_b = torch.empty(ssm.bwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+        a = tm if tok else g
+        o = tm_out if tok else out
+        yy = y_tm if tok else y
+
+        def fwd():
+            ssm.scan_fwd(a["u"], a["delta"], g["A"], g["B"], g["C"], g["D"], a["z"], g["delta_bias"],
+                         y=yy, workspace=ws_f, save_states=True, zoh_exact=not tok, token_major=tok)
+
+        def bwd():
+            ssm.scan_bwd(a["u"], a["delta"], g["A"], g["B"], g["C"], g["D"], a["z"], g["delta_bias"],
+                         a["dy"], out=o, workspace=ws_b, fwd_workspace=ws_f, zoh_exact=not tok,
+                         token_major=tok)
+
+        for _ in range(3):
+            fwd()
+            bwd()
+        torch.cuda.synchronize(dev)
+        ssm.check(ws_f)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        t_f = t_b = 0.0
+        for _ in range(steps):
+            evs[0].record(stream)
+            fwd()
+            evs[1].record(stream)
+            bwd()
+            evs[2].record(stream)
+            torch.cuda.synchronize(dev)
+            t_f += evs[0].elapsed_time(evs[1])
+            t_b += evs[1].elapsed_time(evs[2])
+        barrier()
+        ssm.check(ws_f)
+        res[name] = {"fwd_ms": max_over_ranks(t_f / steps), "bwd_ms": max_over_ranks(t_b / steps),
+                     "fwd_path": ssm.fwd_path(shape),
+                     "bwd_kernel": "k_bwd (general, exact ZOH)" if not tok else "k_bwd16 (token-major)"}
+        del ws_f, ws_b
+    return res
 
 
 def measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks, name):
@@ -427,7 +491,7 @@ def measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks, name)
                          "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                          "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                                        f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"},
-            "gpu_launches": k * (3 if path == "split_l" else 1)}
+            "gpu_launches": k * {"split_l": 3, "lookback_ws": 2}.get(path, 1)}
 
 
 def decode_bytes(w: synth.Workload) -> int:
@@ -631,7 +695,7 @@ def main():
                 "ms_per_step": tr["fwd_ms"] + tr["bwd_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": dict(config_of(w, tr["fwd_path"]), step="fwd+bwd"), "bwd": tr,
-                "roofline": tr["bwd_roofline"], "gpu_launches": 3 * tr["steps"]}
+                "roofline": tr["bwd_roofline"], "gpu_launches": 4 * tr["steps"]}
         if rank == 0:
             print(json.dumps(line), flush=True)
         if world > 1:
@@ -651,7 +715,8 @@ def main():
                            path_id, args.lanes)
     path = ssm.fwd_path(shape)
     ws = torch.empty(ssm.fwd_workspace_bytes(shape), dtype=torch.uint8, device=dev)
-    launches_per_step = {"lookback": 1, "per_group": 1, "split_l": 3, "lookback_ws": 1}[path]
+    # our kernels per forward: the warp-specialised schedule widens B and C first
+    launches_per_step = {"lookback": 1, "per_group": 1, "split_l": 3, "lookback_ws": 2}[path]
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -711,6 +776,32 @@ def main():
         tok = {"layout": "[batch][seqlen][d_inner] u, delta, z, y", "ms_per_step": ms_tm,
                "value": aggregate_value(world, w.bld, ms_tm * 1e-3), "unit": UNIT}
         del tm, y_tm
+
+    # the same forward with the exact zero-order-hold input term, Delta u (e^x - 1)/x B
+    zoh = None
+    if not args.no_bwd and not args.batch:
+        def step_zoh():
+            ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                         g["delta_bias"], y=y, last_state=ls, return_last_state=True,
+                         workspace=ws, zoh_exact=True)
+
+        for _ in range(max(3, args.warmup)):
+            step_zoh()
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step_zoh()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        ssm.check(ws)
+        ms_z = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+        zshape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
+                                ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32,
+                                flags=ssm.SSM_FLAG_ZOH_EXACT)
+        zoh = {"path": ssm.fwd_path(zshape), "ms_per_step": ms_z,
+               "value": aggregate_value(world, w.bld, ms_z * 1e-3), "unit": UNIT}
 
     # end to end through the public API: pinned host inputs in, result out, every step
     e2e = None
@@ -783,6 +874,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": dict(config_of(w, path), parallelism=f"replicas x{world}"),
             "roofline": roofline, "clocks": clocks, "e2e": e2e, "bwd": bwd, "decode": dec, "conv1d": conv, "token_major": tok,
+            "zoh_exact": zoh,
             "mamba_130m_layer": m130, "million_length": mlen,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -94,12 +94,17 @@ def _workspace(nbytes, device, workspace):
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softplus=True,
              initial_state=None, y=None, last_state=None, return_last_state=False,
              workspace=None, path: int = SSM_PATH_AUTO, lanes: int = 0, zoh_exact=False,
-             save_states=False, token_major=False, stream=None):
+             save_states=False, token_major=False, check_status=False, stream=None):
     """Forward selective scan; returns y, or (y, last_state).  zoh_exact selects the
     exact zero-order-hold input term instead of the Euler one (Delta * B).
     save_states also writes the state entering every 16-step chunk into
     ``workspace`` (which must then be given), for scan_bwd(fwd_workspace=...).
-    token_major: u, delta, z and y are (batch, seqlen, dim) instead."""
+    token_major: u, delta, z and y are (batch, seqlen, dim) instead.
+    The look-back schedules hand states between warps with a bounded wait that
+    records a give-up in the workspace's error word instead of trapping:
+    check_status=True synchronises after the launch and raises ScanError
+    (SSM_ERR_DEVICE_TIMEOUT) if that happened; otherwise pass a workspace and
+    call check(workspace) when convenient (an internal workspace is not kept)."""
     import torch
     if token_major:
         batch, seqlen, dim = u.shape
@@ -140,6 +145,8 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
         _ptr(last_state), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(stream))
     if rc != 0:
         raise ScanError(rc, "ssm_scan_fwd")
+    if check_status:
+        check(ws, stream)
     if return_last_state:
         return y, last_state
     return y

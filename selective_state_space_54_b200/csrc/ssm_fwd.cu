@@ -636,8 +636,8 @@ struct __align__(16) WSStage {
   // lane-j stride of the partial sums; with 4 lanes per channel it is padded
   // so that a channel's 4 lanes store into different banks
   static constexpr int YS = CPW * (kTW + 4) + (LPC == 4 ? 8 : 0);
-  float dl[CPW][kTW + 4];
-  float dlu[CPW][kTW + 4];
+  float dl[CPW][kTW + 4];   // Delta
+  float dlu[CPW][kTW + 4];  // Delta u (u in the exact-ZOH instantiation)
   float ys[LPC * YS];  // C.h partial sums of a channel's LPC lanes: [lane j][channel][step]
   __device__ __forceinline__ float *ys_at(int j, int c, int t) { return ys + j * YS + c * (kTW + 4) + t; }
   __device__ __forceinline__ const float *ys_at(int j, int c, int t) const {
@@ -724,6 +724,16 @@ struct Share {
   }
 };
 
+// Exact ZOH in the warp-specialised consumer: (e^x - 1)/x = sum_k x^k/(k+1)!
+// evaluated in the ex2 argument x / ln 2, so term k carries ln2^k / (k+1)!;
+// used for |x| < 1/4, i.e. |x / ln 2| < 0.25 / ln 2.
+constexpr float kZohT1 = 3.465735903e-01f;  // ln2 / 2!
+constexpr float kZohT2 = 8.007550232e-02f;  // ln2^2 / 3!
+constexpr float kZohT3 = 1.387602717e-02f;  // ln2^3 / 4!
+constexpr float kZohT4 = 1.923625822e-03f;  // ln2^4 / 5!
+constexpr float kZohT5 = 2.222259691e-04f;  // ln2^5 / 6!
+constexpr float kZohSmall = 3.606737602e-01f;  // 0.25 / ln2
+
 template <typename T, int NP, int LPC, bool ZOH, bool SAVE>
 __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP, LPC> &sm, int64_t w,
                                             const Share &sh, unsigned bar_full, unsigned bar_ys) {
@@ -737,12 +747,14 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP, LP
     const Lane ln = lane_of<LPC>(p, g);
     const int c = ln.c, j = ln.j;
     f2 A2p[S / 2];
+    f2 rA[ZOH ? S / 2 : 1];  // exact ZOH: 1 / A_n (infinite for A_n = 0, whose x is 0)
 #pragma unroll
     for (int s = 0; s < S; s += 2) {
       const int n = j * S + s;
-      const float a0 = (ln.valid && n < p.N) ? p.A[ln.d * p.N + n] * kLog2e : 0.f;
-      const float a1 = (ln.valid && n + 1 < p.N) ? p.A[ln.d * p.N + n + 1] * kLog2e : 0.f;
-      A2p[s / 2] = pack2(a0, a1);
+      const float a0 = (ln.valid && n < p.N) ? p.A[ln.d * p.N + n] : 0.f;
+      const float a1 = (ln.valid && n + 1 < p.N) ? p.A[ln.d * p.N + n + 1] : 0.f;
+      A2p[s / 2] = pack2(a0 * kLog2e, a1 * kLog2e);
+      if constexpr (ZOH) rA[s / 2] = pack2(__frcp_rn(a0), __frcp_rn(a1));
     }
     float h[S];
     if (k0 > 0) {
@@ -804,15 +816,32 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP, LP
               bv = *reinterpret_cast<const f2 *>(Brow + s);
               cv = *reinterpret_cast<const f2 *>(Crow + s);
             }
+            const f2 xx = mul2(dl2, A2p[s / 2]);  // x / ln 2, x = Delta A_n
             float x0, x1;
-            unpack2(mul2(dl2, A2p[s / 2]), x0, x1);
+            unpack2(xx, x0, x1);
             const float a0 = ex2(x0), a1 = ex2(x1);
             const f2 a = pack2(a0, a1);
-            if constexpr (ZOH)  // exact zero-order hold: Delta u (e^x - 1)/x B, x = Delta A_n
-              hp[s / 2] = fma2(a, hp[s / 2],
-                               mul2(mul2(du2, pack2(expm1_over_x(x0, a0), expm1_over_x(x1, a1))), bv));
-            else
+            if constexpr (ZOH) {
+              // exact zero-order hold: Delta u (e^x - 1)/x B.  Delta (e^x - 1)/x is
+              // (e^x - 1) / A_n for |x| >= 1/4 (Delta cancels; e^x - 1 loses at most
+              // 4 ulp of e^x there), else Delta times the Taylor series of
+              // (e^x - 1)/x to x^5 (remainder below 5e-8).  The stage holds u
+              // itself in this instantiation.
+              const f2 big = mul2(add2(a, splat2(-1.f)), rA[s / 2]);
+              f2 q = fma2(splat2(kZohT5), xx, splat2(kZohT4));
+              q = fma2(q, xx, splat2(kZohT3));
+              q = fma2(q, xx, splat2(kZohT2));
+              q = fma2(q, xx, splat2(kZohT1));
+              q = fma2(q, xx, splat2(1.f));
+              const f2 small = mul2(q, dl2);
+              float b0, b1, s0, s1;
+              unpack2(big, b0, b1);
+              unpack2(small, s0, s1);
+              const f2 wz = pack2(fabsf(x0) < kZohSmall ? s0 : b0, fabsf(x1) < kZohSmall ? s1 : b1);
+              hp[s / 2] = fma2(a, hp[s / 2], mul2(mul2(wz, du2), bv));
+            } else {
               hp[s / 2] = fma2(a, hp[s / 2], mul2(du2, bv));
+            }
             acc = s == 0 ? mul2(cv, hp[0]) : fma2(cv, hp[s / 2], acc);
           }
           float a0, a1;
@@ -983,7 +1012,9 @@ __device__ __forceinline__ void load_row(const float *p, float (&o)[V]) {
   }
 }
 
-template <typename T, int NP, int LPC, bool TOK>
+// ZOH: the stage's second row holds u instead of Delta u (the consumer's
+// exact input term needs u; see ws_consumer)
+template <typename T, int NP, int LPC, bool TOK, bool ZOH>
 __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP, LPC> &sm, const Share &sh,
                                             unsigned bar_full, unsigned bar_ys) {
   constexpr int CPW = 32 / LPC, VPL = kTW / LPC, HP = VPL / 2;
@@ -1110,7 +1141,8 @@ __device__ __forceinline__ void ws_producer(const FwdParams &p, WSPair<T, NP, LP
         }
       }
 #pragma unroll
-      for (int i = 0; i < HP; ++i) dlu2[i] = mul2(dl2[i], pack2(u8[2 * i], u8[2 * i + 1]));
+      for (int i = 0; i < HP; ++i)
+        dlu2[i] = ZOH ? pack2(u8[2 * i], u8[2 * i + 1]) : mul2(dl2[i], pack2(u8[2 * i], u8[2 * i + 1]));
       {
         float *pd = &st.dl[c][jv];
         float *pu = &st.dlu[c][jv];
@@ -1171,7 +1203,7 @@ __global__ void __launch_bounds__(kWSThreads, 2) k_fwd_ws(FwdParams p) {
   if (w >= p.n_workers) return;  // both warps of a pair leave together
   const Share sh(w, p.n_workers, p.n_groups, p.n_chunks);
   const unsigned bar_full = 4 * pair, bar_ys = 4 * pair + 2;
-  if (producer) ws_producer<T, NP, LPC, TOK>(p, sm, sh, bar_full, bar_ys);
+  if (producer) ws_producer<T, NP, LPC, TOK, ZOH>(p, sm, sh, bar_full, bar_ys);
   else ws_consumer<T, NP, LPC, ZOH, SAVE>(p, sm, w, sh, bar_full, bar_ys);
 }
 

@@ -100,6 +100,18 @@ def test_initial_state(cuda_device, path, lanes):
     _check(case, cuda_device, path, h0=h0, lanes=lanes)
 
 
+def test_check_status_after_the_forward(cuda_device):
+    # check_status=True synchronises and reads the error word of the (internal)
+    # workspace: a healthy look-back forward returns normally and matches one without it
+    import selective_state_space_54_b200 as ssm
+    case = synth.make_case(8, 1536, 300, 16, synth.BF16, seed=71)
+    g = upload(case, cuda_device)
+    args = (g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"])
+    y0 = ssm.scan_fwd(*args)
+    y1 = ssm.scan_fwd(*args, check_status=True)
+    assert to_f64(y0).tobytes() == to_f64(y1).tobytes()
+
+
 def test_continuation_matches_one_scan(cuda_device):
     # scan(L1) -> last_state -> scan(L2 from it) == scan(L1 + L2), on the GPU
     import torch

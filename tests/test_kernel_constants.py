@@ -88,3 +88,49 @@ def test_reciprocal_seed_and_newton_steps():
         y = (y.astype(np.float64) + y.astype(np.float64) * e1.astype(np.float64)).astype(np.float32)
     rel = np.abs(y.astype(np.float64) * d.astype(np.float64) - 1.0)
     assert rel.max() <= 3e-7, rel.max()
+
+
+def _zoh_constants():
+    src = open(os.path.join(CSRC, "ssm_fwd.cu")).read()
+    got = {}
+    for name in ("kZohT1", "kZohT2", "kZohT3", "kZohT4", "kZohT5", "kZohSmall"):
+        m = re.search(r"constexpr float " + name + r" = " + FLOAT, src)
+        assert m, name
+        got[name] = float(m.group(1))
+    return got
+
+
+def test_zoh_series_coefficients():
+    # (e^x - 1)/x = sum_k x^k / (k+1)!, evaluated in y = x / ln 2 (the ex2
+    # argument): term k carries ln2^k / (k+1)!; the switch to (e^x - 1)/A is at
+    # |x| = 1/4, i.e. |y| = 0.25 / ln 2
+    import math
+    c = _zoh_constants()
+    for k in range(1, 6):
+        ref = math.log(2) ** k / math.factorial(k + 1)
+        assert abs(c[f"kZohT{k}"] - ref) <= 2 ** -23 * ref, (k, c[f"kZohT{k}"], ref)
+    assert abs(c["kZohSmall"] - 0.25 / math.log(2)) <= 2 ** -23
+
+
+def test_zoh_two_branch_error_bound():
+    # The consumer's Delta (e^x - 1)/x: the series to x^5 below |x| = 1/4, else
+    # (a - 1)/A with a = 2^(x/ln 2) from the special-function unit.  Emulated in
+    # fp32 with a perturbed by the ex2 unit's error (up to 2 ulp, either sign),
+    # relative to the exact value: below 1e-6 everywhere.
+    c = _zoh_constants()
+    T = [np.float32(c[f"kZohT{k}"]) for k in range(5, 0, -1)]
+    x = np.concatenate([-np.geomspace(1e-8, 60.0, 40001), np.geomspace(1e-8, 10.0, 20001)])
+    y = (x / np.log(2)).astype(np.float32)
+    exact = np.expm1(x) / x
+    # series branch, fused Horner in fp32 (one rounding per step)
+    q = np.full_like(y, T[0], dtype=np.float32)
+    for t in T[1:] + [np.float32(1.0)]:
+        q = (q.astype(np.float64) * y.astype(np.float64) + np.float64(t)).astype(np.float32)
+    worst = 0.0
+    for ulps in (-2, 0, 2):
+        a = (np.exp2(y.astype(np.float64)) * (1 + ulps * 2.0 ** -24)).astype(np.float32)
+        # Delta = 1, A = x: (a - 1) * (1/A) against the series
+        big = ((a - np.float32(1)).astype(np.float32) * (np.float32(1) / x.astype(np.float32))).astype(np.float32)
+        got = np.where(np.abs(y) < np.float32(c["kZohSmall"]), q, big).astype(np.float64)
+        worst = max(worst, float(np.max(np.abs(got / exact - 1))))
+    assert worst < 1e-6, worst
