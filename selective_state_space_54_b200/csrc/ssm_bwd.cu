@@ -167,65 +167,55 @@ struct BwdBC {
   }
 };
 
-// packed fp32 pairs (sm_100a f32x2 arithmetic)
-typedef unsigned long long bf2;
-__device__ __forceinline__ bf2 bpack(float lo, float hi) {
-  bf2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void bunpack(bf2 v, float &lo, float &hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ bf2 bfma(bf2 a, bf2 b, bf2 c) {
-  bf2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ bf2 bmul(bf2 a, bf2 b) {
-  bf2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ bf2 badd(bf2 a, bf2 b) {
-  bf2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ bf2 bex2(bf2 x) {
+__device__ __forceinline__ f2 ex2_2(f2 x) {
   float x0, x1;
-  bunpack(x, x0, x1);
-  return bpack(ex2(x0), ex2(x1));
+  unpack2(x, x0, x1);
+  return pack2(ex2(x0), ex2(x1));
 }
 
-// Exact zero-order hold, per half of a pair with x = x2 ln 2 = Delta A_n and
-// a = exp(x): phi = (e^x - 1) / x (the input term is Delta u phi B) and
-// psi = (x e^x - (e^x - 1)) / x^2 (its derivative in A_n is Delta^2 u psi B).
-// For |x| < 1/2 psi is its Taylor series sum_{m<8} x^m (m+1)/(m+2)!
-// (remainder below 1e-8); beyond, the closed form loses at most a few bits.
-__device__ __forceinline__ float xexpm1_over_x2(float x2, float a) {
-  const float x = x2 * kLn2;
-  float q = 2.204585537918871e-05f;        // coefficient of x^m: (m+1)/(m+2)!, m = 7
-  q = fmaf(q, x, 1.736111111111111e-04f);  // m = 6
-  q = fmaf(q, x, 1.190476190476190e-03f);  // m = 5
-  q = fmaf(q, x, 6.944444444444444e-03f);  // m = 4
-  q = fmaf(q, x, 3.333333333333333e-02f);  // m = 3
-  q = fmaf(q, x, 1.250000000000000e-01f);  // m = 2
-  q = fmaf(q, x, 3.333333333333333e-01f);  // m = 1
-  q = fmaf(q, x, 0.5f);                    // m = 0
-  return fabsf(x) < 0.5f ? q : fmaf(x, a, 1.f - a) * rcp_approx(x * x);
+// Exact zero-order hold, on pairs, with y = x / ln 2 the ex2 argument
+// (x = Delta A_n), a = e^x and rA = 1 / A_n:
+//   W = Delta (e^x - 1)/x     (the input term is u W B_n)
+//   Y = Delta^2 psi(x), psi(x) = (x e^x - (e^x - 1)) / x^2   (its A_n derivative is u Y B_n).
+// Above a threshold in |x| Delta cancels: W = (e^x - 1) / A_n and
+// Y = (Delta e^x - W) / A_n, with no reciprocal per element (rA is per state);
+// below it the Taylor series, sum_k x^k/(k+1)! to x^5 for W (|x| < 1/4,
+// remainder below 5e-8) and sum_m x^m (m+1)/(m+2)! to x^7 for psi
+// (|x| < 1/2, remainder below 1e-8), with the ln2^k of y folded into the
+// coefficients.  Where e^x - 1 or Delta e^x - W cancel, the series is used.
+constexpr float kBwdW1 = 3.465735903e-01f, kBwdW2 = 8.007550232e-02f, kBwdW3 = 1.387602717e-02f,
+                kBwdW4 = 1.923625822e-03f, kBwdW5 = 2.222259691e-04f;  // ln2^k / (k+1)!
+constexpr float kBwdWSmall = 3.606737602e-01f;                           // 0.25 / ln2
+constexpr float kBwdP0 = 5.000000000e-01f, kBwdP1 = 2.310490602e-01f, kBwdP2 = 6.005662674e-02f,
+                kBwdP3 = 1.110082173e-02f, kBwdP4 = 1.603021518e-03f, kBwdP5 = 1.904794021e-04f,
+                kBwdP6 = 1.925441299e-05f, kBwdP7 = 1.694748200e-06f;  // ln2^m (m+1) / (m+2)!
+constexpr float kBwdPSmall = 7.213475204e-01f;                           // 0.5 / ln2
+__device__ __forceinline__ f2 zoh_select(f2 y, f2 small, f2 big, float lim) {
+  float y0, y1, s0, s1, b0, b1;
+  unpack2(y, y0, y1);
+  unpack2(small, s0, s1);
+  unpack2(big, b0, b1);
+  return pack2(fabsf(y0) < lim ? s0 : b0, fabsf(y1) < lim ? s1 : b1);
 }
-__device__ __forceinline__ bf2 bphi(bf2 x2, bf2 a) {
-  float x0, x1, a0, a1;
-  bunpack(x2, x0, x1);
-  bunpack(a, a0, a1);
-  return bpack(expm1_over_x(x0, a0), expm1_over_x(x1, a1));
+__device__ __forceinline__ f2 zoh_w(f2 y, f2 a, f2 dl2, f2 rA) {
+  const f2 big = mul2(add2(a, splat2(-1.f)), rA);
+  f2 q = fma2(splat2(kBwdW5), y, splat2(kBwdW4));
+  q = fma2(q, y, splat2(kBwdW3));
+  q = fma2(q, y, splat2(kBwdW2));
+  q = fma2(q, y, splat2(kBwdW1));
+  q = fma2(q, y, splat2(1.f));
+  return zoh_select(y, mul2(q, dl2), big, kBwdWSmall);
 }
-__device__ __forceinline__ bf2 bpsi(bf2 x2, bf2 a) {
-  float x0, x1, a0, a1;
-  bunpack(x2, x0, x1);
-  bunpack(a, a0, a1);
-  return bpack(xexpm1_over_x2(x0, a0), xexpm1_over_x2(x1, a1));
+__device__ __forceinline__ f2 zoh_y(f2 y, f2 a, f2 w, f2 dl2, f2 rA) {
+  const f2 big = mul2(fma2(w, splat2(-1.f), mul2(dl2, a)), rA);
+  f2 q = fma2(splat2(kBwdP7), y, splat2(kBwdP6));
+  q = fma2(q, y, splat2(kBwdP5));
+  q = fma2(q, y, splat2(kBwdP4));
+  q = fma2(q, y, splat2(kBwdP3));
+  q = fma2(q, y, splat2(kBwdP2));
+  q = fma2(q, y, splat2(kBwdP1));
+  q = fma2(q, y, splat2(kBwdP0));
+  return zoh_select(y, mul2(q, mul2(dl2, dl2)), big, kBwdPSmall);
 }
 
 template <typename T, int NP, bool ZOH>
@@ -257,7 +247,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
   const float bias = (p.bias && valid) ? p.bias[d] : 0.f;
   const float Dd = (p.D && valid) ? p.D[d] : 0.f;
   // this lane's states n = j*S + s, as pairs; S = 1 uses the low half only
-  bf2 A2[SP], An[SP];
+  f2 A2[SP], An[SP];
 #pragma unroll
   for (int i = 0; i < SP; ++i) {
     float a[2];
@@ -266,19 +256,29 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
       const int s = 2 * i + h2, n = j * S + s;
       a[h2] = (s < S && valid && n < N) ? p.A[d * N + n] : 0.f;
     }
-    An[i] = bpack(a[0], a[1]);
-    A2[i] = bpack(a[0] * kLog2e, a[1] * kLog2e);
+    An[i] = pack2(a[0], a[1]);
+    A2[i] = pack2(a[0] * kLog2e, a[1] * kLog2e);
+  }
+  // exact ZOH: 1 / A_n per state (infinite for A_n = 0, whose x is 0: the series branch)
+  f2 rA[ZOH ? SP : 1];
+  if constexpr (ZOH) {
+#pragma unroll
+    for (int i = 0; i < SP; ++i) {
+      float a0, a1;
+      unpack2(An[i], a0, a1);
+      rA[i] = pack2(__frcp_rn(a0), __frcp_rn(a1));
+    }
   }
   // saved state entering 16-step chunk k = 8-step saved chunk 2k (padded channels included)
   float *ck = p.ckpt + ckpt_offset(b, d, 0, p.dim, L, NP) + j * S;
   auto ck_at = [&](int64_t k, int i) -> float * { return &ck[2 * k * kCkptChannels * NP + 2 * i]; };
-  auto Bpair = [&](int t, int i) -> bf2 {
-    if constexpr (S >= 2) return *reinterpret_cast<const bf2 *>(&sm.Bs[t][j * S + 2 * i]);
-    else return bpack(sm.Bs[t][j], 0.f);
+  auto Bpair = [&](int t, int i) -> f2 {
+    if constexpr (S >= 2) return *reinterpret_cast<const f2 *>(&sm.Bs[t][j * S + 2 * i]);
+    else return pack2(sm.Bs[t][j], 0.f);
   };
-  auto Cpair = [&](int t, int i) -> bf2 {
-    if constexpr (S >= 2) return *reinterpret_cast<const bf2 *>(&sm.Cs[t][j * S + 2 * i]);
-    else return bpack(sm.Cs[t][j], 0.f);
+  auto Cpair = [&](int t, int i) -> f2 {
+    if constexpr (S >= 2) return *reinterpret_cast<const f2 *>(&sm.Cs[t][j * S + 2 * i]);
+    else return pack2(sm.Cs[t][j], 0.f);
   };
 
   // per (channel, step) quantities for this lane's 4 steps of chunk k
@@ -313,10 +313,14 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
       *reinterpret_cast<float4 *>(&ws.uu[c][4 * q]) = make_float4(u4[0], u4[1], u4[2], u4[3]);
     }
   };
-  // the input term Bbar_n u: Delta u B_n (Euler) or Delta u phi(Delta A_n) B_n (exact ZOH)
-  auto bterm = [&](bf2 du2, bf2 x, bf2 a, bf2 Bv) -> bf2 {
-    if constexpr (ZOH) return bmul(bmul(du2, bphi(x, a)), Bv);
-    else return bmul(du2, Bv);
+  // the input term Bbar_n u: Delta u B_n (Euler) or u W B_n, W = Delta (e^x - 1)/x (exact ZOH)
+  auto bterm = [&](int t, f2 dl2, f2 du2, f2 x, f2 a, int i, f2 Bv) -> f2 {
+    if constexpr (ZOH) {
+      const float uv = ws.uu[c][t];
+      return mul2(mul2(pack2(uv, uv), zoh_w(x, a, dl2, rA[i])), Bv);
+    } else {
+      return mul2(du2, Bv);
+    }
   };
 
   // inputs of one chunk, loaded a chunk ahead of their use
@@ -345,7 +349,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
   };
 
   // ---- phase A: states entering every chunk ----
-  bf2 h[SP];
+  f2 h[SP];
 #pragma unroll
   for (int i = 0; i < SP; ++i) {
     float v[2];
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
       const int s = 2 * i + h2, n = j * S + s;
       v[h2] = (s < S && p.h0 && valid && n < N) ? p.h0[(b * p.dim + d) * N + n] : 0.f;
     }
-    h[i] = bpack(v[0], v[1]);
+    h[i] = pack2(v[0], v[1]);
   }
   ChunkIn nxt;
   if (K > 0 && !p.ckpt_given) load_chunk(0, false, nxt);
@@ -363,7 +367,7 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
 #pragma unroll
     for (int i = 0; i < SP; ++i) {
       float lo, hi;
-      bunpack(h[i], lo, hi);
+      unpack2(h[i], lo, hi);
       float *dst = ck_at(k, i);
       dst[0] = lo;
       if (S >= 2) dst[1] = hi;
@@ -376,20 +380,20 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     __syncthreads();
 #pragma unroll 4
     for (int t = 0; t < kTB; ++t) {
-      const bf2 dl2 = bpack(ws.dl[c][t], ws.dl[c][t]), du2 = bpack(ws.dlu[c][t], ws.dlu[c][t]);
+      const f2 dl2 = pack2(ws.dl[c][t], ws.dl[c][t]), du2 = pack2(ws.dlu[c][t], ws.dlu[c][t]);
 #pragma unroll
       for (int i = 0; i < SP; ++i) {
-        const bf2 x = bmul(dl2, A2[i]), a = bex2(x);
-        h[i] = bfma(a, h[i], bterm(du2, x, a, Bpair(t, i)));
+        const f2 x = mul2(dl2, A2[i]), a = ex2_2(x);
+        h[i] = fma2(a, h[i], bterm(t, dl2, du2, x, a, i, Bpair(t, i)));
       }
     }
     __syncthreads();
   }
 
   // ---- phase B: reverse ----
-  bf2 g[SP], dA_acc[SP];
+  f2 g[SP], dA_acc[SP];
 #pragma unroll
-  for (int i = 0; i < SP; ++i) { g[i] = bpack(0.f, 0.f); dA_acc[i] = g[i]; }
+  for (int i = 0; i < SP; ++i) { g[i] = pack2(0.f, 0.f); dA_acc[i] = g[i]; }
   float dD_acc = 0.f, dbias_acc = 0.f;
   constexpr int kRedOutputs = 4 * 2 * NP / 4;   // float4 outputs of a 4-step group
   if (K > 0) load_chunk(K - 1, true, nxt);
@@ -405,13 +409,13 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     // recompute the chunk's states from its checkpoint, keeping only the
     // state entering each 4-step group (the reverse pass recomputes a group's
     // states again right before it needs them)
-    bf2 H4[kTB / 4][SP];
+    f2 H4[kTB / 4][SP];
     {
-      bf2 hh[SP];
+      f2 hh[SP];
 #pragma unroll
       for (int i = 0; i < SP; ++i) {
         const float *src = ck_at(k, i);  // padded channels: saved states may be unwritten
-        hh[i] = valid ? bpack(src[0], S >= 2 ? src[1] : 0.f) : bpack(0.f, 0.f);
+        hh[i] = valid ? pack2(src[0], S >= 2 ? src[1] : 0.f) : pack2(0.f, 0.f);
       }
 #pragma unroll
     for (int t = 0; t < kTB; t += 4) {
@@ -421,16 +425,16 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
 #pragma unroll
       for (int i4 = 0; i4 < 4; ++i4) {
         const int tt = t + i4;
-        const bf2 dl2 = bpack(ws.dl[c][tt], ws.dl[c][tt]), du2 = bpack(ws.dlu[c][tt], ws.dlu[c][tt]);
-        bf2 acc = bpack(0.f, 0.f);
+        const f2 dl2 = pack2(ws.dl[c][tt], ws.dl[c][tt]), du2 = pack2(ws.dlu[c][tt], ws.dlu[c][tt]);
+        f2 acc = pack2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
-          const bf2 x = bmul(dl2, A2[i]), a = bex2(x);
-          hh[i] = bfma(a, hh[i], bterm(du2, x, a, Bpair(tt, i)));
-          acc = bfma(Cpair(tt, i), hh[i], acc);
+          const f2 x = mul2(dl2, A2[i]), a = ex2_2(x);
+          hh[i] = fma2(a, hh[i], bterm(tt, dl2, du2, x, a, i, Bpair(tt, i)));
+          acc = fma2(Cpair(tt, i), hh[i], acc);
         }
         float a0, a1;
-        bunpack(acc, a0, a1);
+        unpack2(acc, a0, a1);
         yp[i4] = a0 + a1;
       }
       // sum over the channel's 4 lanes; lane j keeps step t + j
@@ -476,71 +480,72 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
     // contributions and adds them to the fp32 accumulators
 #pragma unroll
     for (int grp = kTB / 4 - 1; grp >= 0; --grp) {
-      bf2 hg[4][SP], ag[4][SP];
+      f2 hg[4][SP], ag[4][SP];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int t = 4 * grp + u;
         const float dlv = ws.dl[c][t], duv = ws.dlu[c][t];
-        const bf2 dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
+        const f2 dl2 = pack2(dlv, dlv), du2 = pack2(duv, duv);
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
-          const bf2 x = bmul(dl2, A2[i]);
-          ag[u][i] = bex2(x);
-          hg[u][i] = bfma(ag[u][i], u == 0 ? H4[grp][i] : hg[u - 1][i], bterm(du2, x, ag[u][i], Bpair(t, i)));
+          const f2 x = mul2(dl2, A2[i]);
+          ag[u][i] = ex2_2(x);
+          hg[u][i] = fma2(ag[u][i], u == 0 ? H4[grp][i] : hg[u - 1][i],
+                          bterm(t, dl2, du2, x, ag[u][i], i, Bpair(t, i)));
         }
       }
 #pragma unroll
       for (int u = 3; u >= 0; --u) {
         const int t = 4 * grp + u;
         const float dyv = ws.dy[c][t], dlv = ws.dl[c][t], duv = ws.dlu[c][t];
-        const bf2 dy2 = bpack(dyv, dyv), dl2 = bpack(dlv, dlv), du2 = bpack(duv, duv);
-        bf2 ddl2 = bpack(0.f, 0.f), s12 = ddl2;
-        bf2 u2 = ddl2, ddu2 = ddl2;
+        const f2 dy2 = pack2(dyv, dyv), dl2 = pack2(dlv, dlv), du2 = pack2(duv, duv);
+        f2 ddl2 = pack2(0.f, 0.f), s12 = ddl2;
+        f2 u2 = ddl2;
         if constexpr (ZOH) {
           const float uv = ws.uu[c][t];
-          u2 = bpack(uv, uv);
-          ddu2 = bpack(dlv * duv, dlv * duv);
+          u2 = pack2(uv, uv);
         }
         float *pB = &ws.part[u][0][j][c * S];
         float *pC = &ws.part[u][1][j][c * S];
 #pragma unroll
         for (int i = 0; i < SP; ++i) {
-          g[i] = bfma(dy2, Cpair(t, i), g[i]);
-          const bf2 hp = u == 0 ? H4[grp][i] : hg[u - 1][i];
-          const bf2 ga = bmul(g[i], ag[u][i]);
-          const bf2 qv = bmul(ga, hp);
-          dA_acc[i] = bfma(dl2, qv, dA_acc[i]);
-          ddl2 = bfma(An[i], qv, ddl2);
-          bf2 vB;
+          g[i] = fma2(dy2, Cpair(t, i), g[i]);
+          const f2 hp = u == 0 ? H4[grp][i] : hg[u - 1][i];
+          const f2 ga = mul2(g[i], ag[u][i]);
+          const f2 qv = mul2(ga, hp);
+          dA_acc[i] = fma2(dl2, qv, dA_acc[i]);
+          ddl2 = fma2(An[i], qv, ddl2);
+          f2 vB;
           if constexpr (ZOH) {
-            // h_t = a h_{t-1} + Delta u phi(x) B with x = Delta A: d/dDelta of the
-            // input term is a u B, d/dA is Delta^2 u psi(x) B, d/du is Delta phi B
-            const bf2 x = bmul(dl2, A2[i]);
-            const bf2 phi = bphi(x, ag[u][i]), gB = bmul(g[i], Bpair(t, i));
-            ddl2 = bfma(bmul(ga, Bpair(t, i)), u2, ddl2);
-            dA_acc[i] = bfma(bmul(gB, bpsi(x, ag[u][i])), ddu2, dA_acc[i]);
-            s12 = bfma(gB, phi, s12);
-            vB = bmul(bmul(g[i], du2), phi);
+            // h_t = a h_{t-1} + u W B with W = Delta (e^x - 1)/x, x = Delta A: d/dDelta
+            // of the input term is a u B, d/dA is u Y B (Y = Delta^2 psi(x)), d/du is W B
+            const f2 x = mul2(dl2, A2[i]);
+            const f2 W = zoh_w(x, ag[u][i], dl2, rA[i]);
+            const f2 gB = mul2(g[i], Bpair(t, i));
+            ddl2 = fma2(mul2(ga, Bpair(t, i)), u2, ddl2);
+            dA_acc[i] = fma2(mul2(gB, zoh_y(x, ag[u][i], W, dl2, rA[i])), u2, dA_acc[i]);
+            s12 = fma2(gB, W, s12);
+            vB = mul2(mul2(g[i], u2), W);
           } else {
-            s12 = bfma(g[i], Bpair(t, i), s12);
-            vB = bmul(g[i], du2);
+            s12 = fma2(g[i], Bpair(t, i), s12);
+            vB = mul2(g[i], du2);
           }
-          const bf2 vC = bmul(dy2, hg[u][i]);
+          const f2 vC = mul2(dy2, hg[u][i]);
           g[i] = ga;
           if constexpr (S >= 2) {
-            *reinterpret_cast<bf2 *>(pB + 2 * i) = vB;
-            *reinterpret_cast<bf2 *>(pC + 2 * i) = vC;
+            *reinterpret_cast<f2 *>(pB + 2 * i) = vB;
+            *reinterpret_cast<f2 *>(pC + 2 * i) = vC;
           } else {
             float lo, hi;
-            bunpack(vB, lo, hi);
+            unpack2(vB, lo, hi);
             pB[0] = lo;
-            bunpack(vC, lo, hi);
+            unpack2(vC, lo, hi);
             pC[0] = lo;
           }
         }
         float d0, d1, s0, s1v;
-        bunpack(ddl2, d0, d1);
-        bunpack(s12, s0, s1v);
+        unpack2(ddl2, d0, d1);
+        unpack2(s12, s0, s1v);
         ws.pd[t][c][j] = make_float2(d0 + d1, s0 + s1v);
       }
       __syncthreads();
@@ -553,13 +558,13 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
           const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
           const int which = r4 / NP, n = r4 - which * NP;
           const int jj = n / S, s0 = n - jj * S;
-          bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
+          f2 acc0 = pack2(0.f, 0.f), acc1 = acc0;
 #pragma unroll
           for (int cc = 0; cc < kBCPW; ++cc) {
             const float *src = &ws.part[tl][which][jj][cc * S + s0];
             const ulonglong2 x = *reinterpret_cast<const ulonglong2 *>(src);
-            acc0 = badd(acc0, x.x);
-            acc1 = badd(acc1, x.y);
+            acc0 = add2(acc0, x.x);
+            acc1 = add2(acc1, x.y);
           }
           sm.red[warp][o] = make_ulonglong2(acc0, acc1);
         }
@@ -569,17 +574,17 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
             const int tl = o / (2 * NP / 4), r4 = (o % (2 * NP / 4)) * 4;
             const int which = r4 / NP, n = r4 - which * NP;
             const int t = 4 * grp + tl;
-            bf2 acc0 = bpack(0.f, 0.f), acc1 = acc0;
+            f2 acc0 = pack2(0.f, 0.f), acc1 = acc0;
 #pragma unroll
             for (int w = 0; w < kBW; ++w) {
               const ulonglong2 x = sm.red[w][o];
-              acc0 = badd(acc0, x.x);
-              acc1 = badd(acc1, x.y);
+              acc0 = add2(acc0, x.x);
+              acc1 = add2(acc1, x.y);
             }
             if (t0 + t < L) {
               float4 acc;
-              bunpack(acc0, acc.x, acc.y);
-              bunpack(acc1, acc.z, acc.w);
+              unpack2(acc0, acc.x, acc.y);
+              unpack2(acc1, acc.z, acc.w);
               *reinterpret_cast<float4 *>(p.dBC_part + ((cb * p.batch + b) * L + t0 + t) * 2 * NP +
                                           which * NP + n) = acc;
             }
@@ -618,9 +623,10 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
         const float ddl = (pa.x + pa.z) + (pb.x + pb.z);
         const float s1 = (pa.y + pa.w) + (pb.y + pb.w);
         const float dl = ws.dl[c][t];
-        duv[i] = fmaf(dl, s1, ws.dy[c][t] * Dd);
+        // Euler: du = Delta sum g B + D dy; exact ZOH: s1 = sum g W B already holds Delta
+        duv[i] = fmaf(ZOH ? 1.f : dl, s1, ws.dy[c][t] * Dd);
         // Euler: dDelta = sum g (A a h_prev + B u); exact ZOH: the u term is
-        // already inside ddl (sum g a B u) and s1 = sum g phi B
+        // already inside ddl (sum g a B u)
         float dd = ZOH ? ddl : fmaf(uu[i], s1, ddl);
         if (p.softplus) dd *= sgs[i];
         dd = (valid && t0 + t < L) ? dd : 0.f;
@@ -640,8 +646,8 @@ __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4
 #pragma unroll
     for (int i = 0; i < SP; ++i) {
       float lo[2], gg[2];
-      bunpack(dA_acc[i], lo[0], lo[1]);
-      bunpack(g[i], gg[0], gg[1]);
+      unpack2(dA_acc[i], lo[0], lo[1]);
+      unpack2(g[i], gg[0], gg[1]);
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const int s = 2 * i + h2, n = j * S + s;

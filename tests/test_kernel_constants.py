@@ -134,3 +134,31 @@ def test_zoh_two_branch_error_bound():
         got = np.where(np.abs(y) < np.float32(c["kZohSmall"]), q, big).astype(np.float64)
         worst = max(worst, float(np.max(np.abs(got / exact - 1))))
     assert worst < 1e-6, worst
+
+
+def test_backward_zoh_series_coefficients():
+    # the general backward's exact-ZOH series, in y = x / ln 2: W's terms
+    # ln2^k / (k+1)! (switch at |x| = 1/4) and psi's terms ln2^m (m+1)/(m+2)!
+    # (switch at |x| = 1/2), psi(x) = (x e^x - (e^x - 1)) / x^2
+    import math
+    src = open(os.path.join(CSRC, "ssm_bwd.cu")).read()
+    val = lambda name: float(re.search(name + r" = " + FLOAT, src).group(1))
+    ln2 = math.log(2)
+    for k in range(1, 6):
+        ref = ln2 ** k / math.factorial(k + 1)
+        assert abs(val(f"kBwdW{k}") - ref) <= 2 ** -23 * ref, k
+    for m in range(8):
+        ref = ln2 ** m * (m + 1) / math.factorial(m + 2)
+        assert abs(val(f"kBwdP{m}") - ref) <= 2 ** -23 * ref, m
+    assert abs(val("kBwdWSmall") - 0.25 / ln2) <= 2 ** -23
+    assert abs(val("kBwdPSmall") - 0.5 / ln2) <= 2 ** -22
+    # the psi series against the closed form where that is accurate, and its
+    # remainder at the switch below 1e-8 relative
+    x = np.linspace(-0.5, 0.5, 2001)
+    x = x[np.abs(x) > 1e-3]
+    y = x / ln2
+    q = np.zeros_like(y)
+    for m in range(7, -1, -1):
+        q = q * y + val(f"kBwdP{m}")
+    exact = (x * np.exp(x) - np.expm1(x)) / x ** 2
+    assert np.max(np.abs(q / exact - 1)) < 1e-7
