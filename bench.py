@@ -428,7 +428,7 @@ def measure_training_variants(ssm, torch, dev, g, y, out, w, steps, barrier, max
         ssm.check(ws_f)
         res[name] = {"fwd_ms": max_over_ranks(t_f / steps), "bwd_ms": max_over_ranks(t_b / steps),
                      "fwd_path": ssm.fwd_path(shape),
-                     "bwd_kernel": "k_bwd (general, exact ZOH)" if not tok else "k_bwd16 (token-major)"}
+                     "bwd_kernel": "k_bwd16 (exact ZOH)" if not tok else "k_bwd16 (token-major)"}
         del ws_f, ws_b
     return res
 

@@ -173,51 +173,6 @@ __device__ __forceinline__ f2 ex2_2(f2 x) {
   return pack2(ex2(x0), ex2(x1));
 }
 
-// Exact zero-order hold, on pairs, with y = x / ln 2 the ex2 argument
-// (x = Delta A_n), a = e^x and rA = 1 / A_n:
-//   W = Delta (e^x - 1)/x     (the input term is u W B_n)
-//   Y = Delta^2 psi(x), psi(x) = (x e^x - (e^x - 1)) / x^2   (its A_n derivative is u Y B_n).
-// Above a threshold in |x| Delta cancels: W = (e^x - 1) / A_n and
-// Y = (Delta e^x - W) / A_n, with no reciprocal per element (rA is per state);
-// below it the Taylor series, sum_k x^k/(k+1)! to x^5 for W (|x| < 1/4,
-// remainder below 5e-8) and sum_m x^m (m+1)/(m+2)! to x^7 for psi
-// (|x| < 1/2, remainder below 1e-8), with the ln2^k of y folded into the
-// coefficients.  Where e^x - 1 or Delta e^x - W cancel, the series is used.
-constexpr float kBwdW1 = 3.465735903e-01f, kBwdW2 = 8.007550232e-02f, kBwdW3 = 1.387602717e-02f,
-                kBwdW4 = 1.923625822e-03f, kBwdW5 = 2.222259691e-04f;  // ln2^k / (k+1)!
-constexpr float kBwdWSmall = 3.606737602e-01f;                           // 0.25 / ln2
-constexpr float kBwdP0 = 5.000000000e-01f, kBwdP1 = 2.310490602e-01f, kBwdP2 = 6.005662674e-02f,
-                kBwdP3 = 1.110082173e-02f, kBwdP4 = 1.603021518e-03f, kBwdP5 = 1.904794021e-04f,
-                kBwdP6 = 1.925441299e-05f, kBwdP7 = 1.694748200e-06f;  // ln2^m (m+1) / (m+2)!
-constexpr float kBwdPSmall = 7.213475204e-01f;                           // 0.5 / ln2
-__device__ __forceinline__ f2 zoh_select(f2 y, f2 small, f2 big, float lim) {
-  float y0, y1, s0, s1, b0, b1;
-  unpack2(y, y0, y1);
-  unpack2(small, s0, s1);
-  unpack2(big, b0, b1);
-  return pack2(fabsf(y0) < lim ? s0 : b0, fabsf(y1) < lim ? s1 : b1);
-}
-__device__ __forceinline__ f2 zoh_w(f2 y, f2 a, f2 dl2, f2 rA) {
-  const f2 big = mul2(add2(a, splat2(-1.f)), rA);
-  f2 q = fma2(splat2(kBwdW5), y, splat2(kBwdW4));
-  q = fma2(q, y, splat2(kBwdW3));
-  q = fma2(q, y, splat2(kBwdW2));
-  q = fma2(q, y, splat2(kBwdW1));
-  q = fma2(q, y, splat2(1.f));
-  return zoh_select(y, mul2(q, dl2), big, kBwdWSmall);
-}
-__device__ __forceinline__ f2 zoh_y(f2 y, f2 a, f2 w, f2 dl2, f2 rA) {
-  const f2 big = mul2(fma2(w, splat2(-1.f), mul2(dl2, a)), rA);
-  f2 q = fma2(splat2(kBwdP7), y, splat2(kBwdP6));
-  q = fma2(q, y, splat2(kBwdP5));
-  q = fma2(q, y, splat2(kBwdP4));
-  q = fma2(q, y, splat2(kBwdP3));
-  q = fma2(q, y, splat2(kBwdP2));
-  q = fma2(q, y, splat2(kBwdP1));
-  q = fma2(q, y, splat2(kBwdP0));
-  return zoh_select(y, mul2(q, mul2(dl2, dl2)), big, kBwdPSmall);
-}
-
 template <typename T, int NP, bool ZOH>
 __global__ void __launch_bounds__(kBW * 32, (NP == 8 || NP == 16) ? 4 : (NP == 4 ? 3 : 2)) k_bwd(BwdParams p) {
   constexpr int S = NP / 4;              // states per lane
@@ -745,7 +700,8 @@ cudaError_t launch_bwd16(int io_dtype, BwdParams &p, cudaStream_t s);
 
 // Channel blocks of the dB/dC partials: 64-channel CTAs of k_bwd16 for
 // d_state 16 with the Euler term, 32-channel CTAs of k_bwd otherwise.
-bool bwd_uses_bwd16(int NP, int zoh) { return NP == 16 && !zoh; }
+// d_state 9..16 (padded to 16) takes the d_state-16 kernel, Euler or exact ZOH
+bool bwd_uses_bwd16(int NP, int /*zoh*/) { return NP == 16; }
 
 int64_t bwd_blocks(int64_t dim, int NP, int zoh) {
   return bwd_uses_bwd16(NP, zoh) ? bwd16_blocks(dim) : (dim + kBW * kBCPW - 1) / (kBW * kBCPW);
@@ -769,7 +725,7 @@ cudaError_t launch_bwd(int io_dtype, int NP, BwdParams &p, cudaStream_t s) {
       return cudaGetLastError();
     };
     if constexpr (kNP == 16) {
-      e = p.zoh ? general(k_bwd<T, kNP, true>) : launch_bwd16(io_dtype, p, s);
+      e = launch_bwd16(io_dtype, p, s);  // Euler and exact ZOH
     } else {
       e = p.zoh ? general(k_bwd<T, kNP, true>) : general(k_bwd<T, kNP, false>);
     }

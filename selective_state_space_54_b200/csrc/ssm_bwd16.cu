@@ -9,6 +9,11 @@
 //   dA_n  = sum_{b,t} g_tn Delta_t a_tn h_{t-1,n}
 //   dDelta_t = sum_n g_tn (A_n a_tn h_{t-1,n} + B_tn u_t),  ddelta_t = dDelta_t sigmoid(s_t)
 //   du_t  = dy_t D + Delta_t sum_n g_tn B_tn,  dD = sum dy_t u_t,  ddelta_bias = sum ddelta_t
+// With the exact zero-order hold the input term Delta_t u_t B_tn becomes
+// u_t W_tn B_tn, W = Delta (e^x - 1)/x with x = Delta A_n (reading guide,
+// "Metodo"): dB_tn = sum_d g u W, du_t = dy_t D + sum_n g W B, the input
+// term's part of dDelta_t is u_t sum_n g a B, and dA_n gains
+// sum g u B Delta^2 psi(x), psi(x) = (x e^x - (e^x - 1))/x^2.
 // The states are recomputed from the state entering each 8-step chunk, never
 // stored for every step ("Mamba: Linear-Time Sequence Modeling with Selective
 // State Spaces" reading guide, "Expansao de Estado Ciente de Hardware":
@@ -179,10 +184,11 @@ __device__ __forceinline__ void q_put(uint16_t &dst, float v) {
 __device__ __forceinline__ void q_put(float &dst, float v) { dst = v; }
 
 // Per (channel, step) quantities of chunk k into the stage.  FULL adds what
-// the reverse pass needs (dy, the gate and softplus derivatives, u).
+// the reverse pass needs (dy, the gate and softplus derivatives, u).  ZOH:
+// the (v, v) row du2 holds u instead of Delta u.
 // Thread tid takes channel tid / 2 and steps 4 (tid % 2) .. +3.  Returns this
 // thread's contribution to dD (sum of dy u).
-template <typename T, bool FULL, bool TOK>
+template <typename T, bool FULL, bool TOK, bool ZOH>
 __device__ __forceinline__ float q_prepass(const BwdParams &p, QRaw<T> &raw, QStage &st, int64_t cb,
                                            int64_t k, float bias, float Dd) {
   const int tid = threadIdx.x, pc = tid >> 1, t4 = (tid & 1) * 4;
@@ -206,7 +212,7 @@ __device__ __forceinline__ float q_prepass(const BwdParams &p, QRaw<T> &raw, QSt
     }
     dl = in ? dl : 0.f;
     st.dl2[t][pc] = splat2(dl);
-    st.du2[t][pc] = splat2(dl * u);
+    st.du2[t][pc] = splat2(ZOH ? u : dl * u);
     if (FULL) {
       const float o = in ? q_f(raw.act[3][at<TOK>(pc, t)]) : 0.f;
       float dy = o, fz = 0.f;
@@ -234,7 +240,9 @@ __device__ __forceinline__ float q_prepass(const BwdParams &p, QRaw<T> &raw, QSt
   return dD;
 }
 
-template <typename T, bool TOK>
+// ZOH: the exact zero-order-hold input term u W B, W = Delta (e^x - 1)/x
+// (zoh_w / zoh_y, ssm_common.cuh), a separate instantiation
+template <typename T, bool TOK, bool ZOH>
 __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   QSmem<T> &sm = *reinterpret_cast<QSmem<T> *>(smem_raw);
@@ -255,14 +263,16 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
   }
   // A * log2(e) of the lane's states, per channel, as pairs
   f2 A2[2][2];
+  f2 rA[ZOH ? 2 : 1][2];  // exact ZOH: 1 / A_n (infinite for A_n = 0, whose x is 0)
 #pragma unroll
   for (int c = 0; c < 2; ++c)
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int n = 4 * j + 2 * q;  // padded states (n >= N) have A = B = C = 0
-      const float a0 = (cvalid[c] && n < p.N) ? p.A[(d0 + c) * p.N + n] * kLog2e : 0.f;
-      const float a1 = (cvalid[c] && n + 1 < p.N) ? p.A[(d0 + c) * p.N + n + 1] * kLog2e : 0.f;
-      A2[c][q] = pack2(a0, a1);
+      const float a0 = (cvalid[c] && n < p.N) ? p.A[(d0 + c) * p.N + n] : 0.f;
+      const float a1 = (cvalid[c] && n + 1 < p.N) ? p.A[(d0 + c) * p.N + n + 1] : 0.f;
+      A2[c][q] = pack2(a0 * kLog2e, a1 * kLog2e);
+      if constexpr (ZOH) rA[c][q] = pack2(__frcp_rn(a0), __frcp_rn(a1));
     }
   // the pre-pass thread's channel
   const int64_t pd = cb * kQC + (tid >> 1);
@@ -278,6 +288,12 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
     const ulonglong2 v = *reinterpret_cast<const ulonglong2 *>(&arr[t][4 * j]);
     x0 = v.x;
     x1 = v.y;
+  };
+  // the input term of state pair (c, q): Delta u B (Euler; du = Delta u) or
+  // u W B (exact ZOH; du = u); xx = Delta A log2(e), a = its exp2
+  auto bterm = [&](f2 dl, f2 du, f2 xx, f2 a, int c, int q, f2 Bq) -> f2 {
+    if constexpr (ZOH) return mul2(mul2(du, zoh_w(xx, a, dl, rA[ZOH ? c : 0][q])), Bq);
+    else return mul2(du, Bq);
   };
   float *ck_base[2];
 #pragma unroll
@@ -304,7 +320,7 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
       q_wait_all();
       __syncthreads();
       if (k + 1 < K) q_fetch<T, false, TOK>(p, sm.raw[(k + 1) & 1], b, cb, k + 1);
-      q_prepass<T, false, TOK>(p, sm.raw[k & 1], st, cb, k, pbias, pD);
+      q_prepass<T, false, TOK, ZOH>(p, sm.raw[k & 1], st, cb, k, pbias, pD);
       __syncthreads();
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -319,9 +335,11 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
+            const f2 xx = mul2(dl[c], A2[c][q]);
             float x0, x1;
-            unpack2(mul2(dl[c], A2[c][q]), x0, x1);
-            h[c][q] = fma2(pack2(ex2(x0), ex2(x1)), h[c][q], mul2(du[c], B[q]));
+            unpack2(xx, x0, x1);
+            const f2 a = pack2(ex2(x0), ex2(x1));
+            h[c][q] = fma2(a, h[c][q], bterm(dl[c], du[c], xx, a, c, q, B[q]));
           }
       }
     }
@@ -348,7 +366,7 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
     q_wait_all();
     __syncthreads();
     if (k > 0) q_fetch<T, true, TOK>(p, sm.raw[(k - 1) & 1], b, cb, k - 1);
-    dD_acc += q_prepass<T, true, TOK>(p, raw, st, cb, k, pbias, pD);
+    dD_acc += q_prepass<T, true, TOK, ZOH>(p, raw, st, cb, k, pbias, pD);
     __syncthreads();
 
     // (3) the chunk's states from its entry state; keep the entry of every 2-step group
@@ -376,9 +394,11 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
+            const f2 xx = mul2(dl[c], A2[c][q]);
             float x0, x1;
-            unpack2(mul2(dl[c], A2[c][q]), x0, x1);
-            h[c][q] = fma2(pack2(ex2(x0), ex2(x1)), h[c][q], mul2(du[c], B[q]));
+            unpack2(xx, x0, x1);
+            const f2 a = pack2(ex2(x0), ex2(x1));
+            h[c][q] = fma2(a, h[c][q], bterm(dl[c], du[c], xx, a, c, q, B[q]));
           }
       }
 #pragma unroll
@@ -410,10 +430,12 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
         for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
+            const f2 xx = mul2(dl[c], A2[c][q]);
             float x0, x1;
-            unpack2(mul2(dl[c], A2[c][q]), x0, x1);
+            unpack2(xx, x0, x1);
             as[s][c][q] = pack2(ex2(x0), ex2(x1));
-            hs[s][c][q] = fma2(as[s][c][q], s ? hs[0][c][q] : he[c][q], mul2(du[c], B[q]));
+            hs[s][c][q] = fma2(as[s][c][q], s ? hs[0][c][q] : he[c][q],
+                               bterm(dl[c], du[c], xx, as[s][c][q], c, q, B[q]));
           }
           float lo, hi;
           unpack2(fma2(C[1], hs[s][c][1], mul2(C[0], hs[s][c][0])), lo, hi);
@@ -433,7 +455,7 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
         q_put(raw.act[2][at<TOK>(ch, t)], yss * st.fz[t][ch]);
       }
       // the reverse recurrence over the group's 2 steps
-      float ddv[2][2], s1v[2][2];
+      float ddv[2][2], s1v[2][2], s2v[ZOH ? 2 : 1][2];
 #pragma unroll
       for (int s = 1; s >= 0; --s) {
         const int t = tg + s;
@@ -446,15 +468,29 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
         f2 dBp[2], dCp[2];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          f2 dd, s1;
+          f2 dd, s1, s2;
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             g[c][q] = fma2(dy[c], C[q], g[c][q]);
             dCp[q] = c ? fma2(dy[c], hs[s][c][q], dCp[q]) : mul2(dy[c], hs[s][c][q]);
-            s1 = q ? fma2(g[c][q], B[q], s1) : mul2(g[c][q], B[q]);
-            dBp[q] = c ? fma2(g[c][q], du[c], dBp[q]) : mul2(g[c][q], du[c]);
+            if constexpr (ZOH) {
+              // input term u W B: its u derivative W B (s1 = sum_n g W B is du's sum,
+              // Delta included), its B derivative u W, its A derivative u Y B
+              const f2 xx = mul2(dl[c], A2[c][q]);
+              const f2 W = zoh_w(xx, as[s][c][q], dl[c], rA[ZOH ? c : 0][q]);
+              const f2 gB = mul2(g[c][q], B[q]);
+              s1 = q ? fma2(gB, W, s1) : mul2(gB, W);
+              const f2 uW = mul2(du[c], W);
+              dBp[q] = c ? fma2(g[c][q], uW, dBp[q]) : mul2(g[c][q], uW);
+              dA[c][q] = fma2(mul2(gB, zoh_y(xx, as[s][c][q], W, dl[c], rA[ZOH ? c : 0][q])), du[c], dA[c][q]);
+            } else {
+              s1 = q ? fma2(g[c][q], B[q], s1) : mul2(g[c][q], B[q]);
+              dBp[q] = c ? fma2(g[c][q], du[c], dBp[q]) : mul2(g[c][q], du[c]);
+            }
             // g a_t is both dL/dh_{t-1} and the factor of h_{t-1} in dA and dDelta
             g[c][q] = mul2(g[c][q], as[s][c][q]);
+            // exact ZOH: the input term's Delta derivative is a u B (s2 = sum_n g a B)
+            if constexpr (ZOH) s2 = q ? fma2(g[c][q], B[q], s2) : mul2(g[c][q], B[q]);
             const f2 qv = mul2(g[c][q], s ? hs[0][c][q] : he[c][q]);  // g a_t h_{t-1}
             dA[c][q] = fma2(dl[c], qv, dA[c][q]);
             dd = q ? fma2(A2[c][q], qv, dd) : mul2(A2[c][q], qv);
@@ -464,6 +500,10 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
           ddv[s][c] = lo + hi;
           unpack2(s1, lo, hi);
           s1v[s][c] = lo + hi;
+          if constexpr (ZOH) {
+            unpack2(s2, lo, hi);
+            s2v[ZOH ? s : 0][c] = lo + hi;
+          }
         }
         // dB, dC over the warp's 8 channel pairs: lane keeps output my_out
         f2 k0 = hi16 ? dCp[0] : dBp[0], k1 = hi16 ? dCp[1] : dBp[1];
@@ -489,12 +529,22 @@ __global__ void __launch_bounds__(kQThreads, 16 / kQW) k_bwd16(BwdParams p) {
         float ddsum = my_c ? a1 : a0, s1sum = my_c ? b1 : b0;
         ddsum += __shfl_xor_sync(0xffffffffu, my_c ? a0 : a1, 1);
         s1sum += __shfl_xor_sync(0xffffffffu, my_c ? b0 : b1, 1);
+        // exact ZOH: the Delta derivative's input part is u sum_n g a B (s2)
+        float s2sum = s1sum;
+        if constexpr (ZOH) {
+          float e0 = up ? s2v[ZOH ? 1 : 0][0] : s2v[0][0], e1 = up ? s2v[ZOH ? 1 : 0][1] : s2v[0][1];
+          e0 += __shfl_xor_sync(0xffffffffu, up ? s2v[0][0] : s2v[ZOH ? 1 : 0][0], 2);
+          e1 += __shfl_xor_sync(0xffffffffu, up ? s2v[0][1] : s2v[ZOH ? 1 : 0][1], 2);
+          s2sum = my_c ? e1 : e0;
+          s2sum += __shfl_xor_sync(0xffffffffu, my_c ? e0 : e1, 1);
+        }
         const int t = tg + my_s, ch = ch0 + my_c;
         float dlv, dlv_hi, dyv, dyv_hi;
         unpack2(st.dl2[t][ch], dlv, dlv_hi);
         unpack2(st.dy2[t][ch], dyv, dyv_hi);
-        const float du_v = fmaf(dlv, s1sum, dyv * (my_c ? Dd[1] : Dd[0]));
-        const float ddl = st.sg[t][ch] * fmaf(st.uu[t][ch], s1sum, kLn2f * ddsum);
+        // du = Delta sum g B + D dy (Euler); sum g W B + D dy (exact ZOH: W holds Delta)
+        const float du_v = fmaf(ZOH ? 1.f : dlv, s1sum, dyv * (my_c ? Dd[1] : Dd[0]));
+        const float ddl = st.sg[t][ch] * fmaf(st.uu[t][ch], s2sum, kLn2f * ddsum);
         q_put(raw.act[0][at<TOK>(ch, t)], du_v);
         q_put(raw.act[1][at<TOK>(ch, t)], ddl);
         dbias_acc += ddl;
@@ -586,10 +636,15 @@ cudaError_t launch_bwd16(int io_dtype, BwdParams &p, cudaStream_t s) {
     kern<<<(unsigned)(p.batch * p.cpb), kQThreads, smem, s>>>(p);
     return cudaGetLastError();
   };
-  if (io_dtype == 1)
-    return p.tok ? go(k_bwd16<uint16_t, true>, sizeof(QSmem<uint16_t>))
-                 : go(k_bwd16<uint16_t, false>, sizeof(QSmem<uint16_t>));
-  if (io_dtype == 0 && !p.tok) return go(k_bwd16<float, false>, sizeof(QSmem<float>));
+  if (p.tok && p.zoh) return cudaErrorInvalidValue;  // no forward writes that combination
+  if (io_dtype == 1) {
+    if (p.tok) return go(k_bwd16<uint16_t, true, false>, sizeof(QSmem<uint16_t>));
+    return p.zoh ? go(k_bwd16<uint16_t, false, true>, sizeof(QSmem<uint16_t>))
+                 : go(k_bwd16<uint16_t, false, false>, sizeof(QSmem<uint16_t>));
+  }
+  if (io_dtype == 0 && !p.tok)
+    return p.zoh ? go(k_bwd16<float, false, true>, sizeof(QSmem<float>))
+                 : go(k_bwd16<float, false, false>, sizeof(QSmem<float>));
   return cudaErrorInvalidValue;
 }
 

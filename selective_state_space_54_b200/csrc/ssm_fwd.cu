@@ -724,16 +724,6 @@ struct Share {
   }
 };
 
-// Exact ZOH in the warp-specialised consumer: (e^x - 1)/x = sum_k x^k/(k+1)!
-// evaluated in the ex2 argument x / ln 2, so term k carries ln2^k / (k+1)!;
-// used for |x| < 1/4, i.e. |x / ln 2| < 0.25 / ln 2.
-constexpr float kZohT1 = 3.465735903e-01f;  // ln2 / 2!
-constexpr float kZohT2 = 8.007550232e-02f;  // ln2^2 / 3!
-constexpr float kZohT3 = 1.387602717e-02f;  // ln2^3 / 4!
-constexpr float kZohT4 = 1.923625822e-03f;  // ln2^4 / 5!
-constexpr float kZohT5 = 2.222259691e-04f;  // ln2^5 / 6!
-constexpr float kZohSmall = 3.606737602e-01f;  // 0.25 / ln2
-
 template <typename T, int NP, int LPC, bool ZOH, bool SAVE>
 __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP, LPC> &sm, int64_t w,
                                             const Share &sh, unsigned bar_full, unsigned bar_ys) {
@@ -822,23 +812,10 @@ __device__ __forceinline__ void ws_consumer(const FwdParams &p, WSPair<T, NP, LP
             const float a0 = ex2(x0), a1 = ex2(x1);
             const f2 a = pack2(a0, a1);
             if constexpr (ZOH) {
-              // exact zero-order hold: Delta u (e^x - 1)/x B.  Delta (e^x - 1)/x is
-              // (e^x - 1) / A_n for |x| >= 1/4 (Delta cancels; e^x - 1 loses at most
-              // 4 ulp of e^x there), else Delta times the Taylor series of
-              // (e^x - 1)/x to x^5 (remainder below 5e-8).  The stage holds u
-              // itself in this instantiation.
-              const f2 big = mul2(add2(a, splat2(-1.f)), rA[s / 2]);
-              f2 q = fma2(splat2(kZohT5), xx, splat2(kZohT4));
-              q = fma2(q, xx, splat2(kZohT3));
-              q = fma2(q, xx, splat2(kZohT2));
-              q = fma2(q, xx, splat2(kZohT1));
-              q = fma2(q, xx, splat2(1.f));
-              const f2 small = mul2(q, dl2);
-              float b0, b1, s0, s1;
-              unpack2(big, b0, b1);
-              unpack2(small, s0, s1);
-              const f2 wz = pack2(fabsf(x0) < kZohSmall ? s0 : b0, fabsf(x1) < kZohSmall ? s1 : b1);
-              hp[s / 2] = fma2(a, hp[s / 2], mul2(mul2(wz, du2), bv));
+              // exact zero-order hold: u W B with W = Delta (e^x - 1)/x, formed
+              // without a reciprocal per element (zoh_w); the stage holds u
+              // itself in this instantiation
+              hp[s / 2] = fma2(a, hp[s / 2], mul2(mul2(zoh_w(xx, a, dl2, rA[s / 2]), du2), bv));
             } else {
               hp[s / 2] = fma2(a, hp[s / 2], mul2(du2, bv));
             }

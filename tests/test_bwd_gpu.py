@@ -82,15 +82,15 @@ def test_bwd_initial_state_gradient(cuda_device):
     _check(case, cuda_device, h0=h0)
 
 
-@pytest.mark.parametrize("N", [16, 8])
-def test_bwd_bitwise_repeatable(cuda_device, N):
+@pytest.mark.parametrize("N,zoh", [(16, False), (8, False), (16, True), (8, True)])
+def test_bwd_bitwise_repeatable(cuda_device, N, zoh):
     # every sum over channels, steps or the batch is formed in a fixed order
     # (per-block partials added by a separate pass, no atomics): two runs give
     # bitwise-equal gradients, the cross-channel ones included
     case = _case(3, 200, 777, N, synth.BF16, 7)
     h0 = np.random.default_rng(8).standard_normal((3, 200, N)).astype(np.float32)
-    a = _bwd(case, cuda_device, h0=h0, want_dh0=True)
-    b = _bwd(case, cuda_device, h0=h0, want_dh0=True)
+    a = _bwd(case, cuda_device, h0=h0, want_dh0=True, zoh=zoh)
+    b = _bwd(case, cuda_device, h0=h0, want_dh0=True, zoh=zoh)
     for k in GRADS + ("dinitial_state",):
         assert np.array_equal(a[k], b[k]), k
 
@@ -160,7 +160,7 @@ def test_bwd_full_mamba_1p4b_layer_with_saved_states(cuda_device):
 
 # ---- the exact zero-order-hold input term (reading guide, "Metodo") ----------
 @pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
-@pytest.mark.parametrize("N", [1, 4, 16, 32])
+@pytest.mark.parametrize("N", [1, 4, 12, 16, 32])
 def test_bwd_zoh_exact(cuda_device, dtype, N):
     # 40 channels (a partial block), 333 steps (a partial chunk), an initial state
     case = _case(2, 40, 333, N, dtype, 650 + N)

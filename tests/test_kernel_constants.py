@@ -91,10 +91,11 @@ def test_reciprocal_seed_and_newton_steps():
 
 
 def _zoh_constants():
-    src = open(os.path.join(CSRC, "ssm_fwd.cu")).read()
+    src = open(os.path.join(CSRC, "ssm_common.cuh")).read()
     got = {}
-    for name in ("kZohT1", "kZohT2", "kZohT3", "kZohT4", "kZohT5", "kZohSmall"):
-        m = re.search(r"constexpr float " + name + r" = " + FLOAT, src)
+    for name in ([f"kZohW{k}" for k in range(1, 6)] + [f"kZohP{m}" for m in range(8)]
+                 + ["kZohWSmall", "kZohPSmall"]):
+        m = re.search(r"\b" + name + r" = " + FLOAT, src)
         assert m, name
         got[name] = float(m.group(1))
     return got
@@ -108,8 +109,8 @@ def test_zoh_series_coefficients():
     c = _zoh_constants()
     for k in range(1, 6):
         ref = math.log(2) ** k / math.factorial(k + 1)
-        assert abs(c[f"kZohT{k}"] - ref) <= 2 ** -23 * ref, (k, c[f"kZohT{k}"], ref)
-    assert abs(c["kZohSmall"] - 0.25 / math.log(2)) <= 2 ** -23
+        assert abs(c[f"kZohW{k}"] - ref) <= 2 ** -23 * ref, (k, c[f"kZohW{k}"], ref)
+    assert abs(c["kZohWSmall"] - 0.25 / math.log(2)) <= 2 ** -23
 
 
 def test_zoh_two_branch_error_bound():
@@ -118,7 +119,7 @@ def test_zoh_two_branch_error_bound():
     # fp32 with a perturbed by the ex2 unit's error (up to 2 ulp, either sign),
     # relative to the exact value: below 1e-6 everywhere.
     c = _zoh_constants()
-    T = [np.float32(c[f"kZohT{k}"]) for k in range(5, 0, -1)]
+    T = [np.float32(c[f"kZohW{k}"]) for k in range(5, 0, -1)]
     x = np.concatenate([-np.geomspace(1e-8, 60.0, 40001), np.geomspace(1e-8, 10.0, 20001)])
     y = (x / np.log(2)).astype(np.float32)
     exact = np.expm1(x) / x
@@ -131,34 +132,27 @@ def test_zoh_two_branch_error_bound():
         a = (np.exp2(y.astype(np.float64)) * (1 + ulps * 2.0 ** -24)).astype(np.float32)
         # Delta = 1, A = x: (a - 1) * (1/A) against the series
         big = ((a - np.float32(1)).astype(np.float32) * (np.float32(1) / x.astype(np.float32))).astype(np.float32)
-        got = np.where(np.abs(y) < np.float32(c["kZohSmall"]), q, big).astype(np.float64)
+        got = np.where(np.abs(y) < np.float32(c["kZohWSmall"]), q, big).astype(np.float64)
         worst = max(worst, float(np.max(np.abs(got / exact - 1))))
     assert worst < 1e-6, worst
 
 
-def test_backward_zoh_series_coefficients():
-    # the general backward's exact-ZOH series, in y = x / ln 2: W's terms
-    # ln2^k / (k+1)! (switch at |x| = 1/4) and psi's terms ln2^m (m+1)/(m+2)!
-    # (switch at |x| = 1/2), psi(x) = (x e^x - (e^x - 1)) / x^2
+def test_psi_series_coefficients():
+    # the backward's A derivative Delta^2 psi(x), psi(x) = (x e^x - (e^x - 1)) / x^2:
+    # its series terms ln2^m (m+1)/(m+2)! in y = x / ln 2 (switch at |x| = 1/2),
+    # and the series against the closed form where that is accurate
     import math
-    src = open(os.path.join(CSRC, "ssm_bwd.cu")).read()
-    val = lambda name: float(re.search(name + r" = " + FLOAT, src).group(1))
+    c = _zoh_constants()
     ln2 = math.log(2)
-    for k in range(1, 6):
-        ref = ln2 ** k / math.factorial(k + 1)
-        assert abs(val(f"kBwdW{k}") - ref) <= 2 ** -23 * ref, k
     for m in range(8):
         ref = ln2 ** m * (m + 1) / math.factorial(m + 2)
-        assert abs(val(f"kBwdP{m}") - ref) <= 2 ** -23 * ref, m
-    assert abs(val("kBwdWSmall") - 0.25 / ln2) <= 2 ** -23
-    assert abs(val("kBwdPSmall") - 0.5 / ln2) <= 2 ** -22
-    # the psi series against the closed form where that is accurate, and its
-    # remainder at the switch below 1e-8 relative
+        assert abs(c[f"kZohP{m}"] - ref) <= 2 ** -23 * ref, m
+    assert abs(c["kZohPSmall"] - 0.5 / ln2) <= 2 ** -22
     x = np.linspace(-0.5, 0.5, 2001)
     x = x[np.abs(x) > 1e-3]
     y = x / ln2
     q = np.zeros_like(y)
     for m in range(7, -1, -1):
-        q = q * y + val(f"kBwdP{m}")
+        q = q * y + c[f"kZohP{m}"]
     exact = (x * np.exp(x) - np.expm1(x)) / x ** 2
     assert np.max(np.abs(q / exact - 1)) < 1e-7
