@@ -3,6 +3,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include "ssm_common.cuh"
 #include "ssm_scan.h"
 
@@ -180,14 +182,34 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
       p.total = round_up(p.off_bcf + 2 * sizeof(float) * (size_t)s->batch * (size_t)s->seqlen * p.NP, 256);
     }
   } else if (path == SSM_PATH_SPLIT_L) {
-    // about two waves of resident warps; segments of at least 4 chunks
-    int64_t target = 2 * slots;
-    int64_t segs = (target + G - 1) / G;
-    int64_t max_segs = p.K / 4 > 1 ? p.K / 4 : 1;
-    if (segs > max_segs) segs = max_segs;
-    if (segs < 2 && p.K >= 2) segs = 2;
-    if (segs < 1) segs = 1;
-    p.seg_chunks = (p.K + segs - 1) / segs;
+    // Segments per group.  Both passes launch one warp per (group, segment)
+    // item: pass 1 (end states from zero) at its own occupancy, pass 2 (the
+    // output pass, more registers) at a lower one.  The count minimises the
+    // estimated time  sum over passes of  weight x waves x (segment length +
+    // 2 chunks of per-item start-up), so that neither pass ends on a mostly
+    // idle partial wave (pass 2, which also forms y, weighted 1.3); segments
+    // hold at least 4 chunks, and the search stops at 8 waves of pass 1.
+    int o1 = 0, o2 = 0;
+    if (fwd_segment_occupancy(s->io_dtype, p.NP, lpc, 0, &o1) != cudaSuccess ||
+        fwd_segment_occupancy(s->io_dtype, p.NP, lpc, 1, &o2) != cudaSuccess || o1 <= 0 || o2 <= 0) {
+      cudaGetLastError();
+      return SSM_ERR_CUDA;
+    }
+    const int64_t S1 = (int64_t)sms * o1 * kWarps, S2 = (int64_t)sms * o2 * kWarps;
+    const int64_t max_segs = p.K / 4 > 1 ? p.K / 4 : 1;
+    const int64_t min_segs = p.K >= 2 ? 2 : 1;
+    const int64_t last = std::min(max_segs, std::max(min_segs, 8 * S1 / G));
+    int64_t best = min_segs;
+    double best_cost = 1e300;
+    for (int64_t segs = min_segs; segs <= last; ++segs) {
+      const int64_t sc = (p.K + segs - 1) / segs, ns = (p.K + sc - 1) / sc, items = G * ns;
+      const double cost = (double)(sc + 2) * ((double)((items + S1 - 1) / S1) + 1.3 * (double)((items + S2 - 1) / S2));
+      if (cost < best_cost * (1 - 1e-9)) {
+        best_cost = cost;
+        best = segs;
+      }
+    }
+    p.seg_chunks = (p.K + best - 1) / best;
     p.n_segs = (p.K + p.seg_chunks - 1) / p.seg_chunks;
     const size_t items = (size_t)G * (size_t)p.n_segs;
     p.off_seg_h = kHeaderBytes;

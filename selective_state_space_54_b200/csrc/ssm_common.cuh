@@ -423,6 +423,7 @@ __device__ __forceinline__ bool warp_wait_flag(const unsigned *flag, unsigned *e
 // ---- launchers (defined in ssm_fwd.cu / ssm_bwd.cu) ----------------------------
 int fwd_np_for(int64_t N);
 cudaError_t fwd_occupancy(int io_dtype, int NP, int LPC, int zoh, int *ctas_per_sm);
+cudaError_t fwd_segment_occupancy(int io_dtype, int NP, int LPC, int emit, int *ctas_per_sm);
 cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s);
 int fwd_ws_chunk();

@@ -1279,6 +1279,19 @@ cudaError_t launch_fwd_lookback(int io_dtype, int NP, int LPC, const FwdParams &
   });
 }
 
+// CTAs per SM of the split-L pass (emit = 0: segment end states; 1: the output pass)
+cudaError_t fwd_segment_occupancy(int io_dtype, int NP, int LPC, int emit, int *ctas_per_sm) {
+  return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
+    using T = typename decltype(tt)::type;
+    constexpr int kNP = decltype(np)::value, kLPC = decltype(lpc)::value;
+    const size_t smem = fwd_smem_bytes<kNP, kLPC>();
+    auto kern = emit ? k_fwd_segment<T, kNP, kLPC, true> : k_fwd_segment<T, kNP, kLPC, false>;
+    cudaError_t e = allow_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, kern, kThreads, smem);
+  });
+}
+
 cudaError_t launch_fwd_splitl(int io_dtype, int NP, int LPC, const FwdParams &p, cudaStream_t s) {
   return dispatch(io_dtype, NP, LPC, [&](auto tt, auto np, auto lpc) -> cudaError_t {
     using T = typename decltype(tt)::type;
