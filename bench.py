@@ -62,6 +62,8 @@ def parse():
                     choices=["auto", "lookback", "split_l", "per_group", "lookback_ws"])
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling only)")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (smaller cases for profiling only)")
     return ap.parse_args()
 
 
@@ -652,6 +654,10 @@ def main():
     if args.batch:
         import dataclasses
         w = dataclasses.replace(w, batch=args.batch, name=f"{w.name}[batch={args.batch}]")
+    if args.seqlen:
+        import dataclasses
+        w = dataclasses.replace(w, seqlen=args.seqlen, name=f"{w.name}[seqlen={args.seqlen}]")
+    args.reduced = bool(args.batch or args.seqlen)  # a profiling case: no sub-records
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -753,7 +759,7 @@ def main():
 
     # the same forward on token-major activations (batch, seqlen, d_inner)
     tok = None
-    if not args.no_bwd and not args.batch and w.dtype == synth.BF16 and w.dim % 8 == 0:
+    if not args.no_bwd and not args.reduced and w.dtype == synth.BF16 and w.dim % 8 == 0:
         tm = {k: g[k].transpose(1, 2).contiguous() for k in ("u", "delta", "z")}
         y_tm = torch.empty_like(tm["u"])
 
@@ -779,7 +785,7 @@ def main():
 
     # the same forward with the exact zero-order-hold input term, Delta u (e^x - 1)/x B
     zoh = None
-    if not args.no_bwd and not args.batch:
+    if not args.no_bwd and not args.reduced:
         def step_zoh():
             ssm.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
                          g["delta_bias"], y=y, last_state=ls, return_last_state=True,
@@ -869,7 +875,7 @@ def main():
         del host, dbuf
 
     bwd = dec = conv = m130 = mlen = None
-    if not args.no_bwd and not args.batch:
+    if not args.no_bwd and not args.reduced:
         m130 = measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks,
                                "mamba-130m-layer")
         mlen = measure_forward(ssm, torch, dev, args, world, barrier, max_over_ranks,
