@@ -302,6 +302,15 @@ ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream);
 ssm_status ssm_scan_test_wait_timeout(void *workspace, size_t ws_bytes,
                                       int64_t timeout_us, ssm_stream_t stream);
 
+/* Test hook for callers' error paths: the next `count` calls of
+ * ssm_scan_fwd, ssm_scan_bwd, ssm_scan_step, ssm_causal_conv1d and
+ * ssm_causal_conv1d_bwd (ssm_scan_fwd_noalloc included) that pass their
+ * argument and workspace checks return SSM_ERR_CUDA as if their first launch
+ * had failed with cudaErrorLaunchFailure; they launch nothing and leave every
+ * buffer untouched.  count <= 0 disarms it.  Process-wide, thread-safe;
+ * failures are consumed in call order. */
+void ssm_scan_test_fail_next(int32_t count);
+
 /* Path AUTO would choose for `shape` on the current device (for tests and
  * the benchmark); SSM_PATH_AUTO itself for an invalid shape. */
 int32_t ssm_scan_fwd_path(const ssm_shape *shape);

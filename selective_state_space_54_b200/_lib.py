@@ -39,7 +39,7 @@ EXPORTS = (
     "ssm_scan_fwd_workspace_bytes", "ssm_scan_bwd_workspace_bytes", "ssm_scan_fwd",
     "ssm_scan_bwd", "ssm_scan_check", "ssm_scan_test_wait_timeout", "ssm_scan_fwd_path",
     "ssm_status_string", "ssm_scan_version", "ssm_scan_fwd_noalloc", "ssm_scan_step",
-    "ssm_causal_conv1d", "ssm_causal_conv1d_bwd",
+    "ssm_causal_conv1d", "ssm_causal_conv1d_bwd", "ssm_scan_test_fail_next",
 )
 
 
@@ -88,6 +88,8 @@ def load(path: str | None = None):
     lib.ssm_scan_check.restype = ci
     lib.ssm_scan_test_wait_timeout.argtypes = [vp, sz, i64, vp]
     lib.ssm_scan_test_wait_timeout.restype = ci
+    lib.ssm_scan_test_fail_next.argtypes = [i32]
+    lib.ssm_scan_test_fail_next.restype = None
     lib.ssm_scan_fwd_path.argtypes = [shp]
     lib.ssm_scan_fwd_path.restype = i32
     lib.ssm_status_string.argtypes = [ci]

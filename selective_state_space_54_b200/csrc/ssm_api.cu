@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "ssm_common.cuh"
 #include "ssm_scan.h"
@@ -224,6 +225,19 @@ ssm_status make_fwd_plan(const ssm_shape *s, FwdPlan *pl) {
   return SSM_OK;
 }
 
+// Test hook (ssm_scan_test_fail_next): the number of upcoming entry-point
+// calls that report a launch failure instead of launching.
+std::atomic<int32_t> g_fail_next{0};
+
+// Consumes one armed failure: cudaErrorLaunchFailure in place of the call's
+// first launch (nothing is launched), else cudaSuccess.
+cudaError_t injected_failure() {
+  int32_t v = g_fail_next.load();
+  while (v > 0 && !g_fail_next.compare_exchange_weak(v, v - 1)) {
+  }
+  return v > 0 ? cudaErrorLaunchFailure : cudaSuccess;
+}
+
 ssm_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return SSM_OK;
   fprintf(stderr, "ssm_scan: CUDA error %s\n", cudaGetErrorString(e));
@@ -340,7 +354,8 @@ ssm_status ssm_scan_fwd(const ssm_shape *shape, const void *u, const void *delta
 
   // the error word starts clear on every path, so that ssm_scan_check reads
   // this call's status whatever the workspace held before
-  cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
+  cudaError_t e = injected_failure();
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
   if (e != cudaSuccess) return cuda_status(e);
   if (pl.path == SSM_PATH_LOOKBACK || pl.path == SSM_PATH_LOOKBACK_WS) {
     p.flags = reinterpret_cast<unsigned *>(ws + pl.off_flags);
@@ -392,6 +407,8 @@ ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delt
   p.zoh = (shape->flags & SSM_FLAG_ZOH_EXACT) ? 1 : 0;
   p.vec = shape->dstate % 4 == 0 && aligned(state, 16) && aligned(A, 16) &&
           aligned(B, 4 * es) && aligned(C, 4 * es);
+  const cudaError_t inj = injected_failure();
+  if (inj != cudaSuccess) return cuda_status(inj);
   return cuda_status(launch_step(shape->io_dtype, p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -423,6 +440,8 @@ ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t
   p.x = x; p.w = weight; p.bias = bias; p.s0 = initial_state; p.out = out; p.s1 = final_state;
   p.batch = batch; p.dim = dim; p.L = seqlen; p.K = width; p.silu = silu ? 1 : 0;
   p.vec = ((seqlen * (int64_t)es) % 16 == 0) && aligned(x, 16) && aligned(out, 16);
+  const cudaError_t inj = injected_failure();
+  if (inj != cudaSuccess) return cuda_status(inj);
   return cuda_status(launch_conv(io_dtype, p, s));
 }
 
@@ -458,6 +477,8 @@ ssm_status ssm_causal_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int
   p.dx = dx; p.dw = dweight; p.dbias = dbias; p.ds0 = dinitial_state;
   p.batch = batch; p.dim = dim; p.L = seqlen; p.K = width; p.silu = silu ? 1 : 0;
   p.vec = ((seqlen * (int64_t)es) % 16 == 0) && aligned(x, 16) && aligned(dout, 16) && aligned(dx, 16);
+  const cudaError_t inj = injected_failure();
+  if (inj != cudaSuccess) return cuda_status(inj);
   return cuda_status(launch_conv_bwd(io_dtype, p, s));
 }
 
@@ -534,8 +555,12 @@ ssm_status ssm_scan_bwd(const ssm_shape *shape, const void *u, const void *delta
   if (p.tok && !act16) return SSM_ERR_INVALID_ARG;
   p.io_vec = (p.tok || (L * (int64_t)es) % 16 == 0) && act16;
   p.bc_vec = (N == NP) && ((N * (int64_t)es) % 16 == 0) && aligned(B, 16) && aligned(C, 16);
+  const cudaError_t inj = injected_failure();
+  if (inj != cudaSuccess) return cuda_status(inj);
   return cuda_status(launch_bwd(shape->io_dtype, NP, p, s));
 }
+
+void ssm_scan_test_fail_next(int32_t count) { g_fail_next.store(count > 0 ? count : 0); }
 
 ssm_status ssm_scan_check(void *workspace, ssm_stream_t stream) {
   if (!workspace) return SSM_ERR_WORKSPACE;

@@ -339,3 +339,24 @@ def test_bwd_workspace_holds_every_partial(lib, dstate, blk):
         ckpt = 4 * batch * (4 * -(-dim // 64)) * -(-L // 8) * 16 * np_
         parts = 4 * (-(-dim // blk) * batch * L * 2 * np_ + batch * dim * dstate + 2 * batch * dim)
         assert lib.ssm_scan_bwd_workspace_bytes(ctypes.byref(sh)) >= 256 + ckpt + parts
+
+
+def test_injected_launch_failure_is_consumed_in_call_order(lib, capfd):
+    # ssm_scan_test_fail_next: armed failures replace the first launch of the
+    # next calls that pass their checks (nothing is launched); argument errors
+    # come first and do not consume one.  Every call here is either rejected
+    # by its checks or injected, so none launches.
+    conv = lambda batch=2: lib.ssm_causal_conv1d(batch, 4, 64, 4, _lib.SSM_BF16, ctypes.c_void_p(16),
+                                                 ctypes.c_void_p(16), None, None, 1,
+                                                 ctypes.c_void_p(16), None, None)
+    capfd.readouterr()
+    lib.ssm_scan_test_fail_next(2)
+    assert conv(batch=-1) == _lib.SSM_ERR_INVALID_ARG  # checks first: nothing consumed
+    assert conv() == _lib.SSM_ERR_CUDA
+    assert conv() == _lib.SSM_ERR_CUDA
+    err = capfd.readouterr().err
+    assert err.count("launch failure") == 2, err
+    lib.ssm_scan_test_fail_next(1)
+    lib.ssm_scan_test_fail_next(0)  # disarmed
+    assert conv(batch=-1) == _lib.SSM_ERR_INVALID_ARG
+    assert "launch failure" not in capfd.readouterr().err
