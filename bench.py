@@ -207,8 +207,11 @@ def init_dist(args):
     return world, rank, local
 
 
-def cpu_baseline(w: synth.Workload, case: dict, target_s: float = 12.0) -> dict:
-    """The fp64 oracle as it stands, timed on the host cores on a bounded sample."""
+def cpu_baseline(w: synth.Workload, case: dict, target_s: float = 12.0, y_gpu=None, ls_gpu=None):
+    """The fp64 oracle as it stands, timed on the host cores on a bounded sample.
+    With the GPU's y and last_state of the timed run (host tensors), also their
+    agreement with the oracle on the rows of the final sample (untimed):
+    returns (baseline, parity)."""
     import oracle
     threads = oracle.default_threads()
     nch = w.batch * w.dim
@@ -217,17 +220,36 @@ def cpu_baseline(w: synth.Workload, case: dict, target_s: float = 12.0) -> dict:
     while True:
         chans = synth.sample_channels(w, k)
         subs = synth.subset_case(case, chans)
-        t0 = time.perf_counter()
-        for _, _, sub in subs:
-            oracle.fwd(sub, nthreads=threads)
-        dt = time.perf_counter() - t0
+        dt = 0.0
+        acc = {"y": [0.0, 0.0, 0.0, 0.0], "last_state": [0.0, 0.0, 0.0, 0.0]}  # err2, ref2, max err, max ref
+        for b, dims, sub in subs:
+            t0 = time.perf_counter()
+            ref = oracle.fwd(sub, nthreads=threads)
+            dt += time.perf_counter() - t0
+            if y_gpu is not None:
+                for key, got_t in (("y", y_gpu), ("last_state", ls_gpu)):
+                    got = got_t[b, dims].double().numpy()
+                    r = ref[key][0]
+                    a = acc[key]
+                    a[0] += float(np.sum((got - r) ** 2))
+                    a[1] += float(np.sum(r ** 2))
+                    a[2] = max(a[2], float(np.max(np.abs(got - r))))
+                    a[3] = max(a[3], float(np.max(np.abs(r))))
         t_first = t_first or dt
         if dt >= target_s * 0.5 or k >= nch:
             break
         k = min(nch, int(k * max(2.0, target_s / max(dt, 1e-3))))
-    return {"value": k * w.seqlen / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+    base = {"value": k * w.seqlen / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{k} of {nch} (batch, channel) rows over the full L={w.seqlen}, "
                       f"fp64, {dt:.1f} s"}
+    parity = None
+    if y_gpu is not None:
+        parity = {"against": "the fp64 oracle on the same inputs", "rows": f"{k} of {nch}",
+                  "tolerance": ("rel-L2 <= 2e-3 and max-abs <= 1e-2 max|ref|" if w.dtype == synth.BF16
+                                else "rel-L2 <= 1e-5")}
+        for key, (e2, r2, me, mr) in acc.items():
+            parity[key] = {"rel_l2": (e2 / r2) ** 0.5 if r2 > 0 else 0.0, "max_abs": me, "max_ref": mr}
+    return base, parity
 
 
 def run_reference(args, w):
@@ -756,6 +778,10 @@ def main():
     ssm.check(ws)
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
     clocks = clk.summary()
+    # the timed run's outputs, for the parity check beside the CPU baseline
+    y_keep = ls_keep = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        y_keep, ls_keep = y.cpu(), ls.cpu()
 
     # the same forward on token-major activations (batch, seqlen, d_inner)
     tok = None
@@ -913,7 +939,7 @@ def main():
             "mamba_130m_layer": m130, "million_length": mlen,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, case)
+        line["cpu_baseline"], line["parity"] = cpu_baseline(w, case, y_gpu=y_keep, ls_gpu=ls_keep)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
