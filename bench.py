@@ -924,7 +924,9 @@ def main():
                               f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})",
                 "algorithmic_bytes": alg_bytes(w),
                 "hbm_achieved_gbs": alg_bytes(w) / sec / 1e9, "hbm_peak_gbs": pk["hbm_gbs"],
-                "hbm_frac": alg_bytes(w) / sec / 1e9 / pk["hbm_gbs"]}
+                "hbm_frac": alg_bytes(w) / sec / 1e9 / pk["hbm_gbs"],
+                # against the nominal HBM3e bandwidth too (8 TB/s), for context
+                "hbm_frac_of_nominal_8tbs": alg_bytes(w) / sec / 1e9 / 8000.0}
     if clocks and clocks.get("sm_mhz"):
         at_clock = sm_count * MUFU_EX2_PER_CLK_PER_SM * clocks["sm_mhz"] * 1e6
         roofline["frac_at_measured_clock"] = achieved / at_clock
