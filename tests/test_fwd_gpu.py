@@ -365,6 +365,24 @@ def test_warp_specialised_four_lanes_limits(cuda_device):
     assert ssm.fwd_path(ssm.make_shape(8, 1536, 2048, 16, ssm.SSM_BF16)) == "lookback_ws"
 
 
+def test_auto_warp_specialised_with_fewer_groups_than_subpartitions(cuda_device):
+    # batch 6 x d_inner 1536: 576 groups of 16 channels, at least 3/4 of the
+    # SM sub-partitions of a B200 but fewer than all: AUTO takes the
+    # warp-specialised kernel with one look-back worker per group
+    import torch
+    import selective_state_space_54_b200 as ssm
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    groups = 6 * 1536 // 16
+    if not (4 * groups >= 3 * 4 * sms and groups < 4 * sms):
+        pytest.skip("shape chosen for a 148-SM device")
+    assert ssm.fwd_path(ssm.make_shape(6, 1536, 300, 16, ssm.SSM_BF16)) == "lookback_ws"
+    case = synth.make_case(6, 1536, 300, 16, synth.BF16, seed=470)
+    ref = oracle.fwd(case)
+    y, ls = _run(case, cuda_device)
+    assert_close(y, ref["y"], synth.BF16, "y")
+    assert_close(ls, ref["last_state"], synth.BF16, "last_state", stored_bf16=False)
+
+
 def test_zoh_exact_auto_picks_warp_specialised(cuda_device):
     # a Mamba-layer-like shape: AUTO takes the warp-specialised kernel for ZOH too
     import selective_state_space_54_b200 as ssm
