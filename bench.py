@@ -381,6 +381,14 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
                     "kernel": "k_bwd16", "ex2_per_element": ex2_per_element,
                     "kernel_ex2_per_element": kernel_ex2,
                     "kernel_mufu_frac": kernel_ex2 * w.bldn / (ms_b * 1e-3) / ex2_peak,
+                    # the FP32-pipe view: the gradient formulas need 11 fp32 operations
+                    # per (b, t, d, n) element (a fused multiply-add counted once): the
+                    # state recomputation x = Delta A, Delta u B, a h + b (3); the reverse
+                    # recurrence dy C + (a g) (2); dC, dB, sum_n g B, g a h_{t-1}, dA and
+                    # dDelta's A term (6); peak = SMs x 128 fp32 lanes x clock
+                    "fp32_pipe": {"ops_per_element": 11,
+                                  "peak_tops": sm_count * 128 * pk["sm_max_mhz"] * 1e6 / 1e12,
+                                  "frac": 11 * w.bldn / (ms_b * 1e-3) / (sm_count * 128 * pk["sm_max_mhz"] * 1e6)},
                     "peak_basis": f"{sm_count} SMs x {MUFU_EX2_PER_CLK_PER_SM} ex2/clk x "
                                   f"{pk['sm_max_mhz']:.0f} MHz (sm_max_mhz, {pk['source']})"}
     variants = measure_training_variants(ssm, torch, dev, g, y, out, w, steps, barrier, max_over_ranks)
