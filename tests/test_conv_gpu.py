@@ -155,6 +155,26 @@ def test_conv_bwd_optional_terms(cuda_device, opt):
                with_state=opt != "no_state", silu=opt != "no_silu")
 
 
+@pytest.mark.parametrize("L", [1, 9, 511, 512, 513, 1537, 4096])
+def test_conv_bwd_ragged_lengths_bf16(cuda_device, L):
+    # rows of L * 2 bytes a multiple of 16 (512, 4096) reach shared memory by cp.async,
+    # the others by element loads; 512-step segments, the last one ragged
+    _check_bwd(2, 5, L, 4, synth.BF16, 190 + L, cuda_device)
+
+
+def test_conv_bwd_unaligned_rows_take_the_element_path(cuda_device):
+    _check_bwd(3, 7, 1077, 4, synth.BF16, 12, cuda_device)
+
+
+@pytest.mark.parametrize("dtype,K", [(synth.BF16, 4), (synth.BF16, 7), (synth.F32, 8)])
+def test_conv_bwd_rows_across_warp_ranges(cuda_device, dtype, K):
+    # the backward's warps walk contiguous ranges of 512-step segments: over 16 rows of
+    # 640,024 steps the ranges start and end inside rows (the first inputs before a range
+    # and the da after it come from memory) and hold several segments of one row (lane
+    # 31's second dx half waits for the next segment's first da values)
+    _check_bwd(2, 8, 512 * 1250 + 24, K, dtype, 31 + K, cuda_device)
+
+
 def test_conv_bwd_full_mamba_2p8b_layer(cuda_device):
     # the x_proj shape at full size; dx on sampled rows, parameter sums in full
     w_ = synth.WORKLOADS["mamba-2.8b-layer"]
