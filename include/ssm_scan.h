@@ -283,7 +283,10 @@ ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t
  *  dweight                   [dim][width] fp32, overwritten (required)
  *  dbias                     [dim] fp32, exactly when bias is given
  *  dinitial_state            [batch][dim][width-1] fp32, nullable
- * Argument checks as in the forward.  dx may not alias x or dout. */
+ * Argument checks as in the forward.  dx may not alias x or dout.  dx and
+ * dinitial_state are bitwise repeatable; dweight and dbias are fp32 partial
+ * sums (one per warp and row) added with atomics, so their last bits may
+ * differ between runs. */
 ssm_status ssm_causal_conv1d_bwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
                                  int32_t io_dtype, const void *x, const float *weight,
                                  const float *bias, const float *initial_state, int silu,

@@ -175,6 +175,18 @@ def test_conv_bwd_rows_across_warp_ranges(cuda_device, dtype, K):
     _check_bwd(2, 8, 512 * 1250 + 24, K, dtype, 31 + K, cuda_device)
 
 
+def test_conv_bwd_dx_is_bitwise_repeatable(cuda_device):
+    # dx and the initial state's gradient take no atomics: equal bits on every call
+    # (dweight and dbias are summed with atomics, equal only to rounding)
+    x, w, b, s0 = _inputs(2, 24, 5000, 4, synth.BF16, 44)
+    dout = synth.normal((2, 24, 5000), 44, "dy", synth.BF16)
+    g1 = _run_bwd(x, w, b, s0, dout, synth.BF16, cuda_device)
+    g2 = _run_bwd(x, w, b, s0, dout, synth.BF16, cuda_device)
+    assert np.array_equal(g1["dx"], g2["dx"])
+    assert np.array_equal(g1["dinitial_state"], g2["dinitial_state"])
+    np.testing.assert_allclose(g1["dweight"], g2["dweight"], rtol=1e-5, atol=1e-6)
+
+
 def test_conv_bwd_full_mamba_2p8b_layer(cuda_device):
     # the x_proj shape at full size; dx on sampled rows, parameter sums in full
     w_ = synth.WORKLOADS["mamba-2.8b-layer"]
