@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synth
-from gpu_util import assert_close, to_f64, upload
+from gpu_util import assert_close, to_f64, to_torch, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -75,3 +75,48 @@ def test_random_case_against_the_oracle(cuda_device, i):
         if with_h0:
             assert_close(to_f64(got["dinitial_state"]), refb["dh0"], dtype, "dh0 " + what,
                          stored_bf16=False)
+
+
+@pytest.mark.parametrize("i", range(60))
+def test_random_conv1d_case_against_the_oracle(cuda_device, i):
+    # causal conv1d + SiLU forward and backward: random widths, lengths around the
+    # backward's 512-step segments and the forward's 2048-step warps, row counts that
+    # make the backward's warp ranges start and end inside rows or hold several
+    # segments of one, dtypes, and every optional term
+    import torch
+    import selective_state_space_54_b200 as ssm
+    rng = np.random.default_rng(7000 + i)
+    batch = int(rng.integers(1, 4))
+    dim = int(rng.choice([1, 3, 16, 40, 129]))
+    L = int(rng.choice([1, 2, 7, 8, 100, 511, 512, 513, 1024, 1500, 2049, 5000, 20000]))
+    K = int(rng.integers(1, 9))
+    dtype = synth.BF16 if rng.random() < 0.6 else synth.F32
+    silu = bool(rng.random() < 0.8)
+    with_bias = bool(rng.random() < 0.7)
+    with_state = bool(rng.random() < 0.6)
+    x = synth.normal((batch, dim, L), 7100 + i, "u", dtype)
+    dout = synth.normal((batch, dim, L), 7100 + i, "dy", dtype)
+    w = (rng.standard_normal((dim, K)) / np.sqrt(K)).astype(np.float32)
+    b = rng.standard_normal(dim).astype(np.float32) if with_bias else None
+    s0 = rng.standard_normal((batch, dim, K - 1)).astype(np.float32) if with_state else None
+
+    ref, ref_s = oracle.conv1d(x, w, b, dtype=dtype, initial_state=s0, silu=silu)
+    refb = oracle.conv1d_bwd(x, w, b, dout, dtype=dtype, initial_state=s0, silu=silu)
+    f = lambda a: None if a is None else torch.from_numpy(a).to(cuda_device)
+    xt, gt = to_torch(x, dtype, cuda_device), to_torch(dout, dtype, cuda_device)
+    out, fs = ssm.causal_conv1d(xt, f(w), f(b), initial_state=f(s0), silu=silu,
+                                return_final_state=True)
+    grads = ssm.causal_conv1d_bwd(xt, f(w), f(b), gt, initial_state=f(s0), silu=silu,
+                                  want_dinitial_state=True)
+    torch.cuda.synchronize()
+    tag = f"case {i}: batch {batch} dim {dim} L {L} K {K} {dtype} silu {silu}"
+    assert_close(to_f64(out), ref, dtype, f"{tag} out")
+    if K > 1:
+        assert np.array_equal(to_f64(fs), ref_s), tag
+    assert_close(to_f64(grads["dx"]), refb["dx"], dtype, f"{tag} dx")
+    assert_close(to_f64(grads["dweight"]), refb["dweight"], dtype, f"{tag} dweight", stored_bf16=False)
+    if with_bias:
+        assert_close(to_f64(grads["dbias"]), refb["dbias"], dtype, f"{tag} dbias", stored_bf16=False)
+    if K > 1:
+        assert_close(to_f64(grads["dinitial_state"]), refb["dinitial_state"], dtype,
+                     f"{tag} dinitial_state", stored_bf16=False)
