@@ -314,6 +314,16 @@ ssm_status ssm_scan_test_wait_timeout(void *workspace, size_t ws_bytes,
  * failures are consumed in call order. */
 void ssm_scan_test_fail_next(int32_t count);
 
+/* Test hook for ssm_scan_fwd_noalloc across a device reset: runs it on a
+ * small seeded fp32 problem (batch 2, dim 32, seqlen 200, dstate 16) on
+ * buffers it allocates, calls cudaDeviceReset, allocates afresh and runs it
+ * again.  Returns 0 when both calls give equal bits, 1 when they differ, a
+ * negative ssm_status when a call fails (SSM_ERR_CUDA for a failed
+ * allocation, copy or reset).  The reset ends the process's primary context
+ * on the current device: every earlier device allocation of the process is
+ * gone, so call it only from a process that holds none it still needs. */
+int32_t ssm_scan_test_noalloc_reset_cycle(void);
+
 /* Path AUTO would choose for `shape` on the current device (for tests and
  * the benchmark); SSM_PATH_AUTO itself for an invalid shape. */
 int32_t ssm_scan_fwd_path(const ssm_shape *shape);

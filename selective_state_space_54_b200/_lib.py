@@ -40,6 +40,7 @@ EXPORTS = (
     "ssm_scan_bwd", "ssm_scan_check", "ssm_scan_test_wait_timeout", "ssm_scan_fwd_path",
     "ssm_status_string", "ssm_scan_version", "ssm_scan_fwd_noalloc", "ssm_scan_step",
     "ssm_causal_conv1d", "ssm_causal_conv1d_bwd", "ssm_scan_test_fail_next",
+    "ssm_scan_test_noalloc_reset_cycle",
 )
 
 
@@ -90,6 +91,8 @@ def load(path: str | None = None):
     lib.ssm_scan_test_wait_timeout.restype = ci
     lib.ssm_scan_test_fail_next.argtypes = [i32]
     lib.ssm_scan_test_fail_next.restype = None
+    lib.ssm_scan_test_noalloc_reset_cycle.argtypes = []
+    lib.ssm_scan_test_noalloc_reset_cycle.restype = i32
     lib.ssm_scan_fwd_path.argtypes = [shp]
     lib.ssm_scan_fwd_path.restype = i32
     lib.ssm_status_string.argtypes = [ci]

@@ -25,6 +25,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <cmath>
+#include <vector>
+
 #include "ssm_common.cuh"
 #include "ssm_scan.h"
 
@@ -87,4 +90,76 @@ extern "C" ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u
   // nothing left in the array by an earlier call is read.
   return ssm_scan_fwd(&s, u, delta, A, B, C, D, z, delta_bias, delta_softplus, initial_state, y,
                       last_state, ptr, kStaticScratchBytes, stream);
+}
+
+// Test hook: the no-allocation forward on a small seeded problem, a device
+// reset, then the same call on buffers allocated afresh.  The scratch array's
+// address is looked up again after the reset, so both calls must give equal
+// bits.  0: equal; 1: they differ; negative: the ssm_status of a failed call,
+// or SSM_ERR_CUDA for a failed allocation, copy or reset.
+extern "C" int32_t ssm_scan_test_noalloc_reset_cycle(void) {
+  constexpr int64_t Bt = 2, Dm = 32, Ls = 200, N = 16;
+  const int64_t n_act = Bt * Dm * Ls, n_bc = Bt * Ls * N;
+  std::vector<float> u(n_act), dl(n_act), z(n_act), Bm(n_bc), Cm(n_bc), A(Dm * N), Dd(Dm), bias(Dm);
+  // smooth, deterministic inputs of the layer's ranges (A negative, delta near 0)
+  for (int64_t i = 0; i < n_act; ++i) {
+    u[i] = (float)std::sin(0.37 * (double)i);
+    dl[i] = (float)(0.5 * std::cos(0.11 * (double)i) - 1.0);
+    z[i] = (float)std::sin(0.23 * (double)i + 1.0);
+  }
+  for (int64_t i = 0; i < n_bc; ++i) {
+    Bm[i] = (float)std::cos(0.05 * (double)i);
+    Cm[i] = (float)std::sin(0.07 * (double)i + 0.5);
+  }
+  for (int64_t d = 0; d < Dm; ++d) {
+    for (int64_t n = 0; n < N; ++n) A[d * N + n] = -(float)(n + 1);
+    Dd[d] = 1.f;
+    bias[d] = (float)(0.01 * (double)d);
+  }
+  ssm_shape s;
+  memset(&s, 0, sizeof(s));
+  s.batch = Bt; s.dim = Dm; s.seqlen = Ls; s.dstate = N;
+  s.io_dtype = SSM_F32; s.path = SSM_PATH_AUTO;
+
+  auto run = [&](std::vector<float> &y, std::vector<float> &last) -> int32_t {
+    const std::vector<float> *in[8] = {&u, &dl, &A, &Bm, &Cm, &Dd, &z, &bias};
+    float *dev[8] = {nullptr}, *dy = nullptr, *dls = nullptr;
+    int32_t rc = 0;
+    for (int k = 0; k < 8 && rc == 0; ++k) {
+      const size_t bytes = in[k]->size() * sizeof(float);
+      if (cudaMalloc(&dev[k], bytes) != cudaSuccess ||
+          cudaMemcpy(dev[k], in[k]->data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess)
+        rc = SSM_ERR_CUDA;
+    }
+    if (rc == 0 && (cudaMalloc(&dy, n_act * sizeof(float)) != cudaSuccess ||
+                    cudaMalloc(&dls, Bt * Dm * N * sizeof(float)) != cudaSuccess))
+      rc = SSM_ERR_CUDA;
+    if (rc == 0) {
+      const ssm_status st = ssm_scan_fwd_noalloc(&s, dev[0], dev[1], dev[2], dev[3], dev[4], dev[5], dev[6],
+                                                 dev[7], 1, nullptr, dy, dls, nullptr);
+      if (st != SSM_OK) rc = st;
+    }
+    if (rc == 0 && cudaDeviceSynchronize() != cudaSuccess) rc = SSM_ERR_CUDA;
+    if (rc == 0) {
+      y.resize(n_act);
+      last.resize(Bt * Dm * N);
+      if (cudaMemcpy(y.data(), dy, n_act * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess ||
+          cudaMemcpy(last.data(), dls, last.size() * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess)
+        rc = SSM_ERR_CUDA;
+    }
+    for (float *p : dev) cudaFree(p);
+    cudaFree(dy);
+    cudaFree(dls);
+    return rc;
+  };
+
+  std::vector<float> y1, l1, y2, l2;
+  int32_t rc = run(y1, l1);
+  if (rc != 0) return rc;
+  if (cudaDeviceReset() != cudaSuccess) return SSM_ERR_CUDA;
+  rc = run(y2, l2);
+  if (rc != 0) return rc;
+  const bool same = memcmp(y1.data(), y2.data(), y1.size() * sizeof(float)) == 0 &&
+                    memcmp(l1.data(), l2.data(), l1.size() * sizeof(float)) == 0;
+  return same ? 0 : 1;
 }

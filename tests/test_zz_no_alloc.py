@@ -117,3 +117,21 @@ def test_noalloc_rejects_shapes_beyond_the_static_scratch(cuda_device):
     assert rc == _lib.SSM_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert torch.count_nonzero(buf).item() == 0  # nothing was written
+
+
+def test_noalloc_after_a_device_reset(cuda_device):
+    # The scratch array's address is looked up on every call, so a device reset
+    # between two calls is harmless: the library's self-test runs the entry point,
+    # resets the device, reallocates and runs it again, and the two results must be
+    # equal bit for bit.  It runs in a child process, because the reset ends the
+    # primary context this process's tensors live in.
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys; sys.path.insert(0, %r); "
+            "from selective_state_space_54_b200 import _lib; "
+            "print(_lib.load().ssm_scan_test_noalloc_reset_cycle())") % root
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.strip().splitlines()[-1] == "0", r.stdout + r.stderr
