@@ -97,7 +97,7 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
              save_states=False, token_major=False, check_status=False, stream=None):
     """Forward selective scan; returns y, or (y, last_state).  zoh_exact selects the
     exact zero-order-hold input term instead of the Euler one (Delta * B).
-    save_states also writes the state entering every 16-step chunk into
+    save_states also writes the state entering every 8-step chunk into
     ``workspace`` (which must then be given), for scan_bwd(fwd_workspace=...).
     token_major: u, delta, z and y are (batch, seqlen, dim) instead.
     The look-back schedules hand states between warps with a bounded wait that
