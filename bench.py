@@ -311,6 +311,24 @@ def config_of(w, path):
             "seed": w.seed}
 
 
+def time_fwd_bwd(torch, dev, stream, fwd, bwd, steps):
+    """Device time of `steps` forward + backward steps queued back to back,
+    with events between the two halves of each step and one synchronise on
+    each side of the whole sequence, so the host's launch work overlaps the
+    device's instead of being timed.  Returns the summed forward and backward
+    milliseconds."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        e[0].record(stream)
+        fwd()
+        e[1].record(stream)
+        bwd()
+        e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    return (sum(e[0].elapsed_time(e[1]) for e in evs), sum(e[1].elapsed_time(e[2]) for e in evs))
+
+
 def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None):
     """Forward + recomputation backward on the Mamba-1.4B layer training shape."""
     w = w or synth.WORKLOADS["mamba-1.4b-layer-train"]
@@ -320,7 +338,7 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
         g[k] = torch.from_numpy(np.asarray(case[k], np.float32)).to(dev)
     del case
     y = torch.empty_like(g["u"])
-    # the training step: the forward saves the state entering every 16-step
+    # the training step: the forward saves the state entering every 8-step
     # chunk in its workspace, and the backward starts from those
     shape = ssm.make_shape(w.batch, w.dim, w.seqlen, w.dstate,
                            ssm.SSM_BF16 if w.dtype == synth.BF16 else ssm.SSM_F32,
@@ -348,19 +366,8 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
         bwd()
     torch.cuda.synchronize(dev)
     steps = max(3, min(args.steps, 10))
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     barrier()
-    torch.cuda.synchronize(dev)
-    t_f = t_b = 0.0
-    for _ in range(steps):
-        evs[0].record(stream)
-        fwd()
-        evs[1].record(stream)
-        bwd()
-        evs[2].record(stream)
-        torch.cuda.synchronize(dev)
-        t_f += evs[0].elapsed_time(evs[1])
-        t_b += evs[1].elapsed_time(evs[2])
+    t_f, t_b = time_fwd_bwd(torch, dev, stream, fwd, bwd, steps)
     barrier()
     ms_f = max_over_ranks(t_f / steps)
     ms_b = max_over_ranks(t_b / steps)
@@ -443,19 +450,8 @@ def measure_training_variants(ssm, torch, dev, g, y, out, w, steps, barrier, max
             bwd()
         torch.cuda.synchronize(dev)
         ssm.check(ws_f)
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         barrier()
-        torch.cuda.synchronize(dev)
-        t_f = t_b = 0.0
-        for _ in range(steps):
-            evs[0].record(stream)
-            fwd()
-            evs[1].record(stream)
-            bwd()
-            evs[2].record(stream)
-            torch.cuda.synchronize(dev)
-            t_f += evs[0].elapsed_time(evs[1])
-            t_b += evs[1].elapsed_time(evs[2])
+        t_f, t_b = time_fwd_bwd(torch, dev, stream, fwd, bwd, steps)
         barrier()
         ssm.check(ws_f)
         res[name] = {"fwd_ms": max_over_ranks(t_f / steps), "bwd_ms": max_over_ranks(t_b / steps),
