@@ -65,7 +65,7 @@ def _fwd(lib, shape, ptrs=None, ws=None, ws_bytes=0):
                             v(p["bias"]), 1, v(p["h0"]), v(p["y"]), v(p["ls"]), v(ws), ws_bytes, None)
 
 
-# argument checks passed: no workspace given (a GPU machine) or no device (here)
+# argument checks passed: no workspace given (on a machine with a GPU) or no device
 ACCEPTED = (_lib.SSM_ERR_WORKSPACE, _lib.SSM_ERR_CUDA)
 
 
