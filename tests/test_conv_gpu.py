@@ -187,6 +187,27 @@ def test_conv_bwd_dx_is_bitwise_repeatable(cuda_device):
     np.testing.assert_allclose(g1["dweight"], g2["dweight"], rtol=1e-5, atol=1e-6)
 
 
+@pytest.mark.parametrize("dtype", [synth.F32, synth.BF16])
+def test_conv_saturated_silu(cuda_device, dtype):
+    # pre-activations in the hundreds: e^-a overflows to infinity on the negative side,
+    # where SiLU and its derivative must come out as (signed) zeros, not NaN
+    x, w, b, s0 = _inputs(2, 16, 3000, 4, dtype, 55)
+    xs = (synth.bf16_bits_to_f32(x) * 100.0).astype(np.float32) if dtype == synth.BF16 else x * 100.0
+    if dtype == synth.BF16:
+        xs = synth.f32_to_bf16_bits(xs)
+    dout = synth.normal((2, 16, 3000), 55, "dy", dtype)
+    with np.errstate(over="ignore"):
+        ref, ref_s = oracle.conv1d(xs, w, b, dtype=dtype, initial_state=s0, silu=True)
+        refb = oracle.conv1d_bwd(xs, w, b, dout, dtype=dtype, initial_state=s0, silu=True)
+    out, fs = _run(xs, w, b, s0, dtype, cuda_device)
+    got = _run_bwd(xs, w, b, s0, dout, dtype, cuda_device)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(got["dx"]))
+    assert_close(out, ref, dtype, "out")
+    assert_close(got["dx"], refb["dx"], dtype, "dx")
+    assert_close(got["dweight"], refb["dweight"], dtype, "dweight", stored_bf16=False)
+    assert_close(got["dbias"], refb["dbias"], dtype, "dbias", stored_bf16=False)
+
+
 def test_conv_bwd_full_mamba_2p8b_layer(cuda_device):
     # the x_proj shape at full size; dx on sampled rows, parameter sums in full
     w_ = synth.WORKLOADS["mamba-2.8b-layer"]
