@@ -187,6 +187,46 @@ def test_softplus_accuracy_through_the_kernel(cuda_device):
         assert np.all(rel <= bound), (lanes, float(rel.max()), float(s[np.argmax(rel / bound)]))
 
 
+@pytest.mark.parametrize("path,lanes", PATH_LANES)
+def test_softplus_accuracy_on_every_path(cuda_device, path, lanes):
+    # the construction of the test above through every schedule (the warp-specialised
+    # producer has its own packed softplus), with 8 equal states and C = 1/8 so that
+    # every lane split runs: y_t = 8 (Delta_t / 8) = softplus(s_t) exactly
+    L, N = 4096, 8
+    s = np.linspace(-30.0, 30.0, L).astype(np.float32)
+    case = {"batch": 1, "dim": 1, "seqlen": L, "dstate": N, "dtype": synth.F32,
+            "u": np.ones((1, 1, L), np.float32), "delta": s.reshape(1, 1, L),
+            "A": np.full((1, N), -1e30, np.float32), "B": np.ones((1, L, N), np.float32),
+            "C": np.full((1, L, N), 1.0 / N, np.float32), "D": None, "z": None, "delta_bias": None}
+    ref = oracle.fwd(case)["y"][0, 0]
+    y, _ = _run(case, cuda_device, path, lanes=lanes)
+    rel = np.abs(y[0, 0] - ref) / ref
+    bound = 1e-6 + 1e-7 * np.abs(s.astype(np.float64))
+    assert np.all(rel <= bound), (path, lanes, float(rel.max()), float(s[np.argmax(rel / bound)]))
+
+
+@pytest.mark.parametrize("path,lanes", PATH_LANES)
+def test_gate_over_a_wide_range(cuda_device, path, lanes):
+    # y_t = yss_t * SiLU(z_t) with yss_t = 1 (Abar = 0, Delta = 1 without softplus,
+    # B = u = 1 and C = 1/8 over 8 states): y is SiLU(z) itself, for z over [-200, 200].
+    # Far on the negative side SiLU is below 1e-15 and e^-z overflows fp32: there the
+    # kernels may return any value of that size (the warp-specialised gate clamps
+    # 1 + e^-z at 2^64)
+    L, N = 4096, 8
+    z = np.linspace(-200.0, 200.0, L).astype(np.float32)
+    case = {"batch": 1, "dim": 1, "seqlen": L, "dstate": N, "dtype": synth.F32,
+            "u": np.ones((1, 1, L), np.float32), "delta": np.ones((1, 1, L), np.float32),
+            "A": np.full((1, N), -1e30, np.float32), "B": np.ones((1, L, N), np.float32),
+            "C": np.full((1, L, N), 1.0 / N, np.float32), "D": None, "z": z.reshape(1, 1, L),
+            "delta_bias": None}
+    ref = oracle.fwd(case, delta_softplus=False)["y"][0, 0]
+    y, _ = _run(case, cuda_device, path, softplus=False, lanes=lanes)
+    err = np.abs(y[0, 0] - ref)
+    bound = 2e-6 * np.abs(ref) + 1e-15
+    assert np.all(np.isfinite(y)), (path, lanes)
+    assert np.all(err <= bound), (path, lanes, float((err / bound).max()), float(z[np.argmax(err / bound)]))
+
+
 @pytest.mark.parametrize("path,lanes", [("lookback", 0), ("lookback_ws", 2), ("lookback_ws", 4)])
 def test_deterministic(cuda_device, path, lanes):
     case = synth.make_case(2, 64, 1024, 16, synth.BF16, seed=41)
