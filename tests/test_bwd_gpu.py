@@ -76,6 +76,22 @@ def test_bwd_optional_terms(cuda_device, opt):
     _check(case, cuda_device, softplus=softplus)
 
 
+@pytest.mark.parametrize("N", [4, 16])
+def test_bwd_over_wide_softplus_and_gate_ranges(cuda_device, N):
+    # the raw delta over s in [-30, 30] and z over [-100, 100] in every channel (rolled
+    # differently per channel): the softplus derivative sigmoid(s) and the gate's
+    # SiLU'(z) at saturation on both sides, every gradient against the oracle
+    # (d_state 16 runs the d_state-16 kernel, 4 the general one)
+    D, L = 16, 600
+    case = _case(1, D, L, N, synth.F32, 71)
+    s = np.linspace(-30.0, 30.0, L, dtype=np.float32)
+    z = np.linspace(-100.0, 100.0, L, dtype=np.float32)
+    case["delta"] = np.stack([np.roll(s, 37 * d) for d in range(D)])[None].astype(np.float32)
+    case["z"] = np.stack([np.roll(z, 53 * d) for d in range(D)])[None].astype(np.float32)
+    case["delta_bias"] = np.zeros(D, np.float32)  # s as written
+    _check(case, cuda_device)
+
+
 def test_bwd_initial_state_gradient(cuda_device):
     case = _case(2, 32, 300, 16, synth.F32, 6)
     h0 = np.random.default_rng(2).standard_normal((2, 32, 16)).astype(np.float32)
