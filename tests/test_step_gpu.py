@@ -60,6 +60,33 @@ def test_step_optional_terms(cuda_device, opt):
     _check(case, cuda_device, _state(2, 64, 16, 3), softplus=softplus)
 
 
+@pytest.mark.parametrize("what", ["softplus", "gate"])
+def test_step_over_wide_softplus_and_gate_ranges(cuda_device, what):
+    # one token, one value per channel: with a zero state, Abar = 0, B = u = 1 and
+    # C = 1/16 over 16 states, y = softplus(s) (no gate) over s in [-30, 30], or
+    # y = SiLU(z) (Delta = 1 without softplus) over z in [-200, 200], element by element
+    D, N = 1024, 16
+    v = np.linspace(-30.0, 30.0, D) if what == "softplus" else np.linspace(-200.0, 200.0, D)
+    v = v.astype(np.float32).reshape(1, D, 1)
+    case = {"batch": 1, "dim": D, "seqlen": 1, "dstate": N, "dtype": synth.F32,
+            "u": np.ones((1, D, 1), np.float32),
+            "delta": v if what == "softplus" else np.ones((1, D, 1), np.float32),
+            "A": np.full((D, N), -1e30, np.float32), "B": np.ones((1, 1, N), np.float32),
+            "C": np.full((1, 1, N), 1.0 / N, np.float32), "D": None,
+            "z": None if what == "softplus" else v, "delta_bias": None}
+    softplus = what == "softplus"
+    ref = oracle.fwd(case, delta_softplus=softplus)["y"][0, :, 0]
+    y, _ = _run_step(case, cuda_device, np.zeros((1, D, N), np.float32), softplus=softplus)
+    y = y[0]
+    assert np.all(np.isfinite(y))
+    if softplus:  # relative accuracy of the softplus, as for the scan
+        bound = (1e-6 + 1e-7 * np.abs(v.ravel().astype(np.float64))) * ref
+    else:         # SiLU; far on the negative side any value below 1e-15
+        bound = 2e-6 * np.abs(ref) + 1e-15
+    err = np.abs(y - ref)
+    assert np.all(err <= bound), (what, float((err / bound).max()))
+
+
 @pytest.mark.parametrize("batch,dim", [(1, 1), (1, 7), (5, 33), (2, 1000)])
 def test_step_ragged_channel_counts(cuda_device, batch, dim):
     case = synth.make_case(batch, dim, 1, 16, synth.BF16, seed=batch * 1000 + dim)
