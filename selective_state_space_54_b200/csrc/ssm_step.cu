@@ -155,7 +155,22 @@ static cudaError_t launch_step_k(const StepParams &p, cudaStream_t s) {
 // load-compute-store thread could only match with far more registers.  Each
 // lane reads back only what it copied itself: no block barrier.
 constexpr int kRows = 4;
-static_assert(kRows == 4, "the cp.async wait chain below is written for 4 rows");
+static_assert(kRows >= 1 && kRows <= 8, "the wait below takes up to 7 groups still in flight");
+
+// wait until at most `pending` copy groups are in flight (a constant once the
+// row loop is unrolled)
+__device__ __forceinline__ void step_wait_groups(int pending) {
+  switch (pending) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
+}
 
 // L2 policy for data touched once: evict it first
 __device__ __forceinline__ unsigned long long evict_first_policy() {
@@ -223,11 +238,9 @@ __global__ void __launch_bounds__(kStepThreads) k_step_rows(StepParams p) {
     load_io<S>(static_cast<const T *>(p.C) + b * N, true, n0, N, Cv);
     const float dl = p.softplus ? softplus_fast(ss[r]) : ss[r];
     const float du = dl * uu[r];
-    // wait for this row's copies (groups were committed in row order)
-    if (r == 0) asm volatile("cp.async.wait_group 3;" ::: "memory");
-    if (r == 1) asm volatile("cp.async.wait_group 2;" ::: "memory");
-    if (r == 2) asm volatile("cp.async.wait_group 1;" ::: "memory");
-    if (r == 3) asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // wait for this row's copies (groups were committed in row order: the later
+    // rows' groups may still be in flight)
+    step_wait_groups(kRows - 1 - r);
     float h[S];
 #pragma unroll
     for (int q = 0; q < S / 4; ++q) {
