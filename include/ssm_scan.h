@@ -266,8 +266,9 @@ ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delt
  *  initial_state, final_state [batch][dim][width-1] fp32, nullable
  *                             (oldest input first; unused when width == 1)
  * width is 1..8 (SSM_ERR_UNSUPPORTED above).  out may not alias x.  Rows
- * whose bytes are a multiple of 16 on 16-byte aligned buffers take vector
- * loads and stores. */
+ * whose bytes are a multiple of 32 on 32-byte aligned buffers move 32 bytes
+ * per access, multiples of 16 on 16-byte aligned buffers 16 bytes; other rows
+ * take element accesses. */
 ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t width,
                              int32_t io_dtype, const void *x, const float *weight,
                              const float *bias, const float *initial_state, int silu,

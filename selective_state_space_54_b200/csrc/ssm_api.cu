@@ -439,7 +439,11 @@ ssm_status ssm_causal_conv1d(int64_t batch, int64_t dim, int64_t seqlen, int32_t
   memset(&p, 0, sizeof(p));
   p.x = x; p.w = weight; p.bias = bias; p.s0 = initial_state; p.out = out; p.s1 = final_state;
   p.batch = batch; p.dim = dim; p.L = seqlen; p.K = width; p.silu = silu ? 1 : 0;
-  p.vec = ((seqlen * (int64_t)es) % 16 == 0) && aligned(x, 16) && aligned(out, 16);
+  // 2: rows of whole 32-byte sectors on 32-byte aligned buffers (a lane's 16 steps move
+  // in one 32-byte access); 1: 16-byte rows and buffers; 0: element accesses
+  const bool row16 = ((seqlen * (int64_t)es) % 16 == 0) && aligned(x, 16) && aligned(out, 16);
+  const bool row32 = ((seqlen * (int64_t)es) % 32 == 0) && aligned(x, 32) && aligned(out, 32);
+  p.vec = row32 ? 2 : (row16 ? 1 : 0);
   const cudaError_t inj = injected_failure();
   if (inj != cudaSuccess) return cuda_status(inj);
   return cuda_status(launch_conv(io_dtype, p, s));

@@ -107,7 +107,7 @@ struct ConvParams {
   int64_t batch, dim, L;
   int K;
   int silu;
-  int vec;                             // 16-byte aligned rows: vector loads and stores
+  int vec;                             // 2: 32-byte rows and buffers, 1: 16-byte, 0: neither
 };
 
 // Causal depthwise conv1d backward parameters (ssm_conv.cu).

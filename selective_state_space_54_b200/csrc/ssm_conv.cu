@@ -7,191 +7,210 @@
 //   out_t = act(bias[d] + sum_{k<K} w[d][k] * x_{t-K+1+k}),
 // with x_t for t < 0 taken from the caller's initial state (zeros if none).
 //
-// Design (B200): 2 bytes in and 2 out per (b, d, t) in bf16, a few FMAs:
-// bound by HBM.  A warp takes 2048 consecutive steps of one (b, d) row in 8
-// passes; a lane takes 8 steps per pass with one 16-byte load and store,
-// all 8 loads issued before the first pass computes.  The K-1 steps before a
-// lane's chunk come from neighbouring lanes by shuffles, so every input byte
-// is read once.  Input and output are streamed with evict-first hints.
+// Design (B200): 2 bytes in and 2 out per (b, d, t) in bf16 and a few
+// instructions per element, so HBM sets the pace.  Both kernels give a lane
+// 16 consecutive steps of a row and compute them as 8 packed fp32 pairs
+// (t, t + 8): the convolution, the activation and, in the backward, the
+// dweight sums and dx run as f32x2 operations on aligned register pairs, and
+// only the K-1 pairs at a chunk's edge are assembled from two halves.  The K-1
+// inputs before a chunk come from the previous lane by one shuffle, so every
+// input byte is read once.
 #include "ssm_common.cuh"
+
+#include <algorithm>
 
 namespace ssm {
 
 constexpr int kConvThreads = 256;
 
-constexpr int kConvW = 8;                  // steps per lane and pass
-// Passes per warp, all loads issued first: 8 in the forward, i.e. 8 16-byte
-// loads in flight per lane, with the bf16 kernel held to 64 registers for 4
-// CTAs (32 warps) per SM.  Measured on B200 at the Mamba-2.8B shape (bf16,
-// width 4): 0.123 ms, against 0.133 ms at 3 CTAs per SM, 0.132 ms with 7
-// passes and 0.140 ms with 4; 9, 10, 12 or 16 passes cost registers (fewer
-// resident CTAs) and leave a ragged last segment (0.148-0.169 ms).
-constexpr int kConvR = 8;
-constexpr int kConvSeg = 32 * kConvW * kConvR;  // steps per forward warp
+// ---- shared by forward and backward ----------------------------------------
+__device__ __forceinline__ void conv_cp16(uint32_t dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void conv_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void conv_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-// (row, segment, channel) of this warp; 32-bit divisions when the grid's
-// warp count fits (the launcher checks), 64-bit otherwise
-struct ConvWarp {
-  int64_t row, seg, d;
-  bool live;
-  __device__ __forceinline__ ConvWarp(int64_t segs, int64_t rows, int64_t dim, bool narrow) {
-    if (narrow) {
-      const unsigned w = (blockIdx.x * (unsigned)kConvThreads + threadIdx.x) >> 5;
-      const unsigned r = w / (unsigned)segs;
-      live = r < (unsigned)rows;
-      row = r;
-      seg = w - r * (unsigned)segs;
-      d = r % (unsigned)dim;
-    } else {
-      const int64_t w = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
-      row = w / segs;
-      live = row < rows;
-      seg = w - row * segs;
-      d = row % dim;
-    }
-  }
+// value i of a lane's raw chunk (bf16 pairs per word, or fp32 words)
+template <typename T>
+__device__ __forceinline__ float raw_at(const uint32_t *w, int i) {
+  if constexpr (sizeof(T) == 2)
+    return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+  else
+    return __uint_as_float(w[i]);
+}
+
+__device__ __forceinline__ float lo_of(f2 v) {
+  float lo, hi;
+  unpack2(v, lo, hi);
+  return lo;
+}
+__device__ __forceinline__ float hi_of(f2 v) {
+  float lo, hi;
+  unpack2(v, lo, hi);
+  return hi;
+}
+
+// ---- forward --------------------------------------------------------------
+// Lane-contiguous forward: a warp takes P passes of 512 steps of one row; lane
+// l owns steps 16 l .. 16 l + 15 of each pass, loaded up front with one 32-byte
+// load per pass (two 16-byte ones, or elements, where the row allows less),
+// computed as 8 packed pairs (t, t + 8) and stored with one 32-byte store.
+template <typename T>
+struct ConvFwdPass {
+  static constexpr int S = 16, H = 8, PASS = 32 * S;
+  static constexpr int P = sizeof(T) == 2 ? 4 : 2;  // passes per warp
+  static constexpr int SEG = P * PASS;              // steps per warp
+  static constexpr int W = S * (int)sizeof(T) / 4;  // 32-bit words of one lane's chunk
 };
 
-// raw io vector of 8 values, kept packed until used
-template <typename T> struct Raw8;
-template <> struct Raw8<uint16_t> {
-  uint4 v;
-  __device__ __forceinline__ void load(const uint16_t *row, int64_t t, int64_t L, bool vec) {
-    if (vec && t + 8 <= L) {
-      v = __ldcs(reinterpret_cast<const uint4 *>(row + t));
-    } else {
-      uint32_t w[4];
+template <typename T, int W>
+__device__ __forceinline__ void conv_load_chunk(uint32_t (&w)[W], const T *src, int64_t rem, int vec) {
+  constexpr int S = W * 4 / (int)sizeof(T);
+  if (vec == 2 && rem >= S) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = (t + 2 * i < L) ? row[t + 2 * i] : 0u;
-        const uint32_t hi = (t + 2 * i + 1 < L) ? row[t + 2 * i + 1] : 0u;
-        w[i] = lo | (hi << 16);
+    for (int v = 0; v < W / 8; ++v)
+      asm volatile("ld.global.cs.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=r"(w[8 * v]), "=r"(w[8 * v + 1]), "=r"(w[8 * v + 2]), "=r"(w[8 * v + 3]),
+                     "=r"(w[8 * v + 4]), "=r"(w[8 * v + 5]), "=r"(w[8 * v + 6]), "=r"(w[8 * v + 7])
+                   : "l"(src + v * (32 / (int)sizeof(T))));
+  } else if (vec && rem >= S) {
+#pragma unroll
+    for (int v = 0; v < W / 4; ++v) {
+      const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src) + v);
+      w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < W; ++i) w[i] = 0u;
+#pragma unroll
+    for (int e = 0; e < S; ++e)
+      if (e < rem) {
+        if constexpr (sizeof(T) == 2) w[e >> 1] |= (uint32_t)src[e] << (16 * (e & 1));
+        else w[e] = __float_as_uint(src[e]);
       }
-      v = make_uint4(w[0], w[1], w[2], w[3]);
-    }
   }
-  __device__ __forceinline__ void unpack(float (&o)[8]) const {
-    o[0] = bf16_lo(v.x); o[1] = bf16_hi(v.x); o[2] = bf16_lo(v.y); o[3] = bf16_hi(v.y);
-    o[4] = bf16_lo(v.z); o[5] = bf16_hi(v.z); o[6] = bf16_lo(v.w); o[7] = bf16_hi(v.w);
-  }
-};
-template <> struct Raw8<float> {
-  float4 a, b;
-  __device__ __forceinline__ void load(const float *row, int64_t t, int64_t L, bool vec) {
-    if (vec && t + 8 <= L) {
-      a = __ldcs(reinterpret_cast<const float4 *>(row + t));
-      b = __ldcs(reinterpret_cast<const float4 *>(row + t + 4));
-    } else {
-      float o[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = (t + i < L) ? row[t + i] : 0.f;
-      a = make_float4(o[0], o[1], o[2], o[3]);
-      b = make_float4(o[4], o[5], o[6], o[7]);
-    }
-  }
-  __device__ __forceinline__ void unpack(float (&o)[8]) const {
-    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
-  }
-};
+}
 
-// A warp takes kConvSeg consecutive steps of one row in kConvR passes of 256;
-// all passes' loads are issued before the first is used, so each lane keeps
-// kConvR 16-byte loads in flight.  The K-1 steps before a lane's chunk come
-// from the previous lane (shuffle up), or for lane 0 from lane 31 of the
-// previous pass; only the warp's first pass reads them from memory.
-// NARROW: the grid's thread count fits 32 bits (a separate instantiation:
-// a run-time choice of the index width measured 5 % slower)
-template <typename T, int K, bool NARROW>
-__global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 : 1) k_conv(ConvParams p) {
+template <typename T, int K, bool SILU>
+__global__ void __launch_bounds__(kConvThreads, (sizeof(T) == 2 && K <= 4) ? 4 : 2) k_conv(ConvParams p) {
+  using G = ConvFwdPass<T>;
+  constexpr int S = G::S, H = G::H, W = G::W, KM = K - 1, KA = K > 1 ? K - 1 : 1;
   const int lane = threadIdx.x & 31;
-  const int64_t L = p.L;
-  const ConvWarp cw((L + kConvSeg - 1) / kConvSeg, p.batch * p.dim, p.dim, NARROW);
-  if (!cw.live) return;  // whole warps leave together
-  const int64_t row = cw.row, seg = cw.seg, d = cw.d;
+  const int64_t L = p.L, segs = (L + G::SEG - 1) / G::SEG;
+  const int64_t wid = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) >> 5;
+  const int64_t row = wid / segs, seg = wid - row * segs;
+  if (row >= p.batch * p.dim) return;  // whole warps leave together
+  const int64_t d = row % p.dim;
   const T *xr = static_cast<const T *>(p.x) + row * L;
   T *orow = static_cast<T *>(p.out) + row * L;
-  const bool vec = p.vec != 0;
-  Raw8<T> raw[kConvR];
+  const int64_t tw = seg * G::SEG;
+  uint32_t xw[G::P][W];
 #pragma unroll
-  for (int r = 0; r < kConvR; ++r) raw[r].load(xr, seg * kConvSeg + r * 32 * kConvW + lane * kConvW, L, vec);
-  float w[K];
+  for (int r = 0; r < G::P; ++r) {
+    const int64_t t0 = tw + r * G::PASS + lane * S;
+    conv_load_chunk<T, W>(xw[r], xr + t0, L - t0, p.vec);
+  }
+  f2 w2[K];
 #pragma unroll
-  for (int k = 0; k < K; ++k) w[k] = p.w[d * K + k];
-  const float bias = p.bias ? p.bias[d] : 0.f;
-  float carry[K > 1 ? K - 1 : 1];  // the K-1 inputs before the pass, as lane 31 of the last pass saw them
+  for (int k = 0; k < K; ++k) w2[k] = splat2(p.w[d * K + k]);
+  const f2 bias2 = splat2(p.bias ? p.bias[d] : 0.f);
+  // lane 31's inputs before the next pass reach lane 0 by the shuffle below; before
+  // the warp's first pass they come from memory (lane 31 loads them)
+  float prevtail[KA];
 #pragma unroll
-  for (int r = 0; r < kConvR; ++r) {
-    const int64_t t0 = seg * kConvSeg + r * 32 * kConvW + lane * kConvW;
-    if (seg * kConvSeg + r * 32 * kConvW >= L) break;  // warp-uniform
-    float v[kConvW];
-    raw[r].unpack(v);
-    float halo[K > 1 ? K - 1 : 1];
+  for (int m = 0; m < KM; ++m) prevtail[m] = (lane == 31 && tw > 0) ? IO<T>::get(xr, tw - KM + m) : 0.f;
 #pragma unroll
-    for (int i = 0; i < K - 1; ++i) {
-      const float up = __shfl_up_sync(0xffffffffu, v[kConvW - (K - 1) + i], 1);
-      const float last = __shfl_sync(0xffffffffu, v[kConvW - (K - 1) + i], 31);
-      if (lane > 0) {
-        halo[i] = up;
-      } else if (r > 0) {
-        halo[i] = carry[i];
-      } else {
-        const int64_t t = t0 - (K - 1) + i;  // the warp's first pass: memory or the initial state
-        halo[i] = t >= 0 ? IO<T>::get(xr, t) : (p.s0 ? p.s0[row * (K - 1) + (K - 1) + t] : 0.f);
-      }
-      carry[i] = last;
+  for (int r = 0; r < G::P; ++r) {
+    if (tw + r * G::PASS >= L) break;  // warp-uniform
+    const int64_t t0 = tw + r * G::PASS + lane * S;
+    float hal[KA];
+#pragma unroll
+    for (int m = 0; m < KM; ++m) {
+      const float cur = raw_at<T>(xw[r], S - KM + m);
+      float h = __shfl_sync(0xffffffffu, lane == 31 ? prevtail[m] : cur, (lane + 31) & 31);
+      prevtail[m] = cur;
+      if (lane == 0 && tw == 0 && r == 0) h = p.s0 ? p.s0[row * KM + m] : 0.f;
+      hal[m] = h;
     }
-    float o[kConvW];
+    auto xp = [&](int m) -> f2 {
+      return pack2(m < 0 ? hal[m + KM] : raw_at<T>(xw[r], m), raw_at<T>(xw[r], m + H));
+    };
+    float lo_o[H], hi_o[H];
 #pragma unroll
-    for (int i = 0; i < kConvW; ++i) {
-      float acc = bias;
+    for (int q = 0; q < H; ++q) {
+      f2 a = bias2;
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int idx = i - (K - 1) + k;  // position in [halo | v]
-        acc = fmaf(w[k], idx < 0 ? halo[idx + K - 1] : v[idx], acc);
-      }
-      o[i] = acc;
-    }
-    if (p.silu) {  // SiLU(a) = a / (1 + e^-a), on pairs
-#pragma unroll
-      for (int i = 0; i < kConvW; i += 2) {
-        const f2 a2 = pack2(o[i], o[i + 1]);
+      for (int k = 0; k < K; ++k) a = fma2(w2[k], xp(q - KM + k), a);
+      if constexpr (SILU) {  // SiLU(a) = a / (1 + e^-a), on the pair
         float e0, e1, d0, d1;
-        unpack2(mul2(a2, pack2(-kLog2e, -kLog2e)), e0, e1);
-        unpack2(add2(pack2(ex2(e0), ex2(e1)), pack2(1.f, 1.f)), d0, d1);
-        unpack2(mul2(a2, pack2(rcp_approx(d0), rcp_approx(d1))), o[i], o[i + 1]);
+        unpack2(mul2(a, splat2(-kLog2e)), e0, e1);
+        unpack2(add2(pack2(ex2(e0), ex2(e1)), splat2(1.f)), d0, d1);
+        a = mul2(a, pack2(rcp_approx(d0), rcp_approx(d1)));
       }
+      unpack2(a, lo_o[q], hi_o[q]);
     }
-    if (t0 < L) {
-      if (vec && t0 + kConvW <= L) {
-        if constexpr (sizeof(T) == 2) {
-          uint4 q;
-          q.x = pack_bf16x2(o[0], o[1]); q.y = pack_bf16x2(o[2], o[3]);
-          q.z = pack_bf16x2(o[4], o[5]); q.w = pack_bf16x2(o[6], o[7]);
-          __stcs(reinterpret_cast<uint4 *>(orow + t0), q);
+    const int64_t rem = L - t0;
+    if (rem > 0) {
+      if constexpr (sizeof(T) == 2) {
+        if (p.vec == 2 && rem >= S) {  // the lane's 32 bytes: whole sectors
+          asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(orow + t0),
+                       "r"(pack_bf16x2(lo_o[0], lo_o[1])), "r"(pack_bf16x2(lo_o[2], lo_o[3])),
+                       "r"(pack_bf16x2(lo_o[4], lo_o[5])), "r"(pack_bf16x2(lo_o[6], lo_o[7])),
+                       "r"(pack_bf16x2(hi_o[0], hi_o[1])), "r"(pack_bf16x2(hi_o[2], hi_o[3])),
+                       "r"(pack_bf16x2(hi_o[4], hi_o[5])), "r"(pack_bf16x2(hi_o[6], hi_o[7]))
+                       : "memory");
         } else {
-          __stcs(reinterpret_cast<float4 *>(orow + t0), make_float4(o[0], o[1], o[2], o[3]));
-          __stcs(reinterpret_cast<float4 *>(orow + t0 + 4), make_float4(o[4], o[5], o[6], o[7]));
+          IO<T>::store8(orow, t0, L, p.vec != 0, lo_o);
+          if (rem > H) IO<T>::store8(orow, t0 + H, L, p.vec != 0, hi_o);
         }
       } else {
-        IO<T>::store8(orow, t0, L, false, o);
-      }
-    }
-    // final state: the last K-1 inputs of the row, written by the lane holding step L-1
-    if (K > 1 && p.s1 && t0 <= L - 1 && L - 1 < t0 + kConvW) {
-#pragma unroll
-      for (int i = 0; i < K - 1; ++i) {
-        const int idx = (int)(L - (K - 1) + i - t0);  // position in v, or in halo when negative
-        float val = 0.f;                             // (idx >= -(K - 1) always holds here)
-#pragma unroll
-        for (int m = 0; m < kConvW; ++m)
-          if (m == idx) val = v[m];
-#pragma unroll
-        for (int m = 0; m < K - 1; ++m)
-          if (m - (K - 1) == idx) val = halo[m];
-        p.s1[row * (K - 1) + i] = val;
+        IO<T>::store8(orow, t0, L, p.vec != 0, lo_o);
+        if (rem > H) IO<T>::store8(orow, t0 + H, L, p.vec != 0, hi_o);
       }
     }
   }
+  // final state: the row's last K-1 inputs, by lane 0 of the warp holding step L-1
+  if (KM > 0 && p.s1 && lane == 0 && tw + G::SEG >= L) {
+#pragma unroll
+    for (int m = 0; m < KM; ++m) {
+      const int64_t t = L - KM + m;
+      p.s1[row * KM + m] = t >= 0 ? IO<T>::get(xr, t) : (p.s0 ? p.s0[row * KM + KM + t] : 0.f);
+    }
+  }
+}
+
+template <typename T, int K>
+static cudaError_t launch_conv_fwd_k(const ConvParams &p, cudaStream_t s) {
+  using G = ConvFwdPass<T>;
+  const int64_t segs = (p.L + G::SEG - 1) / G::SEG;
+  const int64_t warps = p.batch * p.dim * segs;
+  const int64_t blocks = (warps * 32 + kConvThreads - 1) / kConvThreads;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  if (p.silu) k_conv<T, K, true><<<(unsigned)blocks, kConvThreads, 0, s>>>(p);
+  else k_conv<T, K, false><<<(unsigned)blocks, kConvThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
+  switch (p.K) {
+    case 1: return launch_conv_fwd_k<T, 1>(p, s);
+    case 2: return launch_conv_fwd_k<T, 2>(p, s);
+    case 3: return launch_conv_fwd_k<T, 3>(p, s);
+    case 4: return launch_conv_fwd_k<T, 4>(p, s);
+    case 5: return launch_conv_fwd_k<T, 5>(p, s);
+    case 6: return launch_conv_fwd_k<T, 6>(p, s);
+    case 7: return launch_conv_fwd_k<T, 7>(p, s);
+    case 8: return launch_conv_fwd_k<T, 8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s) {
+  return io_dtype == 1 ? launch_conv_t<uint16_t>(p, s) : launch_conv_t<float>(p, s);
 }
 
 // ---- backward -------------------------------------------------------------
@@ -240,35 +259,6 @@ struct ConvBwdGeo {
 // Wider filters hold more edge pairs and take 4.
 template <typename T, int K>
 constexpr int conv_bwd_min_blocks() { return sizeof(T) == 2 ? (K <= 4 ? 5 : 4) : 2; }
-
-__device__ __forceinline__ void conv_cp16(uint32_t dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void conv_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void conv_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// value i of a lane's raw chunk (bf16 pairs per word, or fp32 words)
-template <typename T>
-__device__ __forceinline__ float raw_at(const uint32_t *w, int i) {
-  if constexpr (sizeof(T) == 2)
-    return __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
-  else
-    return __uint_as_float(w[i]);
-}
-
-__device__ __forceinline__ float lo_of(f2 v) {
-  float lo, hi;
-  unpack2(v, lo, hi);
-  return lo;
-}
-__device__ __forceinline__ float hi_of(f2 v) {
-  float lo, hi;
-  unpack2(v, lo, hi);
-  return hi;
-}
 
 // da = dout * SiLU'(a) = g s (1 + a (1 - s)), s = 1 / (1 + e^-a), on a pair
 __device__ __forceinline__ f2 silu_grad2(f2 a, f2 g) {
@@ -542,36 +532,6 @@ __global__ void __launch_bounds__(ConvBwdGeo<T>::WARPS * 32, (conv_bwd_min_block
     }
   }
   conv_wait<0>();  // no copy outlives the kernel (the last groups are empty)
-}
-
-template <typename T, bool NARROW>
-static cudaError_t launch_conv_k(const ConvParams &p, unsigned g, cudaStream_t s) {
-  switch (p.K) {
-    case 1: k_conv<T, 1, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 2: k_conv<T, 2, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 3: k_conv<T, 3, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 4: k_conv<T, 4, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 5: k_conv<T, 5, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 6: k_conv<T, 6, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 7: k_conv<T, 7, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    case 8: k_conv<T, 8, NARROW><<<g, kConvThreads, 0, s>>>(p); break;
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-template <typename T>
-static cudaError_t launch_conv_t(const ConvParams &p, cudaStream_t s) {
-  const int64_t segs = (p.L + kConvSeg - 1) / kConvSeg;
-  const int64_t warps = p.batch * p.dim * segs;
-  const int64_t blocks = (warps * 32 + kConvThreads - 1) / kConvThreads;
-  if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  const unsigned g = (unsigned)blocks;
-  return blocks * kConvThreads <= 0xffffffffll ? launch_conv_k<T, true>(p, g, s) : launch_conv_k<T, false>(p, g, s);
-}
-
-cudaError_t launch_conv(int io_dtype, const ConvParams &p, cudaStream_t s) {
-  return io_dtype == 1 ? launch_conv_t<uint16_t>(p, s) : launch_conv_t<float>(p, s);
 }
 
 template <typename T, int K>

@@ -82,6 +82,25 @@ def test_conv_unaligned_rows_take_the_scalar_path(cuda_device):
     _check(3, 7, 77, 4, synth.BF16, 11, cuda_device)
 
 
+def test_conv_sixteen_byte_aligned_buffers(cuda_device):
+    # x 16 bytes into its allocation: rows of 1024 steps take 16-byte accesses instead
+    # of 32-byte ones; same results
+    import torch
+    import selective_state_space_54_b200 as ssm
+    x, w, b, s0 = _inputs(2, 8, 1024, 4, synth.BF16, 61)
+    ref, ref_s = oracle.conv1d(x, w, b, dtype=synth.BF16, initial_state=s0, silu=True)
+    dense = to_torch(x, synth.BF16, cuda_device)
+    flat = torch.empty(dense.numel() + 8, dtype=dense.dtype, device=cuda_device)
+    xv = flat[8:].view(dense.shape)
+    xv.copy_(dense)
+    assert xv.data_ptr() % 32 == 16
+    f = lambda a: torch.from_numpy(a).to(cuda_device)
+    out, fs = ssm.causal_conv1d(xv, f(w), f(b), initial_state=f(s0), silu=True, return_final_state=True)
+    torch.cuda.synchronize()
+    assert_close(to_f64(out), ref, synth.BF16, "out")
+    assert np.array_equal(to_f64(fs), ref_s)
+
+
 def test_conv_full_mamba_2p8b_layer(cuda_device):
     # the Mamba-2.8B layer's x_proj shape (batch 4, d_inner 5120, L 8192), sampled rows
     import torch
