@@ -19,10 +19,11 @@
 // A lane owns S = 8 consecutive states of a channel (LPC = N / 8 lanes per
 // channel), so that per-channel work (softplus, gate, indexing) is shared by
 // 8 states.  On the vector path (N % 8 == 0, 16-byte rows) a block takes
-// kRows batch rows of its channels and starts all their state copies with
-// cp.async before computing the first (k_step_rows); other shapes take one
-// row per block and plain masked loads (k_step).  The state is read and
-// written with evict-first hints: it is touched once per token.  A, B and C
+// kRows batch rows of its channels and loads all their state slices into
+// registers before computing the first, one 32-byte load per row where the
+// state is 32-byte aligned (k_step_rows); other shapes take one row per block
+// and plain masked loads (k_step).  The state is read and written with
+// streaming (evict-first) accesses: it is touched once per token.  A, B and C
 // are re-read across batch elements or channels and are served from L2/L1.
 #include "ssm_common.cuh"
 
@@ -148,46 +149,20 @@ static cudaError_t launch_step_k(const StepParams &p, cudaStream_t s) {
 
 // ---- vector path: several batch rows per block ------------------------------
 // A block owns kStepThreads / LPC channels and kRows batch rows.  Every lane
-// first starts the cp.async copies of its S states for all kRows rows (no
-// registers are held while they are in flight), loads A, D and the bias of
-// its channel once for all rows, and then walks the rows as their copies
-// land.  About kRows * 32 bytes of state per thread are in flight, which a
-// load-compute-store thread could only match with far more registers.  Each
-// lane reads back only what it copied itself: no block barrier.
+// first loads its S states of all kRows rows into registers (one 32-byte load
+// per row; two 16-byte ones when the state is only 16-byte aligned), loads A,
+// D and the bias of its channel once for all rows, and then walks the rows.
+// kRows * 32 bytes of state per thread are in flight before the first row
+// computes.  Held to 80 registers for 3 blocks (24 warps) per SM: on B200 at
+// the Mamba-2.8B decode shape (batch 128) 20.8 us per step, against 22.8 us
+// at 2 blocks per SM (128 registers), 30.0 us at 4 (64 registers, spilling)
+// and 25.0 us for the same rows fed through a cp.async ring in shared memory.
+// 2, 3, 5 or 6 rows per block measured slower than 4.
 constexpr int kRows = 4;
-static_assert(kRows >= 1 && kRows <= 8, "the wait below takes up to 7 groups still in flight");
-
-// wait until at most `pending` copy groups are in flight (a constant once the
-// row loop is unrolled)
-__device__ __forceinline__ void step_wait_groups(int pending) {
-  switch (pending) {
-    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-  }
-}
-
-// L2 policy for data touched once: evict it first
-__device__ __forceinline__ unsigned long long evict_first_policy() {
-  unsigned long long pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-
-__device__ __forceinline__ void cp_async16_ef(void *smem, const void *gmem, unsigned long long pol) {
-  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(sa), "l"(gmem),
-               "l"(pol) : "memory");
-}
 
 template <typename T, int S, int LPC>
-__global__ void __launch_bounds__(kStepThreads) k_step_rows(StepParams p) {
-  extern __shared__ __align__(16) float4 ring[];  // [kRows][S / 4][kStepThreads]
+__global__ void __launch_bounds__(kStepThreads, 3) k_step_rows(StepParams p) {
+  static_assert(S == 8, "a lane's 8 states are one 32-byte access");
   const int tid = threadIdx.x;
   const int64_t slot = (int64_t)blockIdx.x * kStepThreads + tid;
   const int j = (int)(slot % LPC);
@@ -197,16 +172,24 @@ __global__ void __launch_bounds__(kStepThreads) k_step_rows(StepParams p) {
   const int N = p.N, n0 = S * j;
   const int64_t b0 = (int64_t)blockIdx.y * kRows;
   const int rows = (int)(p.batch - b0 < kRows ? p.batch - b0 : kRows);
-  const unsigned long long pol = evict_first_policy();
-  // start every row's state copies (rows past the batch copy row b0 again)
+  // every row's state slice into registers up front (rows past the batch read row b0 again)
+  const bool v32 = (reinterpret_cast<uintptr_t>(p.state) & 31) == 0;
+  float hreg[kRows][S];
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
     const int64_t b = b0 + (r < rows ? r : 0);
     const float *hp = p.state + (b * p.dim + d) * N + n0;
-#pragma unroll
-    for (int q = 0; q < S / 4; ++q)
-      cp_async16_ef(&ring[(r * (S / 4) + q) * kStepThreads + tid], hp + 4 * q, pol);
-    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (v32) {
+      asm volatile("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=f"(hreg[r][0]), "=f"(hreg[r][1]), "=f"(hreg[r][2]), "=f"(hreg[r][3]),
+                     "=f"(hreg[r][4]), "=f"(hreg[r][5]), "=f"(hreg[r][6]), "=f"(hreg[r][7])
+                   : "l"(hp));
+    } else {
+      const float4 h0 = __ldcs(reinterpret_cast<const float4 *>(hp));
+      const float4 h1 = __ldcs(reinterpret_cast<const float4 *>(hp + 4));
+      hreg[r][0] = h0.x; hreg[r][1] = h0.y; hreg[r][2] = h0.z; hreg[r][3] = h0.w;
+      hreg[r][4] = h1.x; hreg[r][5] = h1.y; hreg[r][6] = h1.z; hreg[r][7] = h1.w;
+    }
   }
   // per-channel constants, shared by every row
   float a[S];
@@ -238,15 +221,9 @@ __global__ void __launch_bounds__(kStepThreads) k_step_rows(StepParams p) {
     load_io<S>(static_cast<const T *>(p.C) + b * N, true, n0, N, Cv);
     const float dl = p.softplus ? softplus_fast(ss[r]) : ss[r];
     const float du = dl * uu[r];
-    // wait for this row's copies (groups were committed in row order: the later
-    // rows' groups may still be in flight)
-    step_wait_groups(kRows - 1 - r);
     float h[S];
 #pragma unroll
-    for (int q = 0; q < S / 4; ++q) {
-      const float4 hv = ring[(r * (S / 4) + q) * kStepThreads + tid];
-      h[4 * q] = hv.x; h[4 * q + 1] = hv.y; h[4 * q + 2] = hv.z; h[4 * q + 3] = hv.w;
-    }
+    for (int i = 0; i < S; ++i) h[i] = hreg[r][i];
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int i = 0; i < S; i += 2) {
@@ -264,10 +241,16 @@ __global__ void __launch_bounds__(kStepThreads) k_step_rows(StepParams p) {
     for (int o = LPC / 2; o > 0; o >>= 1) yp += __shfl_xor_sync(0xffffffffu, yp, o);
     if (live && r < rows) {
       float *hp = p.state + (b * p.dim + d) * N + n0;
+      if (v32) {
+        asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(hp), "f"(h[0]), "f"(h[1]),
+                     "f"(h[2]), "f"(h[3]), "f"(h[4]), "f"(h[5]), "f"(h[6]), "f"(h[7])
+                     : "memory");
+      } else {
 #pragma unroll
-      for (int q = 0; q < S / 4; ++q)
-        __stcs(reinterpret_cast<float4 *>(hp + 4 * q),
-               make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
+        for (int q = 0; q < S / 4; ++q)
+          __stcs(reinterpret_cast<float4 *>(hp + 4 * q),
+                 make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
+      }
       if (j == 0) {
         float y = yp + Dd * uu[r];
         if (p.z) y *= silu_fast(zz[r]);
@@ -283,8 +266,7 @@ static cudaError_t launch_step_rows(const StepParams &p, cudaStream_t s) {
   const int64_t bx = (slots + kStepThreads - 1) / kStepThreads;
   const int64_t by = (p.batch + kRows - 1) / kRows;
   if (bx > 0x7fffffff || by > 65535) return launch_step_k<T, S, LPC>(p, s);
-  const size_t smem = (size_t)kRows * S * sizeof(float) * kStepThreads;  // 32 KB at S = 8
-  k_step_rows<T, S, LPC><<<dim3((unsigned)bx, (unsigned)by), kStepThreads, smem, s>>>(p);
+  k_step_rows<T, S, LPC><<<dim3((unsigned)bx, (unsigned)by), kStepThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
