@@ -531,6 +531,51 @@ def decode_bytes(w: synth.Workload) -> int:
             + 4 * w.dim * w.dstate + 8 * w.dim)
 
 
+def copy_same_bytes(torch, dev, stream, nbytes, slots, k, graph, barrier, max_over_ranks):
+    """A plain device-to-device copy moving the same bytes as one step (nbytes/2
+    read, nbytes/2 written), over `slots` buffer pairs cycled like the step's
+    inputs and timed the same way (CUDA graph replay or eager launches).  It is
+    torch's copy kernel, not this library's: the bandwidth a copy reaches at
+    this size, beside the large-copy peak the roofline divides by."""
+    half = (nbytes // 2 + 255) // 256 * 256
+    src = [torch.empty(half, dtype=torch.uint8, device=dev).fill_(i + 1) for i in range(slots)]
+    dst = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(slots)]
+
+    def run():
+        for i in range(k):
+            dst[i % slots].copy_(src[i % slots])
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                run()
+        torch.cuda.synchronize(dev)
+        g.replay()
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    if graph:
+        g.replay()
+    else:
+        run()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / k)
+    if graph:
+        del g
+    del src, dst
+    return {"us_per_copy": ms * 1e3, "bytes": 2 * half, "gbs": 2 * half / (ms * 1e-3) / 1e9,
+            "timing": "CUDA graph replay" if graph else "eager launches", "slots": slots}
+
+
 def measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None):
     """Single-token steps on the decode workload, replayed from a CUDA graph.
 
@@ -600,6 +645,8 @@ def measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None
     nbytes = decode_bytes(w)
     pk = peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
+    cp = copy_same_bytes(torch, dev, stream, nbytes, slots, k, True, barrier, max_over_ranks)
+    cp["step_frac_of_copy"] = achieved / cp["gbs"]
     return {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate,
             "io_dtype": w.dtype, "state_dtype": "f32", "steps": k, "state_slots": slots,
             "l2": f"{slots} state slots of {8 * w.batch * w.dim * w.dstate // 2 / 1e6:.0f} MB cycled",
@@ -610,6 +657,7 @@ def measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None
                          "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
                          "kernel": "k_step", "algorithmic_bytes": nbytes,
                          "peak_basis": f"measured copy bandwidth ({pk['source']})"},
+            "copy_same_bytes": cp,
             "gpu_launches": k}
 
 
@@ -660,6 +708,8 @@ def measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None, 
     nbytes_b = 3 * es * w.bld + 4 * w.dim * (2 * width + 2)
     pk = peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
+    cp = copy_same_bytes(torch, dev, stream, nbytes, 1, k, False, barrier, max_over_ranks)
+    cp["conv_frac_of_copy"] = achieved / cp["gbs"]
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.dim,
             "width": width, "io_dtype": w.dtype, "silu": True, "steps": k,
             "l2": "inputs larger than L2 (no flush)", "ms_per_step": ms,
@@ -671,6 +721,7 @@ def measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None, 
             "bwd": {"ms_per_step": ms_b, "algorithmic_bytes": nbytes_b,
                     "achieved_gbs": nbytes_b / (ms_b * 1e-3) / 1e9,
                     "frac": nbytes_b / (ms_b * 1e-3) / 1e9 / pk["hbm_gbs"], "kernel": "k_conv_bwd"},
+            "copy_same_bytes": cp,
             "gpu_launches": k}
 
 

@@ -18,13 +18,16 @@
 // bound by HBM: the kernel's job is to keep enough state bytes in flight.
 // A lane owns S = 8 consecutive states of a channel (LPC = N / 8 lanes per
 // channel), so that per-channel work (softplus, gate, indexing) is shared by
-// 8 states.  On the vector path (N % 8 == 0, 16-byte rows) a block takes
-// kRows batch rows of its channels and loads all their state slices into
-// registers before computing the first, one 32-byte load per row where the
-// state is 32-byte aligned (k_step_rows); other shapes take one row per block
-// and plain masked loads (k_step).  The state is read and written with
-// streaming (evict-first) accesses: it is touched once per token.  A, B and C
-// are re-read across batch elements or channels and are served from L2/L1.
+// 8 states.  On the vector path (N % 8 == 0, 16-byte rows) persistent blocks
+// walk the batch rows of their channels with the next row's state slices in
+// flight while the current one computes (k_step_rows); other shapes take one
+// row per block and plain masked loads (k_step).  The state is read and
+// written with streaming (evict-first) accesses: it is touched once per token.
+// A, B and C are re-read across batch elements or channels and are served
+// from L2/L1.
+#include <algorithm>
+#include <atomic>
+
 #include "ssm_common.cuh"
 
 namespace ssm {
@@ -147,50 +150,49 @@ static cudaError_t launch_step_k(const StepParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// ---- vector path: several batch rows per block ------------------------------
-// A block owns kStepThreads / LPC channels and kRows batch rows.  Every lane
-// first loads its S states of all kRows rows into registers (one 32-byte load
-// per row; two 16-byte ones when the state is only 16-byte aligned), loads A,
-// D and the bias of its channel once for all rows, and then walks the rows.
-// kRows * 32 bytes of state per thread are in flight before the first row
-// computes.  Held to 80 registers for 3 blocks (24 warps) per SM: on B200 at
-// the Mamba-2.8B decode shape (batch 128) 20.8 us per step, against 22.8 us
-// at 2 blocks per SM (128 registers), 30.0 us at 4 (64 registers, spilling)
-// and 25.0 us for the same rows fed through a cp.async ring in shared memory.
-// 2, 3, 5 or 6 rows per block measured slower than 4.
-constexpr int kRows = 4;
+// ---- vector path: persistent blocks over batch rows ---------------------------
+// A block owns kStepThreads / LPC channels (a channel slice) and walks the
+// batch rows b = kb, kb + bps, ... of that slice, bps blocks per slice, as
+// many as fill the SMs in one wave.  Every lane keeps two row buffers in
+// registers: the next row's S states (one 32-byte load where the state is
+// 32-byte aligned, two 16-byte ones otherwise) and its u, delta and z are
+// loaded before the current row computes, and the state and token lines of
+// the row after that are prefetched into L2, so that each lane has a row in
+// flight while it computes.  A, D and the bias of the lane's channel are
+// loaded once.
+// Held to 64 registers for 4 blocks (32 warps) per SM with bf16 token data
+// (3 blocks with fp32, whose wider loads spill at 64).  On B200 at the
+// Mamba-2.8B decode shape (batch 128, token inputs cycled over 4 slots so
+// that they come from DRAM, CUDA graph replay): 18.3 us per step, against
+// 20.0 us without the token-line prefetch (the 2-byte token loads then wait
+// on DRAM every row), 22.4 us when B and C lines are prefetched as well,
+// 19.9 us with B and C staged through a shared-memory ring, and 20.9 us for
+// non-persistent blocks of 4 rows loaded up front; a plain device copy of the
+// same bytes takes 15.5 us.  With inputs that stay in L2 a third row buffer
+// (two rows in flight) measured 20.7 against 18.6 us, rows taken in pairs at
+// 3 blocks per SM 19.6 us.
+template <typename T>
+constexpr int step_blocks_per_sm() { return sizeof(T) == 2 ? 4 : 3; }
+
+// one batch row of a lane's channel: its state slice and token inputs
+template <int S>
+struct StepRow {
+  float h[S];
+  float u, s, z;  // s = delta + bias
+};
 
 template <typename T, int S, int LPC>
-__global__ void __launch_bounds__(kStepThreads, 3) k_step_rows(StepParams p) {
+__global__ void __launch_bounds__(kStepThreads, step_blocks_per_sm<T>()) k_step_rows(StepParams p, int bps) {
   static_assert(S == 8, "a lane's 8 states are one 32-byte access");
   const int tid = threadIdx.x;
-  const int64_t slot = (int64_t)blockIdx.x * kStepThreads + tid;
+  const int slice = (int)(blockIdx.x / bps), kb = (int)(blockIdx.x - slice * bps);
+  const int64_t slot = (int64_t)slice * kStepThreads + tid;
   const int j = (int)(slot % LPC);
   int64_t d = slot / LPC;
   const bool live = d < p.dim;
   if (!live) d = p.dim - 1;  // lanes past the row compute on its last channel, store nothing
   const int N = p.N, n0 = S * j;
-  const int64_t b0 = (int64_t)blockIdx.y * kRows;
-  const int rows = (int)(p.batch - b0 < kRows ? p.batch - b0 : kRows);
-  // every row's state slice into registers up front (rows past the batch read row b0 again)
   const bool v32 = (reinterpret_cast<uintptr_t>(p.state) & 31) == 0;
-  float hreg[kRows][S];
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) {
-    const int64_t b = b0 + (r < rows ? r : 0);
-    const float *hp = p.state + (b * p.dim + d) * N + n0;
-    if (v32) {
-      asm volatile("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                   : "=f"(hreg[r][0]), "=f"(hreg[r][1]), "=f"(hreg[r][2]), "=f"(hreg[r][3]),
-                     "=f"(hreg[r][4]), "=f"(hreg[r][5]), "=f"(hreg[r][6]), "=f"(hreg[r][7])
-                   : "l"(hp));
-    } else {
-      const float4 h0 = __ldcs(reinterpret_cast<const float4 *>(hp));
-      const float4 h1 = __ldcs(reinterpret_cast<const float4 *>(hp + 4));
-      hreg[r][0] = h0.x; hreg[r][1] = h0.y; hreg[r][2] = h0.z; hreg[r][3] = h0.w;
-      hreg[r][4] = h1.x; hreg[r][5] = h1.y; hreg[r][6] = h1.z; hreg[r][7] = h1.w;
-    }
-  }
   // per-channel constants, shared by every row
   float a[S];
   {
@@ -204,26 +206,47 @@ __global__ void __launch_bounds__(kStepThreads, 3) k_step_rows(StepParams p) {
   }
   const float bias = p.bias ? p.bias[d] : 0.f;
   const float Dd = p.D ? p.D[d] : 0.f;
-  // the token inputs of every row
-  float uu[kRows], ss[kRows], zz[kRows];
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) {
-    const int64_t ch = (b0 + (r < rows ? r : 0)) * p.dim + d;
-    uu[r] = IO<T>::get(static_cast<const T *>(p.u), ch);
-    ss[r] = IO<T>::get(static_cast<const T *>(p.delta), ch) + bias;
-    zz[r] = p.z ? IO<T>::get(static_cast<const T *>(p.z), ch) : 0.f;
-  }
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) {
-    const int64_t b = b0 + (r < rows ? r : 0);
+
+  auto load = [&](StepRow<S> &r, int64_t b) {
+    const float *hp = p.state + (b * p.dim + d) * N + n0;
+    if (v32) {
+      asm volatile("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                   : "=f"(r.h[0]), "=f"(r.h[1]), "=f"(r.h[2]), "=f"(r.h[3]), "=f"(r.h[4]), "=f"(r.h[5]),
+                     "=f"(r.h[6]), "=f"(r.h[7])
+                   : "l"(hp));
+    } else {
+      const float4 h0 = __ldcs(reinterpret_cast<const float4 *>(hp));
+      const float4 h1 = __ldcs(reinterpret_cast<const float4 *>(hp + 4));
+      r.h[0] = h0.x; r.h[1] = h0.y; r.h[2] = h0.z; r.h[3] = h0.w;
+      r.h[4] = h1.x; r.h[5] = h1.y; r.h[6] = h1.z; r.h[7] = h1.w;
+    }
+    const int64_t ch = b * p.dim + d;
+    r.u = IO<T>::get(static_cast<const T *>(p.u), ch);
+    r.s = IO<T>::get(static_cast<const T *>(p.delta), ch) + bias;
+    r.z = p.z ? IO<T>::get(static_cast<const T *>(p.z), ch) : 0.f;
+  };
+  // a later row's state lines and u, delta, z lines into L2, one lane per
+  // 128-byte line (4 lanes of state; 128 / sizeof(T) channels of token data)
+  constexpr int kTokLineLanes = LPC * 128 / (int)sizeof(T);
+  auto prefetch = [&](int64_t b) {
+    if (b < p.batch && (tid & 3) == 0)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p.state + (b * p.dim + d) * N + n0));
+    if (b < p.batch && tid % kTokLineLanes == 0) {
+      const int64_t ch = b * p.dim + d;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const T *>(p.u) + ch));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const T *>(p.delta) + ch));
+      if (p.z) asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const T *>(p.z) + ch));
+    }
+  };
+  auto run = [&](const StepRow<S> &r, int64_t b) {
     float Bv[S], Cv[S];
     load_io<S>(static_cast<const T *>(p.B) + b * N, true, n0, N, Bv);
     load_io<S>(static_cast<const T *>(p.C) + b * N, true, n0, N, Cv);
-    const float dl = p.softplus ? softplus_fast(ss[r]) : ss[r];
-    const float du = dl * uu[r];
+    const float dl = p.softplus ? softplus_fast(r.s) : r.s;
+    const float du = dl * r.u;
     float h[S];
 #pragma unroll
-    for (int i = 0; i < S; ++i) h[i] = hreg[r][i];
+    for (int i = 0; i < S; ++i) h[i] = r.h[i];
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int i = 0; i < S; i += 2) {
@@ -239,34 +262,77 @@ __global__ void __launch_bounds__(kStepThreads, 3) k_step_rows(StepParams p) {
     float yp = y0 + y1;
 #pragma unroll
     for (int o = LPC / 2; o > 0; o >>= 1) yp += __shfl_xor_sync(0xffffffffu, yp, o);
-    if (live && r < rows) {
-      float *hp = p.state + (b * p.dim + d) * N + n0;
-      if (v32) {
-        asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(hp), "f"(h[0]), "f"(h[1]),
-                     "f"(h[2]), "f"(h[3]), "f"(h[4]), "f"(h[5]), "f"(h[6]), "f"(h[7])
-                     : "memory");
-      } else {
+    if (!live) return;
+    float *hp = p.state + (b * p.dim + d) * N + n0;
+    if (v32) {
+      asm volatile("st.global.cs.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(hp), "f"(h[0]), "f"(h[1]),
+                   "f"(h[2]), "f"(h[3]), "f"(h[4]), "f"(h[5]), "f"(h[6]), "f"(h[7])
+                   : "memory");
+    } else {
 #pragma unroll
-        for (int q = 0; q < S / 4; ++q)
-          __stcs(reinterpret_cast<float4 *>(hp + 4 * q),
-                 make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
-      }
-      if (j == 0) {
-        float y = yp + Dd * uu[r];
-        if (p.z) y *= silu_fast(zz[r]);
-        IO<T>::store1(static_cast<T *>(p.y), b * p.dim + d, y);
-      }
+      for (int q = 0; q < S / 4; ++q)
+        __stcs(reinterpret_cast<float4 *>(hp + 4 * q), make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
     }
+    if (j == 0) {
+      float y = yp + Dd * r.u;
+      if (p.z) y *= silu_fast(r.z);
+      IO<T>::store1(static_cast<T *>(p.y), b * p.dim + d, y);
+    }
+  };
+
+  // rows kb, kb + bps, ... through the two buffers; the trip count is the
+  // block's own, so every lane of a warp takes part in each row's shuffles
+  int64_t b = kb;
+  if (b >= p.batch) return;
+  StepRow<S> r0, r1;
+  load(r0, b);
+  for (;;) {
+    const int64_t b1 = b + bps, b2 = b1 + bps;
+    if (b1 < p.batch) load(r1, b1);
+    prefetch(b2);
+    run(r0, b);
+    if (b1 >= p.batch) break;
+    if (b2 < p.batch) load(r0, b2);
+    prefetch(b2 + bps);
+    run(r1, b1);
+    if (b2 >= p.batch) break;
+    b = b2;
   }
 }
 
+// Resident blocks of k_step_rows<T, S, LPC> on the current device (SMs x
+// blocks per SM).  Both are properties of the kernel and the device model, so
+// they are looked up once per device ordinal: a decode step is short enough
+// that three runtime queries per call showed in its host time.  Failures are
+// not cached.
+template <typename T, int S, int LPC>
+static cudaError_t step_rows_slots(int &slots) {
+  constexpr int kDevs = 64;
+  static std::atomic<int> cache[kDevs];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kDevs && (slots = cache[dev].load(std::memory_order_relaxed)) > 0) return cudaSuccess;
+  int sms = 0, occ = 0;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_rows<T, S, LPC>, kStepThreads, 0)) !=
+      cudaSuccess)
+    return e;
+  slots = std::max(sms, 1) * std::max(occ, 1);
+  if (dev >= 0 && dev < kDevs) cache[dev].store(slots, std::memory_order_relaxed);
+  return cudaSuccess;
+}
+
+// grid: slices x bps blocks, block kb of a slice taking rows kb, kb + bps, ...
 template <typename T, int S, int LPC>
 static cudaError_t launch_step_rows(const StepParams &p, cudaStream_t s) {
-  const int64_t slots = p.dim * LPC;
-  const int64_t bx = (slots + kStepThreads - 1) / kStepThreads;
-  const int64_t by = (p.batch + kRows - 1) / kRows;
-  if (bx > 0x7fffffff || by > 65535) return launch_step_k<T, S, LPC>(p, s);
-  k_step_rows<T, S, LPC><<<dim3((unsigned)bx, (unsigned)by), kStepThreads, 0, s>>>(p);
+  const int64_t slices = (p.dim * LPC + kStepThreads - 1) / kStepThreads;
+  int slots = 0;
+  const cudaError_t e = step_rows_slots<T, S, LPC>(slots);
+  if (e != cudaSuccess) return e;
+  const int64_t bps = std::max<int64_t>(1, std::min<int64_t>(p.batch, slots / slices));
+  if (slices * bps > 0x7fffffff) return launch_step_k<T, S, LPC>(p, s);
+  k_step_rows<T, S, LPC><<<(unsigned)(slices * bps), kStepThreads, 0, s>>>(p, (int)bps);
   return cudaGetLastError();
 }
 

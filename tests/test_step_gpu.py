@@ -93,6 +93,35 @@ def test_step_ragged_channel_counts(cuda_device, batch, dim):
     _check(case, cuda_device, _state(batch, dim, 16, dim))
 
 
+# Blocks own a channel slice (128 channels at d_state 16) and walk the batch
+# rows kb, kb + bps, ... with bps blocks per slice: one row per block, rows
+# split unevenly between blocks (odd and even counts through the two row
+# buffers), and more slices than the SMs hold (every block walks every row).
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
+@pytest.mark.parametrize("batch,dim", [(7, 2000), (300, 130), (900, 130), (3, 100000)])
+def test_step_rows_per_block(cuda_device, dtype, batch, dim):
+    case = synth.make_case(batch, dim, 1, 16, dtype, seed=batch + dim)
+    _check(case, cuda_device, _state(batch, dim, 16, batch))
+
+
+def test_step_state_only_16_byte_aligned(cuda_device):
+    # the state 16 bytes past a 32-byte boundary: two 16-byte accesses per
+    # lane instead of one 32-byte access
+    import torch
+    batch, dim, N = 5, 300, 16
+    case = synth.make_case(batch, dim, 1, N, synth.BF16, seed=17)
+    h0 = _state(batch, dim, N, 11)
+    buf = torch.zeros(h0.size + 8, dtype=torch.float32, device=cuda_device)
+    assert buf.data_ptr() % 32 == 0
+    st = buf[4:4 + h0.size].view(batch, dim, N)
+    st.copy_(torch.from_numpy(h0))
+    ref = oracle.fwd(case, h0=h0, delta_softplus=True)
+    y, st = _run_step(case, cuda_device, h0, state=st)
+    assert_close(y, ref["y"][:, :, 0], case["dtype"], "y")
+    assert_close(st, ref["last_state"], synth.F32, "state")
+    assert torch.all(buf[:4] == 0) and torch.all(buf[4 + h0.size:] == 0)
+
+
 def test_step_zero_state_matches_scan_of_one_token(cuda_device):
     case = synth.make_case(2, 48, 1, 16, synth.BF16, seed=9)
     _check(case, cuda_device, np.zeros((2, 48, 16), np.float32))
@@ -196,9 +225,9 @@ def test_step_zoh_exact_matches_oracle(cuda_device, N):
     assert_close(to_f64(st), ref["last_state"], synth.F32, "state")
 
 
-def test_step_batch_beyond_the_grid_y_limit(cuda_device):
-    # more row groups than one grid dimension holds (4 * 65535 rows): the
-    # one-row-per-block kernel with its row loop takes over
+def test_step_batch_far_beyond_the_resident_blocks(cuda_device):
+    # a batch far above the blocks that fit on the GPU (270000 rows of one
+    # channel): each block walks several hundred rows
     batch, dim, N = 270000, 1, 16
     case = synth.make_case(batch, dim, 1, N, synth.BF16, seed=16)
     _check(case, cuda_device, _state(batch, dim, N, 10))
