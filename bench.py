@@ -535,8 +535,9 @@ def copy_same_bytes(torch, dev, stream, nbytes, slots, k, graph, barrier, max_ov
     """A plain device-to-device copy moving the same bytes as one step (nbytes/2
     read, nbytes/2 written), over `slots` buffer pairs cycled like the step's
     inputs and timed the same way (CUDA graph replay or eager launches).  It is
-    torch's copy kernel, not this library's: the bandwidth a copy reaches at
-    this size, beside the large-copy peak the roofline divides by."""
+    torch's copy_ of contiguous same-dtype buffers (a device-to-device memcpy),
+    not this library's work: the bandwidth a plain copy reaches at this size,
+    beside the large-copy peak the roofline divides by."""
     half = (nbytes // 2 + 255) // 256 * 256
     src = [torch.empty(half, dtype=torch.uint8, device=dev).fill_(i + 1) for i in range(slots)]
     dst = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(slots)]
