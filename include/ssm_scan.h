@@ -246,7 +246,9 @@ ssm_status ssm_scan_fwd_noalloc(const ssm_shape *shape, const void *u, const voi
  * seqlen times, feeding each token, gives the same y and final state as
  * ssm_scan_fwd over the seqlen tokens with initial_state = state (up to
  * rounding).  dstate % 4 == 0 with 16-byte aligned state and A (and B/C
- * rows aligned to 4 elements) takes 16-byte accesses. */
+ * rows aligned to 4 elements) takes 16-byte accesses; with dstate % 8 == 0 a
+ * lane's 8 states of a row move as one 32-byte access where the state is
+ * 32-byte aligned. */
 ssm_status ssm_scan_step(const ssm_shape *shape, const void *u, const void *delta,
                          const float *A, const void *B, const void *C,
                          const float *D, const void *z, const float *delta_bias,
