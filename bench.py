@@ -37,12 +37,22 @@ METRIC = "selective-scan fwd/bwd tokens·channels/s and % of HBM/SFU roofline, 1
 UNIT = "tokens·channels/s"
 MUFU_EX2_PER_CLK_PER_SM = 16  # special-function unit ex2 rate per SM and clock
 # ncu summaries holding the DRAM traffic of the dominant kernel, per forward path
+def _csrc(*names):
+    return [os.path.join(ROOT, "selective_state_space_54_b200", "csrc", f) for f in names]
+
+
+# committed ncu summary of each timed kernel and the sources it was captured from
 PROFILE_TRAFFIC = {
-    "lookback": os.path.join(ROOT, "profiles", "fwd_lookback_mamba-2.8b-layer.md"),
-    "lookback_ws": os.path.join(ROOT, "profiles", "fwd_ws_mamba-2.8b-layer.md"),
+    "lookback": (os.path.join(ROOT, "profiles", "fwd_lookback_mamba-2.8b-layer.md"),
+                 _csrc("ssm_fwd.cu", "ssm_common.cuh")),
+    "lookback_ws": (os.path.join(ROOT, "profiles", "fwd_ws_mamba-2.8b-layer.md"),
+                    _csrc("ssm_fwd.cu", "ssm_common.cuh")),
+    "decode": (os.path.join(ROOT, "profiles", "step_mamba-2.8b-decode.md"),
+               _csrc("ssm_step.cu", "ssm_common.cuh")),
+    "conv1d": (os.path.join(ROOT, "profiles", "conv1d_mamba-2.8b-layer.md"),
+               _csrc("ssm_conv.cu", "ssm_common.cuh")),
 }
-KERNEL_SOURCES = [os.path.join(ROOT, "selective_state_space_54_b200", "csrc", f)
-                  for f in ("ssm_fwd.cu", "ssm_common.cuh")]
+KERNEL_SOURCES = _csrc("ssm_fwd.cu", "ssm_common.cuh")
 
 
 def parse():
@@ -89,9 +99,9 @@ def alg_bytes(w: synth.Workload) -> int:
     return b
 
 
-def source_sha() -> str:
+def source_sha(sources=None) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources or KERNEL_SOURCES:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -99,7 +109,7 @@ def source_sha() -> str:
 
 def profiled_traffic(path: str):
     """dram bytes per launch from the committed ncu summary, if the kernel is unchanged."""
-    f = PROFILE_TRAFFIC.get(path)
+    f, sources = PROFILE_TRAFFIC.get(path, (None, None))
     if not f or not os.path.exists(f):
         return None
     vals = {}
@@ -107,7 +117,7 @@ def profiled_traffic(path: str):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != source_sha():
+    if vals.get("kernel_source_sha256_16") != source_sha(sources):
         return None
     try:
         return float(vals["dram_bytes_per_launch_full_size"])
@@ -655,8 +665,9 @@ def measure_decode(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None
             "value": aggregate_value(world, w.batch * w.dim, ms * 1e-3),
             "unit": "tokens·channels/s (single-token steps, CUDA graph replay)",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                         "kernel": "k_step", "algorithmic_bytes": nbytes,
+                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                         "traffic": profiled_traffic("decode"),
+                         "kernel": "k_step_rows", "algorithmic_bytes": nbytes,
                          "peak_basis": f"measured copy bandwidth ({pk['source']})"},
             "copy_same_bytes": cp,
             "gpu_launches": k}
@@ -716,7 +727,8 @@ def measure_conv(ssm, torch, dev, args, world, barrier, max_over_ranks, w=None, 
             "l2": "inputs larger than L2 (no flush)", "ms_per_step": ms,
             "value": aggregate_value(world, w.bld, ms * 1e-3), "unit": UNIT,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": "k_conv",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": profiled_traffic("conv1d"),
+                         "kernel": "k_conv",
                          "algorithmic_bytes": nbytes,
                          "peak_basis": f"measured copy bandwidth ({pk['source']})"},
             "bwd": {"ms_per_step": ms_b, "algorithmic_bytes": nbytes_b,
