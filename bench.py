@@ -36,7 +36,6 @@ import synth  # noqa: E402
 METRIC = "selective-scan fwd/bwd tokens·channels/s and % of HBM/SFU roofline, 1 B200"
 UNIT = "tokens·channels/s"
 MUFU_EX2_PER_CLK_PER_SM = 16  # special-function unit ex2 rate per SM and clock
-# ncu summaries holding the DRAM traffic of the dominant kernel, per forward path
 def _csrc(*names):
     return [os.path.join(ROOT, "selective_state_space_54_b200", "csrc", f) for f in names]
 
@@ -51,6 +50,8 @@ PROFILE_TRAFFIC = {
                _csrc("ssm_step.cu", "ssm_common.cuh")),
     "conv1d": (os.path.join(ROOT, "profiles", "conv1d_mamba-2.8b-layer.md"),
                _csrc("ssm_conv.cu", "ssm_common.cuh")),
+    "bwd16": (os.path.join(ROOT, "profiles", "bwd16_mamba-1.4b-layer-train.md"),
+              _csrc("ssm_bwd16.cu", "ssm_common.cuh")),
 }
 KERNEL_SOURCES = _csrc("ssm_fwd.cu", "ssm_common.cuh")
 
@@ -394,7 +395,9 @@ def measure_training(ssm, torch, dev, args, world, barrier, max_over_ranks, w=No
     ex2_peak = sm_count * MUFU_EX2_PER_CLK_PER_SM * pk["sm_max_mhz"] * 1e6
     bwd_achieved = ex2_per_element * w.bldn / (ms_b * 1e-3)
     bwd_roofline = {"bound": "alu", "achieved": bwd_achieved / 1e12, "peak": ex2_peak / 1e12,
-                    "unit": "Tex2/s", "frac": bwd_achieved / ex2_peak, "traffic": None,
+                    "unit": "Tex2/s", "frac": bwd_achieved / ex2_peak,
+                    # the committed capture is of this workload's Euler, channel-major launch
+                    "traffic": profiled_traffic("bwd16") if w.name == "mamba-1.4b-layer-train" else None,
                     "kernel": "k_bwd16", "ex2_per_element": ex2_per_element,
                     "kernel_ex2_per_element": kernel_ex2,
                     "kernel_mufu_frac": kernel_ex2 * w.bldn / (ms_b * 1e-3) / ex2_peak,
