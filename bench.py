@@ -36,6 +36,8 @@ import synth  # noqa: E402
 METRIC = "selective-scan fwd/bwd tokens·channels/s and % of HBM/SFU roofline, 1 B200"
 UNIT = "tokens·channels/s"
 MUFU_EX2_PER_CLK_PER_SM = 16  # special-function unit ex2 rate per SM and clock
+
+
 def _csrc(*names):
     return [os.path.join(ROOT, "selective_state_space_54_b200", "csrc", f) for f in names]
 
