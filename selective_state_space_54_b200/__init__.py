@@ -16,6 +16,7 @@ dstate) fp32.  io tensors are all bf16 or all fp32.
 from __future__ import annotations
 
 import ctypes
+import functools
 
 from . import _lib
 from ._lib import (PATH_NAMES, SSM_BF16, SSM_F32, SSM_FLAG_SAVE_STATES,  # noqa: F401
@@ -72,14 +73,16 @@ def _stream(stream):
 def _check_io(name, t, shape, dtype, device):
     if t is None:
         return
+    # one combined test on the common path; the message is built only on failure
+    if t.is_cuda and t.device == device and t.shape == tuple(shape) and t.dtype == dtype and t.is_contiguous():
+        return
     if not t.is_cuda or t.device != device:
         raise ValueError(f"{name} must be on {device}")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if t.dtype != dtype:
         raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
+    raise ValueError(f"{name} must be contiguous")
 
 
 def _workspace(nbytes, device, workspace):
@@ -152,6 +155,13 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, delta_softpl
     return y
 
 
+@functools.lru_cache(maxsize=64)
+def _step_shape(batch, dim, dstate, io_dtype, flags):
+    # read-only for the library (a const pointer): one struct per shape serves
+    # every decode step of that shape
+    return make_shape(batch, dim, 1, dstate, io_dtype, flags=flags)
+
+
 def scan_step(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, state,
               delta_softplus=True, zoh_exact=False, y=None, stream=None):
     """One recurrent step for every (batch, channel): updates `state` in place
@@ -175,8 +185,7 @@ def scan_step(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, state,
     if y is None:
         y = torch.empty_like(u)
     _check_io("y", y, (batch, dim), dt, dev)
-    shape = make_shape(batch, dim, 1, dstate, _io_dtype(u),
-                       flags=SSM_FLAG_ZOH_EXACT if zoh_exact else 0)
+    shape = _step_shape(batch, dim, dstate, _io_dtype(u), SSM_FLAG_ZOH_EXACT if zoh_exact else 0)
     rc = _lib.load().ssm_scan_step(
         ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(state), _ptr(y), _stream(stream))

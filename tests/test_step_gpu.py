@@ -231,3 +231,37 @@ def test_step_batch_far_beyond_the_resident_blocks(cuda_device):
     batch, dim, N = 270000, 1, 16
     case = synth.make_case(batch, dim, 1, N, synth.BF16, seed=16)
     _check(case, cuda_device, _state(batch, dim, N, 10))
+
+
+def test_step_rejects_bad_arguments(cuda_device):
+    # the binding checks every tensor before the call: wrong device, shape,
+    # dtype or layout raise, and nothing is launched (the state is untouched)
+    import torch
+    import selective_state_space_54_b200 as ssm
+    batch, dim, N = 2, 40, 16
+    case = synth.make_case(batch, dim, 1, N, synth.BF16, seed=18)
+    g = upload(case, cuda_device)
+    x = _step_inputs(g, 0)
+    st = torch.from_numpy(_state(batch, dim, N, 12)).to(cuda_device)
+    keep = st.clone()
+
+    def call(**over):
+        a = dict(u=x["u"], delta=x["delta"], A=g["A"], B=x["B"], C=x["C"], D=g["D"], z=x["z"],
+                 delta_bias=g["delta_bias"])
+        a.update(over)
+        return ssm.scan_step(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["z"], a["delta_bias"],
+                             state=over.get("state", st))
+
+    with pytest.raises(ValueError, match="must be on"):
+        call(delta=x["delta"].cpu())
+    with pytest.raises(ValueError, match="has shape"):
+        call(z=x["z"][:, :-1].contiguous())
+    with pytest.raises(TypeError, match="has dtype"):
+        call(D=g["D"].double())
+    with pytest.raises(ValueError, match="contiguous"):
+        call(state=torch.empty((batch, N, dim), device=cuda_device).transpose(1, 2))
+    torch.cuda.synchronize()
+    assert torch.equal(st, keep)
+    call()  # and the same arguments, corrected, run
+    torch.cuda.synchronize()
+    assert not torch.equal(st, keep)
